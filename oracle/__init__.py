@@ -1,0 +1,6 @@
+"""fp64 CPU oracle for GPTQ-2D (test infrastructure only; never used by the library)."""
+from .gptq2d_oracle import *  # noqa: F401,F403
+from .gptq2d_oracle import (NEAR_TIE_BAND, Result, babai_kron_sweep, closest_vector_exhaustive,
+                            entry_value, gptq2d, gptq2d_antidiagonal, gptq_1d_obs, grid_bounds,
+                            near_tie, nearest_plane_by_definition, proxy_loss, reverse_cholesky,
+                            round_to_grid, rtn, sphere_decode)

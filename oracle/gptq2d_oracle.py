@@ -1,0 +1,372 @@
+"""fp64 CPU oracle for GPTQ-2D two-sided adaptive rounding.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
+the CUDA library (no kernels, headers, helpers, tables or pre/post-processing),
+and the library never imports it.
+
+What it computes (sources are the two on-topic pages):
+  * mind-verse.de "Neue Ansätze ... durch GPTQ-2D", sections "GPTQ-2D: Eine
+    Weiterentwicklung der adaptiven Rundung" (two-sided problem with bases on
+    both sides of the residual) and "Geometrische Grundlagen und der Bezug zu
+    Babai's Nearest Plane Algorithmus" (vectorisation turns the two-sided
+    problem into a quadratic form whose Gram matrix is a Kronecker product;
+    GPTQ is Babai's nearest-plane algorithm on it).
+  * arxivlens "GPTQ-2D: Cubic-Time Two-Sided Adaptive Rounding", Abstract
+    (same rounding as the quartic Kronecker feedback, cubic work, entries of
+    one anti-diagonal rounded in parallel) and Analysis > Results / Methodology
+    (exact 1-D GPTQ trajectory; rank-one separable feedback kept in a buffer).
+
+Conventions (readings where the pages are silent; each is listed in the design doc):
+  * W is m x n.  H_L (m x m) acts on the row index i, H_R (n x n) on the column
+    index j.  Proxy loss  L(Q) = tr(dW^T H_L dW H_R),  dW = W - diag(s) Q, which
+    is vec(dW)^T (H_R kron H_L) vec(dW) with column-major vec.
+  * Entry (0, 0) is rounded first (GPTQ's index-0-first order).
+  * Grid: q = clamp(rint(t), lo, hi) with rint = round half to even; without
+    clamp the grid is all integers.  The error fed back is W - s q with the
+    clamped q.
+  * Per-row scales s_i are inputs (grid = s_i * Z on row i).
+
+Functions, from most literal to fastest:
+  O0  nearest_plane_by_definition   conditional minimiser, any linear extension
+  O1  babai_kron_sweep              1-D GPTQ sweep over vec(W) on the mn x mn Gram
+  O2  gptq2d_antidiagonal           the cubic anti-diagonal algorithm
+and the special cases used as pins: RTN, 1-D GPTQ in OBS form, exhaustive
+closest-vector search on tiny problems.
+"""
+from __future__ import annotations
+
+import itertools
+import numpy as np
+
+NEAR_TIE_BAND = 1e-6
+
+
+# --------------------------------------------------------------------------- #
+# Grid and loss
+# --------------------------------------------------------------------------- #
+def grid_bounds(bits: int, clamp: bool):
+    """Admissible integers: [-2^(bits-1), 2^(bits-1)-1] when clamping, else all of Z."""
+    if not clamp:
+        return -np.inf, np.inf
+    return float(-(1 << (bits - 1))), float((1 << (bits - 1)) - 1)
+
+
+def round_to_grid(t, lo, hi):
+    """Nearest admissible integer along one coordinate: clamp(rint(t), lo, hi)."""
+    return np.clip(np.rint(t), lo, hi)
+
+
+def proxy_loss(W, Q, s, H_L, H_R) -> float:
+    """L(Q) = tr(dW^T H_L dW H_R), dW = W - diag(s) Q (the two-sided quadratic metric)."""
+    W = np.asarray(W, np.float64)
+    D = W - np.asarray(s, np.float64)[:, None] * np.asarray(Q, np.float64)
+    return float(np.sum(D * (np.asarray(H_L, np.float64) @ D @ np.asarray(H_R, np.float64))))
+
+
+def rtn(W, s, bits, clamp):
+    """Round-to-nearest baseline: each entry independently, q = clamp(rint(W_ij / s_i))."""
+    lo, hi = grid_bounds(bits, clamp)
+    W = np.asarray(W, np.float64)
+    return round_to_grid(W / np.asarray(s, np.float64)[:, None], lo, hi)
+
+
+def near_tie(t, lo, hi, band=NEAR_TIE_BAND):
+    """True where t lies within ``band`` of a rounding boundary k + 1/2 that separates
+    two admissible integers (lo <= k < hi).  Values beyond hi + 1/2 or below lo - 1/2
+    have no boundary: clamping sends both neighbours to the same integer."""
+    t = np.asarray(t, np.float64)
+    h = np.floor(t) + 0.5
+    has_boundary = (h - 0.5 >= lo) & (h + 0.5 <= hi)
+    return has_boundary & (np.abs(t - h) < band)
+
+
+# --------------------------------------------------------------------------- #
+# Factor of a Kronecker factor
+# --------------------------------------------------------------------------- #
+def reverse_cholesky(H):
+    """Lower-triangular M with positive diagonal and M^T M = H.
+
+    With M_L, M_R of this form, M = M_R kron M_L is lower triangular in
+    column-major index order and M^T M = H_R kron H_L, so row p of M(x - z)
+    involves only coordinates <= p: the triangular factor that makes the
+    index-0-first nearest-plane sweep explicit.  Computed through LAPACK's
+    ordinary Cholesky of the index-reversed matrix: if J H J = L L^T then
+    M = J L^T J.
+    """
+    H = np.asarray(H, np.float64)
+    L = np.linalg.cholesky(H[::-1, ::-1])
+    return np.ascontiguousarray(L.T[::-1, ::-1])
+
+
+# --------------------------------------------------------------------------- #
+# O0: the definition
+# --------------------------------------------------------------------------- #
+def nearest_plane_by_definition(W, H_L, H_R, s, bits, clamp, order="row"):
+    """Sequential nearest-plane rounding of vec(W) under G = H_R kron H_L, written
+    as its definition (mind-verse.de, "Geometrische Grundlagen ..."): coordinates
+    are fixed one at a time; the value rounded for coordinate p is the p-th
+    coordinate of the real minimiser of (z - x)^T G (z - x) over the coordinates
+    not yet fixed, with the fixed ones held at s*q.
+
+    ``order`` is any linear extension of the product order on (i, j):
+    "row" (row-major) or "col" (column-major).  Returns (Q, T) with T = y / s.
+    Dense solves of size mn: tiny problems only.
+    """
+    W = np.asarray(W, np.float64)
+    m, n = W.shape
+    lo, hi = grid_bounds(bits, clamp)
+    G = np.kron(np.asarray(H_R, np.float64), np.asarray(H_L, np.float64))
+    x = W.reshape(-1, order="F")                         # p = i + m j
+    sv = np.tile(np.asarray(s, np.float64), n)
+    if order == "row":
+        seq = [i + m * j for i in range(m) for j in range(n)]
+    elif order == "col":
+        seq = list(range(m * n))
+    else:
+        raise ValueError(order)
+    fixed = np.zeros(m * n, bool)
+    z = np.zeros(m * n)
+    T = np.zeros(m * n)
+    Q = np.zeros(m * n)
+    for p in seq:
+        r = np.flatnonzero(~fixed)
+        f = np.flatnonzero(fixed)
+        zr = x[r].copy()
+        if f.size:
+            # stationarity over the free block: G_rr (z_r - x_r) + G_rf (z_f - x_f) = 0
+            zr = x[r] - np.linalg.solve(G[np.ix_(r, r)], G[np.ix_(r, f)] @ (z[f] - x[f]))
+        y = zr[np.searchsorted(r, p)]
+        T[p] = y / sv[p]
+        Q[p] = round_to_grid(T[p], lo, hi)
+        z[p] = sv[p] * Q[p]
+        fixed[p] = True
+    return Q.reshape((m, n), order="F"), T.reshape((m, n), order="F")
+
+
+# --------------------------------------------------------------------------- #
+# O1: naive vectorised Babai / 1-D GPTQ sweep on the full Kronecker Gram
+# --------------------------------------------------------------------------- #
+def babai_kron_sweep(W, H_L, H_R, s, bits, clamp):
+    """The naive vectorised sweep whose trajectory GPTQ-2D reproduces (arxivlens,
+    Analysis > Results; mind-verse.de, "Die algorithmische Neuerung"): one-sided
+    GPTQ over all mn coordinates of vec(W) (column-major), with the Gram
+    G = H_R kron H_L.  GPTQ form: U = upper Cholesky factor of G^{-1}; coordinate
+    p is rounded, and its error, divided by U_pp, is propagated to the later
+    coordinates along row p of U.  Quartic work; 64 x 64 at most.
+    Returns (Q, T) with T = (updated x_p) / s_p.
+    """
+    W = np.asarray(W, np.float64)
+    m, n = W.shape
+    lo, hi = grid_bounds(bits, clamp)
+    G = np.kron(np.asarray(H_R, np.float64), np.asarray(H_L, np.float64))
+    U = np.linalg.cholesky(np.linalg.inv(G)).T            # U^T U = G^{-1}, upper
+    x = W.reshape(-1, order="F").copy()
+    sv = np.tile(np.asarray(s, np.float64), n)
+    N = m * n
+    Q = np.zeros(N)
+    T = np.zeros(N)
+    for p in range(N):
+        T[p] = x[p] / sv[p]
+        Q[p] = round_to_grid(T[p], lo, hi)
+        e = (x[p] - sv[p] * Q[p]) / U[p, p]
+        x[p + 1:] -= e * U[p, p + 1:]
+    return Q.reshape((m, n), order="F"), T.reshape((m, n), order="F")
+
+
+# --------------------------------------------------------------------------- #
+# O2: the cubic anti-diagonal algorithm
+# --------------------------------------------------------------------------- #
+class Result:
+    """Output of gptq2d_antidiagonal: Q, T = y/s, the Babai-identity loss, flags."""
+
+    def __init__(self, Q, T, loss_identity, n_clamped, near_tie_mask, flipped):
+        self.Q = Q
+        self.T = T
+        self.loss_identity = loss_identity
+        self.n_clamped = n_clamped
+        self.near_tie = near_tie_mask
+        self.flipped = flipped
+
+
+def gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=None, band=NEAR_TIE_BAND):
+    """GPTQ-2D: round W anti-diagonal by anti-diagonal (arxivlens Abstract;
+    mind-verse.de "Die algorithmische Neuerung") with the rank-one separable
+    feedback kept in an accumulated buffer (arxivlens, Analysis > Results and
+    Methodology).
+
+    With M_L, M_R the lower factors (M^T M = H), rounding entry (i, j) sees
+        y_ij = W_ij + (sum_{i'<=i, j'<=j, (i',j') != (i,j)} M_L[i,i'] dW[i',j'] M_R[j,j'])
+                       / (M_L[i,i] M_R[j,j]),
+    i.e. row (i,j) of (M_R kron M_L) applied to the errors already made.  The
+    buffer P holds P[i', j] = sum_{j' <= j, done} dW[i', j'] M_R[j, j'] (right
+    feedback); the left factor is applied to a column of P when an entry is
+    rounded.  Entries of anti-diagonal d = i + j only depend on earlier
+    anti-diagonals, so each one is handled as a vector.  Work is mn(m + n).
+
+    ``flip``: optional set of (i, j) where the other neighbouring integer is
+    taken.  Every such entry must be a near-tie (|t - (k + 1/2)| < band) in this
+    run's own trajectory, else ValueError: the flip set only selects among the
+    roundings that the near-tie rule admits.
+
+    Returns a Result with Q, T = y/s, the loss via the Babai identity
+    sum d_ij^2 (y_ij - s_i q_ij)^2, the clamp count and the near-tie mask.
+    """
+    W = np.asarray(W, np.float64)
+    M_L = np.asarray(M_L, np.float64)
+    M_R = np.asarray(M_R, np.float64)
+    s = np.asarray(s, np.float64)
+    m, n = W.shape
+    lo, hi = grid_bounds(bits, clamp)
+    flip = set() if flip is None else set(flip)
+    P = np.zeros((m, n))
+    Q = np.zeros((m, n))
+    T = np.zeros((m, n))
+    tie = np.zeros((m, n), bool)
+    loss = 0.0
+    n_clamped = 0
+    done_flips = set()
+    for d in range(m + n - 1):
+        i = np.arange(max(0, d - n + 1), min(d, m - 1) + 1)
+        j = d - i
+        # left factor applied to column j of P; M_L[i, i'] = 0 for i' > i drops the rest
+        fb = np.einsum("ek,ke->e", M_L[i, :], P[:, j])
+        dij = M_L[i, i] * M_R[j, j]
+        y = W[i, j] + fb / dij
+        t = y / s[i]
+        q_raw = np.rint(t)
+        q = np.clip(q_raw, lo, hi)
+        nt = near_tie(t, lo, hi, band)
+        if flip:
+            for e in range(i.size):
+                key = (int(i[e]), int(j[e]))
+                if key in flip:
+                    if not nt[e]:
+                        raise ValueError(f"flip requested at {key}, not a near-tie (t={t[e]!r})")
+                    h = np.floor(t[e]) + 0.5
+                    q[e] = h + 0.5 if q[e] == h - 0.5 else h - 0.5
+                    done_flips.add(key)
+        n_clamped += int(np.count_nonzero(q != q_raw))
+        delta = W[i, j] - s[i] * q
+        # right feedback: P[i, j'] += delta * M_R[j', j]; zero for j' < j (M_R lower)
+        P[i, :] += delta[:, None] * M_R[:, j].T
+        loss += float(np.sum((dij * (y - s[i] * q)) ** 2))
+        Q[i, j] = q
+        T[i, j] = t
+        tie[i, j] = nt
+    if done_flips != flip:
+        raise ValueError(f"flips never reached: {sorted(flip - done_flips)}")
+    return Result(Q, T, loss, n_clamped, tie, done_flips)
+
+
+def gptq2d(W, H_L, H_R, s, bits, clamp, **kw):
+    """Factor both Kronecker factors, then run the anti-diagonal algorithm."""
+    return gptq2d_antidiagonal(W, reverse_cholesky(H_L), reverse_cholesky(H_R), s, bits, clamp, **kw)
+
+
+def entry_value(W, Q, s, M_L, M_R, i, j):
+    """y_ij computed directly from its definition, given the integers already chosen
+    for the dominated quadrant {i' <= i, j' <= j} minus (i, j) itself.  O(ij) work;
+    used to check single sampled entries of large outputs."""
+    W = np.asarray(W, np.float64)
+    s = np.asarray(s, np.float64)
+    D = W[: i + 1, : j + 1] - s[: i + 1, None] * np.asarray(Q[: i + 1, : j + 1], np.float64)
+    D[i, j] = 0.0
+    fb = np.asarray(M_L[i, : i + 1], np.float64) @ D @ np.asarray(M_R[j, : j + 1], np.float64)
+    return W[i, j] + fb / (float(M_L[i, i]) * float(M_R[j, j]))
+
+
+# --------------------------------------------------------------------------- #
+# Special cases used as pins
+# --------------------------------------------------------------------------- #
+def gptq_1d_obs(w, H, s, bits, clamp):
+    """Textbook one-sided GPTQ on a vector (mind-verse.de, "GPTQ-2D: Eine
+    Weiterentwicklung ...": one-sided rounding with triangular feedback), in the
+    optimal-brain-surgeon form rather than the Cholesky form: round coordinate
+    p, move the remaining coordinates by -err * Hinv[p, rest] / Hinv[p, p],
+    then remove p from the inverse (Hinv -= Hinv[:, p] Hinv[p, :] / Hinv[p, p]).
+    Index 0 first.  Returns q."""
+    w = np.asarray(w, np.float64).copy()
+    s = np.broadcast_to(np.asarray(s, np.float64), w.shape)
+    lo, hi = grid_bounds(bits, clamp)
+    Hinv = np.linalg.inv(np.asarray(H, np.float64))
+    k = w.size
+    q = np.zeros(k)
+    for p in range(k):
+        q[p] = round_to_grid(w[p] / s[p], lo, hi)
+        err = w[p] - s[p] * q[p]
+        w -= err * Hinv[p, :] / Hinv[p, p]
+        Hinv = Hinv - np.outer(Hinv[:, p], Hinv[p, :]) / Hinv[p, p]
+    return q
+
+
+def closest_vector_exhaustive(W, H_L, H_R, s, bits, clamp, radius=2, center=None):
+    """Exact minimiser of the proxy loss over the integer box center +- radius
+    (center defaults to RTN), by evaluating the loss at every point.  Tiny
+    problems only (mn <= 9 with radius 2).  Returns (Q, loss)."""
+    W = np.asarray(W, np.float64)
+    m, n = W.shape
+    lo, hi = grid_bounds(bits, clamp)
+    c = rtn(W, s, bits, clamp) if center is None else np.asarray(center, np.float64)
+    axes = [np.clip(np.arange(c.flat[p] - radius, c.flat[p] + radius + 1), lo, hi)
+            for p in range(m * n)]
+    axes = [np.unique(a) for a in axes]
+    best, bestQ = np.inf, None
+    sv = np.asarray(s, np.float64)
+    H_L = np.asarray(H_L, np.float64)
+    H_R = np.asarray(H_R, np.float64)
+    for combo in itertools.product(*axes):
+        Qc = np.array(combo).reshape(m, n)
+        D = W - sv[:, None] * Qc
+        val = float(np.sum(D * (H_L @ D @ H_R)))
+        if val < best:
+            best, bestQ = val, Qc
+    return bestQ, best
+
+
+def sphere_decode(W, H_L, H_R, s, bits, clamp):
+    """Exact closest-vector point by depth-first Schnorr-Euchner enumeration over
+    coordinates in column-major order, using M = M_R kron M_L (lower) so that the
+    partial sum of squared residual rows is monotone.  The first leaf visited
+    takes the nearest integer at every level, i.e. the nearest-plane point.
+    Returns (Q_opt, loss_opt, Q_first_leaf)."""
+    W = np.asarray(W, np.float64)
+    m, n = W.shape
+    lo, hi = grid_bounds(bits, clamp)
+    M = np.kron(reverse_cholesky(H_R), reverse_cholesky(H_L))
+    x = W.reshape(-1, order="F")
+    sv = np.tile(np.asarray(s, np.float64), n)
+    N = m * n
+    best = [np.inf, None]
+    first = [None]
+    z = np.zeros(N)
+
+    def rec(p, partial):
+        if p == N:
+            if first[0] is None:
+                first[0] = z.copy()
+            if partial < best[0]:
+                best[0], best[1] = partial, z.copy()
+            return
+        # residual row p: M[p,p] (x_p - z_p) + sum_{p'<p} M[p,p'] (x_p' - z_p')
+        off = M[p, :p] @ (x[:p] - z[:p])
+        c = (x[p] + off / M[p, p]) / sv[p]
+        k0 = round_to_grid(c, lo, hi)
+        cand = [k0]
+        for step in range(1, 64):
+            for k in (k0 + step, k0 - step) if c >= k0 else (k0 - step, k0 + step):
+                if lo <= k <= hi:
+                    cand.append(k)
+        cand.sort(key=lambda k: abs(c - k))
+        for k in cand:
+            r = M[p, p] * sv[p] * (c - k)
+            nxt = partial + r * r
+            if nxt >= best[0]:
+                break
+            z[p] = sv[p] * k
+            rec(p + 1, nxt)
+        z[p] = 0.0
+
+    rec(0, 0.0)
+    to_q = lambda v: (v / sv).reshape((m, n), order="F")
+    return to_q(best[1]), best[0], to_q(first[0])
