@@ -1,0 +1,471 @@
+"""Benchmark: GPTQ-2D INT4 rounding of a 4096 x 4096 attention projection on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one independent layer per rank)
+
+One step = the whole path on one layer already resident in HBM: factor
+preparation of both Kronecker factors (H_L, H_R: 4096 x 4096 fp32) and the
+anti-diagonal rounding of W (4096 x 4096 bf16) with INT4 per-row scales.
+Metric: weight entries rounded per second (m*n per step, summed over ranks).
+Rank 0 prints one JSON line.
+
+Reported beside it:
+  roofline      the dominant kernel's algorithmic FLOP/s (CUDA events around
+                its launches, on the launching stream) against the FP64
+                tensor-core peak measured here (cuBLAS DGEMM 8192^3)
+  e2e           the same metric through gptq2d_round_host from pinned host
+                buffers: host->device inputs and device->host Q + statistics
+                inside the timed region
+  cpu_baseline  the fp64 CPU oracle on a bounded sample of the same workload
+  clocks        nvidia-smi samples taken during the timed region
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "weight entries rounded/sec at 4096×4096 INT4 (1 B200); % of pipe roofline"
+TB = 64
+
+
+# --------------------------------------------------------------------------- #
+# workload and algorithmic work
+# --------------------------------------------------------------------------- #
+def make_problem(name, seed, device_gram=True):
+    import torch
+    import workloads as WL
+
+    def gram(X):
+        Xt = torch.from_numpy(X).cuda()
+        return (Xt.T @ Xt).cpu().numpy()
+
+    mm = gram if device_gram else None
+    if name == "attn":
+        return WL.attn(seed, matmul=mm)
+    if name == "mlp":
+        return WL.mlp(seed, matmul=mm)
+    if name == "small":
+        return WL.small(seed)
+    raise ValueError(name)
+
+
+def band_product_flops(m, n):
+    """Useful flops of the band products (right and down feedback between 64-tiles):
+    entry (i, j) feeds 2 * (n - 64 (j//64 + 1)) flops right and 2 * (m - 64 (i//64 + 1)) down."""
+    jt = np.arange(n) // TB
+    it = np.arange(m) // TB
+    right = m * np.sum(2.0 * np.maximum(0, n - TB * (jt + 1)))
+    down = n * np.sum(2.0 * np.maximum(0, m - TB * (it + 1)))
+    return float(right + down)
+
+
+def sweep_flops(m, n):
+    """In-tile flops: entry (a, c) of a rows x cols tile pushes (cols-1-c) + (rows-1-a) FMAs."""
+    tot = 0.0
+    for r in [min(TB, m - r0) for r0 in range(0, m, TB)]:
+        for c in [min(TB, n - c0) for c0 in range(0, n, TB)]:
+            tot += 2.0 * (r * c * (c - 1) / 2 + c * r * (r - 1) / 2)
+    return tot
+
+
+def prep_flops(k):
+    return k ** 3 / 3.0
+
+
+# --------------------------------------------------------------------------- #
+# clocks
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        rows = []
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 10:
+                continue
+            if self.bus_id and self.bus_id[-12:] not in p[1].lower():
+                continue
+            rows.append(p)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[6 + k] == "Active"})
+        pw = [float(r[4]) for r in rows if r[4].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "power_w_max": max(pw) if pw else None, "samples": len(rows)}
+
+
+def bus_id_of(dev):
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    for attr in ("pci_bus_id",):
+        if hasattr(p, attr):
+            dom = getattr(p, "pci_domain_id", 0)
+            return f"{dom:08x}:{getattr(p, attr):02x}:{getattr(p, 'pci_device_id', 0):02x}.0"
+    return ""
+
+
+# --------------------------------------------------------------------------- #
+# ncu traffic figures (profiles/ncu_traffic.txt: kernel, source sha256, bytes per launch, units)
+# --------------------------------------------------------------------------- #
+def ncu_traffic(kernel_class, src_file):
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(src_file, "rb").read()).hexdigest()[:16]
+    for ln in open(path):
+        if ln.startswith("#") or not ln.strip():
+            continue
+        p = ln.split()
+        if len(p) >= 3 and p[0] == kernel_class and p[1] == sha:
+            return float(p[2])
+    return None
+
+
+# --------------------------------------------------------------------------- #
+# our arm
+# --------------------------------------------------------------------------- #
+def measure_dgemm_tflops():
+    import torch
+    n = 8192
+    a = torch.randn(n, n, dtype=torch.float64, device="cuda")
+    b = torch.randn(n, n, dtype=torch.float64, device="cuda")
+    for _ in range(2):
+        torch.matmul(a, b)
+    best = 0.0
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.matmul(a, b)
+        e1.record()
+        e1.synchronize()
+        best = max(best, 2 * n ** 3 / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+    del a, b
+    torch.cuda.empty_cache()
+    return best
+
+
+def cpu_baseline(pb, sample):
+    """The fp64 oracle as it stands on the host cores: LAPACK factors of both full Grams plus
+    the anti-diagonal rounding of the leading sample x sample prefix (the prefix is a GPTQ-2D
+    problem of its own), scaled to the full layer by the work ratio mn(m+n)."""
+    import oracle as O
+    m, n = pb.shape
+    t0 = time.perf_counter()
+    ML = O.reverse_cholesky(pb.H_L)
+    MR = O.reverse_cholesky(pb.H_R)
+    t_prep = time.perf_counter() - t0
+    k = min(sample, m, n)
+    t0 = time.perf_counter()
+    O.gptq2d_antidiagonal(pb.W[:k, :k].astype(np.float64), ML[:k, :k], MR[:k, :k],
+                          pb.scales[:k].astype(np.float64), pb.bits, pb.clamp)
+    t_rnd = time.perf_counter() - t0
+    t_full = t_prep + t_rnd * (m * n * (m + n)) / (k * k * 2 * k)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": m * n / t_full, "unit": "entries/s", "cores": cores, "kind": "oracle",
+            "sample": (f"LAPACK reverse Cholesky of both {m}x{m}/{n}x{n} Grams ({t_prep:.2f} s) + "
+                       f"anti-diagonal oracle on the leading {k}x{k} prefix ({t_rnd:.2f} s), "
+                       f"rounding time scaled by mn(m+n) to {m}x{n}: {t_full:.1f} s per layer")}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import two_sided_adaptive_b200 as g
+    from two_sided_adaptive_b200 import build as gbuild
+
+    if rank == 0:
+        gbuild.build()
+    if world > 1:
+        dist.barrier()
+    g.lib()
+    dev = torch.device("cuda", local_rank)
+    pb = make_problem(args.workload, seed=rank)
+    m, n = pb.shape
+    W = torch.from_numpy(pb.W).to(dev).to(torch.bfloat16 if args.workload != "small" else torch.float32)
+    H_L = torch.from_numpy(pb.H_L).to(dev)
+    H_R = torch.from_numpy(pb.H_R).to(dev)
+    s = torch.from_numpy(pb.scales).to(dev)
+    M_L = torch.empty((m, m), dtype=torch.float64, device=dev)
+    M_R = torch.empty((n, n), dtype=torch.float64, device=dev)
+    wsL = torch.empty(max(g.prepare_workspace_size(m), 256), dtype=torch.uint8, device=dev)
+    wsR = torch.empty(max(g.prepare_workspace_size(n), 256), dtype=torch.uint8, device=dev)
+    wsQ = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
+    Q = torch.empty((m, n), dtype=torch.int8, device=dev)
+    st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+
+    def step():
+        g.prepare(H_L, out=M_L, workspace=wsL, check=False)
+        g.prepare(H_R, out=M_R, workspace=wsR, check=False)
+        g.quantize(W, M_L, M_R, s, pb.bits, pb.clamp, out=Q, stats=st, workspace=wsQ)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    import ctypes
+    for ws in (wsL, wsR):
+        piv = ctypes.c_int64(-1)
+        rc = g.lib().gptq2d_prepare_info(ws.data_ptr(), None, ctypes.byref(piv))
+        assert rc == 0, f"factor not SPD (pivot {piv.value})"
+    stats = g.stats_dict(st)
+    assert stats["status"] == 0, stats
+
+    sampler = ClockSampler(bus_id_of(dev)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    l0 = g.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    launches = g.launch_count() - l0
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * m * n / (ms_step * 1e-3)
+
+    # per-kernel device time of one more step, CUDA events around each launch on its stream
+    g.profile_reset()
+    g.profile_enable(True)
+    step()
+    torch.cuda.synchronize()
+    prof = g.profile_read()
+    g.profile_enable(False)
+    g.profile_reset()
+
+    # end to end through the C ABI from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        wdt = torch.bfloat16 if args.workload != "small" else torch.float32
+        Wh = torch.from_numpy(pb.W).to(wdt).pin_memory()
+        HLh = torch.from_numpy(pb.H_L).pin_memory()
+        HRh = torch.from_numpy(pb.H_R).pin_memory()
+        sh = torch.from_numpy(pb.scales).pin_memory()
+        Qh = torch.empty((m, n), dtype=torch.int8).pin_memory()
+        sth = torch.empty(g.STATS_WORDS, dtype=torch.int64).pin_memory()
+        wsH = torch.empty(g.round_host_workspace_size(m, n, g._dtype_code(Wh), g.DTYPE_F32),
+                          dtype=torch.uint8, device=dev)
+        g.round_host(Wh, HLh, HRh, sh, pb.bits, pb.clamp, workspace=wsH, Q_out=Qh, stats_out=sth)
+        assert torch.equal(Qh, Q.cpu()), "round_host and device path disagree"
+        ke = max(1, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(ke):
+            g.round_host(Wh, HLh, HRh, sh, pb.bits, pb.clamp, workspace=wsH, Q_out=Qh, stats_out=sth)
+        f1.record()
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1) / ke
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = Wh.numel() * Wh.element_size() + (HLh.numel() + HRh.numel() + sh.numel()) * 4
+        d2h = Qh.numel() + sth.numel() * 8
+        e2e = {"value": world * m * n / (ems * 1e-3), "unit": "entries/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": ems, "api": "gptq2d_round_host"}
+
+    if rank != 0:
+        return None
+
+    peak = measure_dgemm_tflops()
+    dom = max(("propagate", "sweep", "prep_trailing", "prep_panel"), key=lambda k: prof[k][1])
+    work = {"propagate": band_product_flops(m, n), "sweep": sweep_flops(m, n),
+            "prep_trailing": prep_flops(m) + prep_flops(n), "prep_panel": None}
+    nl, tms = prof[dom]
+    src = {"propagate": "quantize.cu", "sweep": "quantize.cu", "prep_trailing": "prepare.cu",
+           "prep_panel": "prepare.cu"}[dom]
+    traffic = ncu_traffic(dom, os.path.join(ROOT, "two_sided_adaptive_b200", "csrc", src))
+    achieved = (work[dom] / nl) / (tms / nl * 1e-3) / 1e12 if work[dom] else None
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
+                "traffic": traffic, "launches_per_step": nl, "kernel_ms_per_step": tms,
+                "algorithmic_flops_per_launch": work[dom] / nl if work[dom] else None,
+                "peak_source": "cuBLAS DGEMM 8192^3 (torch.matmul fp64), best of 5, measured in this run"}
+    breakdown = {k: {"launches": v[0], "ms": round(v[1], 4)} for k, v in prof.items()}
+    total_flops = m * n * (m + n) + prep_flops(m) + prep_flops(n)
+    out = {
+        "metric": METRIC, "value": value, "unit": "entries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": pb.name.split("_s")[0], "m": m, "n": n, "bits": pb.bits,
+                   "w_dtype": str(W.dtype).replace("torch.", ""), "h_dtype": "float32",
+                   "step": "prepare(H_L) + prepare(H_R) + quantize(W), inputs resident in HBM",
+                   "l2": "no flush; per-step working set (W, H_L, H_R, factors, 3 fp64 feedback "
+                         "buffers) is %.2f GB > 126 MB L2" % (
+                             (W.numel() * W.element_size() + 2 * 4 * (m * m + n * n) + 8 * (m * m + n * n)
+                              + wsQ_bytes(g, m, n)) / 1e9),
+                   "parallelism": "independent layer per rank" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "gpu_launches": int(launches),
+        "gpu_launches_per_step": launches / args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "stats": stats,
+        "breakdown_ms_per_step": breakdown,
+        "whole_step_fp64_tflops": total_flops / (ms_step * 1e-3) / 1e12,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(pb, args.cpu_sample)
+    return out
+
+
+def wsQ_bytes(g, m, n):
+    return g.quantize_workspace_size(m, n)
+
+
+# --------------------------------------------------------------------------- #
+# reference arm: the fp64 oracle on the host cores
+# --------------------------------------------------------------------------- #
+def run_reference(args):
+    import oracle as O
+    pb = make_problem(args.workload, seed=0, device_gram=False) if args.workload == "small" else None
+    if pb is None:
+        import workloads as WL
+        pb = WL.attn(0) if args.workload == "attn" else WL.mlp(0)
+    m, n = pb.shape
+    k = min(args.ref_sample, m, n)
+
+    def step():
+        ML = O.reverse_cholesky(pb.H_L)
+        MR = O.reverse_cholesky(pb.H_R)
+        t0 = time.perf_counter()
+        O.gptq2d_antidiagonal(pb.W[:k, :k].astype(np.float64), ML[:k, :k], MR[:k, :k],
+                              pb.scales[:k].astype(np.float64), pb.bits, pb.clamp)
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    t_rnd = 0.0
+    for _ in range(args.steps):
+        t_rnd += step()
+    total = time.perf_counter() - t0
+    t_prep = (total - t_rnd) / args.steps
+    t_full = t_prep + (t_rnd / args.steps) * (m * n * (m + n)) / (k * k * 2 * k)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        cores = os.cpu_count()
+    value = m * n / t_full
+    sample = (f"per step: LAPACK reverse Cholesky of both full Grams ({t_prep:.2f} s) + "
+              f"anti-diagonal oracle on the leading {k}x{k} prefix, scaled by mn(m+n) to {m}x{n}")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "entries/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": pb.name.split("_s")[0], "m": m, "n": n, "bits": pb.bits},
+            "cpu_baseline": {"value": value, "unit": "entries/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "entries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=("attn", "mlp", "small"), default="attn")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=768)
+    ap.add_argument("--ref-sample", type=int, default=384)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

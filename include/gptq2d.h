@@ -1,0 +1,194 @@
+/*
+ * gptq2d.h -- C ABI of the B200 (sm_100a) GPTQ-2D two-sided adaptive rounding library.
+ *
+ * The operation (mind-verse.de "Neue Ansätze zur Effizienzsteigerung von Large
+ * Language Models durch GPTQ-2D", sections "GPTQ-2D: Eine Weiterentwicklung der
+ * adaptiven Rundung" and "Geometrische Grundlagen ..."; arxivlens "GPTQ-2D:
+ * Cubic-Time Two-Sided Adaptive Rounding", Abstract and Analysis):
+ *
+ *   Round a real matrix W (m x n) onto per-row integer grids s_i * Z so that the
+ *   rounding follows, entry for entry, the sequential nearest-plane (1-D GPTQ)
+ *   sweep over vec(W) under the Kronecker Gram H = H_R (x) H_L, where H_L (m x m)
+ *   acts on rows and H_R (n x n) on columns.  The proxy loss is
+ *   L(Q) = tr(dW^T H_L dW H_R), dW = W - diag(s) Q.  Entries are rounded anti-
+ *   diagonal by anti-diagonal (entry (0,0) first); every entry of one anti-
+ *   diagonal is rounded in parallel; the rounding error of entry (i,j) feeds
+ *   back as a rank-one, separable update built from column j of the right
+ *   factor and column i of the left factor.  Total work is mn(m + n) flops.
+ *
+ * Conventions shared by every entry point:
+ *   - Matrices are row-major; every leading dimension (ld*) counts ELEMENTS and
+ *     must be >= the row length.
+ *   - All data pointers are DEVICE pointers owned by the caller (except the
+ *     *_host entry point, which takes host pointers).  The library never
+ *     allocates or frees device memory; scratch space is the caller's
+ *     workspace `ws` of at least the size returned by the matching
+ *     *_workspace_size query, aligned to 256 bytes.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  Calls are asynchronous unless stated otherwise.
+ *   - Return value: a gptq2d_status.  Arguments are checked on the host before
+ *     anything is enqueued; an invalid argument returns GPTQ2D_ERR_INVALID_ARG
+ *     and enqueues nothing.  A failed launch returns GPTQ2D_ERR_CUDA.  No C++
+ *     exception crosses the ABI.
+ *   - All floating-point arithmetic on the path is IEEE fp64.
+ *   - Results are deterministic: identical inputs on the same device give a
+ *     bitwise identical Q and statistics.
+ */
+#ifndef GPTQ2D_H_
+#define GPTQ2D_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GPTQ2D_OK = 0,
+  GPTQ2D_ERR_INVALID_ARG = 1, /* null pointer, bad size, ld, dtype, bits or clamp */
+  GPTQ2D_ERR_NOT_SPD = 2,     /* a Kronecker factor is not symmetric positive definite */
+  GPTQ2D_ERR_NONFINITE = 3,   /* NaN/Inf in W or a scale <= 0 / non-finite (reported in stats) */
+  GPTQ2D_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
+  GPTQ2D_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+  GPTQ2D_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed */
+} gptq2d_status;
+
+typedef enum {
+  GPTQ2D_F32 = 0,  /* IEEE binary32 */
+  GPTQ2D_BF16 = 1, /* bfloat16 */
+  GPTQ2D_F64 = 2   /* IEEE binary64 */
+} gptq2d_dtype;
+
+/* Statistics written by gptq2d_quantize on the DEVICE (read them after the
+ * stream has reached the end of the call). */
+typedef struct {
+  double proxy_loss;   /* tr(dW^T H_L dW H_R), accumulated as sum_ij d_ij^2 (y_ij - s_i q_ij)^2
+                          with d_ij = M_L[i,i] M_R[j,j] and y_ij the value rounded at (i,j)
+                          (the nearest-plane residual identity) */
+  int64_t n_clamped;   /* entries where clamping changed rint(y/s) */
+  int64_t n_near_tie;  /* entries whose y/s lies within 1e-6 of a boundary k + 1/2
+                          between two admissible integers */
+  int64_t n_nonfinite; /* entries with non-finite W or y, or rows with an invalid scale */
+  int64_t status;      /* GPTQ2D_OK, or GPTQ2D_ERR_NONFINITE if n_nonfinite > 0 */
+} gptq2d_stats;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gptq2d_status_string(int status);
+
+/* Library version, (major << 16) | minor. */
+int gptq2d_version(void);
+
+/* Number of kernels this library has launched in this process so far (all
+ * devices, all threads).  Lets a caller count launches inside a timed region. */
+int64_t gptq2d_launch_count(void);
+
+/* Optional per-launch timing (off by default).  While enabled, every kernel the
+ * library launches is bracketed by a pair of CUDA events recorded on the
+ * launching stream; events are created on first use and recycled.  Kernel
+ * classes: 0 factor panel (diagonal block + block-row solve), 1 factor trailing
+ * update, 2 anti-diagonal tile sweep, 3 band products (feedback propagation),
+ * 4 other (conversion, diagonals, statistics). */
+void gptq2d_profile_enable(int on);
+/* Number of recorded launches of `kernel_class` and their summed device time
+ * in milliseconds (waits for the recorded events).  GPTQ2D_ERR_INVALID_ARG for
+ * an unknown class. */
+int gptq2d_profile_read(int kernel_class, int64_t* launches, double* total_ms);
+/* Forgets all recorded launches. */
+void gptq2d_profile_reset(void);
+
+/* ------------------------------------------------------------------------- */
+/* Factor preparation (the fixed bases are factored once: arxivlens, Analysis  */
+/* > Limitations, "fixed nonsingular basis matrices"; Future work, "Gram        */
+/* factorizations").                                                           */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace gptq2d_prepare needs for a k x k factor (k >= 0). */
+size_t gptq2d_prepare_workspace_size(int64_t k);
+
+/* Factor one Kronecker factor H (k x k, symmetric positive definite; only its
+ * lower triangle j <= i is read) as H = M^T M with M LOWER triangular with a
+ * positive diagonal (a "reverse" Cholesky factor: the last row is eliminated
+ * first).  With M_L, M_R of this form, M_R (x) M_L is lower triangular in the
+ * column-major order of vec(W), which is the triangular factor of the
+ * index-0-first nearest-plane sweep.
+ *
+ *   H, h_dtype, ldh : device, k x k, GPTQ2D_F32 or GPTQ2D_F64, row-major.
+ *   M, ldm          : device fp64 output, k x k row-major; the strict upper
+ *                     triangle is written as exact zeros.  May not alias H.
+ *   ws, ws_bytes    : device workspace, >= gptq2d_prepare_workspace_size(k).
+ *   bad_pivot       : HOST pointer or NULL.  If non-NULL the call synchronizes
+ *                     `stream`, writes -1 when H is positive definite, else the
+ *                     0-based row index of the first pivot (in elimination
+ *                     order, i.e. the largest such index) that was not
+ *                     positive and finite, and returns GPTQ2D_ERR_NOT_SPD in
+ *                     that case.  If NULL the call is asynchronous and a
+ *                     failure is only visible through gptq2d_prepare_info.
+ * k == 0 is a no-op. */
+int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh,
+                   double* M, int64_t ldm, void* ws, size_t ws_bytes,
+                   void* stream, int64_t* bad_pivot);
+
+/* Reads the pivot word a previous asynchronous gptq2d_prepare left in `ws`
+ * (synchronizes `stream`).  Writes -1 or the failing pivot to *bad_pivot and
+ * returns GPTQ2D_OK or GPTQ2D_ERR_NOT_SPD. */
+int gptq2d_prepare_info(const void* ws, void* stream, int64_t* bad_pivot);
+
+/* ------------------------------------------------------------------------- */
+/* Rounding                                                                    */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace gptq2d_quantize needs for an m x n problem. */
+size_t gptq2d_quantize_workspace_size(int64_t m, int64_t n);
+
+/* GPTQ-2D rounding of W under H_R (x) H_L, given the factors from
+ * gptq2d_prepare (arxivlens Abstract: same rounding as the quartic Kronecker
+ * feedback, cubic work, anti-diagonals in parallel).
+ *
+ *   W, w_dtype, ldw : device, m x n, GPTQ2D_F32, GPTQ2D_BF16 or GPTQ2D_F64.
+ *   M_L, ldl        : device fp64, m x m lower factor of H_L (upper triangle ignored).
+ *   M_R, ldr        : device fp64, n x n lower factor of H_R (upper triangle ignored).
+ *   scales          : device fp32 [m], grid step of each row; must be finite and > 0.
+ *   bits, clamp     : grid [-2^(bits-1), 2^(bits-1)-1] when clamp = 1 (2 <= bits <= 8);
+ *                     clamp = 0 rounds to any integer (results must fit int8).
+ *   Q, ldq          : device int8 output, m x n.
+ *   stats           : device pointer to one gptq2d_stats, written at the end.
+ *   ws, ws_bytes    : device workspace, >= gptq2d_quantize_workspace_size(m, n).
+ *
+ * Rounding: q = clamp(rint(y / s_i)) with rint = round half to even; the error
+ * fed back is W_ij - s_i q_ij with the clamped q.  Entries whose y is not
+ * finite are counted in stats->n_nonfinite and set stats->status.
+ * m == 0 or n == 0 writes zero statistics and returns GPTQ2D_OK. */
+int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                    const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                    const float* scales, int bits, int clamp,
+                    int8_t* Q, int64_t ldq, gptq2d_stats* stats,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* End to end from host memory                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of DEVICE workspace gptq2d_round_host needs. */
+size_t gptq2d_round_host_workspace_size(int64_t m, int64_t n, int w_dtype, int h_dtype);
+
+/* The whole path from HOST buffers: copies W (m x n, dense), H_L (m x m),
+ * H_R (n x n) and scales to the device workspace, factors both Kronecker
+ * factors, rounds, and copies Q (m x n int8, dense) and the statistics back.
+ * Host buffers should be pinned for asynchronous copies.  Synchronizes
+ * `stream` before returning.  Returns GPTQ2D_ERR_NOT_SPD if either factor is
+ * not positive definite (the left factor is checked first; *bad_pivot, if
+ * non-NULL, receives the pivot, and *which_factor, if non-NULL, 0 for H_L and
+ * 1 for H_R), else the statistics' status. */
+int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n,
+                      const void* H_L, const void* H_R, int h_dtype,
+                      const float* scales, int bits, int clamp,
+                      int8_t* Q, gptq2d_stats* stats,
+                      void* ws, size_t ws_bytes, void* stream,
+                      int64_t* bad_pivot, int* which_factor);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ2D_H_ */

@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+entry point declared in include/gptq2d.h, sizes workspaces, and rejects invalid
+arguments before enqueuing anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import two_sided_adaptive_b200 as g
+from two_sided_adaptive_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return g.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "gptq2d.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq2d_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("gptq2d_prepare", "gptq2d_quantize", "gptq2d_round_host",
+                 "gptq2d_prepare_workspace_size", "gptq2d_quantize_workspace_size"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(0, 7):
+        assert L.gptq2d_status_string(code).startswith(b"GPTQ2D_")
+    assert b"unknown" in L.gptq2d_status_string(99)
+
+
+def test_version_and_counter(L):
+    assert L.gptq2d_version() >> 16 == 1
+    assert g.launch_count() >= 0
+
+
+def test_workspace_sizes(L):
+    assert g.prepare_workspace_size(4096) >= 8
+    ws = g.quantize_workspace_size(4096, 4096)
+    assert ws >= 3 * 4096 * 4096 * 8              # P, E and the errors, fp64
+    assert g.quantize_workspace_size(100, 70) >= 3 * 128 * 128 * 8  # padded to 64-tiles
+    assert g.quantize_workspace_size(-1, 5) == 0
+    assert g.quantize_workspace_size(0, 5) > 0
+    assert g.round_host_workspace_size(64, 64, g.DTYPE_F32, g.DTYPE_F32) > g.quantize_workspace_size(64, 64)
+    assert g.round_host_workspace_size(64, 64, 9, g.DTYPE_F32) == 0
+
+
+def _q(L, **kw):
+    a = dict(W=16, wdt=0, m=4, n=4, ldw=4, ML=16, ldl=4, MR=16, ldr=4, s=16, bits=4, clamp=1,
+             Q=16, ldq=4, st=16, ws=256, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return L.gptq2d_quantize(a["W"], a["wdt"], a["m"], a["n"], a["ldw"], a["ML"], a["ldl"], a["MR"],
+                             a["ldr"], a["s"], a["bits"], a["clamp"], a["Q"], a["ldq"], a["st"],
+                             a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [dict(bits=1), dict(bits=9), dict(clamp=2), dict(wdt=7),
+                                 dict(ldw=3), dict(ldl=3), dict(ldr=2), dict(ldq=1), dict(m=-1),
+                                 dict(W=None), dict(ML=None), dict(MR=None), dict(s=None),
+                                 dict(Q=None), dict(st=None), dict(m=1 << 21)])
+def test_quantize_rejects_invalid_arguments(L, bad):
+    assert _q(L, **bad) == g.Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(ws=None), dict(ws=272), dict(wsb=100)])
+def test_quantize_rejects_bad_workspace(L, bad):
+    assert _q(L, **bad) == g.Status.WORKSPACE
+
+
+def test_prepare_rejects_invalid_arguments(L):
+    piv = ctypes.c_int64(0)
+    P = L.gptq2d_prepare
+    assert P(16, 1, 4, 4, 32, 4, 256, 256, None, None) == g.Status.INVALID_ARG   # bf16 H
+    assert P(16, 0, -1, 4, 32, 4, 256, 256, None, None) == g.Status.INVALID_ARG
+    assert P(16, 0, 4, 3, 32, 4, 256, 256, None, None) == g.Status.INVALID_ARG
+    assert P(16, 0, 4, 4, 32, 3, 256, 256, None, None) == g.Status.INVALID_ARG
+    assert P(None, 0, 4, 4, 32, 4, 256, 256, None, None) == g.Status.INVALID_ARG
+    assert P(16, 0, 4, 4, 16, 4, 256, 256, None, None) == g.Status.INVALID_ARG   # M aliases H
+    assert P(16, 0, 4, 4, 32, 4, 264, 256, None, None) == g.Status.WORKSPACE    # misaligned
+    assert P(16, 0, 4, 4, 32, 4, 256, 0, None, None) == g.Status.WORKSPACE
+    assert P(16, 0, 0, 0, 32, 0, 256, 256, None, ctypes.byref(piv)) == g.Status.OK and piv.value == -1
+
+
+def test_round_host_rejects_invalid_arguments(L):
+    R = L.gptq2d_round_host
+    args = [16, 0, 8, 8, 16, 16, 0, 16, 4, 1, 16, 16, 256, 1 << 30, None, None, None]
+    assert R(*args[:6], 1, *args[7:]) == g.Status.INVALID_ARG      # bf16 factors
+    assert R(*args[:2], 0, *args[3:]) == g.Status.INVALID_ARG      # m = 0
+    assert R(*args[:8], 1, *args[9:]) == g.Status.INVALID_ARG      # bits = 1
+    assert R(*args[:12], 256, 10, *args[14:]) == g.Status.WORKSPACE
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(g, "library_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(g, "_LIB", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        g.lib()

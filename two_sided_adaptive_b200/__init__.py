@@ -1,0 +1,258 @@
+"""Python binding of libgptq2d, the sm_100a GPTQ-2D two-sided adaptive rounding library.
+
+Thin ctypes layer over the C ABI in ``include/gptq2d.h``: it turns torch tensors
+into raw device pointers, sizes and the current CUDA stream, allocates outputs
+and workspaces with torch, and raises on a non-OK status.  Every step of the
+path runs in the library's CUDA kernels; there is no CPU fallback, and every
+call fails loudly when the compiled library is missing.
+
+    M_L = prepare(H_L); M_R = prepare(H_R)                # H = M^T M, M lower
+    Q, stats = quantize(W, M_L, M_R, scales, bits=4)      # int8 Q, device stats
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
+    "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
+    "round_host_workspace_size", "profile_enable", "profile_reset", "profile_read",
+    "KERNEL_CLASSES", "STATS_WORDS", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F64",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libgptq2d.so")
+
+DTYPE_F32, DTYPE_BF16, DTYPE_F64 = 0, 1, 2
+STATS_WORDS = 5  # gptq2d_stats: double + 4 x int64
+
+
+class Status:
+    OK = 0
+    INVALID_ARG = 1
+    NOT_SPD = 2
+    NONFINITE = 3
+    WORKSPACE = 4
+    TIMEOUT = 5
+    CUDA = 6
+
+
+class GPTQ2DError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        msg = f"{what}: {lib().gptq2d_status_string(status).decode()}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
+
+
+_LIB = None
+_c_i64 = ctypes.c_int64
+_c_p = ctypes.c_void_p
+
+
+def lib():
+    """The loaded shared library (built in-tree by two_sided_adaptive_b200.build)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(f"libgptq2d.so is not built ({library_path}); "
+                               "run: python -m two_sided_adaptive_b200.build")
+        L = ctypes.CDLL(library_path)
+        L.gptq2d_status_string.restype = ctypes.c_char_p
+        L.gptq2d_status_string.argtypes = [ctypes.c_int]
+        L.gptq2d_version.restype = ctypes.c_int
+        L.gptq2d_launch_count.restype = _c_i64
+        L.gptq2d_profile_enable.restype = None
+        L.gptq2d_profile_enable.argtypes = [ctypes.c_int]
+        L.gptq2d_profile_read.restype = ctypes.c_int
+        L.gptq2d_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(_c_i64),
+                                          ctypes.POINTER(ctypes.c_double)]
+        L.gptq2d_profile_reset.restype = None
+        L.gptq2d_prepare_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_prepare_workspace_size.argtypes = [_c_i64]
+        L.gptq2d_prepare.restype = ctypes.c_int
+        L.gptq2d_prepare.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_i64, _c_p,
+                                     ctypes.c_size_t, _c_p, ctypes.POINTER(_c_i64)]
+        L.gptq2d_prepare_info.restype = ctypes.c_int
+        L.gptq2d_prepare_info.argtypes = [_c_p, _c_p, ctypes.POINTER(_c_i64)]
+        L.gptq2d_quantize_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_quantize_workspace_size.argtypes = [_c_i64, _c_i64]
+        L.gptq2d_quantize.restype = ctypes.c_int
+        L.gptq2d_quantize.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
+                                      _c_p, _c_i64, _c_p, ctypes.c_int, ctypes.c_int, _c_p,
+                                      _c_i64, _c_p, _c_p, ctypes.c_size_t, _c_p]
+        L.gptq2d_round_host_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_round_host_workspace_size.argtypes = [_c_i64, _c_i64, ctypes.c_int, ctypes.c_int]
+        L.gptq2d_round_host.restype = ctypes.c_int
+        L.gptq2d_round_host.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_p,
+                                        ctypes.c_int, _c_p, ctypes.c_int, ctypes.c_int, _c_p,
+                                        _c_p, _c_p, ctypes.c_size_t, _c_p,
+                                        ctypes.POINTER(_c_i64), ctypes.POINTER(ctypes.c_int)]
+        _LIB = L
+    return _LIB
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(lib().gptq2d_launch_count())
+
+
+KERNEL_CLASSES = ("prep_panel", "prep_trailing", "sweep", "propagate", "other")
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library launch with CUDA events on its stream (gptq2d_profile_enable)."""
+    lib().gptq2d_profile_enable(int(on))
+
+
+def profile_reset() -> None:
+    lib().gptq2d_profile_reset()
+
+
+def profile_read() -> dict:
+    """{kernel class: (launches, total device ms)} of the launches recorded so far."""
+    out = {}
+    for k, name in enumerate(KERNEL_CLASSES):
+        n, ms = _c_i64(0), ctypes.c_double(0.0)
+        rc = lib().gptq2d_profile_read(k, ctypes.byref(n), ctypes.byref(ms))
+        if rc != Status.OK:
+            raise GPTQ2DError(rc, "gptq2d_profile_read")
+        out[name] = (int(n.value), float(ms.value))
+    return out
+
+
+def prepare_workspace_size(k: int) -> int:
+    return int(lib().gptq2d_prepare_workspace_size(k))
+
+
+def quantize_workspace_size(m: int, n: int) -> int:
+    return int(lib().gptq2d_quantize_workspace_size(m, n))
+
+
+def round_host_workspace_size(m: int, n: int, w_dtype: int, h_dtype: int) -> int:
+    return int(lib().gptq2d_round_host_workspace_size(m, n, w_dtype, h_dtype))
+
+
+# --------------------------------------------------------------------------- #
+# torch marshalling
+# --------------------------------------------------------------------------- #
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    codes = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float64: DTYPE_F64}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _ld(t) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride (row-major)")
+    return t.stride(0)
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_device(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device")
+
+
+def _workspace(nbytes, device, workspace):
+    torch = _torch()
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError("workspace too small")
+        return workspace
+    # 256-byte alignment: torch's caching allocator hands out 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def prepare(H, *, out=None, workspace=None, stream=None, check: bool = True):
+    """Lower-triangular M with M^T M = H (fp64), by gptq2d_prepare.  H: k x k fp32/fp64 on
+    the GPU (lower triangle read).  ``check`` synchronizes and raises on a non-SPD H."""
+    torch = _torch()
+    _check_device(H)
+    k = H.shape[0]
+    if H.dim() != 2 or H.shape[1] != k:
+        raise ValueError("H must be square")
+    M = out if out is not None else torch.empty((k, k), dtype=torch.float64, device=H.device)
+    ws = _workspace(prepare_workspace_size(k), H.device, workspace)
+    piv = _c_i64(-1)
+    rc = lib().gptq2d_prepare(H.data_ptr(), _dtype_code(H), k, _ld(H), M.data_ptr(), _ld(M),
+                              ws.data_ptr(), ws.numel(), _stream(stream),
+                              ctypes.byref(piv) if check else None)
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_prepare", f"pivot {piv.value}" if rc == Status.NOT_SPD else "")
+    return M
+
+
+def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None, stats=None,
+             workspace=None, stream=None):
+    """GPTQ-2D rounding by gptq2d_quantize.  Returns (Q int8 m x n, stats int64[5] on the
+    device; decode with stats_dict)."""
+    torch = _torch()
+    _check_device(W, M_L, M_R, scales)
+    m, n = W.shape
+    if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous fp32 vector of length m")
+    if M_L.dtype != torch.float64 or M_R.dtype != torch.float64:
+        raise ValueError("factors must be fp64")
+    Q = out if out is not None else torch.empty((m, n), dtype=torch.int8, device=W.device)
+    st = stats if stats is not None else torch.empty(STATS_WORDS, dtype=torch.int64, device=W.device)
+    ws = _workspace(quantize_workspace_size(m, n), W.device, workspace)
+    rc = lib().gptq2d_quantize(W.data_ptr(), _dtype_code(W), m, n, _ld(W), M_L.data_ptr(), _ld(M_L),
+                               M_R.data_ptr(), _ld(M_R), scales.data_ptr(), int(bits), int(clamp),
+                               Q.data_ptr(), _ld(Q), st.data_ptr(), ws.data_ptr(), ws.numel(),
+                               _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_quantize")
+    return Q, st
+
+
+def stats_dict(st) -> dict:
+    """Decodes a gptq2d_stats (int64[5] tensor or array) into a dict."""
+    a = np.asarray(st.cpu() if hasattr(st, "cpu") else st, dtype=np.int64).copy()
+    return {"proxy_loss": float(a[:1].view(np.float64)[0]), "n_clamped": int(a[1]),
+            "n_near_tie": int(a[2]), "n_nonfinite": int(a[3]), "status": int(a[4])}
+
+
+def round_host(W, H_L, H_R, scales, bits: int = 4, clamp: bool = True, *, workspace=None,
+               stream=None, Q_out=None, stats_out=None):
+    """The whole path from HOST tensors through gptq2d_round_host: copies in, factors both
+    Kronecker factors, rounds, copies Q and the statistics out.  Inputs should be pinned CPU
+    tensors; ``workspace`` is a device uint8 tensor of round_host_workspace_size bytes."""
+    torch = _torch()
+    m, n = W.shape
+    for t in (W, H_L, H_R, scales):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("round_host takes contiguous host tensors")
+    if H_L.dtype != H_R.dtype:
+        raise ValueError("H_L and H_R must share a dtype")
+    wdt, hdt = _dtype_code(W), _dtype_code(H_L)
+    need = round_host_workspace_size(m, n, wdt, hdt)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    Q = Q_out if Q_out is not None else torch.empty((m, n), dtype=torch.int8, pin_memory=True)
+    st = stats_out if stats_out is not None else torch.empty(STATS_WORDS, dtype=torch.int64,
+                                                             pin_memory=True)
+    piv, which = _c_i64(-1), ctypes.c_int(-1)
+    rc = lib().gptq2d_round_host(W.data_ptr(), wdt, m, n, H_L.data_ptr(), H_R.data_ptr(), hdt,
+                                 scales.data_ptr(), int(bits), int(clamp), Q.data_ptr(),
+                                 st.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream), ctypes.byref(piv), ctypes.byref(which))
+    if rc not in (Status.OK, Status.NONFINITE):
+        raise GPTQ2DError(rc, "gptq2d_round_host",
+                          f"factor {which.value} pivot {piv.value}" if rc == Status.NOT_SPD else "")
+    return Q, st

@@ -1,0 +1,255 @@
+// extern "C" entry points of libgptq2d (declared and documented in include/gptq2d.h).
+// Argument checks run on the host before anything is enqueued.
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+
+namespace gptq2d {
+std::atomic<int64_t> g_launches{0};
+
+namespace {
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_ev[KC_COUNT];
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+ProfScope::ProfScope(int c, cudaStream_t st) : cls(c), s(st) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  e0 = prof_event();
+  if (e0) cudaEventRecord(e0, s);
+}
+
+ProfScope::~ProfScope() {
+  if (!e0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEvent_t e1 = prof_event();
+  if (e1 && cudaEventRecord(e1, s) == cudaSuccess)
+    g_prof_ev[cls].emplace_back(e0, e1);
+  else
+    g_prof_pool.push_back(e0);
+}
+}  // namespace gptq2d
+
+using namespace gptq2d;
+
+namespace {
+
+// Largest edge handled: keeps every 64-tile count and padded product within int32.
+constexpr int64_t kMaxDim = (int64_t)1 << 20;
+
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+size_t elem_size(int dt) {
+  switch (dt) {
+    case GPTQ2D_F32: return 4;
+    case GPTQ2D_BF16: return 2;
+    case GPTQ2D_F64: return 8;
+    default: return 0;
+  }
+}
+
+struct HostWs {
+  size_t off_W, off_HL, off_HR, off_s, off_ML, off_MR, off_Q, off_stats, off_pl, off_pr, off_q,
+      total;
+};
+
+HostWs host_layout(int64_t m, int64_t n, int w_dtype, int h_dtype) {
+  HostWs L;
+  size_t o = 0;
+  L.off_W = o; o += align256((size_t)m * n * elem_size(w_dtype));
+  L.off_HL = o; o += align256((size_t)m * m * elem_size(h_dtype));
+  L.off_HR = o; o += align256((size_t)n * n * elem_size(h_dtype));
+  L.off_s = o; o += align256((size_t)m * sizeof(float));
+  L.off_ML = o; o += align256((size_t)m * m * sizeof(double));
+  L.off_MR = o; o += align256((size_t)n * n * sizeof(double));
+  L.off_Q = o; o += align256((size_t)m * n);
+  L.off_stats = o; o += align256(sizeof(gptq2d_stats));
+  L.off_pl = o; o += align256(prepare_ws_bytes(m));
+  L.off_pr = o; o += align256(prepare_ws_bytes(n));
+  L.off_q = o; o += align256(quantize_ws_bytes(m, n));
+  L.total = o;
+  return L;
+}
+
+int read_pivot(const void* ws, cudaStream_t s, int64_t* bad_pivot) {
+  long long info = -1;
+  if (cudaMemcpyAsync(&info, ws, sizeof(info), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+  if (bad_pivot) *bad_pivot = info;
+  return info >= 0 ? GPTQ2D_ERR_NOT_SPD : GPTQ2D_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gptq2d_status_string(int status) {
+  switch (status) {
+    case GPTQ2D_OK: return "GPTQ2D_OK";
+    case GPTQ2D_ERR_INVALID_ARG: return "GPTQ2D_ERR_INVALID_ARG: invalid argument";
+    case GPTQ2D_ERR_NOT_SPD: return "GPTQ2D_ERR_NOT_SPD: factor is not positive definite";
+    case GPTQ2D_ERR_NONFINITE: return "GPTQ2D_ERR_NONFINITE: non-finite input or invalid scale";
+    case GPTQ2D_ERR_WORKSPACE: return "GPTQ2D_ERR_WORKSPACE: workspace too small or misaligned";
+    case GPTQ2D_ERR_TIMEOUT: return "GPTQ2D_ERR_TIMEOUT: bounded device wait gave up";
+    case GPTQ2D_ERR_CUDA: return "GPTQ2D_ERR_CUDA: CUDA runtime error";
+    default: return "GPTQ2D: unknown status";
+  }
+}
+
+int gptq2d_version(void) { return (1 << 16) | 0; }
+
+int64_t gptq2d_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void gptq2d_profile_enable(int on) { g_prof_on.store(on != 0); }
+
+int gptq2d_profile_read(int kernel_class, int64_t* launches, double* total_ms) {
+  if (kernel_class < 0 || kernel_class >= KC_COUNT || !launches || !total_ms)
+    return GPTQ2D_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  double ms = 0.0;
+  for (auto& pr : g_prof_ev[kernel_class]) {
+    if (cudaEventSynchronize(pr.second) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, pr.first, pr.second) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+    ms += t;
+  }
+  *launches = (int64_t)g_prof_ev[kernel_class].size();
+  *total_ms = ms;
+  return GPTQ2D_OK;
+}
+
+void gptq2d_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& v : g_prof_ev) {
+    for (auto& pr : v) {
+      g_prof_pool.push_back(pr.first);
+      g_prof_pool.push_back(pr.second);
+    }
+    v.clear();
+  }
+}
+
+size_t gptq2d_prepare_workspace_size(int64_t k) {
+  if (k < 0 || k > kMaxDim) return 0;
+  return prepare_ws_bytes(k);
+}
+
+int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh, double* M, int64_t ldm,
+                   void* ws, size_t ws_bytes, void* stream, int64_t* bad_pivot) {
+  if (k < 0 || k > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  if (h_dtype != GPTQ2D_F32 && h_dtype != GPTQ2D_F64) return GPTQ2D_ERR_INVALID_ARG;
+  if (k == 0) {
+    if (bad_pivot) *bad_pivot = -1;
+    return GPTQ2D_OK;
+  }
+  if (!H || !M || ldh < k || ldm < k) return GPTQ2D_ERR_INVALID_ARG;
+  if (static_cast<const void*>(M) == H) return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < prepare_ws_bytes(k)) return GPTQ2D_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rc = prepare_launch(H, h_dtype, (int)k, ldh, M, ldm, ws, s);
+  if (rc != GPTQ2D_OK) return rc;
+  if (bad_pivot) return read_pivot(ws, s, bad_pivot);
+  return GPTQ2D_OK;
+}
+
+int gptq2d_prepare_info(const void* ws, void* stream, int64_t* bad_pivot) {
+  if (!ws || !bad_pivot) return GPTQ2D_ERR_INVALID_ARG;
+  return read_pivot(ws, static_cast<cudaStream_t>(stream), bad_pivot);
+}
+
+size_t gptq2d_quantize_workspace_size(int64_t m, int64_t n) {
+  if (m < 0 || n < 0 || m > kMaxDim || n > kMaxDim) return 0;
+  if (m == 0 || n == 0) return 256;
+  return quantize_ws_bytes(m, n);
+}
+
+int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                    const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                    const float* scales, int bits, int clamp, int8_t* Q, int64_t ldq,
+                    gptq2d_stats* stats, void* ws, size_t ws_bytes, void* stream) {
+  if (m < 0 || n < 0 || m > kMaxDim || n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  if (elem_size(w_dtype) == 0) return GPTQ2D_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 8 || (clamp != 0 && clamp != 1)) return GPTQ2D_ERR_INVALID_ARG;
+  if (!stats) return GPTQ2D_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (m == 0 || n == 0)
+    return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, scales, bits,
+                           clamp, Q, ldq, stats, ws, s);
+  if (!W || !M_L || !M_R || !scales || !Q) return GPTQ2D_ERR_INVALID_ARG;
+  if (ldw < n || ldl < m || ldr < n || ldq < n) return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(m, n)) return GPTQ2D_ERR_WORKSPACE;
+  return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, scales, bits, clamp,
+                         Q, ldq, stats, ws, s);
+}
+
+size_t gptq2d_round_host_workspace_size(int64_t m, int64_t n, int w_dtype, int h_dtype) {
+  if (m <= 0 || n <= 0 || m > kMaxDim || n > kMaxDim) return 0;
+  if (elem_size(w_dtype) == 0 || (h_dtype != GPTQ2D_F32 && h_dtype != GPTQ2D_F64)) return 0;
+  return host_layout(m, n, w_dtype, h_dtype).total;
+}
+
+int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const void* H_L,
+                      const void* H_R, int h_dtype, const float* scales, int bits, int clamp,
+                      int8_t* Q, gptq2d_stats* stats, void* ws, size_t ws_bytes, void* stream,
+                      int64_t* bad_pivot, int* which_factor) {
+  if (m <= 0 || n <= 0 || m > kMaxDim || n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  if (elem_size(w_dtype) == 0 || (h_dtype != GPTQ2D_F32 && h_dtype != GPTQ2D_F64))
+    return GPTQ2D_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 8 || (clamp != 0 && clamp != 1)) return GPTQ2D_ERR_INVALID_ARG;
+  if (!W || !H_L || !H_R || !scales || !Q || !stats) return GPTQ2D_ERR_INVALID_ARG;
+  const HostWs L = host_layout(m, n, w_dtype, h_dtype);
+  if (!ws || !aligned256(ws) || ws_bytes < L.total) return GPTQ2D_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* b = static_cast<char*>(ws);
+  const size_t hs = elem_size(h_dtype);
+  if (cudaMemcpyAsync(b + L.off_W, W, (size_t)m * n * elem_size(w_dtype), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(b + L.off_HL, H_L, (size_t)m * m * hs, cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(b + L.off_HR, H_R, (size_t)n * n * hs, cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(b + L.off_s, scales, (size_t)m * sizeof(float), cudaMemcpyHostToDevice, s))
+    return GPTQ2D_ERR_CUDA;
+  double* ML = reinterpret_cast<double*>(b + L.off_ML);
+  double* MR = reinterpret_cast<double*>(b + L.off_MR);
+  int rc = prepare_launch(b + L.off_HL, h_dtype, (int)m, m, ML, m, b + L.off_pl, s);
+  if (rc == GPTQ2D_OK) rc = prepare_launch(b + L.off_HR, h_dtype, (int)n, n, MR, n, b + L.off_pr, s);
+  if (rc == GPTQ2D_OK)
+    rc = quantize_launch(b + L.off_W, w_dtype, (int)m, (int)n, n, ML, m, MR, n,
+                         reinterpret_cast<const float*>(b + L.off_s), bits, clamp,
+                         reinterpret_cast<int8_t*>(b + L.off_Q), n,
+                         reinterpret_cast<gptq2d_stats*>(b + L.off_stats), b + L.off_q, s);
+  if (rc != GPTQ2D_OK) return rc;
+  long long piv[2] = {-1, -1};
+  if (cudaMemcpyAsync(Q, b + L.off_Q, (size_t)m * n, cudaMemcpyDeviceToHost, s) ||
+      cudaMemcpyAsync(stats, b + L.off_stats, sizeof(gptq2d_stats), cudaMemcpyDeviceToHost, s) ||
+      cudaMemcpyAsync(&piv[0], b + L.off_pl, sizeof(long long), cudaMemcpyDeviceToHost, s) ||
+      cudaMemcpyAsync(&piv[1], b + L.off_pr, sizeof(long long), cudaMemcpyDeviceToHost, s))
+    return GPTQ2D_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+  for (int f = 0; f < 2; ++f)
+    if (piv[f] >= 0) {
+      if (bad_pivot) *bad_pivot = piv[f];
+      if (which_factor) *which_factor = f;
+      return GPTQ2D_ERR_NOT_SPD;
+    }
+  if (bad_pivot) *bad_pivot = -1;
+  if (which_factor) *which_factor = -1;
+  return (int)stats->status;
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+// Internal helpers shared by the GPTQ-2D kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <atomic>
+
+#include "gptq2d.h"
+
+namespace gptq2d {
+
+// Edge of the square tiles the rounding sweep and the factor preparation work on.
+constexpr int TB = 64;
+
+// Counts every kernel launch the library issues (gptq2d_launch_count).
+extern std::atomic<int64_t> g_launches;
+inline void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Kernel classes of the optional per-launch event profiler (gptq2d_profile_*).
+enum KernelClass {
+  KC_PREP_PANEL = 0,     // factor preparation: diagonal block + block-row solve
+  KC_PREP_TRAILING = 1,  // factor preparation: rank-64 trailing update
+  KC_SWEEP = 2,          // anti-diagonal tile sweep
+  KC_PROPAGATE = 3,      // band products (right / down feedback)
+  KC_OTHER = 4,          // conversions, diagonals, statistics
+  KC_COUNT = 5
+};
+// When profiling is on, records a CUDA event pair around the launch on `s`.
+struct ProfScope {
+  int cls;
+  cudaStream_t s;
+  cudaEvent_t e0 = nullptr;
+  ProfScope(int c, cudaStream_t st);
+  ~ProfScope();
+};
+#define GPTQ2D_LAUNCH(cls, stream, ...)             \
+  do {                                              \
+    ::gptq2d::ProfScope _ps((cls), (stream));       \
+    __VA_ARGS__;                                    \
+    ::gptq2d::count_launch();                       \
+  } while (0)
+
+inline int64_t round_up(int64_t x, int64_t r) { return (x + r - 1) / r * r; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Sets the dynamic shared-memory limit of `fn` once per device.
+template <typename F>
+inline cudaError_t ensure_smem(F* fn, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit && (done_mask.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+// ---------------------------------------------------------------------------
+// Element loads with conversion to fp64
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double to_f64(float v) { return static_cast<double>(v); }
+__device__ __forceinline__ double to_f64(double v) { return v; }
+__device__ __forceinline__ double to_f64(__nv_bfloat16 v) {
+  return static_cast<double>(__bfloat162float(v));
+}
+
+// ---------------------------------------------------------------------------
+// FP64 tensor-core MMA (DMMA), m8n8k4, row.col.
+// Fragments (lane = 4*g + t, g = lane>>2, t = lane&3):
+//   A 8x4 : a = A[g][t]        B 4x8 : b = B[t][g]
+//   C 8x8 : c0 = C[g][2t], c1 = C[g][2t+1]
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void dmma_m8n8k4(double& c0, double& c1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+               : "+d"(c0), "+d"(c1)
+               : "d"(a), "d"(b));
+}
+
+// 64x64x64 product of two shared-memory tiles on 4 warps (128 threads).  Warp w
+// owns the 32x32 quadrant (w>>1, w&1) as 4x4 fragments of 8x8.  `fa(row, k)`
+// and `fb(k, col)` return the operand elements from shared memory.
+template <typename FA, typename FB>
+__device__ __forceinline__ void mma_64x64x64(double (&acc)[4][4][2], FA fa, FB fb, int kmax = TB) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
+#pragma unroll 4
+  for (int kk = 0; kk < kmax; kk += 4) {
+    double a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = fa(wr + i * 8 + g, kk + t);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = fb(kk + t, wc + j * 8 + g);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
+  }
+}
+
+// Per-tile partial statistics of one rounding sweep.
+struct TileStat {
+  double loss;
+  long long clamped, near_tie, nonfinite;
+};
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (defined in prepare.cu / quantize.cu)
+// ---------------------------------------------------------------------------
+size_t prepare_ws_bytes(int64_t k);
+int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
+                   void* ws, cudaStream_t s);
+
+size_t quantize_ws_bytes(int64_t m, int64_t n);
+int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
+                    int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
+                    int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
+                    cudaStream_t s);
+
+}  // namespace gptq2d
