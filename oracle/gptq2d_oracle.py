@@ -96,7 +96,7 @@ def reverse_cholesky(H):
     """
     H = np.asarray(H, np.float64)
     L = np.linalg.cholesky(H[::-1, ::-1])
-    return np.ascontiguousarray(L.T[::-1, ::-1])
+    return np.array(L.T[::-1, ::-1], order="C", copy=True)
 
 
 # --------------------------------------------------------------------------- #
