@@ -217,6 +217,27 @@ def cpu_baseline(pb, sample):
                        f"rounding time scaled by mn(m+n) to {m}x{n}: {t_full:.1f} s per layer")}
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank rounds its own independent layer: the workload seed is the rank."""
+    return rank
+
+
+def aggregate_value(m: int, n: int, world: int, ms_step_max: float) -> float:
+    """Whole-job entries/s: every rank rounds m*n entries per step; time is the slowest rank's."""
+    return world * m * n / (ms_step_max * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -229,7 +250,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     g.lib()
     dev = torch.device("cuda", local_rank)
-    pb = make_problem(args.workload, seed=rank)
+    pb = make_problem(args.workload, seed=rank_seed(rank))
     m, n = pb.shape
     W = torch.from_numpy(pb.W).to(dev).to(torch.bfloat16 if args.workload != "small" else torch.float32)
     H_L = torch.from_numpy(pb.H_L).to(dev)
@@ -247,6 +268,12 @@ def run_ours(args, rank, world, local_rank):
         g.prepare(H_L, out=M_L, workspace=wsL, check=False)
         g.prepare(H_R, out=M_R, workspace=wsR, check=False)
         g.quantize(W, M_L, M_R, s, pb.bits, pb.clamp, out=Q, stats=st, workspace=wsQ)
+
+    if args.profile_step:
+        # one pass of the path and nothing else (for ncu captures of single kernels)
+        step()
+        torch.cuda.synchronize()
+        return None
 
     for _ in range(args.warmup):
         step()
@@ -277,13 +304,9 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop() if sampler else None
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
     ms_step = ms / args.steps
-    value = world * m * n / (ms_step * 1e-3)
+    value = aggregate_value(m, n, world, ms_step)
 
     # per-kernel device time of one more step, CUDA events around each launch on its stream
     g.profile_reset()
@@ -317,14 +340,10 @@ def run_ours(args, rank, world, local_rank):
             g.round_host(Wh, HLh, HRh, sh, pb.bits, pb.clamp, workspace=wsH, Q_out=Qh, stats_out=sth)
         f1.record()
         torch.cuda.synchronize()
-        ems = f0.elapsed_time(f1) / ke
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(f0.elapsed_time(f1) / ke, dev)
         h2d = Wh.numel() * Wh.element_size() + (HLh.numel() + HRh.numel() + sh.numel()) * 4
         d2h = Qh.numel() + sth.numel() * 8
-        e2e = {"value": world * m * n / (ems * 1e-3), "unit": "entries/s",
+        e2e = {"value": aggregate_value(m, n, world, ems), "unit": "entries/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": ems, "api": "gptq2d_round_host"}
 
@@ -437,6 +456,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=768)
     ap.add_argument("--ref-sample", type=int, default=384)
+    ap.add_argument("--profile-step", action="store_true",
+                    help="run one step of the path only (input for ncu captures); prints nothing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -463,7 +484,7 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
-    if rank == 0:
+    if rank == 0 and out is not None:
         print(json.dumps(out), flush=True)
 
 
