@@ -166,6 +166,40 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
                     void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* Rounding without any allocation                                             */
+/* (no counterpart in the GPTQ-2D pages: an interface for callers of this     */
+/* library that may not allocate device memory)                               */
+/* ------------------------------------------------------------------------- */
+
+/* Capacity of the library's static rounding scratch: 32 MiB on every device
+ * that loads the library, held until the process exits. */
+#define GPTQ2D_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* gptq2d_quantize without a workspace argument, for callers that cannot call
+ * cudaMalloc (a framework that owns all device memory through its own pool,
+ * a service that forbids allocation once it is running, or a caller that
+ * cannot afford cudaMalloc's implicit device synchronization).  Arguments,
+ * rounding and statistics are exactly those of gptq2d_quantize; the scratch is
+ * a static device array inside the library instead.
+ *
+ *   - Size limit: the problem must satisfy
+ *     gptq2d_quantize_workspace_size(m, n) <= GPTQ2D_NOALLOC_SCRATCH_BYTES
+ *     (about 1.39 million padded entries: 64*ceil(m/64) * 64*ceil(n/64), e.g.
+ *     1024 x 1024 or 512 x 2048); larger problems return GPTQ2D_ERR_WORKSPACE
+ *     and enqueue nothing.
+ *   - Sharing: every call uses the same array.  Calls whose work overlaps on
+ *     the GPU (two streams, two threads) race on it; order them.  Each call
+ *     clears what must start at zero, so leftovers of earlier calls are harmless.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int gptq2d_quantize_noalloc(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                            const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                            const float* scales, int bits, int clamp,
+                            int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* End to end from host memory                                                 */
 /* ------------------------------------------------------------------------- */
 

@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
-    "round_host_workspace_size", "profile_enable", "profile_reset", "profile_read",
+    "round_host_workspace_size", "quantize_noalloc", "profile_enable", "profile_reset", "profile_read",
     "KERNEL_CLASSES", "STATS_WORDS", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F64",
 ]
 
@@ -83,6 +83,10 @@ def lib():
         L.gptq2d_quantize.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
                                       _c_p, _c_i64, _c_p, ctypes.c_int, ctypes.c_int, _c_p,
                                       _c_i64, _c_p, _c_p, ctypes.c_size_t, _c_p]
+        L.gptq2d_quantize_noalloc.restype = ctypes.c_int
+        L.gptq2d_quantize_noalloc.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p,
+                                              _c_i64, _c_p, _c_i64, _c_p, ctypes.c_int,
+                                              ctypes.c_int, _c_p, _c_i64, _c_p, _c_p]
         L.gptq2d_round_host_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_round_host_workspace_size.argtypes = [_c_i64, _c_i64, ctypes.c_int, ctypes.c_int]
         L.gptq2d_round_host.restype = ctypes.c_int
@@ -218,6 +222,29 @@ def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None
                                _stream(stream))
     if rc != Status.OK:
         raise GPTQ2DError(rc, "gptq2d_quantize")
+    return Q, st
+
+
+def quantize_noalloc(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None,
+                     stats=None, stream=None):
+    """gptq2d_quantize_noalloc: the same rounding with the library's static device scratch
+    (no workspace; for callers that cannot allocate).  Problems must fit
+    GPTQ2D_NOALLOC_SCRATCH_BYTES; calls that overlap on the GPU race on the shared scratch."""
+    torch = _torch()
+    _check_device(W, M_L, M_R, scales)
+    m, n = W.shape
+    if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous fp32 vector of length m")
+    if M_L.dtype != torch.float64 or M_R.dtype != torch.float64:
+        raise ValueError("factors must be fp64")
+    Q = out if out is not None else torch.empty((m, n), dtype=torch.int8, device=W.device)
+    st = stats if stats is not None else torch.empty(STATS_WORDS, dtype=torch.int64, device=W.device)
+    rc = lib().gptq2d_quantize_noalloc(W.data_ptr(), _dtype_code(W), m, n, _ld(W), M_L.data_ptr(),
+                                       _ld(M_L), M_R.data_ptr(), _ld(M_R), scales.data_ptr(),
+                                       int(bits), int(clamp), Q.data_ptr(), _ld(Q), st.data_ptr(),
+                                       _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_quantize_noalloc")
     return Q, st
 
 
