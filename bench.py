@@ -61,23 +61,29 @@ def make_problem(name, seed, device_gram=True):
     raise ValueError(name)
 
 
-def band_product_flops(m, n):
-    """Useful flops of the band products (right and down feedback between 64-tiles):
-    entry (i, j) feeds 2 * (n - 64 (j//64 + 1)) flops right and 2 * (m - 64 (i//64 + 1)) down."""
+def far_flops(m, n):
+    """Useful flops of the band products to tiles two or more 64-tiles away (far_kernel):
+    entry (i, j) feeds 2 * (n - 64 (j//64 + 2)) flops right and 2 * (m - 64 (i//64 + 2)) down."""
     jt = np.arange(n) // TB
     it = np.arange(m) // TB
-    right = m * np.sum(2.0 * np.maximum(0, n - TB * (jt + 1)))
-    down = n * np.sum(2.0 * np.maximum(0, m - TB * (it + 1)))
+    right = m * np.sum(2.0 * np.maximum(0, n - TB * (jt + 2)))
+    down = n * np.sum(2.0 * np.maximum(0, m - TB * (it + 2)))
     return float(right + down)
 
 
 def sweep_flops(m, n):
-    """In-tile flops: entry (a, c) of a rows x cols tile pushes (cols-1-c) + (rows-1-a) FMAs."""
+    """Useful flops inside sweep_kernel: the in-tile pushes (entry (a, c) of a rows x cols tile
+    pushes (cols-1-c) + (rows-1-a) FMAs) plus the pulled contributions of the neighbouring
+    tiles (each entry feeds the next tile to the right and the next tile below)."""
     tot = 0.0
     for r in [min(TB, m - r0) for r0 in range(0, m, TB)]:
         for c in [min(TB, n - c0) for c0 in range(0, n, TB)]:
             tot += 2.0 * (r * c * (c - 1) / 2 + c * r * (r - 1) / 2)
-    return tot
+    jt = np.arange(n) // TB
+    it = np.arange(m) // TB
+    near_r = m * np.sum(2.0 * np.clip(n - TB * (jt + 1), 0, TB))
+    near_d = n * np.sum(2.0 * np.clip(m - TB * (it + 1), 0, TB))
+    return float(tot + near_r + near_d)
 
 
 def prep_flops(k):
@@ -258,15 +264,14 @@ def run_ours(args, rank, world, local_rank):
     s = torch.from_numpy(pb.scales).to(dev)
     M_L = torch.empty((m, m), dtype=torch.float64, device=dev)
     M_R = torch.empty((n, n), dtype=torch.float64, device=dev)
-    wsL = torch.empty(max(g.prepare_workspace_size(m), 256), dtype=torch.uint8, device=dev)
-    wsR = torch.empty(max(g.prepare_workspace_size(n), 256), dtype=torch.uint8, device=dev)
     wsQ = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
     Q = torch.empty((m, n), dtype=torch.int8, device=dev)
     st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
 
+    wsP = torch.empty(512, dtype=torch.uint8, device=dev)
+
     def step():
-        g.prepare(H_L, out=M_L, workspace=wsL, check=False)
-        g.prepare(H_R, out=M_R, workspace=wsR, check=False)
+        g.prepare_pair(H_L, H_R, out_l=M_L, out_r=M_R, workspace=wsP, check=False)
         g.quantize(W, M_L, M_R, s, pb.bits, pb.clamp, out=Q, stats=st, workspace=wsQ)
 
     if args.profile_step:
@@ -279,9 +284,9 @@ def run_ours(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     import ctypes
-    for ws in (wsL, wsR):
+    for off in (0, 256):
         piv = ctypes.c_int64(-1)
-        rc = g.lib().gptq2d_prepare_info(ws.data_ptr(), None, ctypes.byref(piv))
+        rc = g.lib().gptq2d_prepare_info(wsP.data_ptr() + off, None, ctypes.byref(piv))
         assert rc == 0, f"factor not SPD (pivot {piv.value})"
     stats = g.stats_dict(st)
     assert stats["status"] == 0, stats
@@ -352,7 +357,7 @@ def run_ours(args, rank, world, local_rank):
 
     peak = measure_dgemm_tflops()
     dom = max(("propagate", "sweep", "prep_trailing", "prep_panel"), key=lambda k: prof[k][1])
-    work = {"propagate": band_product_flops(m, n), "sweep": sweep_flops(m, n),
+    work = {"propagate": far_flops(m, n), "sweep": sweep_flops(m, n),
             "prep_trailing": prep_flops(m) + prep_flops(n), "prep_panel": None}
     nl, tms = prof[dom]
     src = {"propagate": "quantize.cu", "sweep": "quantize.cu", "prep_trailing": "prepare.cu",
@@ -373,7 +378,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": pb.name.split("_s")[0], "m": m, "n": n, "bits": pb.bits,
                    "w_dtype": str(W.dtype).replace("torch.", ""), "h_dtype": "float32",
-                   "step": "prepare(H_L) + prepare(H_R) + quantize(W), inputs resident in HBM",
+                   "step": "prepare_pair(H_L, H_R) + quantize(W), inputs resident in HBM",
                    "l2": "no flush; per-step working set (W, H_L, H_R, factors, 3 fp64 feedback "
                          "buffers) is %.2f GB > 126 MB L2" % (
                              (W.numel() * W.element_size() + 2 * 4 * (m * m + n * n) + 8 * (m * m + n * n)

@@ -94,6 +94,12 @@ void gptq2d_profile_enable(int on);
  * in milliseconds (waits for the recorded events).  GPTQ2D_ERR_INVALID_ARG for
  * an unknown class. */
 int gptq2d_profile_read(int kernel_class, int64_t* launches, double* total_ms);
+/* Timeline of the recorded launches in enqueue order: kernel class and the
+ * start / end of each launch in milliseconds after the first recorded event
+ * (waits for the events).  Writes min(max_entries, recorded) entries and the
+ * number recorded to *n_out. */
+int gptq2d_profile_timeline(int64_t max_entries, int32_t* cls, double* start_ms, double* end_ms,
+                            int64_t* n_out);
 /* Forgets all recorded launches. */
 void gptq2d_profile_reset(void);
 
@@ -128,6 +134,26 @@ size_t gptq2d_prepare_workspace_size(int64_t k);
 int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh,
                    double* M, int64_t ldm, void* ws, size_t ws_bytes,
                    void* stream, int64_t* bad_pivot);
+
+/* Both Kronecker factors in one call: H_L (m x m) -> M_L and H_R (n x n) -> M_R,
+ * each exactly as gptq2d_prepare computes it.  The two factorizations run
+ * concurrently on two library-internal streams that fork from `stream` and
+ * join back to it, so later work on `stream` sees both factors.
+ *   ws, ws_bytes : device workspace of at least 512 bytes (256-byte aligned);
+ *                  bytes [0,256) hold the left pivot word, [256,512) the right.
+ *   bad_pivot, which_factor : HOST pointers or NULL.  If either is non-NULL
+ *                  the call synchronizes `stream`; on failure it writes the
+ *                  pivot (as gptq2d_prepare does) and 0 for H_L / 1 for H_R
+ *                  (H_L reported first) and returns GPTQ2D_ERR_NOT_SPD; else
+ *                  it writes -1 to both.  If both are NULL the call is
+ *                  asynchronous; gptq2d_prepare_info(ws) and
+ *                  gptq2d_prepare_info(ws + 256) read the two pivot words.
+ * m == 0 or n == 0 skips that factor. */
+int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl,
+                        const void* H_R, int64_t n, int64_t ldhr, int h_dtype,
+                        double* M_L, int64_t ldml, double* M_R, int64_t ldmr,
+                        void* ws, size_t ws_bytes, void* stream,
+                        int64_t* bad_pivot, int* which_factor);
 
 /* Reads the pivot word a previous asynchronous gptq2d_prepare left in `ws`
  * (synchronizes `stream`).  Writes -1 or the failing pivot to *bad_pivot and
@@ -171,9 +197,9 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
 /* library that may not allocate device memory)                               */
 /* ------------------------------------------------------------------------- */
 
-/* Capacity of the library's static rounding scratch: 32 MiB on every device
+/* Capacity of the library's static rounding scratch: 48 MiB on every device
  * that loads the library, held until the process exits. */
-#define GPTQ2D_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define GPTQ2D_NOALLOC_SCRATCH_BYTES (48u << 20)
 
 /* gptq2d_quantize without a workspace argument, for callers that cannot call
  * cudaMalloc (a framework that owns all device memory through its own pool,
@@ -184,9 +210,8 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
  *
  *   - Size limit: the problem must satisfy
  *     gptq2d_quantize_workspace_size(m, n) <= GPTQ2D_NOALLOC_SCRATCH_BYTES
- *     (about 1.39 million padded entries: 64*ceil(m/64) * 64*ceil(n/64), e.g.
- *     1024 x 1024 or 512 x 2048); larger problems return GPTQ2D_ERR_WORKSPACE
- *     and enqueue nothing.
+ *     (for example 1024 x 1024, which needs 40 MiB); larger problems return
+ *     GPTQ2D_ERR_WORKSPACE and enqueue nothing.
  *   - Sharing: every call uses the same array.  Calls whose work overlaps on
  *     the GPU (two streams, two threads) race on it; order them.  Each call
  *     clears what must start at zero, so leftovers of earlier calls are harmless.

@@ -260,3 +260,26 @@ def test_attention_layer_4096(g):
     assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
     rtn_loss = O.proxy_loss(W64, O.rtn(W64, s64, pb.bits, pb.clamp), s64, pb.H_L, pb.H_R)
     assert st["proxy_loss"] < rtn_loss
+
+
+# --------------------------------------------------------------------------- #
+# both factors in one call
+# --------------------------------------------------------------------------- #
+def test_prepare_pair_matches_single_factors(g):
+    rng = np.random.default_rng(21)
+    H_L = WL.damped_gram(WL.student_t_activations(rng, 700, 130))
+    H_R = WL.damped_gram(WL.student_t_activations(rng, 900, 200))
+    ML, MR = g.prepare_pair(dev(H_L), dev(H_R))
+    assert torch.equal(ML, g.prepare(dev(H_L))) and torch.equal(MR, g.prepare(dev(H_R)))
+    np.testing.assert_allclose(MR.cpu().numpy(), O.reverse_cholesky(H_R.astype(np.float64)),
+                               rtol=1e-9, atol=1e-11 * np.abs(MR.cpu().numpy()).max())
+
+
+@pytest.mark.parametrize("bad_side", [0, 1])
+def test_prepare_pair_reports_which_factor(g, bad_side):
+    H_L, H_R = np.eye(70), np.eye(90)
+    (H_L if bad_side == 0 else H_R)[33, 33] = -1.0
+    with pytest.raises(g.GPTQ2DError) as ei:
+        g.prepare_pair(dev(H_L), dev(H_R))
+    assert ei.value.status == g.Status.NOT_SPD
+    assert f"factor {bad_side} pivot 33" in str(ei.value)

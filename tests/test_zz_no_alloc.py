@@ -68,7 +68,7 @@ def test_noalloc_matches_workspace_entry_point(g):
 
 
 def test_noalloc_rejects_problems_beyond_the_static_scratch(g):
-    cap = 32 << 20
+    cap = 48 << 20
     assert g.quantize_workspace_size(1024, 1024) <= cap < g.quantize_workspace_size(2048, 2048)
     rc = g.lib().gptq2d_quantize_noalloc(16, 0, 2048, 2048, 2048, 16, 2048, 16, 2048, 16, 4, 1,
                                          16, 2048, 16, None)

@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
-    "round_host_workspace_size", "quantize_noalloc", "profile_enable", "profile_reset", "profile_read",
+    "round_host_workspace_size", "quantize_noalloc", "profile_enable", "profile_reset", "profile_read", "profile_timeline",
     "KERNEL_CLASSES", "STATS_WORDS", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F64",
 ]
 
@@ -70,11 +70,17 @@ def lib():
         L.gptq2d_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(_c_i64),
                                           ctypes.POINTER(ctypes.c_double)]
         L.gptq2d_profile_reset.restype = None
+        L.gptq2d_profile_timeline.restype = ctypes.c_int
+        L.gptq2d_profile_timeline.argtypes = [_c_i64, _c_p, _c_p, _c_p, ctypes.POINTER(_c_i64)]
         L.gptq2d_prepare_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_prepare_workspace_size.argtypes = [_c_i64]
         L.gptq2d_prepare.restype = ctypes.c_int
         L.gptq2d_prepare.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_i64, _c_p,
                                      ctypes.c_size_t, _c_p, ctypes.POINTER(_c_i64)]
+        L.gptq2d_prepare_pair.restype = ctypes.c_int
+        L.gptq2d_prepare_pair.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, ctypes.c_int,
+                                          _c_p, _c_i64, _c_p, _c_i64, _c_p, ctypes.c_size_t, _c_p,
+                                          ctypes.POINTER(_c_i64), ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_prepare_info.restype = ctypes.c_int
         L.gptq2d_prepare_info.argtypes = [_c_p, _c_p, ctypes.POINTER(_c_i64)]
         L.gptq2d_quantize_workspace_size.restype = ctypes.c_size_t
@@ -125,6 +131,21 @@ def profile_read() -> dict:
             raise GPTQ2DError(rc, "gptq2d_profile_read")
         out[name] = (int(n.value), float(ms.value))
     return out
+
+
+def profile_timeline():
+    """[(kernel class, start ms, end ms)] of the recorded launches, relative to the first."""
+    n = _c_i64(0)
+    rc = lib().gptq2d_profile_timeline(0, None, None, None, ctypes.byref(n))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_profile_timeline")
+    cls = (ctypes.c_int32 * max(1, n.value))()
+    t0 = (ctypes.c_double * max(1, n.value))()
+    t1 = (ctypes.c_double * max(1, n.value))()
+    rc = lib().gptq2d_profile_timeline(n.value, cls, t0, t1, ctypes.byref(n))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_profile_timeline")
+    return [(KERNEL_CLASSES[cls[i]], t0[i], t1[i]) for i in range(n.value)]
 
 
 def prepare_workspace_size(k: int) -> int:
@@ -200,6 +221,30 @@ def prepare(H, *, out=None, workspace=None, stream=None, check: bool = True):
     if rc != Status.OK:
         raise GPTQ2DError(rc, "gptq2d_prepare", f"pivot {piv.value}" if rc == Status.NOT_SPD else "")
     return M
+
+
+def prepare_pair(H_L, H_R, *, out_l=None, out_r=None, workspace=None, stream=None,
+                 check: bool = True):
+    """Both factors at once (gptq2d_prepare_pair): the two factorizations run concurrently
+    on library-internal streams joined back to ``stream``.  Returns (M_L, M_R)."""
+    torch = _torch()
+    _check_device(H_L, H_R)
+    if H_L.dtype != H_R.dtype:
+        raise ValueError("H_L and H_R must share a dtype")
+    m, n = H_L.shape[0], H_R.shape[0]
+    ML = out_l if out_l is not None else torch.empty((m, m), dtype=torch.float64, device=H_L.device)
+    MR = out_r if out_r is not None else torch.empty((n, n), dtype=torch.float64, device=H_L.device)
+    ws = _workspace(512, H_L.device, workspace)
+    piv, which = _c_i64(-1), ctypes.c_int(-1)
+    rc = lib().gptq2d_prepare_pair(H_L.data_ptr(), m, _ld(H_L), H_R.data_ptr(), n, _ld(H_R),
+                                   _dtype_code(H_L), ML.data_ptr(), _ld(ML), MR.data_ptr(), _ld(MR),
+                                   ws.data_ptr(), ws.numel(), _stream(stream),
+                                   ctypes.byref(piv) if check else None,
+                                   ctypes.byref(which) if check else None)
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_prepare_pair",
+                          f"factor {which.value} pivot {piv.value}" if rc == Status.NOT_SPD else "")
+    return ML, MR
 
 
 def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None, stats=None,

@@ -1,5 +1,6 @@
 // extern "C" entry points of libgptq2d (declared and documented in include/gptq2d.h).
 // Argument checks run on the host before anything is enqueued.
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -14,6 +15,8 @@ namespace {
 std::atomic<bool> g_prof_on{false};
 std::mutex g_prof_mu;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_ev[KC_COUNT];
+struct ProfRec { int cls; cudaEvent_t e0, e1; };
+std::vector<ProfRec> g_prof_order;  // every recorded launch, in enqueue order
 std::vector<cudaEvent_t> g_prof_pool;
 
 cudaEvent_t prof_event() {
@@ -40,7 +43,10 @@ ProfScope::~ProfScope() {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   cudaEvent_t e1 = prof_event();
   if (e1 && cudaEventRecord(e1, s) == cudaSuccess)
+  {
     g_prof_ev[cls].emplace_back(e0, e1);
+    g_prof_order.push_back(ProfRec{cls, e0, e1});
+  }
   else
     g_prof_pool.push_back(e0);
 }
@@ -135,8 +141,31 @@ int gptq2d_profile_read(int kernel_class, int64_t* launches, double* total_ms) {
   return GPTQ2D_OK;
 }
 
+int gptq2d_profile_timeline(int64_t max_entries, int32_t* cls, double* start_ms, double* end_ms,
+                            int64_t* n_out) {
+  if (!n_out || (max_entries > 0 && (!cls || !start_ms || !end_ms))) return GPTQ2D_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  *n_out = (int64_t)g_prof_order.size();
+  if (g_prof_order.empty()) return GPTQ2D_OK;
+  const cudaEvent_t base = g_prof_order.front().e0;
+  for (auto& r : g_prof_order)
+    if (cudaEventSynchronize(r.e1) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+  const int64_t n = std::min<int64_t>(max_entries, (int64_t)g_prof_order.size());
+  for (int64_t i = 0; i < n; ++i) {
+    float a = 0.f, b = 0.f;
+    if (cudaEventElapsedTime(&a, base, g_prof_order[i].e0) != cudaSuccess ||
+        cudaEventElapsedTime(&b, base, g_prof_order[i].e1) != cudaSuccess)
+      return GPTQ2D_ERR_CUDA;
+    cls[i] = g_prof_order[i].cls;
+    start_ms[i] = a;
+    end_ms[i] = b;
+  }
+  return GPTQ2D_OK;
+}
+
 void gptq2d_profile_reset(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_order.clear();
   for (auto& v : g_prof_ev) {
     for (auto& pr : v) {
       g_prof_pool.push_back(pr.first);
@@ -166,6 +195,40 @@ int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh, double* M
   const int rc = prepare_launch(H, h_dtype, (int)k, ldh, M, ldm, ws, s);
   if (rc != GPTQ2D_OK) return rc;
   if (bad_pivot) return read_pivot(ws, s, bad_pivot);
+  return GPTQ2D_OK;
+}
+
+int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
+                        int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
+                        int64_t ldmr, void* ws, size_t ws_bytes, void* stream,
+                        int64_t* bad_pivot, int* which_factor) {
+  if (m < 0 || n < 0 || m > kMaxDim || n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  if (h_dtype != GPTQ2D_F32 && h_dtype != GPTQ2D_F64) return GPTQ2D_ERR_INVALID_ARG;
+  if (m > 0 && (!H_L || !M_L || ldhl < m || ldml < m || static_cast<const void*>(M_L) == H_L))
+    return GPTQ2D_ERR_INVALID_ARG;
+  if (n > 0 && (!H_R || !M_R || ldhr < n || ldmr < n || static_cast<const void*>(M_R) == H_R))
+    return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < 512) return GPTQ2D_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* b = static_cast<char*>(ws);
+  const int rc = prepare_pair_launch(H_L, m, ldhl, H_R, n, ldhr, h_dtype, M_L, ldml, M_R, ldmr,
+                                     b, b + 256, s);
+  if (rc != GPTQ2D_OK) return rc;
+  if (!bad_pivot && !which_factor) return GPTQ2D_OK;
+  long long piv[2] = {-1, -1};
+  if (m > 0 && cudaMemcpyAsync(&piv[0], b, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  if (n > 0 && cudaMemcpyAsync(&piv[1], b + 256, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+  for (int f = 0; f < 2; ++f)
+    if (piv[f] >= 0) {
+      if (bad_pivot) *bad_pivot = piv[f];
+      if (which_factor) *which_factor = f;
+      return GPTQ2D_ERR_NOT_SPD;
+    }
+  if (bad_pivot) *bad_pivot = -1;
+  if (which_factor) *which_factor = -1;
   return GPTQ2D_OK;
 }
 
@@ -226,8 +289,8 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
     return GPTQ2D_ERR_CUDA;
   double* ML = reinterpret_cast<double*>(b + L.off_ML);
   double* MR = reinterpret_cast<double*>(b + L.off_MR);
-  int rc = prepare_launch(b + L.off_HL, h_dtype, (int)m, m, ML, m, b + L.off_pl, s);
-  if (rc == GPTQ2D_OK) rc = prepare_launch(b + L.off_HR, h_dtype, (int)n, n, MR, n, b + L.off_pr, s);
+  int rc = prepare_pair_launch(b + L.off_HL, m, m, b + L.off_HR, n, n, h_dtype, ML, m, MR, n,
+                               b + L.off_pl, b + L.off_pr, s);
   if (rc == GPTQ2D_OK)
     rc = quantize_launch(b + L.off_W, w_dtype, (int)m, (int)n, n, ML, m, MR, n,
                          reinterpret_cast<const float*>(b + L.off_s), bits, clamp,

@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 #include <atomic>
+#include <mutex>
 
 #include "gptq2d.h"
 
@@ -101,6 +102,27 @@ __device__ __forceinline__ void mma_64x64x64(double (&acc)[4][4][2], FA fa, FB f
   }
 }
 
+// ---------------------------------------------------------------------------
+// cp.async helpers (Ampere-style asynchronous copies, available on sm_100a)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 16 : 0;  // src-size 0: nothing is read, 16 zero bytes are written
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async8_zfill(void* smem, const void* gmem, bool valid) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 8 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit_group() {
+  asm volatile("cp.async.commit_group;\n" ::);
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
 // Per-tile partial statistics of one rounding sweep.
 struct TileStat {
   double loss;
@@ -108,11 +130,33 @@ struct TileStat {
 };
 
 // ---------------------------------------------------------------------------
+// Per-device internal streams (streams.cu): a highest-priority and a lowest-
+// priority non-blocking stream plus events to fork from / join to the caller's
+// stream.  `mu` serialises the enqueue sequences that use them.
+// ---------------------------------------------------------------------------
+constexpr int RING = 4;
+struct DevStreams {
+  std::mutex mu;
+  bool ready = false;
+  int sms = 148;
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t fork = nullptr, setup = nullptr, join_hi = nullptr, join_lo = nullptr;
+  cudaEvent_t sw[RING] = {}, far[RING] = {};
+};
+int dev_streams(DevStreams** out);
+
+// ---------------------------------------------------------------------------
 // Host-side launchers (defined in prepare.cu / quantize.cu)
 // ---------------------------------------------------------------------------
 size_t prepare_ws_bytes(int64_t k);
 int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
                    void* ws, cudaStream_t s);
+
+// Both factors at once: H_L on the high-priority internal stream, H_R on the
+// low-priority one, forked from and joined back to `s`.
+int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
+                        int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
+                        int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s);
 
 size_t quantize_ws_bytes(int64_t m, int64_t n);
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,

@@ -15,14 +15,18 @@
 //   3. A_IJ -= M_KI^T M_KJ, J<=I<K   (rank-64 trailing update on FP64 tensor cores)
 // Everything is fp64.  A pivot that is not positive and finite stops the
 // factorization and is reported through a pivot word in the workspace.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace gptq2d {
 
 namespace {
 
-constexpr int PLD = TB + 1;   // leading dimension of the in-SM factor / panel tiles
-constexpr int SLD = TB + 8;   // leading dimension of [k][*] operand tiles (72: conflict-free fragments)
+constexpr int PLD = TB + 1;  // leading dimension of the in-SM factor / panel tiles
+constexpr int KLD = TB + 8;  // leading dimension of [k][*] operand tiles (72: conflict-free fragments)
+constexpr int TR_THREADS = 128;
+constexpr int MAX_TR_GROUPS = 512;
 
 template <typename TH>
 __global__ void __launch_bounds__(256) convert_lower_kernel(const TH* __restrict__ H, int64_t ldh,
@@ -39,13 +43,16 @@ __global__ void __launch_bounds__(256) convert_lower_kernel(const TH* __restrict
 
 // One launch per block row K.  CTA K factors the diagonal block and writes it;
 // CTAs b < K factor the same block redundantly in shared memory (cheaper than a
-// separate launch) and solve their block M_Kb.
+// separate launch) and solve their block M_Kb.  One barrier per pivot: the
+// scaling of a finished row is deferred to the next pivot's phase, when no
+// thread reads that row any more.
 __global__ void __launch_bounds__(256) panel_kernel(double* __restrict__ M, int64_t ldm, int k,
                                                     int K, long long* info) {
   if (*(volatile long long*)info >= 0) return;
   extern __shared__ double psm[];
-  double* S = psm;            // diagonal block, factored in place
-  double* X = psm + TB * PLD; // block M_Kb being solved
+  double* S = psm;             // diagonal block, factored in place
+  double* X = psm + TB * PLD;  // block M_Kb being solved
+  __shared__ double dd[TB], invd[TB];
   const int tid = threadIdx.x;
   const int rb = K * TB, nb = min(TB, k - rb);
   const int b = blockIdx.x;
@@ -61,20 +68,41 @@ __global__ void __launch_bounds__(256) panel_kernel(double* __restrict__ M, int6
   for (int p = nb - 1; p >= 0; --p) {
     const double piv = S[p * PLD + p];
     if (!(piv > 0.0) || !isfinite(piv)) {  // uniform: every thread read the same value
-      if (tid == 0) *info = rb + p;  // every CTA of this launch finds the same pivot
+      if (tid == 0) *info = rb + p;        // every CTA of this launch finds the same pivot
       return;
     }
     const double dp = sqrt(piv);
-    __syncthreads();
-    for (int j = tid; j < p; j += blockDim.x) S[p * PLD + j] /= dp;
-    if (tid == 0) S[p * PLD + p] = dp;
-    __syncthreads();
-    for (int e = tid; e < p * TB; e += blockDim.x) {
-      const int i = e >> 6, j = e & 63;
-      if (j <= i) S[i * PLD + j] -= S[p * PLD + i] * S[p * PLD + j];
+    const double inv = 1.0 / dp;
+    if (p + 1 < nb) {  // row p+1 is final: scale it
+      const double iv = invd[p + 1];
+      for (int j = tid; j <= p; j += blockDim.x) S[(p + 1) * PLD + j] *= iv;
+      if (tid == 0) S[(p + 1) * PLD + p + 1] = dd[p + 1];
+    }
+    {  // rows i = i0 + 4u of column j: one pivot-row value per thread, 16 batched updates
+      const int j = tid & 63, i0 = tid >> 6;
+      const double bj = S[p * PLD + j] * inv;
+      double ai[16], cij[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + 4 * u;
+        const bool ok = i < p && j <= i;
+        ai[u] = ok ? S[p * PLD + i] : 0.0;
+        cij[u] = ok ? S[i * PLD + j] : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + 4 * u;
+        if (i < p && j <= i) S[i * PLD + j] = cij[u] - (ai[u] * inv) * bj;
+      }
+    }
+    if (tid == 0) {
+      dd[p] = dp;
+      invd[p] = inv;
     }
     __syncthreads();
   }
+  if (tid == 0) S[0] = dd[0];
+  __syncthreads();
 
   if (b == K) {
     for (int e = tid; e < nb * TB; e += blockDim.x) {
@@ -84,82 +112,146 @@ __global__ void __launch_bounds__(256) panel_kernel(double* __restrict__ M, int6
     return;
   }
 
-  // X <- M_KK^{-T} X by back substitution (M_KK^T is upper triangular).
+  // X <- M_KK^{-T} X by back substitution (M_KK^T is upper triangular); row r's
+  // final scaling by 1/M_KK[r][r] is applied in the next phase.
   for (int r = nb - 1; r >= 0; --r) {
-    if (tid < TB) X[r * PLD + tid] /= S[r * PLD + r];
-    __syncthreads();
-    for (int e = tid; e < r * TB; e += blockDim.x) {
-      const int r2 = e >> 6, c = e & 63;
-      X[r2 * PLD + c] -= S[r * PLD + r2] * X[r * PLD + c];
+    const double iv = invd[r];
+    if (r + 1 < nb)
+      for (int c = tid; c < TB; c += blockDim.x) X[(r + 1) * PLD + c] *= invd[r + 1];
+    {  // rows r2 = i0 + 4u of column c, batched
+      const int c = tid & 63, i0 = tid >> 6;
+      const double xr = X[r * PLD + c] * iv;
+      double sv[16], xv[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int r2 = i0 + 4 * u;
+        const bool ok = r2 < r;
+        sv[u] = ok ? S[r * PLD + r2] : 0.0;
+        xv[u] = ok ? X[r2 * PLD + c] : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (i0 + 4 * u < r) X[(i0 + 4 * u) * PLD + c] = xv[u] - sv[u] * xr;
     }
     __syncthreads();
   }
+  for (int c = tid; c < TB; c += blockDim.x) X[c] *= invd[0];
+  __syncthreads();
   for (int e = tid; e < nb * TB; e += blockDim.x) {
     const int r = e >> 6, c = e & 63;
     M[(int64_t)(rb + r) * ldm + (int64_t)b * TB + c] = X[r * PLD + c];
   }
 }
 
-// A_IJ -= M_KI^T M_KJ for the lower block pairs J <= I < K (blockIdx.x enumerates them).
-__global__ void __launch_bounds__(128) trailing_kernel(double* __restrict__ M, int64_t ldm, int k,
-                                                       int K, const long long* info) {
-  if (*(volatile const long long*)info >= 0) return;
-  extern __shared__ double sm[];
-  double* Xs = sm;             // Xs[r][i] = M[rb + r][64 I + i]
-  double* Ys = sm + TB * SLD;  // Ys[r][j] = M[rb + r][64 J + j]
-  const int e = blockIdx.x;
-  int I = (int)((sqrt(8.0 * e + 1.0) - 1.0) * 0.5);
-  while ((I + 1) * (I + 2) / 2 <= e) ++I;
-  while (I * (I + 1) / 2 > e) --I;
-  const int J = e - I * (I + 1) / 2;
-  const int rb = K * TB, nb = min(TB, k - rb);
-  const int tid = threadIdx.x;
-
-  for (int x = tid; x < TB * TB / 2; x += blockDim.x) {
-    const int r = x >> 5, c2 = (x & 31) * 2;
-    double2 vx = make_double2(0.0, 0.0), vy = make_double2(0.0, 0.0);
-    if (r < nb) {
-      const double* row = M + (int64_t)(rb + r) * ldm;
-      vx = make_double2(row[(int64_t)I * TB + c2], row[(int64_t)I * TB + c2 + 1]);
-      vy = make_double2(row[(int64_t)J * TB + c2], row[(int64_t)J * TB + c2 + 1]);
+// Copies the nb x 64 block of M at (row0, col0) into shared memory [r][c] with
+// row stride KLD, zero rows beyond nb.  16-byte copies when every row start is
+// 16-byte aligned, else 8-byte copies.
+template <bool V16>
+__device__ __forceinline__ void load_rows(double* dst, const double* M, int64_t ldm, int row0,
+                                          int col0, int nb) {
+  if (V16) {
+    for (int x = threadIdx.x; x < TB * TB / 2; x += TR_THREADS) {
+      const int r = x >> 5, c2 = (x & 31) * 2;
+      const bool ok = r < nb;
+      const double* src = ok ? M + (int64_t)(row0 + r) * ldm + col0 + c2 : M;
+      cp_async16_zfill(dst + r * KLD + c2, src, ok);
     }
-    Xs[r * SLD + c2] = vx.x;
-    Xs[r * SLD + c2 + 1] = vx.y;
-    Ys[r * SLD + c2] = vy.x;
-    Ys[r * SLD + c2 + 1] = vy.y;
+  } else {
+    for (int x = threadIdx.x; x < TB * TB; x += TR_THREADS) {
+      const int r = x >> 6, c = x & 63;
+      const bool ok = r < nb;
+      const double* src = ok ? M + (int64_t)(row0 + r) * ldm + col0 + c : M;
+      cp_async8_zfill(dst + r * KLD + c, src, ok);
+    }
   }
-  __syncthreads();
-
-  double acc[4][4][2] = {};
-  mma_64x64x64(
-      acc, [&](int row, int kk) { return Xs[kk * SLD + row]; },
-      [&](int kk, int col) { return Ys[kk * SLD + col]; }, (nb + 3) & ~3);
-
-  const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
-  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t;
-      double* dst = M + (int64_t)(I * TB + r) * ldm + (int64_t)J * TB + c;
-      if (I != J || c <= r) dst[0] -= acc[i][j][0];
-      if (I != J || c + 1 <= r) dst[1] -= acc[i][j][1];
-    }
 }
 
-std::atomic<uint64_t> g_trailing_smem_set{0};
+struct TrailPlan {
+  int K, I0, ng;                 // block row, first group, number of groups
+  int per_cta;                   // blocks J per CTA
+  int start[MAX_TR_GROUPS + 1];  // first CTA of each group; group g updates A[I0+g][0..I0+g]
+};
+
+constexpr int TR_SMEM = 3 * TB * KLD * (int)sizeof(double);
+
+// A_IJ -= M_KI^T M_KJ.  Each CTA keeps M_KI in shared memory and streams the
+// M_KJ blocks of its range of J through a double buffer.
+template <bool V16>
+__global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restrict__ M,
+                                                                 int64_t ldm, int k,
+                                                                 const long long* info,
+                                                                 TrailPlan pl) {
+  if (*(volatile const long long*)info >= 0) return;
+  extern __shared__ __align__(16) double sm[];
+  double* Xs = sm;  // Xs[r][i] = M[rb + r][64 I + i]
+  double* const Y0 = sm + TB * KLD;
+  auto ybuf = [&](int bsel) { return Y0 + bsel * (TB * KLD); };
+  const int cta = blockIdx.x;
+  int g;
+  {
+    int lo = 0, hi = pl.ng;  // largest g with start[g] <= cta
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pl.start[mid] <= cta) lo = mid; else hi = mid;
+    }
+    g = lo;
+  }
+  const int I = pl.I0 + g;
+  const int first = (cta - pl.start[g]) * pl.per_cta;
+  const int last = min(first + pl.per_cta, I + 1);
+  if (first >= last) return;
+  const int rb = pl.K * TB, nb = min(TB, k - rb);
+
+  load_rows<V16>(Xs, M, ldm, rb, I * TB, nb);
+  load_rows<V16>(ybuf(0), M, ldm, rb, first * TB, nb);
+  cp_async_commit_group();
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, t4 = lane & 3;
+  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
+  for (int J = first; J < last; ++J) {
+    const int bsel = (J - first) & 1;
+    if (J + 1 < last) {
+      load_rows<V16>(ybuf(bsel ^ 1), M, ldm, rb, (J + 1) * TB, nb);
+      cp_async_commit_group();
+      cp_async_wait_group<1>();
+    } else {
+      cp_async_wait_group<0>();
+    }
+    __syncthreads();
+    const double* Ys = ybuf(bsel);
+    double acc[4][4][2] = {};
+    mma_64x64x64(
+        acc, [&](int row, int kk) { return Xs[kk * KLD + row]; },
+        [&](int kk, int col) { return Ys[kk * KLD + col]; }, (nb + 3) & ~3);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = wr + i * 8 + g8, c = wc + j * 8 + 2 * t4;
+        double* dst = M + (int64_t)(I * TB + r) * ldm + (int64_t)J * TB + c;
+        if (I != J || c <= r) dst[0] -= acc[i][j][0];
+        if (I != J || c + 1 <= r) dst[1] -= acc[i][j][1];
+      }
+    __syncthreads();
+  }
+}
+
+std::atomic<uint64_t> g_trailing_smem_set[2];
 std::atomic<uint64_t> g_panel_smem_set{0};
 
-}  // namespace
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
 
-size_t prepare_ws_bytes(int64_t) { return 256; }
-
-int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
-                   void* ws, cudaStream_t s) {
+int prepare_enqueue(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
+                    void* ws, cudaStream_t s, int sms) {
   long long* info = static_cast<long long*>(ws);
   const int T = (k + TB - 1) / TB;
-  const int cblocks = (int)std::min<int64_t>(((int64_t)k * k + 255) / 256, 148 * 16);
+  const int cblocks = (int)std::min<int64_t>(((int64_t)k * k + 255) / 256, (int64_t)sms * 16);
   if (h_dtype == GPTQ2D_F32)
     GPTQ2D_LAUNCH(KC_OTHER, s,
                   convert_lower_kernel<float><<<cblocks, 256, 0, s>>>(
@@ -168,18 +260,70 @@ int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
     GPTQ2D_LAUNCH(KC_OTHER, s,
                   convert_lower_kernel<double><<<cblocks, 256, 0, s>>>(
                       static_cast<const double*>(H), ldh, k, M, ldm, info));
-  const int tsmem = 2 * TB * SLD * (int)sizeof(double);
   const int psmem = 2 * TB * PLD * (int)sizeof(double);
-  if (ensure_smem(trailing_kernel, tsmem, g_trailing_smem_set) != cudaSuccess ||
+  const bool v16 = (ldm % 2 == 0) && ((reinterpret_cast<uintptr_t>(M) & 15u) == 0);
+  if (ensure_smem(trailing_kernel<true>, TR_SMEM, g_trailing_smem_set[0]) != cudaSuccess ||
+      ensure_smem(trailing_kernel<false>, TR_SMEM, g_trailing_smem_set[1]) != cudaSuccess ||
       ensure_smem(panel_kernel, psmem, g_panel_smem_set) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
+  const int target = 2 * sms;
   for (int K = T - 1; K >= 0; --K) {
     GPTQ2D_LAUNCH(KC_PREP_PANEL, s, panel_kernel<<<K + 1, 256, psmem, s>>>(M, ldm, k, K, info));
-    if (K > 0)
-      GPTQ2D_LAUNCH(KC_PREP_TRAILING, s,
-                    trailing_kernel<<<K * (K + 1) / 2, 128, tsmem, s>>>(M, ldm, k, K, info));
+    if (K == 0) continue;
+    const long long total = (long long)K * (K + 1) / 2;
+    const int per_cta = (int)std::max<long long>(1, (total + target - 1) / target);
+    for (int g0 = 0; g0 < K; g0 += MAX_TR_GROUPS) {
+      TrailPlan pl;
+      pl.K = K;
+      pl.I0 = g0;
+      pl.ng = std::min(K - g0, MAX_TR_GROUPS);
+      pl.per_cta = per_cta;
+      int ctas = 0;
+      for (int gi = 0; gi < pl.ng; ++gi) {
+        pl.start[gi] = ctas;
+        ctas += (g0 + gi + 1 + per_cta - 1) / per_cta;
+      }
+      pl.start[pl.ng] = ctas;
+      if (v16)
+        GPTQ2D_LAUNCH(KC_PREP_TRAILING, s,
+                      trailing_kernel<true><<<ctas, TR_THREADS, TR_SMEM, s>>>(M, ldm, k, info, pl));
+      else
+        GPTQ2D_LAUNCH(KC_PREP_TRAILING, s,
+                      trailing_kernel<false><<<ctas, TR_THREADS, TR_SMEM, s>>>(M, ldm, k, info, pl));
+    }
   }
   return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t prepare_ws_bytes(int64_t) { return 256; }
+
+int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
+                   void* ws, cudaStream_t s) {
+  return prepare_enqueue(H, h_dtype, k, ldh, M, ldm, ws, s, sm_count());
+}
+
+int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
+                        int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
+                        int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s) {
+  DevStreams* ds = nullptr;
+  int rc = dev_streams(&ds);
+  if (rc != GPTQ2D_OK) return rc;
+  std::lock_guard<std::mutex> lk(ds->mu);
+  if (cudaEventRecord(ds->fork, s) != cudaSuccess ||
+      cudaStreamWaitEvent(ds->hi, ds->fork, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(ds->lo, ds->fork, 0) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  if (m > 0) rc = prepare_enqueue(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ds->hi, ds->sms);
+  if (rc == GPTQ2D_OK && n > 0)
+    rc = prepare_enqueue(H_R, h_dtype, (int)n, ldhr, M_R, ldmr, ws_r, ds->lo, ds->sms);
+  const bool ok = cudaEventRecord(ds->join_hi, ds->hi) == cudaSuccess &&
+                  cudaEventRecord(ds->join_lo, ds->lo) == cudaSuccess &&
+                  cudaStreamWaitEvent(s, ds->join_hi, 0) == cudaSuccess &&
+                  cudaStreamWaitEvent(s, ds->join_lo, 0) == cudaSuccess;
+  if (rc != GPTQ2D_OK) return rc;
+  return ok ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
 }  // namespace gptq2d

@@ -12,30 +12,41 @@
 // so far.  y_ij depends only on the dominated quadrant, so all entries of one
 // anti-diagonal are independent.
 //
-// Data layout in HBM (workspace, row-major, padded to 64 x 64 tiles):
-//   P  (mp x np)  right feedback  P[i,j]  = sum_{done j'<=j} dW[i,j'] Rh[j,j']
-//   E  (mp x np)  down feedback   E[i,j]  = sum_{i' < tile row of i} Lh[i,i'] P[i',j]
+// Data layout in HBM (workspace, row-major, padded to whole 64 x 64 tiles):
+//   Lh (mp x mp), Rh (np x np)  normalised factors, strictly lower (diagonal
+//                               stored as 0), zero padding
+//   P  (mp x np)  right feedback  P[i,j] = sum_{done j'<=j} dW[i,j'] Rh[j,j']
+//   E  (mp x np)  down feedback   E[i,j] = sum_{i' in tile rows <= I-2} Lh[i,i'] P[i',j]
 //   Dl (mp x np)  errors dW of finished tiles
-// Schedule: 64 x 64 tiles, one tile wavefront (tile row + tile column = D) at a time:
-//   sweep_kernel      one CTA per tile of the wavefront; the tile's 127 local
-//                     anti-diagonals run in shared memory with the rank-one,
-//                     separable updates applied as a row push (along Rh) and
-//                     a column push (along Lh)
-//   propagate_kernel  the band products that carry a finished tile's errors to
-//                     the tiles right of it (P += dW Rh^T) and its final P to
-//                     the tiles below it (E += Lh P); 64x64x64 FP64 tensor-core
-//                     (DMMA) tiles
-// Exactness: every contribution to a tile comes from tiles on earlier
-// wavefronts (through P and E) or from the tile itself (through the sweep).
+//
+// Schedule: 64 x 64 tiles, one tile wavefront D (tile row + tile column = D)
+// at a time, on two internal streams forked from the caller's stream:
+//   high priority  sweep_kernel(D): one CTA per tile.  It first pulls the
+//                  contributions of its left and upper neighbours (wavefront
+//                  D-1) with FP64 tensor-core products, then runs the tile's
+//                  127 local anti-diagonals in shared memory, applying the
+//                  rank-one separable update of every rounded entry as a row
+//                  push (along Rh) and a column push (along Lh).
+//   low priority   far_kernel(D): the band products that carry the tiles of
+//                  wavefront D to tiles two or more tiles away (to the right:
+//                  P += dW Rh^T; below: E += Lh P), 64x64x64 DMMA tiles with
+//                  double-buffered cp.async operand streams.
+// sweep_kernel(D) waits for far_kernel(D-2) only, so far_kernel(D) runs under
+// sweep_kernel(D+1).  Exactness: every contribution to a tile comes from
+// earlier wavefronts (far: through P and E, near: pulled by the sweep) or from
+// the tile itself (the sweep).
+#include <mutex>
+
 #include "common.cuh"
 
 namespace gptq2d {
 
 namespace {
 
-constexpr int SLD = TB + 4;    // 68 doubles: shared tiles accessed along rows and anti-diagonals
-constexpr int KLD = TB + 8;    // 72 doubles: [k][n] operand tiles of the band products
+constexpr int SLD = TB + 4;  // 68 doubles: [row][k] tiles (conflict-free DMMA fragments)
+constexpr int KLD = TB + 8;  // 72 doubles: [k][col] tiles
 constexpr int SWEEP_THREADS = 256;  // 4 threads per tile row
+constexpr int FAR_THREADS = 128;
 
 struct QArgs {
   const void* W;
@@ -50,127 +61,318 @@ struct QArgs {
   int clamp;
   int8_t* Q;
   int64_t ldq;
-  double* P;
-  double* E;
-  double* Dl;
-  int64_t lds;  // leading dimension of P, E, Dl (np)
-  const double* dL;     // M_L[i,i]   (mp, zero-padded)
-  const double* dR;     // M_R[j,j]   (np)
-  const double* invdL;  // 1/M_L[i,i] (mp)
-  const double* invdR;  // 1/M_R[j,j] (np)
-  TileStat* part;       // Tm x Tn
+  double* Lh;     // mp x mp
+  double* Rh;     // np x np
+  double* P;      // mp x np
+  double* E;      // mp x np
+  double* Dl;     // mp x np
+  int64_t mp, np;
+  double* dL;     // M_L[i,i] (mp)
+  double* dR;     // M_R[j,j] (np)
+  TileStat* part; // Tm x Tn
   int Tm, Tn;
 };
 
-template <typename TW>
-__device__ __forceinline__ double load_w(const QArgs& a, int64_t idx) {
-  return to_f64(static_cast<const TW*>(a.W)[idx]);
+// ---------------------------------------------------------------------------
+// small PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint64_t pol) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
+               "l"(pol));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+__device__ __forceinline__ double2 ld_hint(const double* p, uint64_t pol) {
+  double2 v;
+  asm volatile("ld.global.L2::cache_hint.v2.f64 {%0,%1}, [%2], %3;\n"
+               : "=d"(v.x), "=d"(v.y)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_hint(double* p, double2 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v2.f64 [%0], {%1,%2}, %3;\n" ::"l"(p), "d"(v.x), "d"(v.y),
+               "l"(pol));
 }
 
-// Diagonals of both factors and their reciprocals, zero beyond m / n.
-__global__ void diag_kernel(QArgs a, int mp, int np) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < mp + np; i += gridDim.x * blockDim.x) {
-    if (i < mp) {
-      const double d = (i < a.m) ? a.ML[(int64_t)i * a.ldl + i] : 0.0;
-      const_cast<double*>(a.dL)[i] = d;
-      const_cast<double*>(a.invdL)[i] = (i < a.m) ? 1.0 / d : 0.0;
+// Copies a 64x64 fp64 tile (row stride `ld` elements, 16-byte aligned rows) into
+// shared memory with row stride `sld`, 16 bytes per cp.async.
+template <int NT>
+__device__ __forceinline__ void tile_cp_async(double* dst, int sld, const double* src, int64_t ld,
+                                              uint64_t pol) {
+  for (int x = threadIdx.x; x < TB * TB / 2; x += NT) {
+    const int r = x >> 5, c2 = (x & 31) * 2;
+    cp_async16(dst + r * sld + c2, src + (int64_t)r * ld + c2, pol);
+  }
+}
+
+// 64x64x64 product on 8 warps: warp w owns rows (w>>1)*16..+16, cols (w&1)*32..+32.
+template <typename FA, typename FB>
+__device__ __forceinline__ void mma8w(double (&acc)[2][4][2], FA fa, FB fb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wr = (warp >> 1) * 16, wc = (warp & 1) * 32;
+#pragma unroll 4
+  for (int kk = 0; kk < TB; kk += 4) {
+    double av[2], bv[4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) av[i] = fa(wr + i * 8 + g, kk + t);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bv[j] = fb(kk + t, wc + j * 8 + g);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// set-up: normalised, tile-padded factors and their diagonals
+// ---------------------------------------------------------------------------
+__global__ void normalize_kernel(QArgs a) {
+  const int64_t nl = a.mp * a.mp, nr = a.np * a.np;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nl + nr;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    if (e < nl) {
+      const int i = (int)(e / a.mp), k = (int)(e % a.mp);
+      double v = 0.0;
+      if (i < a.m && k < i) v = a.ML[(int64_t)i * a.ldl + k] / a.ML[(int64_t)i * a.ldl + i];
+      a.Lh[e] = v;
+      if (k == 0) a.dL[i] = (i < a.m) ? a.ML[(int64_t)i * a.ldl + i] : 0.0;
     } else {
-      const int j = i - mp;
-      const double d = (j < a.n) ? a.MR[(int64_t)j * a.ldr + j] : 0.0;
-      const_cast<double*>(a.dR)[j] = d;
-      const_cast<double*>(a.invdR)[j] = (j < a.n) ? 1.0 / d : 0.0;
+      const int64_t f = e - nl;
+      const int j = (int)(f / a.np), k = (int)(f % a.np);
+      double v = 0.0;
+      if (j < a.n && k < j) v = a.MR[(int64_t)j * a.ldr + k] / a.MR[(int64_t)j * a.ldr + j];
+      a.Rh[f] = v;
+      if (k == 0) a.dR[j] = (j < a.n) ? a.MR[(int64_t)j * a.ldr + j] : 0.0;
     }
   }
 }
 
+// ---------------------------------------------------------------------------
+// the tile sweep
+// ---------------------------------------------------------------------------
+template <typename TW>
+struct WStore { using T = float; };          // f32 and bf16 are exact in f32
+template <>
+struct WStore<__nv_bfloat16> { using T = __nv_bfloat16; };
+template <>
+struct WStore<double> { using T = double; };
+
+template <typename TW>
+constexpr int sweep_smem_bytes() {
+  return 3 * TB * SLD * (int)sizeof(double) + TB * TB * (int)sizeof(typename WStore<TW>::T);
+}
+
 // One CTA per tile (I, J) with I = I0 + blockIdx.x, J = D - I.
 template <typename TW>
-__global__ void __launch_bounds__(SWEEP_THREADS) sweep_kernel(QArgs a, int D, int I0) {
-  extern __shared__ double sm[];
-  double* Ws = sm;                // W, overwritten by dW as entries are rounded
-  double* V = Ws + TB * SLD;      // W + E + in-tile column feedback
-  double* Pt = V + TB * SLD;      // P of the tile (left feedback + in-tile row feedback)
-  double* Lh = Pt + TB * SLD;     // Lh[a][a'] = M_L[r0+a][r0+a'] / M_L[r0+a][r0+a], a' < a
-  double* Rh = Lh + TB * SLD;     // Rh[c'][c] = M_R[c0+c'][c0+c] / M_R[c0+c'][c0+c'], c < c'
-  signed char* Qs = reinterpret_cast<signed char*>(Rh + TB * SLD);  // TB x TB
+__global__ void __launch_bounds__(SWEEP_THREADS, 2) sweep_kernel(QArgs a, int D, int I0) {
+  using WT = typename WStore<TW>::T;
+  extern __shared__ __align__(16) double sm[];
+  double* V = sm;               // W + E + pulled down feedback + in-tile column feedback
+  double* Ps = V + TB * SLD;    // P of the tile: far + pulled right feedback + in-tile row feedback
+  double* RT = Ps + TB * SLD;   // RT[c][c'] = Rh[c0+c'][c0+c] (c < c'), the row-push coefficients
+  WT* Ws = reinterpret_cast<WT*>(RT + TB * SLD);  // W of the tile
 
   const int I = I0 + blockIdx.x, J = D - I;
   const int r0 = I * TB, c0 = J * TB;
   const int rows = min(TB, a.m - r0), cols = min(TB, a.n - c0);
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
+  const int wr = (warp >> 1) * 16, wc = (warp & 1) * 32;
+  const int64_t ts = (int64_t)r0 * a.np + c0;  // tile origin in the workspace matrices
 
-  for (int e = tid; e < TB * TB; e += SWEEP_THREADS) {
-    const int r = e >> 6, c = e & 63;
-    const int64_t wi = (int64_t)(r0 + r) * a.lds + c0 + c;
-    const double w = (r < rows && c < cols) ? load_w<TW>(a, (int64_t)(r0 + r) * a.ldw + c0 + c) : 0.0;
-    Ws[r * SLD + c] = w;
-    V[r * SLD + c] = w + a.E[wi];
-    Pt[r * SLD + c] = a.P[wi];
-    Lh[r * SLD + c] =
-        (r < rows && c < r) ? a.ML[(int64_t)(r0 + r) * a.ldl + r0 + c] * a.invdL[r0 + r] : 0.0;
-    Rh[r * SLD + c] =
-        (r < cols && c < r) ? a.MR[(int64_t)(c0 + r) * a.ldr + c0 + c] * a.invdR[c0 + r] : 0.0;
+  // ---- right feedback: P[I,J] (far part) + dW[I,J-1] Rh[J, J-1]^T (near part) -> Ps
+  {
+    double acc[2][4][2] = {};
+    if (J > 0) {
+      const double* A = a.Dl + ts - TB;                           // [a][k]
+      const double* B = a.Rh + (int64_t)c0 * a.np + (c0 - TB);    // [c][k]
+      for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+        const int r = x >> 5, k2 = (x & 31) * 2;
+        *reinterpret_cast<double2*>(V + r * SLD + k2) =
+            *reinterpret_cast<const double2*>(A + (int64_t)r * a.np + k2);
+        *reinterpret_cast<double2*>(RT + r * SLD + k2) =
+            *reinterpret_cast<const double2*>(B + (int64_t)r * a.np + k2);
+      }
+      __syncthreads();
+      mma8w(acc, [&](int r, int k) { return V[r * SLD + k]; },
+            [&](int k, int c) { return RT[c * SLD + k]; });
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t4;
+        const double2 p = *reinterpret_cast<const double2*>(a.P + ts + (int64_t)r * a.np + c);
+        Ps[r * SLD + c] = p.x + acc[i][j][0];
+        Ps[r * SLD + c + 1] = p.y + acc[i][j][1];
+      }
+  }
+
+  // ---- down feedback: W + E[I,J] (far part) + Lh[I, I-1] P[I-1, J] (near part) -> V
+  {
+    double acc[2][4][2] = {};
+    if (I > 0) {
+      const double* A = a.Lh + (int64_t)r0 * a.mp + (r0 - TB);  // [a][k]
+      const double* B = a.P + ts - (int64_t)TB * a.np;          // [k][c], final P of tile (I-1, J)
+      for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+        const int r = x >> 5, k2 = (x & 31) * 2;
+        *reinterpret_cast<double2*>(RT + r * SLD + k2) =
+            *reinterpret_cast<const double2*>(A + (int64_t)r * a.mp + k2);
+        const double2 b = *reinterpret_cast<const double2*>(B + (int64_t)r * a.np + k2);
+        V[k2 * SLD + r] = b.x;  // transposed: V[c][k]
+        V[(k2 + 1) * SLD + r] = b.y;
+      }
+      __syncthreads();
+      mma8w(acc, [&](int r, int k) { return RT[r * SLD + k]; },
+            [&](int k, int c) { return V[c * SLD + k]; });
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t4;
+        const double2 e = *reinterpret_cast<const double2*>(a.E + ts + (int64_t)r * a.np + c);
+        double w0 = 0.0, w1 = 0.0;
+        if (r < rows) {
+          const TW* wrow = static_cast<const TW*>(a.W) + (int64_t)(r0 + r) * a.ldw + c0;
+          if (c < cols) w0 = to_f64(wrow[c]);
+          if (c + 1 < cols) w1 = to_f64(wrow[c + 1]);
+        }
+        V[r * SLD + c] = w0 + e.x + acc[i][j][0];
+        V[r * SLD + c + 1] = w1 + e.y + acc[i][j][1];
+        Ws[r * TB + c] = static_cast<WT>(w0);
+        Ws[r * TB + c + 1] = static_cast<WT>(w1);
+      }
+  }
+
+  // ---- row-push coefficients, transposed: RT[c][c'] = Rh[c0+c'][c0+c]
+  for (int x = tid; x < TB * TB; x += SWEEP_THREADS) {
+    const int cp = x >> 6, c = x & 63;
+    RT[c * SLD + cp] = a.Rh[(int64_t)(c0 + cp) * a.np + c0 + c];
+  }
+
+  // ---- diagonal of M_R over the tile's columns (for the loss identity)
+  __shared__ double dRs[TB];
+  if (tid < TB) dRs[tid] = a.dR[c0 + tid];
+
+  // ---- column-push coefficients of this thread's row, in registers
+  const int ra = tid >> 2, k4 = tid & 3;
+  double colL[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int aa = ra + 1 + k4 + 4 * u;
+    colL[u] = (aa < TB) ? a.Lh[(int64_t)(r0 + aa) * a.mp + r0 + ra] : 0.0;
   }
   __syncthreads();
 
-  const int ra = tid >> 2, k4 = tid & 3;
   const bool row_ok = ra < rows;
   const double s = row_ok ? (double)a.scales[r0 + ra] : 1.0;
+  const double inv_s = 1.0 / s;
   const double dl = a.dL[r0 + ra];
   const bool s_bad = row_ok && !(s > 0.0 && isfinite(s));
   double loss = 0.0;
   long long ncl = 0, nnt = 0, nnf = 0;
+  double* const Prow = Ps + ra * SLD;
+  int8_t* const Qrow = a.Q + (int64_t)(r0 + ra) * a.ldq + c0;
+  double* const Drow = a.Dl + ts + (int64_t)ra * a.np;
 
+  // Each step: the push targets are loaded before the entry's rounding (they do
+  // not depend on it), in two batches of 8 per thread, so that one shared-memory
+  // latency is paid per batch instead of one per element.
   const int steps = rows + cols - 1;
   for (int t = 0; t < steps; ++t) {
     const int c = t - ra;
     const bool act = row_ok && c >= 0 && c < cols;
-    double delta = 0.0, pf = 0.0, q = 0.0;
+    const int cs = act ? c : 0;
+    const double* rt = RT + cs * SLD;
+    double pv[8], rc[8], vv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
+      const bool okr = act && cc < cols, okc = act && aa < rows;
+      pv[u] = okr ? Prow[cc] : 0.0;
+      rc[u] = okr ? rt[cc] : 0.0;
+      vv[u] = okc ? V[aa * SLD + cs] : 0.0;
+    }
+    double delta = 0.0, pf = 0.0;
     if (act) {
-      const double w = Ws[ra * SLD + c];
-      const double p = Pt[ra * SLD + c];
+      const double p = Prow[c];
       const double y = V[ra * SLD + c] + p;
-      const double tq = y / s;
+      const double tq = y * inv_s;
       const double qr = rint(tq);
-      q = a.clamp ? fmin(fmax(qr, a.lo), a.hi) : qr;
-      delta = w - s * q;
+      const double q = a.clamp ? fmin(fmax(qr, a.lo), a.hi) : qr;
+      delta = to_f64(Ws[ra * TB + c]) - s * q;
       pf = p + delta;
       if (k4 == 0) {
-        const double res = (dl * a.dR[c0 + c]) * (y - s * q);
+        const double res = (dl * dRs[c]) * (y - s * q);
         loss += res * res;
         ncl += (q != qr);
         const double h = floor(tq) + 0.5;
         nnt += (fabs(tq - h) < 1e-6) && (h - 0.5 >= a.lo) && (h + 0.5 <= a.hi);
         nnf += !isfinite(y);
+        Qrow[c] = (int8_t)(int)q;
+        Drow[c] = delta;
       }
     }
     __syncwarp();
-    if (act) {
-      if (k4 == 0) {
-        Pt[ra * SLD + c] = pf;
-        Ws[ra * SLD + c] = delta;
-        Qs[ra * TB + c] = (signed char)(int)q;
+    if (act && k4 == 0) Prow[c] = pf;
+    // row push P[ra][c'] += dW Rh[c'][c] (c' > c); column push V[a'][c] += Lh[a'][ra] P_final
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
+      if (act && cc < cols) Prow[cc] = fma(delta, rc[u], pv[u]);
+      if (act && aa < rows) V[aa * SLD + cs] = fma(pf, colL[u], vv[u]);
+    }
+    if (act && (cs + 33 + k4 < cols || ra + 33 + k4 < rows)) {
+#pragma unroll
+      for (int u = 8; u < 16; ++u) {
+        const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
+        const bool okr = cc < cols, okc = aa < rows;
+        pv[u - 8] = okr ? Prow[cc] : 0.0;
+        rc[u - 8] = okr ? rt[cc] : 0.0;
+        vv[u - 8] = okc ? V[aa * SLD + cs] : 0.0;
       }
-      // row push: P[ra][c'] += dW * Rh[c'][c], c' > c
-      for (int cc = c + 1 + k4; cc < cols; cc += 4)
-        Pt[ra * SLD + cc] = fma(delta, Rh[cc * SLD + c], Pt[ra * SLD + cc]);
-      // column push: V[a'][c] += Lh[a'][ra] * P_final[ra][c], a' > ra
-      for (int aa = ra + 1 + k4; aa < rows; aa += 4)
-        V[aa * SLD + c] = fma(pf, Lh[aa * SLD + ra], V[aa * SLD + c]);
+#pragma unroll
+      for (int u = 8; u < 16; ++u) {
+        const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
+        if (cc < cols) Prow[cc] = fma(delta, rc[u - 8], pv[u - 8]);
+        if (aa < rows) V[aa * SLD + cs] = fma(pf, colL[u], vv[u - 8]);
+      }
     }
     __syncthreads();
   }
 
-  // write back Q, dW, final P of the tile
-  for (int e = tid; e < TB * TB; e += SWEEP_THREADS) {
-    const int r = e >> 6, c = e & 63;
-    const int64_t wi = (int64_t)(r0 + r) * a.lds + c0 + c;
-    a.Dl[wi] = Ws[r * SLD + c];
-    a.P[wi] = Pt[r * SLD + c];
-    if (r < rows && c < cols) a.Q[(int64_t)(r0 + r) * a.ldq + c0 + c] = Qs[r * TB + c];
+  // ---- final P of the tile; zeros into the padding of dW (the band products read whole tiles)
+  for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+    const int r = x >> 5, c2 = (x & 31) * 2;
+    *reinterpret_cast<double2*>(a.P + ts + (int64_t)r * a.np + c2) =
+        make_double2(Ps[r * SLD + c2], Ps[r * SLD + c2 + 1]);
+    if (r >= rows || c2 + 1 >= cols) {
+      double* d = a.Dl + ts + (int64_t)r * a.np + c2;
+      if (r >= rows || c2 >= cols) d[0] = 0.0;
+      d[1] = 0.0;
+    }
   }
 
-  // tile statistics (fixed reduction order: deterministic)
+  // ---- tile statistics (fixed reduction order: deterministic)
   if (k4 == 0 && c0 == 0 && s_bad) ++nnf;
   __shared__ double red_l[SWEEP_THREADS / 32];
   __shared__ long long red_c[SWEEP_THREADS / 32][3];
@@ -180,11 +382,11 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_kernel(QArgs a, int D, in
     nnt += __shfl_down_sync(0xffffffffu, nnt, o);
     nnf += __shfl_down_sync(0xffffffffu, nnf, o);
   }
-  if ((tid & 31) == 0) {
-    red_l[tid >> 5] = loss;
-    red_c[tid >> 5][0] = ncl;
-    red_c[tid >> 5][1] = nnt;
-    red_c[tid >> 5][2] = nnf;
+  if (lane == 0) {
+    red_l[warp] = loss;
+    red_c[warp][0] = ncl;
+    red_c[warp][1] = nnt;
+    red_c[warp][2] = nnf;
   }
   __syncthreads();
   if (tid == 0) {
@@ -199,73 +401,89 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_kernel(QArgs a, int D, in
   }
 }
 
-// Band products of the tiles of wavefront D.  blockIdx.y = tile, blockIdx.z:
-//   0: right,  P[I, J+1+x] += (dW[I,J] M_R[J+1+x, J]^T) * diag(1/M_R)   (columns scaled)
-//   1: down,   E[I+1+x, J] += diag(1/M_L) (M_L[I+1+x, I] P[I,J])        (rows scaled)
-__global__ void __launch_bounds__(128) propagate_kernel(QArgs a, int D, int I0) {
-  extern __shared__ double sm[];
-  double* As = sm;             // [64][SLD]: A[row][k]
-  double* Bs = sm + TB * SLD;  // right: [n][k] with SLD; down: [k][n] with KLD
-  const int I = I0 + blockIdx.y, J = D - I;
-  const int x = blockIdx.x;
-  const bool down = blockIdx.z == 1;
-  const int tid = threadIdx.x;
-  int R0, C0;  // output tile origin in the workspace
-  if (!down) {
-    const int Jp = J + 1 + x;
-    if (Jp >= a.Tn) return;
-    R0 = I * TB;
-    C0 = Jp * TB;
-    for (int e = tid; e < TB * TB; e += blockDim.x) {
-      const int r = e >> 6, c = e & 63;
-      As[r * SLD + c] = a.Dl[(int64_t)(I * TB + r) * a.lds + J * TB + c];
-      const int jr = Jp * TB + r, jc = J * TB + c;  // M_R[jr][jc], jr > jc always
-      Bs[r * SLD + c] = (jr < a.n && jc < a.n) ? a.MR[(int64_t)jr * a.ldr + jc] : 0.0;
+// ---------------------------------------------------------------------------
+// band products to tiles two or more tiles away
+// ---------------------------------------------------------------------------
+constexpr int MAX_GROUPS = 512;  // 2 groups per tile: 256 tiles per launch
+struct FarPlan {
+  int D, I0, nt;
+  int per_cta;               // tasks (64x64 output tiles) per CTA
+  int start[MAX_GROUPS + 1]; // first CTA of each group; group g < nt: right tasks of tile
+                             // I0+g, else down tasks of tile I0+g-nt
+};
+
+constexpr int FAR_SMEM = (TB * KLD + 2 * TB * SLD) * (int)sizeof(double);
+
+__global__ void __launch_bounds__(FAR_THREADS, 2) far_kernel(QArgs a, FarPlan pl) {
+  extern __shared__ __align__(16) double sm[];
+  double* Sh = sm;                       // shared operand of the CTA's tasks
+  double* const Bf0 = sm + TB * KLD;     // per-task operand, double-buffered
+  auto bufp = [&](int b) { return Bf0 + b * (TB * SLD); };
+  const int cta = blockIdx.x;
+  int g = 0;
+  {
+    int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= cta
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pl.start[mid] <= cta) lo = mid; else hi = mid;
     }
-  } else {
-    const int Ip = I + 1 + x;
-    if (Ip >= a.Tm) return;
-    R0 = Ip * TB;
-    C0 = J * TB;
-    for (int e = tid; e < TB * TB; e += blockDim.x) {
-      const int r = e >> 6, c = e & 63;
-      const int ir = Ip * TB + r, ic = I * TB + c;
-      As[r * SLD + c] = (ir < a.m && ic < a.m) ? a.ML[(int64_t)ir * a.ldl + ic] : 0.0;
-      Bs[r * KLD + c] = a.P[(int64_t)(I * TB + r) * a.lds + J * TB + c];
-    }
+    g = lo;
   }
-  __syncthreads();
+  const bool down = g >= pl.nt;
+  const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
+  const int count = down ? a.Tm - I - 2 : a.Tn - J - 2;
+  const int first = (cta - pl.start[g]) * pl.per_cta;
+  const int last = min(first + pl.per_cta, count);
+  if (first >= last) return;
 
-  double acc[4][4][2] = {};
+  const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+  const int64_t np = a.np;
+  // shared operand: right -> dW[I,J] as [a][k]; down -> P[I,J] as [k][c]
   if (!down)
-    mma_64x64x64(
-        acc, [&](int row, int kk) { return As[row * SLD + kk]; },
-        [&](int kk, int col) { return Bs[col * SLD + kk]; });
+    tile_cp_async<FAR_THREADS>(Sh, SLD, a.Dl + (int64_t)I * TB * np + J * TB, np, stream);
   else
-    mma_64x64x64(
-        acc, [&](int row, int kk) { return As[row * SLD + kk]; },
-        [&](int kk, int col) { return Bs[kk * KLD + col]; });
+    tile_cp_async<FAR_THREADS>(Sh, KLD, a.P + (int64_t)I * TB * np + J * TB, np, stream);
+  auto task_operand = [&](int x) -> const double* {
+    // right: Rh[(J+2+x) block rows][J block cols] as [c][k]; down: Lh[(I+2+x) rows][I cols] as [a][k]
+    return down ? a.Lh + (int64_t)(I + 2 + x) * TB * a.mp + I * TB
+                : a.Rh + (int64_t)(J + 2 + x) * TB * np + J * TB;
+  };
+  const int64_t opld = down ? a.mp : np;
+  tile_cp_async<FAR_THREADS>(bufp(0), SLD, task_operand(first), opld, keep);
+  cp_async_commit();
 
-  double* C = down ? a.E : a.P;
-  const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = R0 + wr + i * 8 + g, c = C0 + wc + j * 8 + 2 * t;
-      double2* dst = reinterpret_cast<double2*>(C + (int64_t)r * a.lds + c);
-      double2 v = *dst;
-      if (down) {
-        const double sc = a.invdL[r];
-        v.x = fma(sc, acc[i][j][0], v.x);
-        v.y = fma(sc, acc[i][j][1], v.y);
-      } else {
-        v.x = fma(a.invdR[c], acc[i][j][0], v.x);
-        v.y = fma(a.invdR[c + 1], acc[i][j][1], v.y);
-      }
-      *dst = v;
+  for (int x = first; x < last; ++x) {
+    const int buf = (x - first) & 1;
+    if (x + 1 < last) {
+      tile_cp_async<FAR_THREADS>(bufp(buf ^ 1), SLD, task_operand(x + 1), opld, keep);
+      cp_async_commit();
     }
+    double* C = down ? a.E + (int64_t)(I + 2 + x) * TB * np + J * TB
+                     : a.P + (int64_t)I * TB * np + (J + 2 + x) * TB;
+    if (x + 1 < last) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncthreads();
+    double acc[4][4][2] = {};
+    const double* B = bufp(buf);
+    if (!down)
+      mma_64x64x64(acc, [&](int r, int k) { return Sh[r * SLD + k]; },
+                   [&](int k, int c) { return B[c * SLD + k]; });
+    else
+      mma_64x64x64(acc, [&](int r, int k) { return B[r * SLD + k]; },
+                   [&](int k, int c) { return Sh[k * KLD + c]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        double* cp = C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4;
+        double2 v = ld_hint(cp, stream);
+        v.x += acc[i][j][0];
+        v.y += acc[i][j][1];
+        st_hint(cp, v, stream);
+      }
+    __syncthreads();
+  }
 }
 
 // Sums the per-tile statistics in a fixed order into the caller's gptq2d_stats.
@@ -312,10 +530,13 @@ __global__ void zero_stats_kernel(gptq2d_stats* out) {
   *out = st;
 }
 
+// ---------------------------------------------------------------------------
+// workspace and streams
+// ---------------------------------------------------------------------------
 struct WsLayout {
   int64_t mp, np;
   int Tm, Tn;
-  size_t off_P, off_E, off_D, off_dL, off_dR, off_idL, off_idR, off_part, total;
+  size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_part, total;
 };
 
 WsLayout layout(int64_t m, int64_t n) {
@@ -326,42 +547,93 @@ WsLayout layout(int64_t m, int64_t n) {
   L.Tn = (int)(L.np / TB);
   const size_t mat = align256((size_t)L.mp * L.np * sizeof(double));
   size_t o = 0;
+  L.off_Lh = o; o += align256((size_t)L.mp * L.mp * sizeof(double));
+  L.off_Rh = o; o += align256((size_t)L.np * L.np * sizeof(double));
   L.off_P = o; o += mat;
   L.off_E = o; o += mat;
   L.off_D = o; o += mat;
   L.off_dL = o; o += align256(L.mp * sizeof(double));
   L.off_dR = o; o += align256(L.np * sizeof(double));
-  L.off_idL = o; o += align256(L.mp * sizeof(double));
-  L.off_idR = o; o += align256(L.np * sizeof(double));
   L.off_part = o; o += align256((size_t)L.Tm * L.Tn * sizeof(TileStat));
   L.total = o;
   return L;
 }
 
 std::atomic<uint64_t> g_sweep_smem_set[3];
-std::atomic<uint64_t> g_prop_smem_set{0};
-
-constexpr int SWEEP_SMEM = 5 * TB * SLD * (int)sizeof(double) + TB * TB;
-constexpr int PROP_SMEM = (TB * SLD + TB * KLD) * (int)sizeof(double);
+std::atomic<uint64_t> g_far_smem_set{0};
 
 template <typename TW>
 int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s, int wslot) {
-  if (ensure_smem(sweep_kernel<TW>, SWEEP_SMEM, g_sweep_smem_set[wslot]) != cudaSuccess ||
-      ensure_smem(propagate_kernel, PROP_SMEM, g_prop_smem_set) != cudaSuccess)
+  constexpr int SW_SMEM = sweep_smem_bytes<TW>();
+  if (ensure_smem(sweep_kernel<TW>, SW_SMEM, g_sweep_smem_set[wslot]) != cudaSuccess ||
+      ensure_smem(far_kernel, FAR_SMEM, g_far_smem_set) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
+  DevStreams* ds = nullptr;
+  int rc = dev_streams(&ds);
+  if (rc != GPTQ2D_OK) return rc;
+  std::lock_guard<std::mutex> lk(ds->mu);
+  cudaStream_t hi = ds->hi, lo = ds->lo;
+  bool ok = cudaEventRecord(ds->fork, s) == cudaSuccess &&
+            cudaStreamWaitEvent(hi, ds->fork, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(lo, ds->fork, 0) == cudaSuccess;
+  if (!ok) return GPTQ2D_ERR_CUDA;
+
+  // set-up on the high-priority stream: zero P and E, normalised factors
+  ok = cudaMemsetAsync(a.P, 0, (size_t)(L.off_D - L.off_P), hi) == cudaSuccess;
+  const int64_t nnorm = L.mp * L.mp + L.np * L.np;
+  const int nblk = (int)std::min<int64_t>((nnorm + 255) / 256, (int64_t)ds->sms * 8);
+  GPTQ2D_LAUNCH(KC_OTHER, hi, normalize_kernel<<<nblk, 256, 0, hi>>>(a));
+  ok = ok && cudaEventRecord(ds->setup, hi) == cudaSuccess &&
+       cudaStreamWaitEvent(lo, ds->setup, 0) == cudaSuccess;
+
   const int nd = a.Tm + a.Tn - 1;
-  const int gx = (a.Tm > a.Tn ? a.Tm : a.Tn) - 1;
-  for (int D = 0; D < nd; ++D) {
+  const int target_ctas = 2 * ds->sms;
+  bool far_recorded[RING] = {};
+  for (int D = 0; D < nd && ok; ++D) {
     const int I0 = D - (a.Tn - 1) > 0 ? D - (a.Tn - 1) : 0;
     const int I1 = D < a.Tm - 1 ? D : a.Tm - 1;
     const int nt = I1 - I0 + 1;
-    GPTQ2D_LAUNCH(KC_SWEEP, s, sweep_kernel<TW><<<nt, SWEEP_THREADS, SWEEP_SMEM, s>>>(a, D, I0));
-    if (D < nd - 1 && gx > 0)
-      GPTQ2D_LAUNCH(KC_PROPAGATE, s,
-                    propagate_kernel<<<dim3(gx, nt, 2), 128, PROP_SMEM, s>>>(a, D, I0));
+    if (D >= 2 && far_recorded[(D - 2) % RING])
+      ok = cudaStreamWaitEvent(hi, ds->far[(D - 2) % RING], 0) == cudaSuccess;
+    far_recorded[D % RING] = false;
+    GPTQ2D_LAUNCH(KC_SWEEP, hi,
+                  sweep_kernel<TW><<<nt, SWEEP_THREADS, SW_SMEM, hi>>>(a, D, I0));
+    // band products of wavefront D to tiles two or more tiles away
+    long long total = 0;
+    for (int i = 0; i < nt; ++i) {
+      const int I = I0 + i, J = D - I;
+      total += std::max(0, a.Tn - J - 2) + std::max(0, a.Tm - I - 2);
+    }
+    if (total == 0) continue;
+    const int per_cta = (int)std::max<long long>(1, (total + target_ctas - 1) / target_ctas);
+    ok = ok && cudaEventRecord(ds->sw[D % RING], hi) == cudaSuccess &&
+         cudaStreamWaitEvent(lo, ds->sw[D % RING], 0) == cudaSuccess;
+    for (int tb = 0; tb < nt && ok; tb += MAX_GROUPS / 2) {  // tiles per launch
+      FarPlan pl;
+      pl.D = D;
+      pl.I0 = I0 + tb;
+      pl.nt = std::min(nt - tb, MAX_GROUPS / 2);
+      pl.per_cta = per_cta;
+      int ctas = 0;
+      for (int gidx = 0; gidx < 2 * pl.nt; ++gidx) {
+        const int I = pl.I0 + (gidx < pl.nt ? gidx : gidx - pl.nt), J = D - I;
+        const int cnt = gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
+        pl.start[gidx] = ctas;
+        ctas += (cnt + per_cta - 1) / per_cta;
+      }
+      pl.start[2 * pl.nt] = ctas;
+      if (ctas > 0)
+        GPTQ2D_LAUNCH(KC_PROPAGATE, lo, far_kernel<<<ctas, FAR_THREADS, FAR_SMEM, lo>>>(a, pl));
+    }
+    ok = ok && cudaEventRecord(ds->far[D % RING], lo) == cudaSuccess;
+    far_recorded[D % RING] = true;
   }
-  GPTQ2D_LAUNCH(KC_OTHER, s, finalize_kernel<<<1, 256, 0, s>>>(a.part, a.Tm * a.Tn, stats));
-  return GPTQ2D_OK;
+  GPTQ2D_LAUNCH(KC_OTHER, hi, finalize_kernel<<<1, 256, 0, hi>>>(a.part, a.Tm * a.Tn, stats));
+  ok = ok && cudaEventRecord(ds->join_hi, hi) == cudaSuccess &&
+       cudaEventRecord(ds->join_lo, lo) == cudaSuccess &&
+       cudaStreamWaitEvent(s, ds->join_hi, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(s, ds->join_lo, 0) == cudaSuccess;
+  return ok ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
 }  // namespace
@@ -393,21 +665,18 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
   a.clamp = clamp;
   a.Q = Q;
   a.ldq = ldq;
+  a.Lh = reinterpret_cast<double*>(base + L.off_Lh);
+  a.Rh = reinterpret_cast<double*>(base + L.off_Rh);
   a.P = reinterpret_cast<double*>(base + L.off_P);
   a.E = reinterpret_cast<double*>(base + L.off_E);
   a.Dl = reinterpret_cast<double*>(base + L.off_D);
-  a.lds = L.np;
+  a.mp = L.mp;
+  a.np = L.np;
   a.dL = reinterpret_cast<double*>(base + L.off_dL);
   a.dR = reinterpret_cast<double*>(base + L.off_dR);
-  a.invdL = reinterpret_cast<double*>(base + L.off_idL);
-  a.invdR = reinterpret_cast<double*>(base + L.off_idR);
   a.part = reinterpret_cast<TileStat*>(base + L.off_part);
   a.Tm = L.Tm;
   a.Tn = L.Tn;
-
-  // P and E start at zero (E and P are contiguous).
-  if (cudaMemsetAsync(a.P, 0, L.off_D - L.off_P, s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
-  GPTQ2D_LAUNCH(KC_OTHER, s, diag_kernel<<<64, 256, 0, s>>>(a, (int)L.mp, (int)L.np));
   int rc;
   switch (w_dtype) {
     case GPTQ2D_F32: rc = launch_all<float>(a, L, stats, s, 0); break;

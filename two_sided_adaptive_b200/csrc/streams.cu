@@ -1,0 +1,36 @@
+// Per-device internal streams and events (created once per device, on first use).
+#include "common.cuh"
+
+namespace gptq2d {
+
+namespace {
+constexpr int kMaxDevices = 64;
+DevStreams g_dev[kMaxDevices];
+}  // namespace
+
+int dev_streams(DevStreams** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GPTQ2D_ERR_CUDA;
+  DevStreams& d = g_dev[dev];
+  std::lock_guard<std::mutex> lk(d.mu);
+  if (!d.ready) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+    if (cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&d.lo, cudaStreamNonBlocking, least) != cudaSuccess)
+      return GPTQ2D_ERR_CUDA;
+    cudaEvent_t* evs[] = {&d.fork, &d.setup, &d.join_hi, &d.join_lo};
+    for (auto* e : evs)
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+    for (int r = 0; r < RING; ++r)
+      if (cudaEventCreateWithFlags(&d.sw[r], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.far[r], cudaEventDisableTiming) != cudaSuccess)
+        return GPTQ2D_ERR_CUDA;
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    d.ready = true;
+  }
+  *out = &d;
+  return GPTQ2D_OK;
+}
+
+}  // namespace gptq2d
