@@ -42,104 +42,110 @@ __global__ void __launch_bounds__(256) convert_lower_kernel(const TH* __restrict
 }
 
 // One launch per block row K.  CTA K factors the diagonal block and writes it;
-// CTAs b < K factor the same block redundantly in shared memory (cheaper than a
-// separate launch) and solve their block M_Kb.  One barrier per pivot: the
-// scaling of a finished row is deferred to the next pivot's phase, when no
-// thread reads that row any more.
+// CTAs b < K factor the same block redundantly (cheaper than a separate launch)
+// and solve their block M_Kb = M_KK^{-T} A_Kb.
+//
+// Both phases keep their 64 x 64 block in registers: thread (i = tid/4, q =
+// tid%4) holds row i, columns q + 4u (u < 16).  The pivot and solve loops are
+// unrolled so that every register index is a compile-time constant.  Per pivot
+// p (last row first): the four threads of row p scale it by 1/sqrt(A[p][p]) and
+// publish it to a double-buffered shared row; after one barrier every row i < p
+// applies A[i][j] -= M[p][i] M[p][j] from broadcast reads.  The strict upper
+// part of the register block is never read (published rows are zero beyond p).
 __global__ void __launch_bounds__(256) panel_kernel(double* __restrict__ M, int64_t ldm, int k,
                                                     int K, long long* info) {
   if (*(volatile long long*)info >= 0) return;
-  extern __shared__ double psm[];
-  double* S = psm;             // diagonal block, factored in place
-  double* X = psm + TB * PLD;  // block M_Kb being solved
-  __shared__ double dd[TB], invd[TB];
-  const int tid = threadIdx.x;
+  __shared__ double S[TB * PLD];      // the factored diagonal block M_KK
+  __shared__ double rowb[2][TB];      // published pivot row / solved row
+  __shared__ double invd[TB];         // 1 / M_KK[p][p]
+  __shared__ int bad;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int i = tid >> 2, q = tid & 3;
   const int rb = K * TB, nb = min(TB, k - rb);
   const int b = blockIdx.x;
+  if (tid == 0) bad = -1;
 
-  for (int e = tid; e < TB * TB; e += blockDim.x) {
-    const int r = e >> 6, c = e & 63;
-    S[r * PLD + c] = (r < nb && c <= r) ? M[(int64_t)(rb + r) * ldm + rb + c] : 0.0;
-    if (b < K) X[r * PLD + c] = (r < nb) ? M[(int64_t)(rb + r) * ldm + (int64_t)b * TB + c] : 0.0;
+  double v[TB / 4];
+#pragma unroll
+  for (int u = 0; u < TB / 4; ++u) {
+    const int j = q + 4 * u;
+    v[u] = (i < nb && j <= i) ? M[(int64_t)(rb + i) * ldm + rb + j] : 0.0;
   }
   __syncthreads();
 
-  // Reverse factorization of the diagonal block: the last row first.
-  for (int p = nb - 1; p >= 0; --p) {
-    const double piv = S[p * PLD + p];
-    if (!(piv > 0.0) || !isfinite(piv)) {  // uniform: every thread read the same value
-      if (tid == 0) *info = rb + p;        // every CTA of this launch finds the same pivot
-      return;
-    }
-    const double dp = sqrt(piv);
-    const double inv = 1.0 / dp;
-    if (p + 1 < nb) {  // row p+1 is final: scale it
-      const double iv = invd[p + 1];
-      for (int j = tid; j <= p; j += blockDim.x) S[(p + 1) * PLD + j] *= iv;
-      if (tid == 0) S[(p + 1) * PLD + p + 1] = dd[p + 1];
-    }
-    {  // rows i = i0 + 4u of column j: one pivot-row value per thread, 16 batched updates
-      const int j = tid & 63, i0 = tid >> 6;
-      const double bj = S[p * PLD + j] * inv;
-      double ai[16], cij[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + 4 * u;
-        const bool ok = i < p && j <= i;
-        ai[u] = ok ? S[p * PLD + i] : 0.0;
-        cij[u] = ok ? S[i * PLD + j] : 0.0;
-      }
+  for (int p = TB - 1; p >= 0; --p) {
+    if (p < nb) {
+      // every lane takes part in the shuffle; row p's four threads use the value
+      const double piv = __shfl_sync(0xffffffffu, v[p >> 2], (lane & ~3) | (p & 3));
+      if (i == p) {
+        const bool ok = piv > 0.0 && isfinite(piv);
+        const double r = ok ? rsqrt(piv) : 0.0;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + 4 * u;
-        if (i < p && j <= i) S[i * PLD + j] = cij[u] - (ai[u] * inv) * bj;
+        for (int u = 0; u < TB / 4; ++u) {
+          const int j = q + 4 * u;
+          v[u] = (j <= p) ? v[u] * r : 0.0;
+          rowb[p & 1][j] = v[u];
+        }
+        if (q == 0) {
+          invd[p] = r;
+          if (!ok) bad = rb + p;
+        }
+      }
+      __syncthreads();
+      if (bad >= 0) {  // uniform: every thread reads the flag after the barrier
+        if (tid == 0) *info = bad;
+        return;
+      }
+      if (i < p) {
+        const double mi = rowb[p & 1][i];
+#pragma unroll
+        for (int u = 0; u < TB / 4; ++u) v[u] = fma(-mi, rowb[p & 1][q + 4 * u], v[u]);
       }
     }
-    if (tid == 0) {
-      dd[p] = dp;
-      invd[p] = inv;
-    }
-    __syncthreads();
   }
-  if (tid == 0) S[0] = dd[0];
+  // registers now hold M_KK (lower part); the diagonal is A[p][p] * (1/sqrt(A[p][p]))
+#pragma unroll
+  for (int u = 0; u < TB / 4; ++u) {
+    const int j = q + 4 * u;
+    S[i * PLD + j] = (i < nb && j <= i) ? v[u] : 0.0;
+  }
   __syncthreads();
-
   if (b == K) {
     for (int e = tid; e < nb * TB; e += blockDim.x) {
       const int r = e >> 6, c = e & 63;
-      if (c < nb) M[(int64_t)(rb + r) * ldm + rb + c] = (c <= r) ? S[r * PLD + c] : 0.0;
+      if (c < nb) M[(int64_t)(rb + r) * ldm + rb + c] = S[r * PLD + c];
     }
     return;
   }
 
-  // X <- M_KK^{-T} X by back substitution (M_KK^T is upper triangular); row r's
-  // final scaling by 1/M_KK[r][r] is applied in the next phase.
-  for (int r = nb - 1; r >= 0; --r) {
-    const double iv = invd[r];
-    if (r + 1 < nb)
-      for (int c = tid; c < TB; c += blockDim.x) X[(r + 1) * PLD + c] *= invd[r + 1];
-    {  // rows r2 = i0 + 4u of column c, batched
-      const int c = tid & 63, i0 = tid >> 6;
-      const double xr = X[r * PLD + c] * iv;
-      double sv[16], xv[16];
+  // X <- M_KK^{-T} X by back substitution (M_KK^T is upper triangular)
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int r2 = i0 + 4 * u;
-        const bool ok = r2 < r;
-        sv[u] = ok ? S[r * PLD + r2] : 0.0;
-        xv[u] = ok ? X[r2 * PLD + c] : 0.0;
+  for (int u = 0; u < TB / 4; ++u)
+    v[u] = (i < nb) ? M[(int64_t)(rb + i) * ldm + (int64_t)b * TB + q + 4 * u] : 0.0;
+#pragma unroll
+  for (int r = TB - 1; r >= 0; --r) {
+    if (r < nb) {
+      if (i == r) {
+        const double iv = invd[r];
+#pragma unroll
+        for (int u = 0; u < TB / 4; ++u) {
+          v[u] *= iv;
+          rowb[r & 1][q + 4 * u] = v[u];
+        }
       }
+      __syncthreads();
+      if (i < r) {
+        const double mr = S[r * PLD + i];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        if (i0 + 4 * u < r) X[(i0 + 4 * u) * PLD + c] = xv[u] - sv[u] * xr;
+        for (int u = 0; u < TB / 4; ++u) v[u] = fma(-mr, rowb[r & 1][q + 4 * u], v[u]);
+      }
     }
-    __syncthreads();
   }
-  for (int c = tid; c < TB; c += blockDim.x) X[c] *= invd[0];
-  __syncthreads();
-  for (int e = tid; e < nb * TB; e += blockDim.x) {
-    const int r = e >> 6, c = e & 63;
-    M[(int64_t)(rb + r) * ldm + (int64_t)b * TB + c] = X[r * PLD + c];
+  if (i < nb) {
+#pragma unroll
+    for (int u = 0; u < TB / 4; ++u)
+      M[(int64_t)(rb + i) * ldm + (int64_t)b * TB + q + 4 * u] = v[u];
   }
 }
 
@@ -260,7 +266,7 @@ int prepare_enqueue(const void* H, int h_dtype, int k, int64_t ldh, double* M, i
     GPTQ2D_LAUNCH(KC_OTHER, s,
                   convert_lower_kernel<double><<<cblocks, 256, 0, s>>>(
                       static_cast<const double*>(H), ldh, k, M, ldm, info));
-  const int psmem = 2 * TB * PLD * (int)sizeof(double);
+  const int psmem = 0;
   const bool v16 = (ldm % 2 == 0) && ((reinterpret_cast<uintptr_t>(M) & 15u) == 0);
   if (ensure_smem(trailing_kernel<true>, TR_SMEM, g_trailing_smem_set[0]) != cudaSuccess ||
       ensure_smem(trailing_kernel<false>, TR_SMEM, g_trailing_smem_set[1]) != cudaSuccess ||

@@ -45,7 +45,7 @@ namespace {
 
 constexpr int SLD = TB + 4;  // 68 doubles: [row][k] tiles (conflict-free DMMA fragments)
 constexpr int KLD = TB + 8;  // 72 doubles: [k][col] tiles
-constexpr int SWEEP_THREADS = 256;  // 4 threads per tile row
+constexpr int SWEEP_THREADS = 512;
 constexpr int FAR_THREADS = 128;
 
 struct QArgs {
@@ -139,6 +139,26 @@ __device__ __forceinline__ void mma8w(double (&acc)[2][4][2], FA fa, FB fb) {
   }
 }
 
+// 64x64x64 product on 16 warps: warp w owns rows (w>>2)*16..+16, cols (w&3)*16..+16.
+template <typename FA, typename FB>
+__device__ __forceinline__ void mma16w(double (&acc)[2][2][2], FA fa, FB fb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wr = (warp >> 2) * 16, wc = (warp & 3) * 16;
+#pragma unroll 4
+  for (int kk = 0; kk < TB; kk += 4) {
+    double av[2], bv[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) av[i] = fa(wr + i * 8 + g, kk + t);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) bv[j] = fb(kk + t, wc + j * 8 + g);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // set-up: normalised, tile-padded factors and their diagonals
 // ---------------------------------------------------------------------------
@@ -173,207 +193,253 @@ struct WStore<__nv_bfloat16> { using T = __nv_bfloat16; };
 template <>
 struct WStore<double> { using T = double; };
 
+// Shared memory of the sweep: six 64 x SLD fp64 tiles: P, V, W-then-dW, the
+// diagonal blocks of Rh and Lh, and t = y / s of every rounded entry.
 template <typename TW>
 constexpr int sweep_smem_bytes() {
-  return 3 * TB * SLD * (int)sizeof(double) + TB * TB * (int)sizeof(typename WStore<TW>::T);
+  return 6 * TB * SLD * (int)sizeof(double);
 }
 
+constexpr int SUB = 8;             // sub-tile edge
+constexpr int NSUB = TB / SUB;     // sub-tiles per tile edge
+
 // One CTA per tile (I, J) with I = I0 + blockIdx.x, J = D - I.
+//
+// The tile is swept as 8 x 8 sub-tiles, one sub-tile wavefront (p + q = w) at a
+// time.  A sub-tile's 15 local anti-diagonals run in one warp, warp-
+// synchronously: lane (a = lane/4, cq = lane%4) holds row a, columns cq and
+// cq + 4 of P (right feedback), V (down feedback) and W / dW in registers; the
+// rank-one updates of each rounded entry inside the sub-tile go through warp
+// shuffles (dW along its row, P_final down its column).  After each sub-tile
+// wavefront, every finished sub-tile (p, q) pushes its errors to the sub-tiles
+// right of it (P[p][q'] += dW[p][q] Rh[q'][q]^T) and its final P below it
+// (V[p'][q] += Lh[p'][p] P[p][q]) as 8x8x8 FP64 tensor-core products, one warp
+// per target sub-tile.
 template <typename TW>
-__global__ void __launch_bounds__(SWEEP_THREADS, 2) sweep_kernel(QArgs a, int D, int I0) {
-  using WT = typename WStore<TW>::T;
+__global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D, int I0) {
   extern __shared__ __align__(16) double sm[];
-  double* V = sm;               // W + E + pulled down feedback + in-tile column feedback
-  double* Ps = V + TB * SLD;    // P of the tile: far + pulled right feedback + in-tile row feedback
-  double* RT = Ps + TB * SLD;   // RT[c][c'] = Rh[c0+c'][c0+c] (c < c'), the row-push coefficients
-  WT* Ws = reinterpret_cast<WT*>(RT + TB * SLD);  // W of the tile
+  double* Pt = sm;                 // P of the tile
+  double* Vt = Pt + TB * SLD;      // V of the tile
+  double* Dt = Vt + TB * SLD;      // W, overwritten by dW entry by entry
+  double* Rt = Dt + TB * SLD;      // Rt[c'][c] = Rh[c0+c'][c0+c] (strictly lower)
+  double* Lt = Rt + TB * SLD;      // Lt[a'][a] = Lh[r0+a'][r0+a]
+  double* Tq = Lt + TB * SLD;      // t = y / s of each rounded entry (Q and statistics come from it)
 
   const int I = I0 + blockIdx.x, J = D - I;
   const int r0 = I * TB, c0 = J * TB;
   const int rows = min(TB, a.m - r0), cols = min(TB, a.n - c0);
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
-  const int wr = (warp >> 1) * 16, wc = (warp & 1) * 32;
-  const int64_t ts = (int64_t)r0 * a.np + c0;  // tile origin in the workspace matrices
+  const int wr = (warp >> 2) * 16, wc = (warp & 3) * 16;
+  const int64_t np = a.np;
+  const int64_t ts = (int64_t)r0 * np + c0;  // tile origin in the workspace matrices
 
-  // ---- right feedback: P[I,J] (far part) + dW[I,J-1] Rh[J, J-1]^T (near part) -> Ps
+  // ---- right feedback: P (far part, in HBM) + dW[I,J-1] Rh[J,J-1]^T (pulled); staged in Rt/Lt
   {
-    double acc[2][4][2] = {};
+    double acc[2][2][2] = {};
     if (J > 0) {
-      const double* A = a.Dl + ts - TB;                           // [a][k]
-      const double* B = a.Rh + (int64_t)c0 * a.np + (c0 - TB);    // [c][k]
+      const double* A = a.Dl + ts - TB;                       // [a][k]
+      const double* B = a.Rh + (int64_t)c0 * np + (c0 - TB);  // [c][k]
       for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
         const int r = x >> 5, k2 = (x & 31) * 2;
-        *reinterpret_cast<double2*>(V + r * SLD + k2) =
-            *reinterpret_cast<const double2*>(A + (int64_t)r * a.np + k2);
-        *reinterpret_cast<double2*>(RT + r * SLD + k2) =
-            *reinterpret_cast<const double2*>(B + (int64_t)r * a.np + k2);
+        *reinterpret_cast<double2*>(Rt + r * SLD + k2) =
+            *reinterpret_cast<const double2*>(A + (int64_t)r * np + k2);
+        *reinterpret_cast<double2*>(Lt + r * SLD + k2) =
+            *reinterpret_cast<const double2*>(B + (int64_t)r * np + k2);
       }
       __syncthreads();
-      mma8w(acc, [&](int r, int k) { return V[r * SLD + k]; },
-            [&](int k, int c) { return RT[c * SLD + k]; });
-      __syncthreads();
+      mma16w(acc, [&](int r, int kk) { return Rt[r * SLD + kk]; },
+             [&](int kk, int c) { return Lt[c * SLD + kk]; });
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t4;
-        const double2 p = *reinterpret_cast<const double2*>(a.P + ts + (int64_t)r * a.np + c);
-        Ps[r * SLD + c] = p.x + acc[i][j][0];
-        Ps[r * SLD + c + 1] = p.y + acc[i][j][1];
+        const double2 p = *reinterpret_cast<const double2*>(a.P + ts + (int64_t)r * np + c);
+        Pt[r * SLD + c] = p.x + acc[i][j][0];
+        Pt[r * SLD + c + 1] = p.y + acc[i][j][1];
       }
+    __syncthreads();
   }
-
-  // ---- down feedback: W + E[I,J] (far part) + Lh[I, I-1] P[I-1, J] (near part) -> V
+  // ---- down feedback: V = W + E (far part) + Lh[I,I-1] P_final[I-1,J] (pulled); W -> Dt
   {
-    double acc[2][4][2] = {};
+    double acc[2][2][2] = {};
     if (I > 0) {
       const double* A = a.Lh + (int64_t)r0 * a.mp + (r0 - TB);  // [a][k]
-      const double* B = a.P + ts - (int64_t)TB * a.np;          // [k][c], final P of tile (I-1, J)
+      const double* B = a.P + ts - (int64_t)TB * np;            // [k][c]: final P of tile (I-1, J)
       for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
         const int r = x >> 5, k2 = (x & 31) * 2;
-        *reinterpret_cast<double2*>(RT + r * SLD + k2) =
+        *reinterpret_cast<double2*>(Rt + r * SLD + k2) =
             *reinterpret_cast<const double2*>(A + (int64_t)r * a.mp + k2);
-        const double2 b = *reinterpret_cast<const double2*>(B + (int64_t)r * a.np + k2);
-        V[k2 * SLD + r] = b.x;  // transposed: V[c][k]
-        V[(k2 + 1) * SLD + r] = b.y;
+        const double2 b = *reinterpret_cast<const double2*>(B + (int64_t)r * np + k2);
+        Lt[k2 * SLD + r] = b.x;  // transposed: [c][k]
+        Lt[(k2 + 1) * SLD + r] = b.y;
       }
       __syncthreads();
-      mma8w(acc, [&](int r, int k) { return RT[r * SLD + k]; },
-            [&](int k, int c) { return V[c * SLD + k]; });
-      __syncthreads();
+      mma16w(acc, [&](int r, int kk) { return Rt[r * SLD + kk]; },
+             [&](int kk, int c) { return Lt[c * SLD + kk]; });
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t4;
-        const double2 e = *reinterpret_cast<const double2*>(a.E + ts + (int64_t)r * a.np + c);
+        const double2 e = *reinterpret_cast<const double2*>(a.E + ts + (int64_t)r * np + c);
         double w0 = 0.0, w1 = 0.0;
         if (r < rows) {
           const TW* wrow = static_cast<const TW*>(a.W) + (int64_t)(r0 + r) * a.ldw + c0;
           if (c < cols) w0 = to_f64(wrow[c]);
           if (c + 1 < cols) w1 = to_f64(wrow[c + 1]);
         }
-        V[r * SLD + c] = w0 + e.x + acc[i][j][0];
-        V[r * SLD + c + 1] = w1 + e.y + acc[i][j][1];
-        Ws[r * TB + c] = static_cast<WT>(w0);
-        Ws[r * TB + c + 1] = static_cast<WT>(w1);
+        Vt[r * SLD + c] = w0 + e.x + acc[i][j][0];
+        Vt[r * SLD + c + 1] = w1 + e.y + acc[i][j][1];
+        Dt[r * SLD + c] = w0;
+        Dt[r * SLD + c + 1] = w1;
       }
+    __syncthreads();
   }
-
-  // ---- row-push coefficients, transposed: RT[c][c'] = Rh[c0+c'][c0+c]
-  for (int x = tid; x < TB * TB; x += SWEEP_THREADS) {
-    const int cp = x >> 6, c = x & 63;
-    RT[c * SLD + cp] = a.Rh[(int64_t)(c0 + cp) * a.np + c0 + c];
+  // ---- diagonal blocks of the normalised factors
+  for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+    const int r = x >> 5, k2 = (x & 31) * 2;
+    cp_async16_zfill(Rt + r * SLD + k2, a.Rh + (int64_t)(c0 + r) * np + c0 + k2, true);
+    cp_async16_zfill(Lt + r * SLD + k2, a.Lh + (int64_t)(r0 + r) * a.mp + r0 + k2, true);
   }
-
-  // ---- diagonal of M_R over the tile's columns (for the loss identity)
-  __shared__ double dRs[TB];
-  if (tid < TB) dRs[tid] = a.dR[c0 + tid];
-
-  // ---- column-push coefficients of this thread's row, in registers
-  const int ra = tid >> 2, k4 = tid & 3;
-  double colL[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int aa = ra + 1 + k4 + 4 * u;
-    colL[u] = (aa < TB) ? a.Lh[(int64_t)(r0 + aa) * a.mp + r0 + ra] : 0.0;
-  }
+  cp_async_commit_group();
+  cp_async_wait_group<0>();
   __syncthreads();
 
-  const bool row_ok = ra < rows;
-  const double s = row_ok ? (double)a.scales[r0 + ra] : 1.0;
-  const double inv_s = 1.0 / s;
-  const double dl = a.dL[r0 + ra];
-  const bool s_bad = row_ok && !(s > 0.0 && isfinite(s));
   double loss = 0.0;
   long long ncl = 0, nnt = 0, nnf = 0;
-  double* const Prow = Ps + ra * SLD;
-  int8_t* const Qrow = a.Q + (int64_t)(r0 + ra) * a.ldq + c0;
-  double* const Drow = a.Dl + ts + (int64_t)ra * a.np;
+  const int sa = lane >> 2, cq = lane & 3;  // row inside a sub-tile, column group (cq, cq + 4)
+  for (int w = 0; w < 2 * NSUB - 1; ++w) {
+    const int p0 = w - (NSUB - 1) > 0 ? w - (NSUB - 1) : 0;
+    const int p1 = w < NSUB - 1 ? w : NSUB - 1;
+    const int nsub = p1 - p0 + 1;
 
-  // Each step: the push targets are loaded before the entry's rounding (they do
-  // not depend on it), in two batches of 8 per thread, so that one shared-memory
-  // latency is paid per batch instead of one per element.
-  const int steps = rows + cols - 1;
-  for (int t = 0; t < steps; ++t) {
-    const int c = t - ra;
-    const bool act = row_ok && c >= 0 && c < cols;
-    const int cs = act ? c : 0;
-    const double* rt = RT + cs * SLD;
-    double pv[8], rc[8], vv[8];
+    // ---- sweep: warp i takes sub-tile (p0 + i, w - p0 - i)
+    if (warp < nsub) {
+      const int p = p0 + warp, q = w - p;
+      const int R0 = SUB * p, C0 = SUB * q;
+      if (R0 < rows && C0 < cols) {
+        const int ar = R0 + sa;
+        const bool rok = ar < rows;
+        const double s = rok ? (double)a.scales[r0 + ar] : 1.0;
+        const double inv_s = 1.0 / s;
+        double P[2], V[2], Wd[2];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
-      const bool okr = act && cc < cols, okc = act && aa < rows;
-      pv[u] = okr ? Prow[cc] : 0.0;
-      rc[u] = okr ? rt[cc] : 0.0;
-      vv[u] = okc ? V[aa * SLD + cs] : 0.0;
-    }
-    double delta = 0.0, pf = 0.0;
-    if (act) {
-      const double p = Prow[c];
-      const double y = V[ra * SLD + c] + p;
-      const double tq = y * inv_s;
-      const double qr = rint(tq);
-      const double q = a.clamp ? fmin(fmax(qr, a.lo), a.hi) : qr;
-      delta = to_f64(Ws[ra * TB + c]) - s * q;
-      pf = p + delta;
-      if (k4 == 0) {
-        const double res = (dl * dRs[c]) * (y - s * q);
-        loss += res * res;
-        ncl += (q != qr);
-        const double h = floor(tq) + 0.5;
-        nnt += (fabs(tq - h) < 1e-6) && (h - 0.5 >= a.lo) && (h + 0.5 <= a.hi);
-        nnf += !isfinite(y);
-        Qrow[c] = (int8_t)(int)q;
-        Drow[c] = delta;
+        for (int sl = 0; sl < 2; ++sl) {
+          const int cc = C0 + cq + 4 * sl;
+          P[sl] = Pt[ar * SLD + cc];
+          V[sl] = Vt[ar * SLD + cc];
+          Wd[sl] = Dt[ar * SLD + cc];
+        }
+#pragma unroll
+        for (int t = 0; t < 2 * SUB - 1; ++t) {
+          // The entry of this lane on local anti-diagonal t, if any: at most one of
+          // its two slots lies on it.  One branch-free chain for all owner lanes.
+          const bool o1 = sa + cq + 4 == t;
+          const bool mine = (sa + cq == t || o1) && rok && C0 + cq + (o1 ? 4 : 0) < cols;
+          const double Px = o1 ? P[1] : P[0];
+          const double y = (o1 ? V[1] : V[0]) + Px;
+          const double tq = y * inv_s;
+          const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;  // rint, |t| <= 2^51
+          const double qv = qr < a.lo ? a.lo : (qr > a.hi ? a.hi : qr);  // lo/hi infinite: no clamp
+          const double delta = fma(-s, qv, o1 ? Wd[1] : Wd[0]);
+          const double pf = Px + delta;
+          const double dO = mine ? delta : 0.0, pO = mine ? pf : 0.0;
+          if (mine && !o1) { P[0] = pf; Wd[0] = delta; }
+          if (mine && o1) { P[1] = pf; Wd[1] = delta; }
+          // dW of this row's entry (column t - sa) and P_final of each column's entry (row t - col)
+          const int cl = t - sa;
+          const double dRow = __shfl_sync(0xffffffffu, dO, (sa << 2) | (cl & 3));
+          double pCol[2];
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl)
+            pCol[sl] = __shfl_sync(0xffffffffu, pO, (((t - cq - 4 * sl) & 7) << 2) | cq);
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            const int col = cq + 4 * sl, ae = t - col;
+            if (cl >= 0 && cl < col)  // row push: P[sa][col] += dW[sa][cl] Rh[col][cl]
+              P[sl] = fma(dRow, Rt[(C0 + col) * SLD + C0 + cl], P[sl]);
+            if (ae >= 0 && ae < sa)   // column push: V[sa][col] += Lh[sa][ae] P_final[ae][col]
+              V[sl] = fma(pCol[sl], Lt[(R0 + sa) * SLD + R0 + ae], V[sl]);
+          }
+          if (mine) Tq[ar * SLD + C0 + cq + (o1 ? 4 : 0)] = tq;  // off the chain
+        }
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const int cc = C0 + cq + 4 * sl;
+          Pt[ar * SLD + cc] = P[sl];
+          Dt[ar * SLD + cc] = Wd[sl];
+        }
       }
     }
-    __syncwarp();
-    if (act && k4 == 0) Prow[c] = pf;
-    // row push P[ra][c'] += dW Rh[c'][c] (c' > c); column push V[a'][c] += Lh[a'][ra] P_final
+    __syncthreads();
+    if (w == 2 * NSUB - 2) break;
+
+    // ---- block updates from the finished sub-tiles: 8x8x8 DMMA products, one warp per target
+    const int per = 2 * NSUB - 2 - w;  // targets per source: (7 - q) right + (7 - p) down
+    for (int x = warp; x < nsub * per; x += SWEEP_THREADS / 32) {
+      const int p = p0 + x / per, q = w - p, j = x % per;
+      const int R0 = SUB * p, C0 = SUB * q;
+      double c0v, c1v;
+      if (j < NSUB - 1 - q) {  // right: P[p][q'] += dW[p][q] Rh[q'][q]^T
+        const int Q0 = SUB * (q + 1 + j);
+        double* C = Pt + (R0 + g) * SLD + Q0 + 2 * t4;
+        c0v = C[0];
+        c1v = C[1];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
-      if (act && cc < cols) Prow[cc] = fma(delta, rc[u], pv[u]);
-      if (act && aa < rows) V[aa * SLD + cs] = fma(pf, colL[u], vv[u]);
-    }
-    if (act && (cs + 33 + k4 < cols || ra + 33 + k4 < rows)) {
+        for (int kk = 0; kk < SUB; kk += 4)
+          dmma_m8n8k4(c0v, c1v, Dt[(R0 + g) * SLD + C0 + kk + t4],
+                      Rt[(Q0 + g) * SLD + C0 + kk + t4]);
+        C[0] = c0v;
+        C[1] = c1v;
+      } else {                 // down: V[p'][q] += Lh[p'][p] P_final[p][q]
+        const int S0 = SUB * (p + 1 + j - (NSUB - 1 - q));
+        double* C = Vt + (S0 + g) * SLD + C0 + 2 * t4;
+        c0v = C[0];
+        c1v = C[1];
 #pragma unroll
-      for (int u = 8; u < 16; ++u) {
-        const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
-        const bool okr = cc < cols, okc = aa < rows;
-        pv[u - 8] = okr ? Prow[cc] : 0.0;
-        rc[u - 8] = okr ? rt[cc] : 0.0;
-        vv[u - 8] = okc ? V[aa * SLD + cs] : 0.0;
-      }
-#pragma unroll
-      for (int u = 8; u < 16; ++u) {
-        const int cc = cs + 1 + k4 + 4 * u, aa = ra + 1 + k4 + 4 * u;
-        if (cc < cols) Prow[cc] = fma(delta, rc[u - 8], pv[u - 8]);
-        if (aa < rows) V[aa * SLD + cs] = fma(pf, colL[u], vv[u - 8]);
+        for (int kk = 0; kk < SUB; kk += 4)
+          dmma_m8n8k4(c0v, c1v, Lt[(S0 + g) * SLD + R0 + kk + t4],
+                      Pt[(R0 + kk + t4) * SLD + C0 + g]);
+        C[0] = c0v;
+        C[1] = c1v;
       }
     }
     __syncthreads();
   }
 
-  // ---- final P of the tile; zeros into the padding of dW (the band products read whole tiles)
+  // ---- outputs: final P and dW of the tile (whole tile, padding included), Q
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
     const int r = x >> 5, c2 = (x & 31) * 2;
-    *reinterpret_cast<double2*>(a.P + ts + (int64_t)r * a.np + c2) =
-        make_double2(Ps[r * SLD + c2], Ps[r * SLD + c2 + 1]);
-    if (r >= rows || c2 + 1 >= cols) {
-      double* d = a.Dl + ts + (int64_t)r * a.np + c2;
-      if (r >= rows || c2 >= cols) d[0] = 0.0;
-      d[1] = 0.0;
+    *reinterpret_cast<double2*>(a.P + ts + (int64_t)r * np + c2) =
+        make_double2(Pt[r * SLD + c2], Pt[r * SLD + c2 + 1]);
+    *reinterpret_cast<double2*>(a.Dl + ts + (int64_t)r * np + c2) =
+        make_double2(Dt[r * SLD + c2], Dt[r * SLD + c2 + 1]);
+  }
+  // Q and the statistics of every rounded entry, from its t = y / s:
+  // loss term (M_L[i,i] M_R[j,j] s_i (t - q))^2 (the nearest-plane residual identity)
+  for (int x = tid; x < TB * TB; x += SWEEP_THREADS) {
+    const int r = x >> 6, c = x & 63;
+    if (r < rows && c < cols) {
+      const double sr = (double)a.scales[r0 + r];
+      const double tq = Tq[r * SLD + c];
+      const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;
+      const double qv = qr < a.lo ? a.lo : (qr > a.hi ? a.hi : qr);
+      a.Q[(int64_t)(r0 + r) * a.ldq + c0 + c] = (int8_t)(int)qv;
+      const double res = a.dL[r0 + r] * a.dR[c0 + c] * sr * (tq - qv);
+      loss += res * res;
+      ncl += (qv != qr);
+      const double qn = qr + (tq >= qr ? 1.0 : -1.0);
+      nnt += (0.5 - fabs(tq - qr) < 1e-6) && (fmin(qr, qn) >= a.lo) && (fmax(qr, qn) <= a.hi);
+      nnf += !isfinite(tq);
+      if (c == 0 && J == 0 && !(sr > 0.0 && isfinite(sr))) ++nnf;
     }
   }
 
   // ---- tile statistics (fixed reduction order: deterministic)
-  if (k4 == 0 && c0 == 0 && s_bad) ++nnf;
   __shared__ double red_l[SWEEP_THREADS / 32];
   __shared__ long long red_c[SWEEP_THREADS / 32][3];
   for (int o = 16; o > 0; o >>= 1) {
@@ -391,11 +457,11 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 2) sweep_kernel(QArgs a, int D,
   __syncthreads();
   if (tid == 0) {
     TileStat st{0.0, 0, 0, 0};
-    for (int w = 0; w < SWEEP_THREADS / 32; ++w) {
-      st.loss += red_l[w];
-      st.clamped += red_c[w][0];
-      st.near_tie += red_c[w][1];
-      st.nonfinite += red_c[w][2];
+    for (int w2 = 0; w2 < SWEEP_THREADS / 32; ++w2) {
+      st.loss += red_l[w2];
+      st.clamped += red_c[w2][0];
+      st.near_tie += red_c[w2][1];
+      st.nonfinite += red_c[w2][2];
     }
     a.part[(int64_t)I * a.Tn + J] = st;
   }
