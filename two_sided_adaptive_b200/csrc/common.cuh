@@ -84,8 +84,9 @@ __device__ __forceinline__ void dmma_m8n8k4(double& c0, double& c1, double a, do
 // owns the 32x32 quadrant (w>>1, w&1) as 4x4 fragments of 8x8.  `fa(row, k)`
 // and `fb(k, col)` return the operand elements from shared memory.
 template <typename FA, typename FB>
-__device__ __forceinline__ void mma_64x64x64(double (&acc)[4][4][2], FA fa, FB fb, int kmax = TB) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ void mma_64x64x64_w(double (&acc)[4][4][2], int warp, FA fa, FB fb,
+                                               int kmax = TB) {
+  const int lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
 #pragma unroll 4
@@ -100,6 +101,11 @@ __device__ __forceinline__ void mma_64x64x64(double (&acc)[4][4][2], FA fa, FB f
 #pragma unroll
       for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
   }
+}
+
+template <typename FA, typename FB>
+__device__ __forceinline__ void mma_64x64x64(double (&acc)[4][4][2], FA fa, FB fb, int kmax = TB) {
+  mma_64x64x64_w(acc, (int)(threadIdx.x >> 5), fa, fb, kmax);
 }
 
 // ---------------------------------------------------------------------------

@@ -46,7 +46,7 @@ namespace {
 constexpr int SLD = TB + 4;  // 68 doubles: [row][k] tiles (conflict-free DMMA fragments)
 constexpr int KLD = TB + 8;  // 72 doubles: [k][col] tiles
 constexpr int SWEEP_THREADS = 512;
-constexpr int FAR_THREADS = 128;
+constexpr int FAR_THREADS = 256;  // two independent 4-warp task streams
 
 struct QArgs {
   const void* W;
@@ -112,8 +112,8 @@ __device__ __forceinline__ void st_hint(double* p, double2 v, uint64_t pol) {
 // shared memory with row stride `sld`, 16 bytes per cp.async.
 template <int NT>
 __device__ __forceinline__ void tile_cp_async(double* dst, int sld, const double* src, int64_t ld,
-                                              uint64_t pol) {
-  for (int x = threadIdx.x; x < TB * TB / 2; x += NT) {
+                                              uint64_t pol, int tix) {
+  for (int x = tix; x < TB * TB / 2; x += NT) {
     const int r = x >> 5, c2 = (x & 31) * 2;
     cp_async16(dst + r * sld + c2, src + (int64_t)r * ld + c2, pol);
   }
@@ -299,6 +299,13 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       }
     __syncthreads();
   }
+  // ---- the tile's row scales and their reciprocals
+  __shared__ double Ss[TB], Si[TB];
+  if (tid < TB) {
+    const double sv = tid < rows ? (double)a.scales[r0 + tid] : 1.0;
+    Ss[tid] = sv;
+    Si[tid] = 1.0 / sv;
+  }
   // ---- diagonal blocks of the normalised factors
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
     const int r = x >> 5, k2 = (x & 31) * 2;
@@ -308,6 +315,23 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   cp_async_commit_group();
   cp_async_wait_group<0>();
   __syncthreads();
+
+  // One 8x8x8 FP64 tensor-core product: the finished sub-tile (p, q) pushes to
+  //   right (p, tgt):  P[p][tgt] += dW[p][q] Rh[tgt][q]^T
+  //   down  (tgt, q):  V[tgt][q] += Lh[tgt][p] P_final[p][q]
+  auto sub_update = [&](int p, int q, bool right, int tgt) {
+    const int R0 = SUB * p, C0 = SUB * q, T0 = SUB * tgt;
+    double* C = right ? Pt + (R0 + g) * SLD + T0 + 2 * t4 : Vt + (T0 + g) * SLD + C0 + 2 * t4;
+    double c0v = C[0], c1v = C[1];
+#pragma unroll
+    for (int kk = 0; kk < SUB; kk += 4) {
+      const double av = right ? Dt[(R0 + g) * SLD + C0 + kk + t4] : Lt[(T0 + g) * SLD + R0 + kk + t4];
+      const double bv = right ? Rt[(T0 + g) * SLD + C0 + kk + t4] : Pt[(R0 + kk + t4) * SLD + C0 + g];
+      dmma_m8n8k4(c0v, c1v, av, bv);
+    }
+    C[0] = c0v;
+    C[1] = c1v;
+  };
 
   double loss = 0.0;
   long long ncl = 0, nnt = 0, nnf = 0;
@@ -324,8 +348,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       if (R0 < rows && C0 < cols) {
         const int ar = R0 + sa;
         const bool rok = ar < rows;
-        const double s = rok ? (double)a.scales[r0 + ar] : 1.0;
-        const double inv_s = 1.0 / s;
+        const double s = Ss[ar], inv_s = Si[ar];
         double P[2], V[2], Wd[2];
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
@@ -375,37 +398,35 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
         }
       }
     }
+    // ---- meanwhile, warps NSUB.. apply the updates of sub-wavefront w-1 that are not
+    // needed before sub-wavefront w+2 (targets two or more sub-tiles away); they
+    // touch sub-tiles no sweep of wave w reads or writes
+    if (warp >= NSUB && w >= 1) {
+      const int wp = w - 1;
+      const int pp0 = wp - (NSUB - 1) > 0 ? wp - (NSUB - 1) : 0;
+      const int pp1 = wp < NSUB - 1 ? wp : NSUB - 1;
+      int x = warp - NSUB;
+      for (int pp = pp0; pp <= pp1; ++pp) {
+        const int qq = wp - pp;
+        const int nr = NSUB - 2 - qq > 0 ? NSUB - 2 - qq : 0;  // right targets qq+2 ..
+        const int nd = NSUB - 2 - pp > 0 ? NSUB - 2 - pp : 0;  // down targets pp+2 ..
+        for (; x < nr + nd; x += SWEEP_THREADS / 32 - NSUB) {
+          if (x < nr) sub_update(pp, qq, true, qq + 2 + x);
+          else sub_update(pp, qq, false, pp + 2 + (x - nr));
+        }
+        x -= nr + nd;
+      }
+    }
     __syncthreads();
     if (w == 2 * NSUB - 2) break;
 
-    // ---- block updates from the finished sub-tiles: 8x8x8 DMMA products, one warp per target
-    const int per = 2 * NSUB - 2 - w;  // targets per source: (7 - q) right + (7 - p) down
-    for (int x = warp; x < nsub * per; x += SWEEP_THREADS / 32) {
-      const int p = p0 + x / per, q = w - p, j = x % per;
-      const int R0 = SUB * p, C0 = SUB * q;
-      double c0v, c1v;
-      if (j < NSUB - 1 - q) {  // right: P[p][q'] += dW[p][q] Rh[q'][q]^T
-        const int Q0 = SUB * (q + 1 + j);
-        double* C = Pt + (R0 + g) * SLD + Q0 + 2 * t4;
-        c0v = C[0];
-        c1v = C[1];
-#pragma unroll
-        for (int kk = 0; kk < SUB; kk += 4)
-          dmma_m8n8k4(c0v, c1v, Dt[(R0 + g) * SLD + C0 + kk + t4],
-                      Rt[(Q0 + g) * SLD + C0 + kk + t4]);
-        C[0] = c0v;
-        C[1] = c1v;
-      } else {                 // down: V[p'][q] += Lh[p'][p] P_final[p][q]
-        const int S0 = SUB * (p + 1 + j - (NSUB - 1 - q));
-        double* C = Vt + (S0 + g) * SLD + C0 + 2 * t4;
-        c0v = C[0];
-        c1v = C[1];
-#pragma unroll
-        for (int kk = 0; kk < SUB; kk += 4)
-          dmma_m8n8k4(c0v, c1v, Lt[(S0 + g) * SLD + R0 + kk + t4],
-                      Pt[(R0 + kk + t4) * SLD + C0 + g]);
-        C[0] = c0v;
-        C[1] = c1v;
+    // ---- the urgent updates of sub-wavefront w: its right and lower neighbours
+    if (warp < 2 * nsub) {
+      const int p = p0 + (warp >> 1), q = w - p;
+      if ((warp & 1) == 0) {
+        if (q + 1 < NSUB) sub_update(p, q, true, q + 1);
+      } else {
+        if (p + 1 < NSUB) sub_update(p, q, false, p + 1);
       }
     }
     __syncthreads();
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   for (int x = tid; x < TB * TB; x += SWEEP_THREADS) {
     const int r = x >> 6, c = x & 63;
     if (r < rows && c < cols) {
-      const double sr = (double)a.scales[r0 + r];
+      const double sr = Ss[r];
       const double tq = Tq[r * SLD + c];
       const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;
       const double qv = qr < a.lo ? a.lo : (qr > a.hi ? a.hi : qr);
@@ -473,82 +494,107 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
 constexpr int MAX_GROUPS = 512;  // 2 groups per tile: 256 tiles per launch
 struct FarPlan {
   int D, I0, nt;
-  int per_cta;               // tasks (64x64 output tiles) per CTA
-  int start[MAX_GROUPS + 1]; // first CTA of each group; group g < nt: right tasks of tile
-                             // I0+g, else down tasks of tile I0+g-nt
+  // start[g] = first task of group g in launch order; group g < nt holds the right
+  // tasks of tile I0+g, group g >= nt the down tasks of tile I0+g-nt.
+  int start[MAX_GROUPS + 1];
 };
 
-constexpr int FAR_SMEM = (TB * KLD + 2 * TB * SLD) * (int)sizeof(double);
+constexpr int FAR_GROUP_DOUBLES = TB * KLD + 2 * TB * SLD;  // shared operand + 2 task operands
+constexpr int FAR_SMEM = 2 * FAR_GROUP_DOUBLES * (int)sizeof(double);
 
-__global__ void __launch_bounds__(FAR_THREADS, 2) far_kernel(QArgs a, FarPlan pl) {
+__device__ __forceinline__ void group_barrier(int h) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(1 + h), "r"(128) : "memory");
+}
+
+// Persistent: each CTA runs two independent task streams (4 warps each, own shared
+// buffers, own named barrier).  Stream s of S = 2 gridDim.x takes tasks
+// [s T / S, (s+1) T / S) of the launch's T tasks, walking across groups.  A task is
+// one 64x64x64 DMMA product accumulated into a P or E tile; within a group the next
+// task's operand is copied in (cp.async) and the task's C tile is loaded into
+// registers while the previous copy lands.
+__global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl) {
   extern __shared__ __align__(16) double sm[];
-  double* Sh = sm;                       // shared operand of the CTA's tasks
-  double* const Bf0 = sm + TB * KLD;     // per-task operand, double-buffered
+  const int h = threadIdx.x >> 7, ht = threadIdx.x & 127;
+  double* Sh = sm + h * FAR_GROUP_DOUBLES;  // shared operand of the group's tasks
+  double* const Bf0 = Sh + TB * KLD;        // per-task operand, double-buffered
   auto bufp = [&](int b) { return Bf0 + b * (TB * SLD); };
-  const int cta = blockIdx.x;
-  int g = 0;
-  {
-    int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= cta
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (pl.start[mid] <= cta) lo = mid; else hi = mid;
-    }
-    g = lo;
-  }
-  const bool down = g >= pl.nt;
-  const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
-  const int count = down ? a.Tm - I - 2 : a.Tn - J - 2;
-  const int first = (cta - pl.start[g]) * pl.per_cta;
-  const int last = min(first + pl.per_cta, count);
-  if (first >= last) return;
-
   const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
   const int64_t np = a.np;
-  // shared operand: right -> dW[I,J] as [a][k]; down -> P[I,J] as [k][c]
-  if (!down)
-    tile_cp_async<FAR_THREADS>(Sh, SLD, a.Dl + (int64_t)I * TB * np + J * TB, np, stream);
-  else
-    tile_cp_async<FAR_THREADS>(Sh, KLD, a.P + (int64_t)I * TB * np + J * TB, np, stream);
-  auto task_operand = [&](int x) -> const double* {
-    // right: Rh[(J+2+x) block rows][J block cols] as [c][k]; down: Lh[(I+2+x) rows][I cols] as [a][k]
-    return down ? a.Lh + (int64_t)(I + 2 + x) * TB * a.mp + I * TB
-                : a.Rh + (int64_t)(J + 2 + x) * TB * np + J * TB;
-  };
-  const int64_t opld = down ? a.mp : np;
-  tile_cp_async<FAR_THREADS>(bufp(0), SLD, task_operand(first), opld, keep);
-  cp_async_commit();
-
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
+  const int lane = ht & 31, warp = ht >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
-  for (int x = first; x < last; ++x) {
-    const int buf = (x - first) & 1;
-    if (x + 1 < last) {
-      tile_cp_async<FAR_THREADS>(bufp(buf ^ 1), SLD, task_operand(x + 1), opld, keep);
-      cp_async_commit();
-    }
-    double* C = down ? a.E + (int64_t)(I + 2 + x) * TB * np + J * TB
-                     : a.P + (int64_t)I * TB * np + (J + 2 + x) * TB;
-    if (x + 1 < last) cp_async_wait<1>(); else cp_async_wait<0>();
-    __syncthreads();
-    double acc[4][4][2] = {};
-    const double* B = bufp(buf);
-    if (!down)
-      mma_64x64x64(acc, [&](int r, int k) { return Sh[r * SLD + k]; },
-                   [&](int k, int c) { return B[c * SLD + k]; });
-    else
-      mma_64x64x64(acc, [&](int r, int k) { return B[r * SLD + k]; },
-                   [&](int k, int c) { return Sh[k * KLD + c]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        double* cp = C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4;
-        double2 v = ld_hint(cp, stream);
-        v.x += acc[i][j][0];
-        v.y += acc[i][j][1];
-        st_hint(cp, v, stream);
+  const int64_t total = pl.start[2 * pl.nt];
+  const int64_t S = 2 * (int64_t)gridDim.x, sid = 2 * (int64_t)blockIdx.x + h;
+  const int t_end = (int)((sid + 1) * total / S);
+  int t_cur = (int)(sid * total / S);
+
+  while (t_cur < t_end) {
+    int g;
+    {
+      int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= t_cur
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pl.start[mid] <= t_cur) lo = mid; else hi = mid;
       }
-    __syncthreads();
+      g = lo;
+    }
+    const bool down = g >= pl.nt;
+    const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
+    const int first = t_cur - pl.start[g];
+    const int last = min(pl.start[g + 1], t_end) - pl.start[g];
+    t_cur = pl.start[g] + last;
+
+    // shared operand: right -> dW[I,J] as [a][k]; down -> P[I,J] as [k][c]
+    if (!down)
+      tile_cp_async<128>(Sh, SLD, a.Dl + (int64_t)I * TB * np + J * TB, np, stream, ht);
+    else
+      tile_cp_async<128>(Sh, KLD, a.P + (int64_t)I * TB * np + J * TB, np, stream, ht);
+    auto task_operand = [&](int x) -> const double* {
+      // right: Rh[(J+2+x) rows][J cols] as [c][k]; down: Lh[(I+2+x) rows][I cols] as [a][k]
+      return down ? a.Lh + (int64_t)(I + 2 + x) * TB * a.mp + I * TB
+                  : a.Rh + (int64_t)(J + 2 + x) * TB * np + J * TB;
+    };
+    auto task_c = [&](int x) -> double* {
+      return down ? a.E + (int64_t)(I + 2 + x) * TB * np + J * TB
+                  : a.P + (int64_t)I * TB * np + (J + 2 + x) * TB;
+    };
+    const int64_t opld = down ? a.mp : np;
+    tile_cp_async<128>(bufp(0), SLD, task_operand(first), opld, keep, ht);
+    cp_async_commit();
+
+    for (int x = first; x < last; ++x) {
+      const int buf = (x - first) & 1;
+      if (x + 1 < last) {
+        tile_cp_async<128>(bufp(buf ^ 1), SLD, task_operand(x + 1), opld, keep, ht);
+        cp_async_commit();
+      }
+      double* C = task_c(x);
+      double2 cv[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          cv[i][j] = ld_hint(C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4, stream);
+      if (x + 1 < last) cp_async_wait<1>(); else cp_async_wait<0>();
+      group_barrier(h);
+      double acc[4][4][2] = {};
+      const double* B = bufp(buf);
+      if (!down)
+        mma_64x64x64_w(acc, warp, [&](int r, int k) { return Sh[r * SLD + k]; },
+                       [&](int k, int c) { return B[c * SLD + k]; });
+      else
+        mma_64x64x64_w(acc, warp, [&](int r, int k) { return B[r * SLD + k]; },
+                       [&](int k, int c) { return Sh[k * KLD + c]; });
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          double2 v = cv[i][j];
+          v.x += acc[i][j][0];
+          v.y += acc[i][j][1];
+          st_hint(C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4, v, stream);
+        }
+      group_barrier(h);
+    }
   }
 }
 
@@ -653,7 +699,6 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
        cudaStreamWaitEvent(lo, ds->setup, 0) == cudaSuccess;
 
   const int nd = a.Tm + a.Tn - 1;
-  const int target_ctas = 2 * ds->sms;
   bool far_recorded[RING] = {};
   for (int D = 0; D < nd && ok; ++D) {
     const int I0 = D - (a.Tn - 1) > 0 ? D - (a.Tn - 1) : 0;
@@ -671,23 +716,25 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
       total += std::max(0, a.Tn - J - 2) + std::max(0, a.Tm - I - 2);
     }
     if (total == 0) continue;
-    const int per_cta = (int)std::max<long long>(1, (total + target_ctas - 1) / target_ctas);
     ok = ok && cudaEventRecord(ds->sw[D % RING], hi) == cudaSuccess &&
          cudaStreamWaitEvent(lo, ds->sw[D % RING], 0) == cudaSuccess;
+    // far(D) runs beside sweep(D+1): leave that sweep's CTAs their SMs
+    const int nt_next = std::max(0, std::min(D + 1, a.Tm - 1) -
+                                        std::max(0, D + 1 - (a.Tn - 1)) + 1);
+    const int far_ctas = std::max(ds->sms / 4, ds->sms - nt_next);
     for (int tb = 0; tb < nt && ok; tb += MAX_GROUPS / 2) {  // tiles per launch
       FarPlan pl;
       pl.D = D;
       pl.I0 = I0 + tb;
       pl.nt = std::min(nt - tb, MAX_GROUPS / 2);
-      pl.per_cta = per_cta;
-      int ctas = 0;
+      int tasks = 0;
       for (int gidx = 0; gidx < 2 * pl.nt; ++gidx) {
         const int I = pl.I0 + (gidx < pl.nt ? gidx : gidx - pl.nt), J = D - I;
-        const int cnt = gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
-        pl.start[gidx] = ctas;
-        ctas += (cnt + per_cta - 1) / per_cta;
+        pl.start[gidx] = tasks;
+        tasks += gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
       }
-      pl.start[2 * pl.nt] = ctas;
+      pl.start[2 * pl.nt] = tasks;
+      const int ctas = std::min(far_ctas, (tasks + 1) / 2);
       if (ctas > 0)
         GPTQ2D_LAUNCH(KC_PROPAGATE, lo, far_kernel<<<ctas, FAR_THREADS, FAR_SMEM, lo>>>(a, pl));
     }
