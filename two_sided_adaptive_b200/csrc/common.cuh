@@ -136,18 +136,20 @@ struct TileStat {
 };
 
 // ---------------------------------------------------------------------------
-// Per-device internal streams (streams.cu): a highest-priority and a lowest-
-// priority non-blocking stream plus events to fork from / join to the caller's
-// stream.  `mu` serialises the enqueue sequences that use them.
+// Per-device internal streams (streams.cu): two highest-priority and two
+// lowest-priority non-blocking streams plus events to fork from / join to the
+// caller's stream.  `mu` serialises the enqueue sequences that use them.
 // ---------------------------------------------------------------------------
 constexpr int RING = 4;
 struct DevStreams {
   std::mutex mu;
   bool ready = false;
   int sms = 148;
-  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaStream_t hi = nullptr, lo = nullptr, hi2 = nullptr, lo2 = nullptr;
   cudaEvent_t fork = nullptr, setup = nullptr, join_hi = nullptr, join_lo = nullptr;
-  cudaEvent_t sw[RING] = {}, far[RING] = {};
+  cudaEvent_t join_hi2 = nullptr, join_lo2 = nullptr;
+  cudaEvent_t sw[RING] = {}, far[RING] = {}, farb[RING] = {};
+  cudaEvent_t panel_done[2][RING] = {}, rest_done[2][RING] = {};  // factor preparation
 };
 int dev_streams(DevStreams** out);
 
@@ -158,8 +160,9 @@ size_t prepare_ws_bytes(int64_t k);
 int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
                    void* ws, cudaStream_t s);
 
-// Both factors at once: H_L on the high-priority internal stream, H_R on the
-// low-priority one, forked from and joined back to `s`.
+// Both factors at once, interleaved step by step on the internal streams
+// (panels on the high-priority ones, trailing updates on the low-priority
+// ones), forked from and joined back to `s`.
 int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
                         int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s);

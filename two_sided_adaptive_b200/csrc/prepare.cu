@@ -13,8 +13,12 @@
 //   1. M_KK^T M_KK = A_KK            (in-SM factorization of one 64x64 block)
 //   2. M_Kb = M_KK^{-T} A_Kb, b < K  (triangular solve of the block row)
 //   3. A_IJ -= M_KI^T M_KJ, J<=I<K   (rank-64 trailing update on FP64 tensor cores)
-// Everything is fp64.  A pivot that is not positive and finite stops the
-// factorization and is reported through a pivot word in the workspace.
+// Step 3 is split with a lookahead of one block row: the update of row K-1 by
+// M row K is done inside panel(K-1) itself, and the rest (rows I <= K-2) runs
+// on a second stream beside panel(K-1).  panel(K-1) therefore waits only for
+// the rest-update of step K+1.  Everything is fp64.  A pivot that is not
+// positive and finite stops the factorization and is reported through a pivot
+// word in the workspace.
 #include <algorithm>
 
 #include "common.cuh"
@@ -23,9 +27,9 @@ namespace gptq2d {
 
 namespace {
 
-constexpr int PLD = TB + 1;  // leading dimension of the in-SM factor / panel tiles
-constexpr int KLD = TB + 8;  // leading dimension of [k][*] operand tiles (72: conflict-free fragments)
+constexpr int OLD = TB + 4;  // 68: row stride of shared 64x64 tiles (conflict-free DMMA fragments)
 constexpr int TR_THREADS = 128;
+constexpr int PANEL_THREADS = 256;
 constexpr int MAX_TR_GROUPS = 512;
 
 template <typename TH>
@@ -41,147 +45,263 @@ __global__ void __launch_bounds__(256) convert_lower_kernel(const TH* __restrict
   }
 }
 
+// Copies the rows x cols block of M at (row0, col0) into shared memory [r][c]
+// with row stride OLD, zero outside.  V16: 16-byte copies, which needs 16-byte
+// aligned row starts and an even `cols`; else 8-byte copies.
+template <bool V16, int NT>
+__device__ __forceinline__ void load_block(double* dst, const double* M, int64_t ldm, int row0,
+                                           int col0, int rows, int cols) {
+  if (V16) {
+    for (int x = threadIdx.x; x < TB * TB / 2; x += NT) {
+      const int r = x >> 5, c2 = (x & 31) * 2;
+      const bool ok = r < rows && c2 < cols;
+      const double* src = ok ? M + (int64_t)(row0 + r) * ldm + col0 + c2 : M;
+      cp_async16_zfill(dst + r * OLD + c2, src, ok);
+    }
+  } else {
+    for (int x = threadIdx.x; x < TB * TB; x += NT) {
+      const int r = x >> 6, c = x & 63;
+      const bool ok = r < rows && c < cols;
+      const double* src = ok ? M + (int64_t)(row0 + r) * ldm + col0 + c : M;
+      cp_async8_zfill(dst + r * OLD + c, src, ok);
+    }
+  }
+}
+
+// Subtracts Xs^T Ys from the 64x64 shared tile Cs, all [r][c] with stride OLD:
+// Cs[i][j] -= sum_r Xs[r][i] Ys[r][j].  8 warps; warp w owns rows (w>>1)*16..+16
+// and columns (w&1)*32..+32 of Cs, so every element has one owner.
+__device__ __forceinline__ void sub_xty_8w(double* Cs, const double* Xs, const double* Ys) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wr = (warp >> 1) * 16, wc = (warp & 1) * 32;
+  double acc[2][4][2] = {};
+#pragma unroll 4
+  for (int kk = 0; kk < TB; kk += 4) {
+    double a[2], b[4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) a[i] = Xs[(kk + t) * OLD + wr + i * 8 + g];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = Ys[(kk + t) * OLD + wc + j * 8 + g];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double* c = Cs + (wr + i * 8 + g) * OLD + wc + j * 8 + 2 * t;
+      c[0] -= acc[i][j][0];
+      c[1] -= acc[i][j][1];
+    }
+}
+
+constexpr int PANEL_SMEM = 4 * TB * OLD * (int)sizeof(double);
+
+// Reverse Cholesky of the 8x8 block D = A[R0..R0+8)^2 of the shared tile A into
+// registers: L (lower) = M_D and inv[p] = 1/M_D[p][p].  Every calling thread
+// computes the same factor; nothing is shared, so no barrier is needed between
+// the factor and its use.  Returns the first bad pivot (elimination order,
+// local index) or -1.
+__device__ __forceinline__ int factor_diag8_regs(const double* A, int R0, double (&L)[8][8],
+                                                 double (&inv)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j <= i; ++j) L[i][j] = A[(R0 + i) * OLD + R0 + j];
+  int bad = -1;
+#pragma unroll
+  for (int p = 7; p >= 0; --p) {
+    const double piv = L[p][p];
+    const bool ok = piv > 0.0 && isfinite(piv);
+    if (!ok && bad < 0) bad = p;
+    const double r = ok ? rsqrt(piv) : 0.0;
+    const double r2 = r * r;
+#pragma unroll
+    for (int i = p - 1; i >= 0; --i) {  // row p-1 first: it carries the next pivot
+      const double mi = L[p][i] * r2;
+#pragma unroll
+      for (int j = 0; j <= i; ++j) L[i][j] = fma(-mi, L[p][j], L[i][j]);
+    }
+#pragma unroll
+    for (int j = 0; j <= p; ++j) L[p][j] *= r;
+    inv[p] = r;
+  }
+  return bad;
+}
+
+// X <- M_D^{-T} X for the 8 rows R0..R0+8 of column c of the shared tile X,
+// with M_D the 8x8 diagonal block of the shared factor F (back substitution).
+__device__ __forceinline__ void solve_col8(double* X, const double* F, const double* invd, int R0,
+                                           int c) {
+  double x[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) x[a] = X[(R0 + a) * OLD + c];
+#pragma unroll
+  for (int p = 7; p >= 0; --p) {
+    x[p] *= invd[R0 + p];
+#pragma unroll
+    for (int i = 0; i < p; ++i) x[i] = fma(-F[(R0 + p) * OLD + R0 + i], x[p], x[i]);
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a) X[(R0 + a) * OLD + c] = x[a];
+}
+
+// The same with the factor in registers.
+__device__ __forceinline__ void solve_col8_regs(double* X, const double (&L)[8][8],
+                                                const double (&inv)[8], int R0, int c) {
+  double x[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) x[a] = X[(R0 + a) * OLD + c];
+#pragma unroll
+  for (int p = 7; p >= 0; --p) {
+    x[p] *= inv[p];
+#pragma unroll
+    for (int i = 0; i < p; ++i) x[i] = fma(-L[p][i], x[p], x[i]);
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a) X[(R0 + a) * OLD + c] = x[a];
+}
+
+// C[8bi.., 8bj..] -= sum_{a<8} S[R0+a][8bi + r] T[R0+a][8bj + c] for the 8x8 block
+// (bi, bj) of shared tile C, on one warp (two m8n8k4 DMMA steps).
+__device__ __forceinline__ void rank8_block(double* C, const double* S, const double* T, int R0,
+                                            int bi, int bj) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  double c0 = 0.0, c1 = 0.0;
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 4)
+    dmma_m8n8k4(c0, c1, S[(R0 + kk + t) * OLD + 8 * bi + g], T[(R0 + kk + t) * OLD + 8 * bj + g]);
+  double* dst = C + (8 * bi + g) * OLD + 8 * bj + 2 * t;
+  dst[0] -= c0;
+  dst[1] -= c1;
+}
+
 // One launch per block row K.  CTA K factors the diagonal block and writes it;
 // CTAs b < K factor the same block redundantly (cheaper than a separate launch)
-// and solve their block M_Kb = M_KK^{-T} A_Kb.
+// and solve their block M_Kb = M_KK^{-T} A_Kb.  When a factored block row K+1
+// exists, each CTA first applies its update to the blocks it reads:
+// A_KK -= M_{K+1,K}^T M_{K+1,K} and A_Kb -= M_{K+1,K}^T M_{K+1,b}.
 //
-// Both phases keep their 64 x 64 block in registers: thread (i = tid/4, q =
-// tid%4) holds row i, columns q + 4u (u < 16).  The pivot and solve loops are
-// unrolled so that every register index is a compile-time constant.  Per pivot
-// p (last row first): the four threads of row p scale it by 1/sqrt(A[p][p]) and
-// publish it to a double-buffered shared row; after one barrier every row i < p
-// applies A[i][j] -= M[p][i] M[p][j] from broadcast reads.  The strict upper
-// part of the register block is never read (published rows are zero beyond p).
-__global__ void __launch_bounds__(256) panel_kernel(double* __restrict__ M, int64_t ldm, int k,
-                                                    int K, long long* info) {
+// The 64x64 factorization runs in 8-row strips from the bottom: warp 0 factors
+// the strip's 8x8 diagonal block (factor_diag8); one thread per column solves
+// the strip left of it (solve_col8); the strip's rank-8 update of the leading
+// block runs on the DMMA units of all warps (rank8_block).  The solve of A_Kb
+// goes the same way.  Rows beyond a ragged edge get a unit diagonal, which
+// leaves the factor of the leading part unchanged.
+template <bool V16>
+__global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict__ M, int64_t ldm,
+                                                              int k, int K, long long* info) {
   if (*(volatile long long*)info >= 0) return;
-  __shared__ double S[TB * PLD];      // the factored diagonal block M_KK
-  __shared__ double rowb[2][TB];      // published pivot row / solved row
-  __shared__ double invd[TB];         // 1 / M_KK[p][p]
+  extern __shared__ __align__(16) double sm[];
+  double* Ad = sm;              // A_KK, then M_KK
+  double* Ab = Ad + TB * OLD;   // A_Kb, then M_Kb
+  double* Mn = Ab + TB * OLD;   // M_{K+1,K}
+  double* Mb = Mn + TB * OLD;   // M_{K+1,b}
+  __shared__ double invd[TB];
   __shared__ int bad;
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int i = tid >> 2, q = tid & 3;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int rb = K * TB, nb = min(TB, k - rb);
+  const int rn = rb + TB, nn = max(0, min(TB, k - rn));  // block row K+1, if any
   const int b = blockIdx.x;
   if (tid == 0) bad = -1;
 
-  double v[TB / 4];
-#pragma unroll
-  for (int u = 0; u < TB / 4; ++u) {
-    const int j = q + 4 * u;
-    v[u] = (i < nb && j <= i) ? M[(int64_t)(rb + i) * ldm + rb + j] : 0.0;
+  load_block<V16, PANEL_THREADS>(Ad, M, ldm, rb, rb, nb, nb);
+  if (b < K) load_block<V16, PANEL_THREADS>(Ab, M, ldm, rb, b * TB, nb, TB);
+  if (nn > 0) {
+    load_block<V16, PANEL_THREADS>(Mn, M, ldm, rn, rb, nn, nb);
+    if (b < K) load_block<V16, PANEL_THREADS>(Mb, M, ldm, rn, b * TB, nn, TB);
   }
+  cp_async_commit_group();
+  cp_async_wait_group<0>();
+  __syncthreads();
+  if (nn > 0) {
+    sub_xty_8w(Ad, Mn, Mn);
+    if (b < K) sub_xty_8w(Ab, Mn, Mb);
+  }
+  // unit diagonal past a ragged edge (only the last block row is ragged, and it
+  // has no lookahead update, so no other thread writes these elements)
+  if (tid < TB && tid >= nb) Ad[tid * OLD + tid] = 1.0;
   __syncthreads();
 
+  // factor A_KK in place, strips s = 7..0
+#pragma unroll 1
+  for (int s = TB / 8 - 1; s >= 0; --s) {
+    const int R0 = 8 * s;
+    if (tid <= R0) {  // threads < R0 solve a column of the strip, thread R0 stores M_D
+      double L[8][8], inv[8];
+      const int bp = factor_diag8_regs(Ad, R0, L, inv);
+      if (tid < R0) {
+        solve_col8_regs(Ad, L, inv, R0, tid);
+      } else {
 #pragma unroll
-  for (int p = TB - 1; p >= 0; --p) {
-    if (p < nb) {
-      // every lane takes part in the shuffle; row p's four threads use the value
-      const double piv = __shfl_sync(0xffffffffu, v[p >> 2], (lane & ~3) | (p & 3));
-      if (i == p) {
-        const bool ok = piv > 0.0 && isfinite(piv);
-        const double r = ok ? rsqrt(piv) : 0.0;
+        for (int i = 0; i < 8; ++i) {
+          invd[R0 + i] = inv[i];
 #pragma unroll
-        for (int u = 0; u < TB / 4; ++u) {
-          const int j = q + 4 * u;
-          v[u] = (j <= p) ? v[u] * r : 0.0;
-          rowb[p & 1][j] = v[u];
+          for (int j = 0; j < 8; ++j) Ad[(R0 + i) * OLD + R0 + j] = j <= i ? L[i][j] : 0.0;
         }
-        if (q == 0) {
-          invd[p] = r;
-          if (!ok) bad = rb + p;
-        }
-      }
-      __syncthreads();
-      if (bad >= 0) {  // uniform: every thread reads the flag after the barrier
-        if (tid == 0) *info = bad;
-        return;
-      }
-      if (i < p) {
-        const double mi = rowb[p & 1][i];
-#pragma unroll
-        for (int u = 0; u < TB / 4; ++u) v[u] = fma(-mi, rowb[p & 1][q + 4 * u], v[u]);
+        if (bp >= 0 && bad < 0) bad = rb + R0 + bp;
       }
     }
+    __syncthreads();
+    // A_lead[i][j] -= sum_a M[R0+a][i] M[R0+a][j], lower 8x8 blocks (bi >= bj) of the lead
+    const int nblk = s * (s + 1) / 2;
+    for (int x = warp; x < nblk; x += PANEL_THREADS / 32) {
+      int bi = 0;
+      while ((bi + 1) * (bi + 2) / 2 <= x) ++bi;
+      rank8_block(Ad, Ad, Ad, R0, bi, x - bi * (bi + 1) / 2);
+    }
+    __syncthreads();
   }
-  // registers now hold M_KK (lower part); the diagonal is A[p][p] * (1/sqrt(A[p][p]))
-#pragma unroll
-  for (int u = 0; u < TB / 4; ++u) {
-    const int j = q + 4 * u;
-    S[i * PLD + j] = (i < nb && j <= i) ? v[u] : 0.0;
+  if (bad >= 0) {  // uniform: read after the last barrier
+    if (tid == 0) *info = bad;
+    return;
+  }
+  // zero the strict upper part of the 8x8 blocks above the diagonal blocks
+  for (int e = tid; e < TB * TB; e += PANEL_THREADS) {
+    const int r = e >> 6, c = e & 63;
+    if (c > r) Ad[r * OLD + c] = 0.0;
   }
   __syncthreads();
   if (b == K) {
-    for (int e = tid; e < nb * TB; e += blockDim.x) {
+    for (int e = tid; e < nb * TB; e += PANEL_THREADS) {
       const int r = e >> 6, c = e & 63;
-      if (c < nb) M[(int64_t)(rb + r) * ldm + rb + c] = S[r * PLD + c];
+      if (c < nb) M[(int64_t)(rb + r) * ldm + rb + c] = Ad[r * OLD + c];
     }
     return;
   }
 
-  // X <- M_KK^{-T} X by back substitution (M_KK^T is upper triangular)
-#pragma unroll
-  for (int u = 0; u < TB / 4; ++u)
-    v[u] = (i < nb) ? M[(int64_t)(rb + i) * ldm + (int64_t)b * TB + q + 4 * u] : 0.0;
-#pragma unroll
-  for (int r = TB - 1; r >= 0; --r) {
-    if (r < nb) {
-      if (i == r) {
-        const double iv = invd[r];
-#pragma unroll
-        for (int u = 0; u < TB / 4; ++u) {
-          v[u] *= iv;
-          rowb[r & 1][q + 4 * u] = v[u];
-        }
-      }
-      __syncthreads();
-      if (i < r) {
-        const double mr = S[r * PLD + i];
-#pragma unroll
-        for (int u = 0; u < TB / 4; ++u) v[u] = fma(-mr, rowb[r & 1][q + 4 * u], v[u]);
-      }
-    }
+  // X <- M_KK^{-T} X in strips from the bottom
+#pragma unroll 1
+  for (int s = TB / 8 - 1; s >= 0; --s) {
+    const int R0 = 8 * s;
+    if (tid < TB) solve_col8(Ab, Ad, invd, R0, tid);
+    __syncthreads();
+    // X[i][c] -= sum_a M[R0+a][i] X[R0+a][c] for rows i < R0
+    for (int x = warp; x < s * 8; x += PANEL_THREADS / 32) rank8_block(Ab, Ad, Ab, R0, x >> 3, x & 7);
+    __syncthreads();
   }
-  if (i < nb) {
-#pragma unroll
-    for (int u = 0; u < TB / 4; ++u)
-      M[(int64_t)(rb + i) * ldm + (int64_t)b * TB + q + 4 * u] = v[u];
-  }
-}
-
-// Copies the nb x 64 block of M at (row0, col0) into shared memory [r][c] with
-// row stride KLD, zero rows beyond nb.  16-byte copies when every row start is
-// 16-byte aligned, else 8-byte copies.
-template <bool V16>
-__device__ __forceinline__ void load_rows(double* dst, const double* M, int64_t ldm, int row0,
-                                          int col0, int nb) {
-  if (V16) {
-    for (int x = threadIdx.x; x < TB * TB / 2; x += TR_THREADS) {
-      const int r = x >> 5, c2 = (x & 31) * 2;
-      const bool ok = r < nb;
-      const double* src = ok ? M + (int64_t)(row0 + r) * ldm + col0 + c2 : M;
-      cp_async16_zfill(dst + r * KLD + c2, src, ok);
-    }
-  } else {
-    for (int x = threadIdx.x; x < TB * TB; x += TR_THREADS) {
-      const int r = x >> 6, c = x & 63;
-      const bool ok = r < nb;
-      const double* src = ok ? M + (int64_t)(row0 + r) * ldm + col0 + c : M;
-      cp_async8_zfill(dst + r * KLD + c, src, ok);
-    }
+  for (int e = tid; e < nb * TB; e += PANEL_THREADS) {
+    const int r = e >> 6, c = e & 63;
+    M[(int64_t)(rb + r) * ldm + (int64_t)b * TB + c] = Ab[r * OLD + c];
   }
 }
 
 struct TrailPlan {
-  int K, I0, ng;                 // block row, first group, number of groups
+  int K, I0, ng;                 // factored block row, first group, number of groups
   int per_cta;                   // blocks J per CTA
   int start[MAX_TR_GROUPS + 1];  // first CTA of each group; group g updates A[I0+g][0..I0+g]
 };
 
-constexpr int TR_SMEM = 3 * TB * KLD * (int)sizeof(double);
+constexpr int TR_SMEM = 3 * TB * OLD * (int)sizeof(double);
 
-// A_IJ -= M_KI^T M_KJ.  Each CTA keeps M_KI in shared memory and streams the
-// M_KJ blocks of its range of J through a double buffer.
+// A_IJ -= M_KI^T M_KJ for J <= I, over a range of J of one block row I.  Each
+// CTA keeps M_KI in shared memory and streams the M_KJ blocks through a double
+// buffer; the A_IJ block is loaded into registers before the product so that
+// its latency overlaps the tensor-core work.  Only the lower part of A_II is
+// written.
 template <bool V16>
 __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restrict__ M,
                                                                  int64_t ldm, int k,
@@ -190,8 +310,8 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
   if (*(volatile const long long*)info >= 0) return;
   extern __shared__ __align__(16) double sm[];
   double* Xs = sm;  // Xs[r][i] = M[rb + r][64 I + i]
-  double* const Y0 = sm + TB * KLD;
-  auto ybuf = [&](int bsel) { return Y0 + bsel * (TB * KLD); };
+  double* const Y0 = sm + TB * OLD;
+  auto ybuf = [&](int bsel) { return Y0 + bsel * (TB * OLD); };
   const int cta = blockIdx.x;
   int g;
   {
@@ -208,97 +328,193 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
   if (first >= last) return;
   const int rb = pl.K * TB, nb = min(TB, k - rb);
 
-  load_rows<V16>(Xs, M, ldm, rb, I * TB, nb);
-  load_rows<V16>(ybuf(0), M, ldm, rb, first * TB, nb);
+  load_block<V16, TR_THREADS>(Xs, M, ldm, rb, I * TB, nb, TB);
+  load_block<V16, TR_THREADS>(ybuf(0), M, ldm, rb, first * TB, nb, TB);
   cp_async_commit_group();
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
+  const int kmax = (nb + 3) & ~3;
   for (int J = first; J < last; ++J) {
     const int bsel = (J - first) & 1;
     if (J + 1 < last) {
-      load_rows<V16>(ybuf(bsel ^ 1), M, ldm, rb, (J + 1) * TB, nb);
+      load_block<V16, TR_THREADS>(ybuf(bsel ^ 1), M, ldm, rb, (J + 1) * TB, nb, TB);
       cp_async_commit_group();
-      cp_async_wait_group<1>();
-    } else {
-      cp_async_wait_group<0>();
     }
+    double* Cg = M + (int64_t)(I * TB + wr + g8) * ldm + (int64_t)J * TB + wc + 2 * t4;
+    double cv[4][4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const double* src = Cg + (int64_t)i * 8 * ldm + j * 8;
+        if (V16) {
+          const double2 x = *reinterpret_cast<const double2*>(src);
+          cv[i][j][0] = x.x;
+          cv[i][j][1] = x.y;
+        } else {
+          cv[i][j][0] = src[0];
+          cv[i][j][1] = src[1];
+        }
+      }
+    if (J + 1 < last) cp_async_wait_group<1>(); else cp_async_wait_group<0>();
     __syncthreads();
     const double* Ys = ybuf(bsel);
     double acc[4][4][2] = {};
     mma_64x64x64(
-        acc, [&](int row, int kk) { return Xs[kk * KLD + row]; },
-        [&](int kk, int col) { return Ys[kk * KLD + col]; }, (nb + 3) & ~3);
+        acc, [&](int row, int kk) { return Xs[kk * OLD + row]; },
+        [&](int kk, int col) { return Ys[kk * OLD + col]; }, kmax);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int r = wr + i * 8 + g8, c = wc + j * 8 + 2 * t4;
-        double* dst = M + (int64_t)(I * TB + r) * ldm + (int64_t)J * TB + c;
-        if (I != J || c <= r) dst[0] -= acc[i][j][0];
-        if (I != J || c + 1 <= r) dst[1] -= acc[i][j][1];
+        double* dst = Cg + (int64_t)i * 8 * ldm + j * 8;
+        const double x0 = cv[i][j][0] - acc[i][j][0], x1 = cv[i][j][1] - acc[i][j][1];
+        if (I != J) {
+          if (V16) {
+            *reinterpret_cast<double2*>(dst) = make_double2(x0, x1);
+          } else {
+            dst[0] = x0;
+            dst[1] = x1;
+          }
+        } else {
+          if (c <= r) dst[0] = x0;
+          if (c + 1 <= r) dst[1] = x1;
+        }
       }
     __syncthreads();
   }
 }
 
 std::atomic<uint64_t> g_trailing_smem_set[2];
-std::atomic<uint64_t> g_panel_smem_set{0};
+std::atomic<uint64_t> g_panel_smem_set[2];
 
-int sm_count() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms > 0 ? sms : 148;
+
+// One factor's enqueue state: panels on `ps`, trailing updates on `us`.
+struct FactorJob {
+  const void* H;
+  int h_dtype, k, T;
+  int64_t ldh, ldm;
+  double* M;
+  long long* info;
+  bool v16;
+  cudaStream_t ps, us;
+  cudaEvent_t* panel_done;  // [RING]
+  cudaEvent_t* rest_done;   // [RING]
+};
+
+int enqueue_convert(const FactorJob& f, int sms) {
+  const int cblocks = (int)std::min<int64_t>(((int64_t)f.k * f.k + 255) / 256, (int64_t)sms * 16);
+  if (f.h_dtype == GPTQ2D_F32)
+    GPTQ2D_LAUNCH(KC_OTHER, f.ps,
+                  convert_lower_kernel<float><<<cblocks, 256, 0, f.ps>>>(
+                      static_cast<const float*>(f.H), f.ldh, f.k, f.M, f.ldm, f.info));
+  else
+    GPTQ2D_LAUNCH(KC_OTHER, f.ps,
+                  convert_lower_kernel<double><<<cblocks, 256, 0, f.ps>>>(
+                      static_cast<const double*>(f.H), f.ldh, f.k, f.M, f.ldm, f.info));
+  return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
-int prepare_enqueue(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
-                    void* ws, cudaStream_t s, int sms) {
-  long long* info = static_cast<long long*>(ws);
-  const int T = (k + TB - 1) / TB;
-  const int cblocks = (int)std::min<int64_t>(((int64_t)k * k + 255) / 256, (int64_t)sms * 16);
-  if (h_dtype == GPTQ2D_F32)
-    GPTQ2D_LAUNCH(KC_OTHER, s,
-                  convert_lower_kernel<float><<<cblocks, 256, 0, s>>>(
-                      static_cast<const float*>(H), ldh, k, M, ldm, info));
+// Step K of one factor: panel(K) after the trailing update of step K+2, then the
+// trailing update of rows I <= K-2 by M row K.
+int enqueue_step(const FactorJob& f, int K, int sms) {
+  bool ok = true;
+  if (K + 2 < f.T) ok = cudaStreamWaitEvent(f.ps, f.rest_done[(K + 2) % RING], 0) == cudaSuccess;
+  if (f.v16)
+    GPTQ2D_LAUNCH(KC_PREP_PANEL, f.ps,
+                  panel_kernel<true><<<K + 1, PANEL_THREADS, PANEL_SMEM, f.ps>>>(f.M, f.ldm, f.k,
+                                                                                   K, f.info));
   else
-    GPTQ2D_LAUNCH(KC_OTHER, s,
-                  convert_lower_kernel<double><<<cblocks, 256, 0, s>>>(
-                      static_cast<const double*>(H), ldh, k, M, ldm, info));
-  const int psmem = 0;
-  const bool v16 = (ldm % 2 == 0) && ((reinterpret_cast<uintptr_t>(M) & 15u) == 0);
+    GPTQ2D_LAUNCH(KC_PREP_PANEL, f.ps,
+                  panel_kernel<false><<<K + 1, PANEL_THREADS, PANEL_SMEM, f.ps>>>(f.M, f.ldm, f.k,
+                                                                                    K, f.info));
+  if (K < 2) return ok && cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
+  ok = ok && cudaEventRecord(f.panel_done[K % RING], f.ps) == cudaSuccess &&
+       cudaStreamWaitEvent(f.us, f.panel_done[K % RING], 0) == cudaSuccess;
+  const int rows = K - 1;  // block rows I = 0..K-2
+  const long long total = (long long)rows * (rows + 1) / 2;
+  const int target = 2 * sms;
+  const int per_cta = (int)std::max<long long>(1, (total + target - 1) / target);
+  for (int g0 = 0; g0 < rows && ok; g0 += MAX_TR_GROUPS) {
+    TrailPlan pl;
+    pl.K = K;
+    pl.I0 = g0;
+    pl.ng = std::min(rows - g0, MAX_TR_GROUPS);
+    pl.per_cta = per_cta;
+    int ctas = 0;
+    for (int gi = 0; gi < pl.ng; ++gi) {
+      pl.start[gi] = ctas;
+      ctas += (g0 + gi + 1 + per_cta - 1) / per_cta;
+    }
+    pl.start[pl.ng] = ctas;
+    if (f.v16)
+      GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
+                    trailing_kernel<true><<<ctas, TR_THREADS, TR_SMEM, f.us>>>(f.M, f.ldm, f.k,
+                                                                                 f.info, pl));
+    else
+      GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
+                    trailing_kernel<false><<<ctas, TR_THREADS, TR_SMEM, f.us>>>(f.M, f.ldm, f.k,
+                                                                                  f.info, pl));
+  }
+  ok = ok && cudaEventRecord(f.rest_done[K % RING], f.us) == cudaSuccess;
+  return ok && cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
+}
+
+int ensure_prepare_smem() {
   if (ensure_smem(trailing_kernel<true>, TR_SMEM, g_trailing_smem_set[0]) != cudaSuccess ||
       ensure_smem(trailing_kernel<false>, TR_SMEM, g_trailing_smem_set[1]) != cudaSuccess ||
-      ensure_smem(panel_kernel, psmem, g_panel_smem_set) != cudaSuccess)
+      ensure_smem(panel_kernel<true>, PANEL_SMEM, g_panel_smem_set[0]) != cudaSuccess ||
+      ensure_smem(panel_kernel<false>, PANEL_SMEM, g_panel_smem_set[1]) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
-  const int target = 2 * sms;
-  for (int K = T - 1; K >= 0; --K) {
-    GPTQ2D_LAUNCH(KC_PREP_PANEL, s, panel_kernel<<<K + 1, 256, psmem, s>>>(M, ldm, k, K, info));
-    if (K == 0) continue;
-    const long long total = (long long)K * (K + 1) / 2;
-    const int per_cta = (int)std::max<long long>(1, (total + target - 1) / target);
-    for (int g0 = 0; g0 < K; g0 += MAX_TR_GROUPS) {
-      TrailPlan pl;
-      pl.K = K;
-      pl.I0 = g0;
-      pl.ng = std::min(K - g0, MAX_TR_GROUPS);
-      pl.per_cta = per_cta;
-      int ctas = 0;
-      for (int gi = 0; gi < pl.ng; ++gi) {
-        pl.start[gi] = ctas;
-        ctas += (g0 + gi + 1 + per_cta - 1) / per_cta;
-      }
-      pl.start[pl.ng] = ctas;
-      if (v16)
-        GPTQ2D_LAUNCH(KC_PREP_TRAILING, s,
-                      trailing_kernel<true><<<ctas, TR_THREADS, TR_SMEM, s>>>(M, ldm, k, info, pl));
-      else
-        GPTQ2D_LAUNCH(KC_PREP_TRAILING, s,
-                      trailing_kernel<false><<<ctas, TR_THREADS, TR_SMEM, s>>>(M, ldm, k, info, pl));
-    }
-  }
-  return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
+  return GPTQ2D_OK;
+}
+
+FactorJob make_job(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
+                   void* ws, cudaStream_t ps, cudaStream_t us, cudaEvent_t* pd, cudaEvent_t* rd) {
+  FactorJob f;
+  f.H = H;
+  f.h_dtype = h_dtype;
+  f.k = k;
+  f.T = (k + TB - 1) / TB;
+  f.ldh = ldh;
+  f.ldm = ldm;
+  f.M = M;
+  f.info = static_cast<long long*>(ws);
+  // 16-byte copies need aligned row starts and even block widths
+  f.v16 = (ldm % 2 == 0) && (k % 2 == 0) && ((reinterpret_cast<uintptr_t>(M) & 15u) == 0);
+  f.ps = ps;
+  f.us = us;
+  f.panel_done = pd;
+  f.rest_done = rd;
+  return f;
+}
+
+// Enqueues the factorizations of `jobs` (1 or 2), forked from and joined back to s.
+int enqueue_factors(FactorJob* jobs, int nj, cudaStream_t s, DevStreams* ds) {
+  int rc = ensure_prepare_smem();
+  if (rc != GPTQ2D_OK) return rc;
+  bool ok = cudaEventRecord(ds->fork, s) == cudaSuccess;
+  for (int j = 0; j < nj && ok; ++j)
+    ok = cudaStreamWaitEvent(jobs[j].ps, ds->fork, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(jobs[j].us, ds->fork, 0) == cudaSuccess;
+  if (!ok) return GPTQ2D_ERR_CUDA;
+  for (int j = 0; j < nj && rc == GPTQ2D_OK; ++j) rc = enqueue_convert(jobs[j], ds->sms);
+  int steps = 0;
+  for (int j = 0; j < nj; ++j) steps = std::max(steps, jobs[j].T);
+  for (int st = 0; st < steps && rc == GPTQ2D_OK; ++st)
+    for (int j = 0; j < nj && rc == GPTQ2D_OK; ++j)
+      if (st < jobs[j].T) rc = enqueue_step(jobs[j], jobs[j].T - 1 - st, ds->sms);
+  cudaEvent_t joins[4] = {ds->join_hi, ds->join_lo, ds->join_hi2, ds->join_lo2};
+  for (int j = 0; j < nj && ok; ++j)
+    ok = cudaEventRecord(joins[2 * j], jobs[j].ps) == cudaSuccess &&
+         cudaEventRecord(joins[2 * j + 1], jobs[j].us) == cudaSuccess &&
+         cudaStreamWaitEvent(s, joins[2 * j], 0) == cudaSuccess &&
+         cudaStreamWaitEvent(s, joins[2 * j + 1], 0) == cudaSuccess;
+  if (rc != GPTQ2D_OK) return rc;
+  return ok ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
 }  // namespace
@@ -307,7 +523,13 @@ size_t prepare_ws_bytes(int64_t) { return 256; }
 
 int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
                    void* ws, cudaStream_t s) {
-  return prepare_enqueue(H, h_dtype, k, ldh, M, ldm, ws, s, sm_count());
+  DevStreams* ds = nullptr;
+  int rc = dev_streams(&ds);
+  if (rc != GPTQ2D_OK) return rc;
+  std::lock_guard<std::mutex> lk(ds->mu);
+  FactorJob f = make_job(H, h_dtype, k, ldh, M, ldm, ws, ds->hi, ds->lo, ds->panel_done[0],
+                         ds->rest_done[0]);
+  return enqueue_factors(&f, 1, s, ds);
 }
 
 int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
@@ -317,19 +539,18 @@ int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
   std::lock_guard<std::mutex> lk(ds->mu);
-  if (cudaEventRecord(ds->fork, s) != cudaSuccess ||
-      cudaStreamWaitEvent(ds->hi, ds->fork, 0) != cudaSuccess ||
-      cudaStreamWaitEvent(ds->lo, ds->fork, 0) != cudaSuccess)
-    return GPTQ2D_ERR_CUDA;
-  if (m > 0) rc = prepare_enqueue(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ds->hi, ds->sms);
-  if (rc == GPTQ2D_OK && n > 0)
-    rc = prepare_enqueue(H_R, h_dtype, (int)n, ldhr, M_R, ldmr, ws_r, ds->lo, ds->sms);
-  const bool ok = cudaEventRecord(ds->join_hi, ds->hi) == cudaSuccess &&
-                  cudaEventRecord(ds->join_lo, ds->lo) == cudaSuccess &&
-                  cudaStreamWaitEvent(s, ds->join_hi, 0) == cudaSuccess &&
-                  cudaStreamWaitEvent(s, ds->join_lo, 0) == cudaSuccess;
-  if (rc != GPTQ2D_OK) return rc;
-  return ok ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
+  FactorJob jobs[2];
+  int nj = 0;
+  if (m > 0)
+    jobs[nj++] = make_job(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ds->hi, ds->lo,
+                          ds->panel_done[0], ds->rest_done[0]);
+  if (n > 0) {
+    jobs[nj] = make_job(H_R, h_dtype, (int)n, ldhr, M_R, ldmr, ws_r, nj ? ds->hi2 : ds->hi,
+                        nj ? ds->lo2 : ds->lo, ds->panel_done[nj], ds->rest_done[nj]);
+    ++nj;
+  }
+  if (nj == 0) return GPTQ2D_OK;
+  return enqueue_factors(jobs, nj, s, ds);
 }
 
 }  // namespace gptq2d

@@ -35,7 +35,9 @@
 // sweep_kernel(D+1).  Exactness: every contribution to a tile comes from
 // earlier wavefronts (far: through P and E, near: pulled by the sweep) or from
 // the tile itself (the sweep).
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -44,7 +46,6 @@ namespace gptq2d {
 namespace {
 
 constexpr int SLD = TB + 4;  // 68 doubles: [row][k] tiles (conflict-free DMMA fragments)
-constexpr int KLD = TB + 8;  // 72 doubles: [k][col] tiles
 constexpr int SWEEP_THREADS = 512;
 constexpr int FAR_THREADS = 256;  // two independent 4-warp task streams
 
@@ -494,60 +495,64 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
 constexpr int MAX_GROUPS = 512;  // 2 groups per tile: 256 tiles per launch
 struct FarPlan {
   int D, I0, nt;
-  // start[g] = first task of group g in launch order; group g < nt holds the right
-  // tasks of tile I0+g, group g >= nt the down tasks of tile I0+g-nt.
+  int per_chunk;  // tasks per chunk
+  int* counter;   // chunk dispenser, zero before the first launch on this plan
+  // start[g] = first chunk of group g; group g < nt holds the right tasks of tile
+  // I0+g, group g >= nt the down tasks of tile I0+g-nt.
   int start[MAX_GROUPS + 1];
 };
 
-constexpr int FAR_GROUP_DOUBLES = TB * KLD + 2 * TB * SLD;  // shared operand + 2 task operands
+constexpr int FAR_GROUP_DOUBLES = 3 * TB * SLD;  // shared operand + 2 task operands
 constexpr int FAR_SMEM = 2 * FAR_GROUP_DOUBLES * (int)sizeof(double);
 
 __device__ __forceinline__ void group_barrier(int h) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(1 + h), "r"(128) : "memory");
 }
 
-// Persistent: each CTA runs two independent task streams (4 warps each, own shared
-// buffers, own named barrier).  Stream s of S = 2 gridDim.x takes tasks
-// [s T / S, (s+1) T / S) of the launch's T tasks, walking across groups.  A task is
-// one 64x64x64 DMMA product accumulated into a P or E tile; within a group the next
-// task's operand is copied in (cp.async) and the task's C tile is loaded into
-// registers while the previous copy lands.
+// Each CTA runs two independent task streams (4 warps each, own shared buffers, own
+// named barrier) that take chunks from the plan's dispenser until it runs dry, so
+// several launches on one plan (one beside the next sweep, one on the SMs that
+// sweep frees) share the work.  A chunk is a run of tasks of one group (same
+// shared operand); a task is one 64x64x64 DMMA product accumulated into a P or E
+// tile.  Within a chunk the next task's operand is copied in (cp.async) and the
+// task's C tile is loaded into registers while the previous copy lands.
 __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl) {
   extern __shared__ __align__(16) double sm[];
+  __shared__ int next_chunk[2];
   const int h = threadIdx.x >> 7, ht = threadIdx.x & 127;
-  double* Sh = sm + h * FAR_GROUP_DOUBLES;  // shared operand of the group's tasks
-  double* const Bf0 = Sh + TB * KLD;        // per-task operand, double-buffered
+  double* Sh = sm + h * FAR_GROUP_DOUBLES;  // shared operand of the chunk's tasks
+  double* const Bf0 = Sh + TB * SLD;        // per-task operand, double-buffered
   auto bufp = [&](int b) { return Bf0 + b * (TB * SLD); };
   const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
   const int64_t np = a.np;
   const int lane = ht & 31, warp = ht >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
-  const int64_t total = pl.start[2 * pl.nt];
-  const int64_t S = 2 * (int64_t)gridDim.x, sid = 2 * (int64_t)blockIdx.x + h;
-  const int t_end = (int)((sid + 1) * total / S);
-  int t_cur = (int)(sid * total / S);
+  const int nchunks = pl.start[2 * pl.nt];
 
-  while (t_cur < t_end) {
+  if (ht == 0) next_chunk[h] = atomicAdd(pl.counter, 1);
+  group_barrier(h);
+  int ch = next_chunk[h];
+  while (ch < nchunks) {
+    group_barrier(h);  // every thread has read next_chunk[h]
+    if (ht == 0) next_chunk[h] = atomicAdd(pl.counter, 1);
     int g;
     {
-      int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= t_cur
+      int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= ch
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (pl.start[mid] <= t_cur) lo = mid; else hi = mid;
+        if (pl.start[mid] <= ch) lo = mid; else hi = mid;
       }
       g = lo;
     }
     const bool down = g >= pl.nt;
     const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
-    const int first = t_cur - pl.start[g];
-    const int last = min(pl.start[g + 1], t_end) - pl.start[g];
-    t_cur = pl.start[g] + last;
+    const int count = down ? a.Tm - I - 2 : a.Tn - J - 2;
+    const int first = (ch - pl.start[g]) * pl.per_chunk;
+    const int last = min(first + pl.per_chunk, count);
 
     // shared operand: right -> dW[I,J] as [a][k]; down -> P[I,J] as [k][c]
-    if (!down)
-      tile_cp_async<128>(Sh, SLD, a.Dl + (int64_t)I * TB * np + J * TB, np, stream, ht);
-    else
-      tile_cp_async<128>(Sh, KLD, a.P + (int64_t)I * TB * np + J * TB, np, stream, ht);
+    tile_cp_async<128>(Sh, SLD, (down ? a.P : a.Dl) + (int64_t)I * TB * np + J * TB, np, stream,
+                       ht);
     auto task_operand = [&](int x) -> const double* {
       // right: Rh[(J+2+x) rows][J cols] as [c][k]; down: Lh[(I+2+x) rows][I cols] as [a][k]
       return down ? a.Lh + (int64_t)(I + 2 + x) * TB * a.mp + I * TB
@@ -583,7 +588,7 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
                        [&](int k, int c) { return B[c * SLD + k]; });
       else
         mma_64x64x64_w(acc, warp, [&](int r, int k) { return B[r * SLD + k]; },
-                       [&](int k, int c) { return Sh[k * KLD + c]; });
+                       [&](int k, int c) { return Sh[k * SLD + c]; });
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -595,6 +600,7 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
         }
       group_barrier(h);
     }
+    ch = next_chunk[h];
   }
 }
 
@@ -648,8 +654,16 @@ __global__ void zero_stats_kernel(gptq2d_stats* out) {
 struct WsLayout {
   int64_t mp, np;
   int Tm, Tn;
-  size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_part, total;
+  size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_part, off_cnt, total;
+  int n_cnt;  // far-field chunk dispensers, one per far plan
 };
+
+// Tiles of wavefront D, and the first of them.
+inline int wave_i0(int D, int Tn) { return D - (Tn - 1) > 0 ? D - (Tn - 1) : 0; }
+inline int wave_tiles(int D, int Tm, int Tn) {
+  if (D < 0 || D > Tm + Tn - 2) return 0;
+  return std::min(D, Tm - 1) - wave_i0(D, Tn) + 1;
+}
 
 WsLayout layout(int64_t m, int64_t n) {
   WsLayout L;
@@ -667,6 +681,10 @@ WsLayout layout(int64_t m, int64_t n) {
   L.off_dL = o; o += align256(L.mp * sizeof(double));
   L.off_dR = o; o += align256(L.np * sizeof(double));
   L.off_part = o; o += align256((size_t)L.Tm * L.Tn * sizeof(TileStat));
+  L.n_cnt = 0;
+  for (int D = 0; D < L.Tm + L.Tn - 1; ++D)
+    L.n_cnt += (wave_tiles(D, L.Tm, L.Tn) + MAX_GROUPS / 2 - 1) / (MAX_GROUPS / 2);
+  L.off_cnt = o; o += align256((size_t)L.n_cnt * sizeof(int));
   L.total = o;
   return L;
 }
@@ -698,17 +716,32 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
   ok = ok && cudaEventRecord(ds->setup, hi) == cudaSuccess &&
        cudaStreamWaitEvent(lo, ds->setup, 0) == cudaSuccess;
 
+  int* counters = reinterpret_cast<int*>(reinterpret_cast<char*>(a.P) - L.off_P + L.off_cnt);
+  ok = ok && cudaMemsetAsync(counters, 0, (size_t)L.n_cnt * sizeof(int), hi) == cudaSuccess;
   const int nd = a.Tm + a.Tn - 1;
+  const int sms = ds->sms;
+  int next_cnt = 0;
+  // far(D) = one launch on the low-priority stream beside sweep(D+1), on the SMs that
+  // sweep leaves free, plus (when the work outlasts that sweep) one on the
+  // high-priority stream after sweep(D+1), on the SMs it frees; both draw chunks from
+  // the same dispenser.  sweep(D+2) waits for both.
+  std::vector<FarPlan> prev_plans;  // far(D-1), still to get its second launch
+  int prev_b_ctas = 0;
   bool far_recorded[RING] = {};
   for (int D = 0; D < nd && ok; ++D) {
-    const int I0 = D - (a.Tn - 1) > 0 ? D - (a.Tn - 1) : 0;
-    const int I1 = D < a.Tm - 1 ? D : a.Tm - 1;
-    const int nt = I1 - I0 + 1;
+    const int I0 = wave_i0(D, a.Tn);
+    const int nt = wave_tiles(D, a.Tm, a.Tn);
     if (D >= 2 && far_recorded[(D - 2) % RING])
       ok = cudaStreamWaitEvent(hi, ds->far[(D - 2) % RING], 0) == cudaSuccess;
     far_recorded[D % RING] = false;
     GPTQ2D_LAUNCH(KC_SWEEP, hi,
                   sweep_kernel<TW><<<nt, SWEEP_THREADS, SW_SMEM, hi>>>(a, D, I0));
+    const bool b_launched = !prev_plans.empty();
+    for (const FarPlan& pl : prev_plans)
+      GPTQ2D_LAUNCH(KC_PROPAGATE, hi,
+                    far_kernel<<<prev_b_ctas, FAR_THREADS, FAR_SMEM, hi>>>(a, pl));
+    prev_plans.clear();
+
     // band products of wavefront D to tiles two or more tiles away
     long long total = 0;
     for (int i = 0; i < nt; ++i) {
@@ -716,28 +749,38 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
       total += std::max(0, a.Tn - J - 2) + std::max(0, a.Tm - I - 2);
     }
     if (total == 0) continue;
-    ok = ok && cudaEventRecord(ds->sw[D % RING], hi) == cudaSuccess &&
-         cudaStreamWaitEvent(lo, ds->sw[D % RING], 0) == cudaSuccess;
-    // far(D) runs beside sweep(D+1): leave that sweep's CTAs their SMs
-    const int nt_next = std::max(0, std::min(D + 1, a.Tm - 1) -
-                                        std::max(0, D + 1 - (a.Tn - 1)) + 1);
-    const int far_ctas = std::max(ds->sms / 4, ds->sms - nt_next);
-    for (int tb = 0; tb < nt && ok; tb += MAX_GROUPS / 2) {  // tiles per launch
+    const int nt_next = wave_tiles(D + 1, a.Tm, a.Tn);
+    const int a_ctas = std::max(sms / 4, sms - nt_next);
+    // a second launch pays when the work outlasts the next sweep on a_ctas SMs
+    // (about 24 tasks per CTA fit in one sweep's time)
+    const bool want_b = nt_next > 0 && total > 24LL * a_ctas;
+    const long long streams = 2LL * (a_ctas + (want_b ? nt_next : 0));
+    const int per_chunk = (int)std::min<long long>(8, std::max<long long>(1, total / (4 * streams)));
+    ok = ok && cudaEventRecord(b_launched ? ds->farb[(D - 1) % RING] : ds->sw[D % RING], hi) ==
+                   cudaSuccess &&
+         cudaStreamWaitEvent(lo, b_launched ? ds->farb[(D - 1) % RING] : ds->sw[D % RING], 0) ==
+             cudaSuccess;
+    for (int tb = 0; tb < nt && ok; tb += MAX_GROUPS / 2) {  // tiles per plan
       FarPlan pl;
       pl.D = D;
       pl.I0 = I0 + tb;
       pl.nt = std::min(nt - tb, MAX_GROUPS / 2);
-      int tasks = 0;
+      pl.per_chunk = per_chunk;
+      pl.counter = counters + next_cnt++;
+      int chunks = 0;
       for (int gidx = 0; gidx < 2 * pl.nt; ++gidx) {
         const int I = pl.I0 + (gidx < pl.nt ? gidx : gidx - pl.nt), J = D - I;
-        pl.start[gidx] = tasks;
-        tasks += gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
+        const int cnt = gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
+        pl.start[gidx] = chunks;
+        chunks += (cnt + per_chunk - 1) / per_chunk;
       }
-      pl.start[2 * pl.nt] = tasks;
-      const int ctas = std::min(far_ctas, (tasks + 1) / 2);
-      if (ctas > 0)
-        GPTQ2D_LAUNCH(KC_PROPAGATE, lo, far_kernel<<<ctas, FAR_THREADS, FAR_SMEM, lo>>>(a, pl));
+      pl.start[2 * pl.nt] = chunks;
+      if (chunks == 0) continue;
+      const int ctas = std::min(a_ctas, (chunks + 1) / 2);
+      GPTQ2D_LAUNCH(KC_PROPAGATE, lo, far_kernel<<<ctas, FAR_THREADS, FAR_SMEM, lo>>>(a, pl));
+      if (want_b && chunks > 2 * ctas) prev_plans.push_back(pl);
     }
+    prev_b_ctas = nt_next;
     ok = ok && cudaEventRecord(ds->far[D % RING], lo) == cudaSuccess;
     far_recorded[D % RING] = true;
   }

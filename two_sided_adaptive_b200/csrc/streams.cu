@@ -17,14 +17,21 @@ int dev_streams(DevStreams** out) {
     int least = 0, greatest = 0;
     if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ2D_ERR_CUDA;
     if (cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
-        cudaStreamCreateWithPriority(&d.lo, cudaStreamNonBlocking, least) != cudaSuccess)
+        cudaStreamCreateWithPriority(&d.lo, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&d.hi2, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&d.lo2, cudaStreamNonBlocking, least) != cudaSuccess)
       return GPTQ2D_ERR_CUDA;
-    cudaEvent_t* evs[] = {&d.fork, &d.setup, &d.join_hi, &d.join_lo};
+    cudaEvent_t* evs[] = {&d.fork, &d.setup, &d.join_hi, &d.join_lo, &d.join_hi2, &d.join_lo2};
     for (auto* e : evs)
       if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GPTQ2D_ERR_CUDA;
     for (int r = 0; r < RING; ++r)
       if (cudaEventCreateWithFlags(&d.sw[r], cudaEventDisableTiming) != cudaSuccess ||
-          cudaEventCreateWithFlags(&d.far[r], cudaEventDisableTiming) != cudaSuccess)
+          cudaEventCreateWithFlags(&d.far[r], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.farb[r], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.panel_done[0][r], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.panel_done[1][r], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.rest_done[0][r], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&d.rest_done[1][r], cudaEventDisableTiming) != cudaSuccess)
         return GPTQ2D_ERR_CUDA;
     cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     d.ready = true;
