@@ -87,8 +87,9 @@ int64_t gptq2d_launch_count(void);
  * library launches is bracketed by a pair of CUDA events recorded on the
  * launching stream; events are created on first use and recycled.  Kernel
  * classes: 0 factor panel (diagonal block + block-row solve), 1 factor trailing
- * update, 2 anti-diagonal tile sweep, 3 band products (feedback propagation),
- * 4 other (conversion, diagonals, statistics). */
+ * update, 2 anti-diagonal tile sweep (near feedback included), 3 band products
+ * to tiles two or more tiles away (far-field feedback), 4 other (conversion,
+ * diagonals, statistics). */
 void gptq2d_profile_enable(int on);
 /* Number of recorded launches of `kernel_class` and their summed device time
  * in milliseconds (waits for the recorded events).  GPTQ2D_ERR_INVALID_ARG for

@@ -23,7 +23,7 @@ enum KernelClass {
   KC_PREP_PANEL = 0,     // factor preparation: diagonal block + block-row solve
   KC_PREP_TRAILING = 1,  // factor preparation: rank-64 trailing update
   KC_SWEEP = 2,          // anti-diagonal tile sweep
-  KC_PROPAGATE = 3,      // band products (right / down feedback)
+  KC_PROPAGATE = 3,      // band products to tiles two or more tiles away
   KC_OTHER = 4,          // conversions, diagonals, statistics
   KC_COUNT = 5
 };

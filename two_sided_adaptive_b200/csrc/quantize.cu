@@ -97,16 +97,11 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
-__device__ __forceinline__ double2 ld_hint(const double* p, uint64_t pol) {
-  double2 v;
-  asm volatile("ld.global.L2::cache_hint.v2.f64 {%0,%1}, [%2], %3;\n"
-               : "=d"(v.x), "=d"(v.y)
-               : "l"(p), "l"(pol));
-  return v;
-}
-__device__ __forceinline__ void st_hint(double* p, double2 v, uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.v2.f64 [%0], {%1,%2}, %3;\n" ::"l"(p), "d"(v.x), "d"(v.y),
-               "l"(pol));
+// C += v without reading C back: each C element gets one contribution per
+// far-field launch and launches on one plan are stream-ordered, so the sum is
+// the same as a load, add and store.
+__device__ __forceinline__ void red_add(double* p, double v) {
+  asm volatile("red.global.add.f64 [%0], %1;\n" ::"l"(p), "d"(v) : "memory");
 }
 
 // Copies a 64x64 fp64 tile (row stride `ld` elements, 16-byte aligned rows) into
@@ -235,85 +230,102 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   const int64_t np = a.np;
   const int64_t ts = (int64_t)r0 * np + c0;  // tile origin in the workspace matrices
 
-  // ---- right feedback: P (far part, in HBM) + dW[I,J-1] Rh[J,J-1]^T (pulled); staged in Rt/Lt
-  {
-    double acc[2][2][2] = {};
-    if (J > 0) {
-      const double* A = a.Dl + ts - TB;                       // [a][k]
-      const double* B = a.Rh + (int64_t)c0 * np + (c0 - TB);  // [c][k]
-      for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
-        const int r = x >> 5, k2 = (x & 31) * 2;
-        *reinterpret_cast<double2*>(Rt + r * SLD + k2) =
-            *reinterpret_cast<const double2*>(A + (int64_t)r * np + k2);
-        *reinterpret_cast<double2*>(Lt + r * SLD + k2) =
-            *reinterpret_cast<const double2*>(B + (int64_t)r * np + k2);
-      }
-      __syncthreads();
-      mma16w(acc, [&](int r, int kk) { return Rt[r * SLD + kk]; },
-             [&](int kk, int c) { return Lt[c * SLD + kk]; });
+  // ---- near-neighbour feedback, pulled from the tiles finished one wavefront ago:
+  //   right: P += dW[I,J-1] Rh[J,J-1]^T      (warps 0..7)
+  //   down:  V += Lh[I,I-1] P_final[I-1,J]   (warps 8..15)
+  // All operand tiles and the tile's own P and E arrive in two async batches; the
+  // two products run side by side on the DMMA units.
+  const bool has_r = J > 0, has_d = I > 0;
+  for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+    const int r = x >> 5, c2 = (x & 31) * 2;
+    if (has_r) {
+      cp_async16_zfill(Dt + r * SLD + c2, a.Dl + ts - TB + (int64_t)r * np + c2, true);
+      cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 - TB + c2, true);
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t4;
-        const double2 p = *reinterpret_cast<const double2*>(a.P + ts + (int64_t)r * np + c);
-        Pt[r * SLD + c] = p.x + acc[i][j][0];
-        Pt[r * SLD + c + 1] = p.y + acc[i][j][1];
-      }
-    __syncthreads();
-  }
-  // ---- down feedback: V = W + E (far part) + Lh[I,I-1] P_final[I-1,J] (pulled); W -> Dt
-  {
-    double acc[2][2][2] = {};
-    if (I > 0) {
-      const double* A = a.Lh + (int64_t)r0 * a.mp + (r0 - TB);  // [a][k]
-      const double* B = a.P + ts - (int64_t)TB * np;            // [k][c]: final P of tile (I-1, J)
-      for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
-        const int r = x >> 5, k2 = (x & 31) * 2;
-        *reinterpret_cast<double2*>(Rt + r * SLD + k2) =
-            *reinterpret_cast<const double2*>(A + (int64_t)r * a.mp + k2);
-        const double2 b = *reinterpret_cast<const double2*>(B + (int64_t)r * np + k2);
-        Lt[k2 * SLD + r] = b.x;  // transposed: [c][k]
-        Lt[(k2 + 1) * SLD + r] = b.y;
-      }
-      __syncthreads();
-      mma16w(acc, [&](int r, int kk) { return Rt[r * SLD + kk]; },
-             [&](int kk, int c) { return Lt[c * SLD + kk]; });
+    if (has_d) {
+      cp_async16_zfill(Lt + r * SLD + c2, a.Lh + (int64_t)(r0 + r) * a.mp + r0 - TB + c2, true);
+      cp_async16_zfill(Tq + r * SLD + c2, a.P + ts - (int64_t)TB * np + (int64_t)r * np + c2, true);
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int r = wr + i * 8 + g, c = wc + j * 8 + 2 * t4;
-        const double2 e = *reinterpret_cast<const double2*>(a.E + ts + (int64_t)r * np + c);
-        double w0 = 0.0, w1 = 0.0;
-        if (r < rows) {
-          const TW* wrow = static_cast<const TW*>(a.W) + (int64_t)(r0 + r) * a.ldw + c0;
-          if (c < cols) w0 = to_f64(wrow[c]);
-          if (c + 1 < cols) w1 = to_f64(wrow[c + 1]);
-        }
-        Vt[r * SLD + c] = w0 + e.x + acc[i][j][0];
-        Vt[r * SLD + c + 1] = w1 + e.y + acc[i][j][1];
-        Dt[r * SLD + c] = w0;
-        Dt[r * SLD + c + 1] = w1;
-      }
-    __syncthreads();
   }
-  // ---- the tile's row scales and their reciprocals
-  __shared__ double Ss[TB], Si[TB];
+  cp_async_commit_group();
+  for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+    const int r = x >> 5, c2 = (x & 31) * 2;
+    cp_async16_zfill(Pt + r * SLD + c2, a.P + ts + (int64_t)r * np + c2, true);
+    cp_async16_zfill(Vt + r * SLD + c2, a.E + ts + (int64_t)r * np + c2, true);
+  }
+  cp_async_commit_group();
+  // row scales, their reciprocals and the factor diagonals of the tile
+  __shared__ double Ss[TB], Si[TB], Sdl[TB], Sdr[TB];
   if (tid < TB) {
     const double sv = tid < rows ? (double)a.scales[r0 + tid] : 1.0;
     Ss[tid] = sv;
     Si[tid] = 1.0 / sv;
+    Sdl[tid] = a.dL[r0 + tid];
+    Sdr[tid] = a.dR[c0 + tid];
   }
-  // ---- diagonal blocks of the normalised factors
+  // W of the tile (zero outside the matrix)
+  constexpr int WPT = TB * TB / SWEEP_THREADS;
+  double wv[WPT];
+#pragma unroll
+  for (int u = 0; u < WPT; ++u) {
+    const int x = tid + u * SWEEP_THREADS, r = x >> 6, c = x & 63;
+    wv[u] = (r < rows && c < cols)
+                ? to_f64(static_cast<const TW*>(a.W)[(int64_t)(r0 + r) * a.ldw + c0 + c])
+                : 0.0;
+  }
+  cp_async_wait_group<1>();
+  __syncthreads();
+  {
+    // warp w8 = warp % 8 owns rows (w8>>1)*16..+16, columns (w8&1)*32..+32
+    const int w8 = warp & 7, nr = (w8 >> 1) * 16, nc = (w8 & 1) * 32;
+    const bool right = warp < 8;
+    double acc[2][4][2] = {};
+    if (right ? has_r : has_d) {
+#pragma unroll 4
+      for (int kk = 0; kk < TB; kk += 4) {
+        double av[2], bv[4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = nr + i * 8 + g;
+          av[i] = right ? Dt[r * SLD + kk + t4] : Lt[r * SLD + kk + t4];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = nc + j * 8 + g;
+          bv[j] = right ? Rt[c * SLD + kk + t4] : Tq[(kk + t4) * SLD + c];
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
+      }
+    }
+    cp_async_wait_group<0>();
+    __syncthreads();
+    double* C = right ? Pt : Vt;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        double* c = C + (nr + i * 8 + g) * SLD + nc + j * 8 + 2 * t4;
+        c[0] += acc[i][j][0];
+        c[1] += acc[i][j][1];
+      }
+  }
+  __syncthreads();
+  // ---- W -> Dt, V += W; diagonal blocks of the normalised factors -> Rt, Lt
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
-    const int r = x >> 5, k2 = (x & 31) * 2;
-    cp_async16_zfill(Rt + r * SLD + k2, a.Rh + (int64_t)(c0 + r) * np + c0 + k2, true);
-    cp_async16_zfill(Lt + r * SLD + k2, a.Lh + (int64_t)(r0 + r) * a.mp + r0 + k2, true);
+    const int r = x >> 5, c2 = (x & 31) * 2;
+    cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 + c2, true);
+    cp_async16_zfill(Lt + r * SLD + c2, a.Lh + (int64_t)(r0 + r) * a.mp + r0 + c2, true);
   }
   cp_async_commit_group();
+#pragma unroll
+  for (int u = 0; u < WPT; ++u) {
+    const int x = tid + u * SWEEP_THREADS, r = x >> 6, c = x & 63;
+    Dt[r * SLD + c] = wv[u];
+    Vt[r * SLD + c] += wv[u];
+  }
   cp_async_wait_group<0>();
   __syncthreads();
 
@@ -451,7 +463,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;
       const double qv = qr < a.lo ? a.lo : (qr > a.hi ? a.hi : qr);
       a.Q[(int64_t)(r0 + r) * a.ldq + c0 + c] = (int8_t)(int)qv;
-      const double res = a.dL[r0 + r] * a.dR[c0 + c] * sr * (tq - qv);
+      const double res = Sdl[r] * Sdr[c] * sr * (tq - qv);
       loss += res * res;
       ncl += (qv != qr);
       const double qn = qr + (tq >= qr ? 1.0 : -1.0);
@@ -494,7 +506,9 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
 // ---------------------------------------------------------------------------
 constexpr int MAX_GROUPS = 512;  // 2 groups per tile: 256 tiles per launch
 struct FarPlan {
-  int D, I0, nt;
+  int D, I0, nt;  // source tiles: I0..I0+nt-1 of wavefront D
+  int dist0;      // distance of the first target tile (2: far field, 1: near neighbours)
+  int cap;        // most tasks per group
   int per_chunk;  // tasks per chunk
   int* counter;   // chunk dispenser, zero before the first launch on this plan
   // start[g] = first chunk of group g; group g < nt holds the right tasks of tile
@@ -513,9 +527,9 @@ __device__ __forceinline__ void group_barrier(int h) {
 // named barrier) that take chunks from the plan's dispenser until it runs dry, so
 // several launches on one plan (one beside the next sweep, one on the SMs that
 // sweep frees) share the work.  A chunk is a run of tasks of one group (same
-// shared operand); a task is one 64x64x64 DMMA product accumulated into a P or E
-// tile.  Within a chunk the next task's operand is copied in (cp.async) and the
-// task's C tile is loaded into registers while the previous copy lands.
+// shared operand); a task is one 64x64x64 DMMA product added into a P or E tile
+// by reductions in L2 (red_add).  Within a chunk the next task's operand is
+// copied in (cp.async) while the current product runs.
 __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl) {
   extern __shared__ __align__(16) double sm[];
   __shared__ int next_chunk[2];
@@ -546,7 +560,7 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
     }
     const bool down = g >= pl.nt;
     const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
-    const int count = down ? a.Tm - I - 2 : a.Tn - J - 2;
+    const int count = min(pl.cap, down ? a.Tm - I - pl.dist0 : a.Tn - J - pl.dist0);
     const int first = (ch - pl.start[g]) * pl.per_chunk;
     const int last = min(first + pl.per_chunk, count);
 
@@ -554,13 +568,13 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
     tile_cp_async<128>(Sh, SLD, (down ? a.P : a.Dl) + (int64_t)I * TB * np + J * TB, np, stream,
                        ht);
     auto task_operand = [&](int x) -> const double* {
-      // right: Rh[(J+2+x) rows][J cols] as [c][k]; down: Lh[(I+2+x) rows][I cols] as [a][k]
-      return down ? a.Lh + (int64_t)(I + 2 + x) * TB * a.mp + I * TB
-                  : a.Rh + (int64_t)(J + 2 + x) * TB * np + J * TB;
+      // right: Rh[(J+d+x) rows][J cols] as [c][k]; down: Lh[(I+d+x) rows][I cols] as [a][k]
+      return down ? a.Lh + (int64_t)(I + pl.dist0 + x) * TB * a.mp + I * TB
+                  : a.Rh + (int64_t)(J + pl.dist0 + x) * TB * np + J * TB;
     };
     auto task_c = [&](int x) -> double* {
-      return down ? a.E + (int64_t)(I + 2 + x) * TB * np + J * TB
-                  : a.P + (int64_t)I * TB * np + (J + 2 + x) * TB;
+      return down ? a.E + (int64_t)(I + pl.dist0 + x) * TB * np + J * TB
+                  : a.P + (int64_t)I * TB * np + (J + pl.dist0 + x) * TB;
     };
     const int64_t opld = down ? a.mp : np;
     tile_cp_async<128>(bufp(0), SLD, task_operand(first), opld, keep, ht);
@@ -573,12 +587,6 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
         cp_async_commit();
       }
       double* C = task_c(x);
-      double2 cv[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          cv[i][j] = ld_hint(C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4, stream);
       if (x + 1 < last) cp_async_wait<1>(); else cp_async_wait<0>();
       group_barrier(h);
       double acc[4][4][2] = {};
@@ -593,10 +601,9 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          double2 v = cv[i][j];
-          v.x += acc[i][j][0];
-          v.y += acc[i][j][1];
-          st_hint(C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4, v, stream);
+          double* p = C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4;
+          red_add(p, acc[i][j][0]);
+          red_add(p + 1, acc[i][j][1]);
         }
       group_barrier(h);
     }
@@ -655,7 +662,7 @@ struct WsLayout {
   int64_t mp, np;
   int Tm, Tn;
   size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_part, off_cnt, total;
-  int n_cnt;  // far-field chunk dispensers, one per far plan
+  int n_cnt;  // chunk dispensers, one per far-field plan
 };
 
 // Tiles of wavefront D, and the first of them.
@@ -682,7 +689,7 @@ WsLayout layout(int64_t m, int64_t n) {
   L.off_dR = o; o += align256(L.np * sizeof(double));
   L.off_part = o; o += align256((size_t)L.Tm * L.Tn * sizeof(TileStat));
   L.n_cnt = 0;
-  for (int D = 0; D < L.Tm + L.Tn - 1; ++D)
+  for (int D = 0; D < L.Tm + L.Tn - 1; ++D)  // one far-field plan per MAX_GROUPS/2 tiles
     L.n_cnt += (wave_tiles(D, L.Tm, L.Tn) + MAX_GROUPS / 2 - 1) / (MAX_GROUPS / 2);
   L.off_cnt = o; o += align256((size_t)L.n_cnt * sizeof(int));
   L.total = o;
@@ -765,6 +772,8 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
       pl.D = D;
       pl.I0 = I0 + tb;
       pl.nt = std::min(nt - tb, MAX_GROUPS / 2);
+      pl.dist0 = 2;
+      pl.cap = 1 << 30;
       pl.per_chunk = per_chunk;
       pl.counter = counters + next_cnt++;
       int chunks = 0;
