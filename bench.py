@@ -313,14 +313,33 @@ def run_ours(args, rank, world, local_rank):
     ms_step = ms / args.steps
     value = aggregate_value(m, n, world, ms_step)
 
-    # per-kernel device time of one more step, CUDA events around each launch on its stream
+    # per-kernel device time: the same K steps again with a CUDA event pair around every
+    # launch on its own stream; per-step figures are the totals / K
     g.profile_reset()
     g.profile_enable(True)
-    step()
+    for _ in range(args.steps):
+        step()
     torch.cuda.synchronize()
-    prof = g.profile_read()
+    prof = {k: (v[0] / args.steps, v[1] / args.steps) for k, v in g.profile_read().items()}
     g.profile_enable(False)
     g.profile_reset()
+
+    # the two calls of a step on their own (events on the caller stream)
+    def timed(fn, reps):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(reps):
+            fn()
+        f1.record()
+        torch.cuda.synchronize()
+        return f0.elapsed_time(f1) / reps
+    reps = max(3, min(args.steps, 10))
+    phases = {
+        "prepare_pair": timed(lambda: g.prepare_pair(H_L, H_R, out_l=M_L, out_r=M_R,
+                                                     workspace=wsP, check=False), reps),
+        "quantize": timed(lambda: g.quantize(W, M_L, M_R, s, pb.bits, pb.clamp, out=Q, stats=st,
+                                             workspace=wsQ), reps),
+    }
 
     # end to end through the C ABI from pinned host memory
     e2e = None
@@ -368,8 +387,13 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
                 "traffic": traffic, "launches_per_step": nl, "kernel_ms_per_step": tms,
                 "algorithmic_flops_per_launch": work[dom] / nl if work[dom] else None,
-                "peak_source": "cuBLAS DGEMM 8192^3 (torch.matmul fp64), best of 5, measured in this run"}
+                "peak_source": "cuBLAS DGEMM 8192^3 (torch.matmul fp64), best of 5, measured in this run",
+                "timing": "CUDA events around every launch of this kernel over K profiled steps "
+                          "run right after the timed region, averaged per launch"}
     breakdown = {k: {"launches": v[0], "ms": round(v[1], 4)} for k, v in prof.items()}
+    phase_out = {k: {"ms": round(v, 4), "entries_per_s": m * n / (v * 1e-3)} for k, v in phases.items()}
+    phase_out["quantize"]["fp64_tflops"] = m * n * (m + n) / (phases["quantize"] * 1e-3) / 1e12
+    phase_out["quantize"]["frac_of_dgemm"] = phase_out["quantize"]["fp64_tflops"] / peak
     total_flops = m * n * (m + n) + prep_flops(m) + prep_flops(n)
     out = {
         "metric": METRIC, "value": value, "unit": "entries/s", "n_gpus": world,
@@ -391,6 +415,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "stats": stats,
         "breakdown_ms_per_step": breakdown,
+        "phases": phase_out,
         "whole_step_fp64_tflops": total_flops / (ms_step * 1e-3) / 1e12,
     }
     if world == 1 and not args.no_cpu_baseline:
