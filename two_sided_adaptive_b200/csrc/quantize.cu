@@ -23,18 +23,25 @@
 // at a time, on two internal streams forked from the caller's stream:
 //   high priority  sweep_kernel(D): one CTA per tile.  It first pulls the
 //                  contributions of its left and upper neighbours (wavefront
-//                  D-1) with FP64 tensor-core products, then runs the tile's
-//                  127 local anti-diagonals in shared memory, applying the
-//                  rank-one separable update of every rounded entry as a row
-//                  push (along Rh) and a column push (along Lh).
+//                  D-1) with two FP64 tensor-core products run side by side,
+//                  then sweeps the tile as 8 x 8 sub-tiles: the sub-tiles of one
+//                  sub-wavefront go to one warp each, which walks the 15 local
+//                  anti-diagonals warp-synchronously (row and column pushes by
+//                  shuffles); between sub-wavefronts the finished sub-tiles push
+//                  to their neighbours with 8x8x8 DMMA products, and the pushes
+//                  two or more sub-tiles away run on helper warps during the
+//                  next sub-wavefront.
 //   low priority   far_kernel(D): the band products that carry the tiles of
 //                  wavefront D to tiles two or more tiles away (to the right:
-//                  P += dW Rh^T; below: E += Lh P), 64x64x64 DMMA tiles with
-//                  double-buffered cp.async operand streams.
-// sweep_kernel(D) waits for far_kernel(D-2) only, so far_kernel(D) runs under
-// sweep_kernel(D+1).  Exactness: every contribution to a tile comes from
-// earlier wavefronts (far: through P and E, near: pulled by the sweep) or from
-// the tile itself (the sweep).
+//                  P += dW Rh^T; below: E += Lh P), 64x64x64 DMMA tasks handed
+//                  out in chunks by a dispenser.  One launch runs beside
+//                  sweep_kernel(D+1) on the SMs that sweep leaves free; when the
+//                  work outlasts that sweep a second launch on the high-priority
+//                  stream, after sweep_kernel(D+1), takes the rest on the SMs the
+//                  sweep frees.
+// sweep_kernel(D) waits for far_kernel(D-2) only.  Exactness: every
+// contribution to a tile comes from earlier wavefronts (far: through P and E,
+// near: pulled by the sweep) or from the tile itself (the sweep).
 #include <algorithm>
 #include <mutex>
 #include <vector>
