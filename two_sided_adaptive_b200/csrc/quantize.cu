@@ -54,7 +54,6 @@ namespace {
 
 constexpr int SLD = TB + 4;  // 68 doubles: [row][k] tiles (conflict-free DMMA fragments)
 constexpr int SWEEP_THREADS = 512;
-constexpr int FAR_THREADS = 256;  // two independent 4-warp task streams
 
 struct QArgs {
   const void* W;
@@ -69,6 +68,7 @@ struct QArgs {
   int clamp;
   int8_t* Q;
   int64_t ldq;
+  int* err;       // nonzero: a bounded wait in a kernel timed out
   double* Lh;     // mp x mp
   double* Rh;     // np x np
   double* P;      // mp x np
@@ -109,6 +109,56 @@ __device__ __forceinline__ void cp_async_wait() {
 // the same as a load, add and store.
 __device__ __forceinline__ void red_add(double* p, double v) {
   asm volatile("red.global.add.f64 [%0], %1;\n" ::"l"(p), "d"(v) : "memory");
+}
+
+// ---- mbarriers and bulk copies (the far-field kernel's producer/consumer pipeline)
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+// Waits for the phase of `bar` with the given parity to complete; gives up after
+// kWaitLimitNs and returns false (the caller reports a timeout).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+// One bulk copy global -> shared (TMA engine, no multicast), completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar,
+                                         uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;\n" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
 }
 
 // Copies a 64x64 fp64 tile (row stride `ld` elements, 16-byte aligned rows) into
@@ -523,104 +573,221 @@ struct FarPlan {
   int start[MAX_GROUPS + 1];
 };
 
-constexpr int FAR_GROUP_DOUBLES = 3 * TB * SLD;  // shared operand + 2 task operands
-constexpr int FAR_SMEM = 2 * FAR_GROUP_DOUBLES * (int)sizeof(double);
+constexpr int FAR_CONS = 128;                    // consumer threads per task stream (4 warps)
+constexpr int FAR_THREADS = 2 * FAR_CONS + 64;   // 2 streams + one producer warp each
+constexpr int FAR_SLOTS = 3;                     // 64x64 tile buffers per stream
+constexpr int FAR_DQ = 4;                        // task descriptors in flight per stream
+constexpr int FAR_TILE_BYTES = TB * TB * (int)sizeof(double);
+constexpr int FAR_STREAM_DOUBLES = FAR_SLOTS * TB * SLD;
+constexpr int FAR_SMEM = 2 * FAR_STREAM_DOUBLES * (int)sizeof(double);
 
-__device__ __forceinline__ void group_barrier(int h) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(1 + h), "r"(128) : "memory");
-}
+// One task for the consumers: the slots of its operands and its target tile.
+struct FarDesc {
+  double* C;      // 64x64 target tile (row stride np)
+  int task_slot;  // buffer holding R^[J+d+x, J] ([c][k]) or L^[I+d+x, I] ([a][k])
+  int sh_slot;    // buffer holding dW[I,J] ([a][k]) or P_final[I,J] ([k][c])
+  int flags;      // FD_* bits
+};
+constexpr int FD_DOWN = 1, FD_FIRST = 2, FD_LAST = 4, FD_END = 8;
 
-// Each CTA runs two independent task streams (4 warps each, own shared buffers, own
-// named barrier) that take chunks from the plan's dispenser until it runs dry, so
-// several launches on one plan (one beside the next sweep, one on the SMs that
-// sweep frees) share the work.  A chunk is a run of tasks of one group (same
-// shared operand); a task is one 64x64x64 DMMA product added into a P or E tile
-// by reductions in L2 (red_add).  Within a chunk the next task's operand is
-// copied in (cp.async) while the current product runs.
+// mbarriers of one stream:
+//   full[s]  : producer's expect_tx + the 64 row copies into slot s (count 1)
+//   empty[s] : one arrival per consumer warp when it is done with slot s (count 4)
+//   dqf[e]   : descriptor e written (count 1); dqe[e]: descriptor e read (count 4)
+struct FarSync {
+  uint64_t full[FAR_SLOTS], empty[FAR_SLOTS], dqf[FAR_DQ], dqe[FAR_DQ];
+  FarDesc desc[FAR_DQ];
+};
+
+// Each CTA runs two independent task streams.  A stream is one producer warp and
+// four consumer warps.  The producer takes chunks from the plan's dispenser (a
+// chunk is a run of tasks of one source tile and direction, which share one
+// operand) and brings every operand tile in with 512-byte bulk row copies (TMA
+// engine) that complete on the slot's mbarrier.  Slots are handed out in the
+// order the consumers free them, so a chunk's shared operand is fetched while
+// the previous chunk still runs.  The consumers wait for a descriptor and its
+// slots, run the 64x64x64 DMMA product, free the slots, and add the product into
+// P or E by reductions in L2 (red_add: each element gets one contribution per
+// launch, so the sum equals a load, add and store).  Several launches on one plan
+// (one beside the next sweep, one on the SMs that sweep frees) share the
+// dispenser.  Every wait gives up after kWaitLimitNs, sets *a.err and leaves the
+// kernel (the call then reports GPTQ2D_ERR_TIMEOUT); a producer that gives up
+// first waits, again bounded, for the copies it has in flight.
 __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl) {
-  extern __shared__ __align__(16) double sm[];
-  __shared__ int next_chunk[2];
-  const int h = threadIdx.x >> 7, ht = threadIdx.x & 127;
-  double* Sh = sm + h * FAR_GROUP_DOUBLES;  // shared operand of the chunk's tasks
-  double* const Bf0 = Sh + TB * SLD;        // per-task operand, double-buffered
-  auto bufp = [&](int b) { return Bf0 + b * (TB * SLD); };
-  const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
-  const int64_t np = a.np;
-  const int lane = ht & 31, warp = ht >> 5, g8 = lane >> 2, t4 = lane & 3;
-  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
-  const int nchunks = pl.start[2 * pl.nt];
-
-  if (ht == 0) next_chunk[h] = atomicAdd(pl.counter, 1);
-  group_barrier(h);
-  int ch = next_chunk[h];
-  while (ch < nchunks) {
-    group_barrier(h);  // every thread has read next_chunk[h]
-    if (ht == 0) next_chunk[h] = atomicAdd(pl.counter, 1);
-    int g;
-    {
-      int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= ch
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (pl.start[mid] <= ch) lo = mid; else hi = mid;
-      }
-      g = lo;
+  extern __shared__ __align__(128) double sm[];
+  __shared__ FarSync sync[2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool producer = warp >= 8;
+  const int h = producer ? warp - 8 : warp >> 2;  // task stream
+  double* const Slot0 = sm + h * FAR_STREAM_DOUBLES;
+  auto slot_ptr = [&](int s) { return Slot0 + s * (TB * SLD); };
+  FarSync& S = sync[h];
+  if (threadIdx.x < 2) {
+    FarSync& T = sync[threadIdx.x];
+    for (int s = 0; s < FAR_SLOTS; ++s) {
+      mbar_init(&T.full[s], 1);
+      mbar_init(&T.empty[s], 4);
     }
-    const bool down = g >= pl.nt;
-    const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
-    const int count = min(pl.cap, down ? a.Tm - I - pl.dist0 : a.Tn - J - pl.dist0);
-    const int first = (ch - pl.start[g]) * pl.per_chunk;
-    const int last = min(first + pl.per_chunk, count);
+    for (int e = 0; e < FAR_DQ; ++e) {
+      mbar_init(&T.dqf[e], 1);
+      mbar_init(&T.dqe[e], 4);
+    }
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  __syncthreads();
+  const int64_t np = a.np;
 
-    // shared operand: right -> dW[I,J] as [a][k]; down -> P[I,J] as [k][c]
-    tile_cp_async<128>(Sh, SLD, (down ? a.P : a.Dl) + (int64_t)I * TB * np + J * TB, np, stream,
-                       ht);
-    auto task_operand = [&](int x) -> const double* {
-      // right: Rh[(J+d+x) rows][J cols] as [c][k]; down: Lh[(I+d+x) rows][I cols] as [a][k]
-      return down ? a.Lh + (int64_t)(I + pl.dist0 + x) * TB * a.mp + I * TB
-                  : a.Rh + (int64_t)(J + pl.dist0 + x) * TB * np + J * TB;
+  if (producer) {
+    const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+    const int nchunks = pl.start[2 * pl.nt];
+    int fills[FAR_SLOTS] = {0, 0, 0};  // fills issued per slot
+    int fifo[4] = {0, 1, 2, 0};        // slots in the order the consumers free them
+    int fh = 0, ft = FAR_SLOTS, nd = 0;
+    bool ok = true;
+    // the next slot in release order, once the consumers have freed it
+    auto acquire = [&](int& s) -> bool {
+      s = fifo[fh & 3];
+      ++fh;
+      const int k = fills[s];
+      if (k > 0 && !mbar_wait(&S.empty[s], (k - 1) & 1)) return false;
+      fills[s] = k + 1;
+      return true;
     };
-    auto task_c = [&](int x) -> double* {
-      return down ? a.E + (int64_t)(I + pl.dist0 + x) * TB * np + J * TB
-                  : a.P + (int64_t)I * TB * np + (J + pl.dist0 + x) * TB;
+    auto release_later = [&](int s) {
+      fifo[ft & 3] = s;
+      ++ft;
     };
-    const int64_t opld = down ? a.mp : np;
-    tile_cp_async<128>(bufp(0), SLD, task_operand(first), opld, keep, ht);
-    cp_async_commit();
-
-    for (int x = first; x < last; ++x) {
-      const int buf = (x - first) & 1;
-      if (x + 1 < last) {
-        tile_cp_async<128>(bufp(buf ^ 1), SLD, task_operand(x + 1), opld, keep, ht);
-        cp_async_commit();
+    auto fill = [&](int s, const double* src, int64_t ld, uint64_t pol) {
+      if (lane == 0) mbar_arrive_expect_tx(&S.full[s], FAR_TILE_BYTES);
+      __syncwarp();
+      double* dst = slot_ptr(s);
+      for (int r = lane; r < TB; r += 32)
+        bulk_g2s(dst + r * SLD, src + (int64_t)r * ld, TB * sizeof(double), &S.full[s], pol);
+    };
+    auto put_desc = [&](double* C, int ts, int shs, int flags) -> bool {
+      const int e = nd % FAR_DQ, k = nd / FAR_DQ;
+      if (k > 0 && !mbar_wait(&S.dqe[e], (k - 1) & 1)) return false;
+      if (lane == 0) {
+        S.desc[e].C = C;
+        S.desc[e].task_slot = ts;
+        S.desc[e].sh_slot = shs;
+        S.desc[e].flags = flags;
+        mbar_arrive(&S.dqf[e]);
       }
-      double* C = task_c(x);
-      if (x + 1 < last) cp_async_wait<1>(); else cp_async_wait<0>();
-      group_barrier(h);
-      double acc[4][4][2] = {};
-      const double* B = bufp(buf);
-      if (!down)
-        mma_64x64x64_w(acc, warp, [&](int r, int k) { return Sh[r * SLD + k]; },
-                       [&](int k, int c) { return B[c * SLD + k]; });
-      else
-        mma_64x64x64_w(acc, warp, [&](int r, int k) { return B[r * SLD + k]; },
-                       [&](int k, int c) { return Sh[k * SLD + c]; });
+      __syncwarp();
+      ++nd;
+      return true;
+    };
+    while (ok) {
+      int ch = 0;
+      if (lane == 0) ch = atomicAdd(pl.counter, 1);
+      ch = __shfl_sync(0xffffffffu, ch, 0);
+      if (ch >= nchunks) break;
+      int g;
+      {
+        int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= ch
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (pl.start[mid] <= ch) lo = mid; else hi = mid;
+        }
+        g = lo;
+      }
+      const bool down = g >= pl.nt;
+      const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
+      const int count = min(pl.cap, down ? a.Tm - I - pl.dist0 : a.Tn - J - pl.dist0);
+      const int first = (ch - pl.start[g]) * pl.per_chunk;
+      const int last = min(first + pl.per_chunk, count);
+      // shared operand: right -> dW[I,J] as [a][k]; down -> P_final[I,J] as [k][c]
+      int shs;
+      ok = acquire(shs);
+      if (!ok) break;
+      fill(shs, (down ? a.P : a.Dl) + (int64_t)I * TB * np + J * TB, np, stream);
+      const int64_t opld = down ? a.mp : np;
+      for (int x = first; x < last && ok; ++x) {
+        int ts;
+        ok = acquire(ts);
+        if (!ok) break;
+        // right: Rh[(J+d+x) rows][J cols] as [c][k]; down: Lh[(I+d+x) rows][I cols] as [a][k]
+        fill(ts,
+             down ? a.Lh + (int64_t)(I + pl.dist0 + x) * TB * a.mp + I * TB
+                  : a.Rh + (int64_t)(J + pl.dist0 + x) * TB * np + J * TB,
+             opld, keep);
+        release_later(ts);
+        if (x + 1 == last) release_later(shs);
+        double* C = down ? a.E + (int64_t)(I + pl.dist0 + x) * TB * np + J * TB
+                         : a.P + (int64_t)I * TB * np + (J + pl.dist0 + x) * TB;
+        ok = put_desc(C, ts, shs,
+                      (down ? FD_DOWN : 0) | (x == first ? FD_FIRST : 0) |
+                          (x + 1 == last ? FD_LAST : 0));
+      }
+    }
+    if (ok) ok = put_desc(nullptr, 0, 0, FD_END);
+    if (!ok) {
+      if (lane == 0) atomicExch(a.err, 1);
+      for (int s = 0; s < FAR_SLOTS; ++s)  // let this warp's copies land before the CTA exits
+        if (fills[s] > 0) mbar_wait(&S.full[s], (fills[s] - 1) & 1);
+    }
+    return;
+  }
+
+  // consumers: warp cw of this stream owns the 32x32 quadrant (cw>>1, cw&1)
+  const int cw = warp & 3, g8 = lane >> 2, t4 = lane & 3;
+  const int wr = (cw >> 1) * 32, wc = (cw & 1) * 32;
+  unsigned par = 0;  // bit s: parity of the next phase of full[s] to wait for
+  for (int n = 0;; ++n) {
+    const int e = n % FAR_DQ;
+    if (!mbar_wait(&S.dqf[e], (n / FAR_DQ) & 1)) break;
+    const FarDesc d = S.desc[e];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.dqe[e]);
+    if (d.flags & FD_END) return;
+    if (d.flags & FD_FIRST) {
+      if (!mbar_wait(&S.full[d.sh_slot], (par >> d.sh_slot) & 1)) break;
+      par ^= 1u << d.sh_slot;
+    }
+    if (!mbar_wait(&S.full[d.task_slot], (par >> d.task_slot) & 1)) break;
+    par ^= 1u << d.task_slot;
+    const bool down = (d.flags & FD_DOWN) != 0;
+    const double* Ts = slot_ptr(d.task_slot);
+    const double* Hs = slot_ptr(d.sh_slot);
+    const double* As = down ? Ts : Hs;  // A(r, k) = As[r * SLD + k]
+    const double* Bs = down ? Hs : Ts;  // B(k, c) = down ? Bs[k * SLD + c] : Bs[c * SLD + k]
+    double acc[4][4][2] = {};
+#pragma unroll 4
+    for (int kk = 0; kk < TB; kk += 4) {
+      double av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[(wr + i * 8 + g8) * SLD + kk + t4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = wc + j * 8 + g8;
+        bv[j] = down ? Bs[(kk + t4) * SLD + c] : Bs[c * SLD + kk + t4];
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          double* p = C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4;
-          red_add(p, acc[i][j][0]);
-          red_add(p + 1, acc[i][j][1]);
-        }
-      group_barrier(h);
+        for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
     }
-    ch = next_chunk[h];
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&S.empty[d.task_slot]);
+      if (d.flags & FD_LAST) mbar_arrive(&S.empty[d.sh_slot]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        double* p = d.C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4;
+        red_add(p, acc[i][j][0]);
+        red_add(p + 1, acc[i][j][1]);
+      }
   }
+  if (lane == 0) atomicExch(a.err, 1);  // a wait gave up
 }
 
 // Sums the per-tile statistics in a fixed order into the caller's gptq2d_stats.
 __global__ void __launch_bounds__(256) finalize_kernel(const TileStat* part, int ntiles,
-                                                       gptq2d_stats* out) {
+                                                       const int* err, gptq2d_stats* out) {
   __shared__ double sl[256];
   __shared__ long long sc[256][3];
   const int tid = threadIdx.x;
@@ -652,7 +819,8 @@ __global__ void __launch_bounds__(256) finalize_kernel(const TileStat* part, int
     st.n_clamped = sc[0][0];
     st.n_near_tie = sc[0][1];
     st.n_nonfinite = sc[0][2];
-    st.status = sc[0][2] > 0 ? GPTQ2D_ERR_NONFINITE : GPTQ2D_OK;
+    st.status = *err != 0 ? GPTQ2D_ERR_TIMEOUT
+                : sc[0][2] > 0 ? GPTQ2D_ERR_NONFINITE : GPTQ2D_OK;
     *out = st;
   }
 }
@@ -698,7 +866,7 @@ WsLayout layout(int64_t m, int64_t n) {
   L.n_cnt = 0;
   for (int D = 0; D < L.Tm + L.Tn - 1; ++D)  // one far-field plan per MAX_GROUPS/2 tiles
     L.n_cnt += (wave_tiles(D, L.Tm, L.Tn) + MAX_GROUPS / 2 - 1) / (MAX_GROUPS / 2);
-  L.off_cnt = o; o += align256((size_t)L.n_cnt * sizeof(int));
+  L.off_cnt = o; o += align256((size_t)(L.n_cnt + 1) * sizeof(int));  // error word + dispensers
   L.total = o;
   return L;
 }
@@ -730,8 +898,8 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
   ok = ok && cudaEventRecord(ds->setup, hi) == cudaSuccess &&
        cudaStreamWaitEvent(lo, ds->setup, 0) == cudaSuccess;
 
-  int* counters = reinterpret_cast<int*>(reinterpret_cast<char*>(a.P) - L.off_P + L.off_cnt);
-  ok = ok && cudaMemsetAsync(counters, 0, (size_t)L.n_cnt * sizeof(int), hi) == cudaSuccess;
+  int* counters = a.err + 1;
+  ok = ok && cudaMemsetAsync(a.err, 0, (size_t)(L.n_cnt + 1) * sizeof(int), hi) == cudaSuccess;
   const int nd = a.Tm + a.Tn - 1;
   const int sms = ds->sms;
   int next_cnt = 0;
@@ -800,7 +968,7 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
     ok = ok && cudaEventRecord(ds->far[D % RING], lo) == cudaSuccess;
     far_recorded[D % RING] = true;
   }
-  GPTQ2D_LAUNCH(KC_OTHER, hi, finalize_kernel<<<1, 256, 0, hi>>>(a.part, a.Tm * a.Tn, stats));
+  GPTQ2D_LAUNCH(KC_OTHER, hi, finalize_kernel<<<1, 256, 0, hi>>>(a.part, a.Tm * a.Tn, a.err, stats));
   ok = ok && cudaEventRecord(ds->join_hi, hi) == cudaSuccess &&
        cudaEventRecord(ds->join_lo, lo) == cudaSuccess &&
        cudaStreamWaitEvent(s, ds->join_hi, 0) == cudaSuccess &&
@@ -847,6 +1015,7 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
   a.dL = reinterpret_cast<double*>(base + L.off_dL);
   a.dR = reinterpret_cast<double*>(base + L.off_dR);
   a.part = reinterpret_cast<TileStat*>(base + L.off_part);
+  a.err = reinterpret_cast<int*>(base + L.off_cnt);
   a.Tm = L.Tm;
   a.Tn = L.Tn;
   int rc;
