@@ -33,8 +33,8 @@
 //                  next sub-wavefront.
 //   low priority   far_kernel(D): the band products that carry the tiles of
 //                  wavefront D to tiles two or more tiles away (to the right:
-//                  P += dW Rh^T; below: E += Lh P), 64x64x64 DMMA tasks handed
-//                  out in chunks by a dispenser.  One launch runs beside
+//                  P += dW Rh^T; below: E += Lh P), 64x64x64 DMMA tasks
+//                  claimed one at a time per group.  One launch runs beside
 //                  sweep_kernel(D+1) on the SMs that sweep leaves free; when the
 //                  work outlasts that sweep a second launch on the high-priority
 //                  stream, after sweep_kernel(D+1), takes the rest on the SMs the
@@ -562,15 +562,26 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
 // band products to tiles two or more tiles away
 // ---------------------------------------------------------------------------
 constexpr int MAX_GROUPS = 512;  // 2 groups per tile: 256 tiles per launch
+constexpr int MAX_STREAMS = 640;  // task streams of one plan over both of its launches
+constexpr int FAR_HELP = 16;      // groups a stream helps once its own run dry
+constexpr int FAR_CLAIM = 2;      // tasks a stream claims from a group at a time
+// One wavefront's far-field tasks.  Group g < nt holds the right tasks of source
+// tile I0+g, group g >= nt its down tasks; the tasks of a group share one
+// operand.  Each group has a task counter in the workspace, so the streams on a
+// group take its tasks one at a time; stream s works on own[s] (or, when there
+// are fewer streams than groups, on every rr-th group from its own index) and
+// then helps the groups in help[].
 struct FarPlan {
-  int D, I0, nt;  // source tiles: I0..I0+nt-1 of wavefront D
-  int dist0;      // distance of the first target tile (2: far field, 1: near neighbours)
-  int cap;        // most tasks per group
-  int per_chunk;  // tasks per chunk
-  int* counter;   // chunk dispenser, zero before the first launch on this plan
-  // start[g] = first chunk of group g; group g < nt holds the right tasks of tile
-  // I0+g, group g >= nt the down tasks of tile I0+g-nt.
-  int start[MAX_GROUPS + 1];
+  int D, I0, nt;     // source tiles: I0..I0+nt-1 of wavefront D
+  int dist0;         // distance of the first target tile (2: far field)
+  int cap;           // most tasks per group
+  int* gcnt;         // per-group task counters, zero before the first launch on this plan
+  int stream_base;   // index of this launch's first stream
+  int nstreams;      // streams planned over both launches
+  int rr_a, rr_b;    // nonzero: streams < rr_a take every rr_a-th group, the rest every rr_b-th
+  int nhelp;
+  short help[FAR_HELP];
+  short own[MAX_STREAMS];
 };
 
 constexpr int FAR_CONS = 128;                    // consumer threads per task stream (4 warps)
@@ -600,19 +611,20 @@ struct FarSync {
 };
 
 // Each CTA runs two independent task streams.  A stream is one producer warp and
-// four consumer warps.  The producer takes chunks from the plan's dispenser (a
-// chunk is a run of tasks of one source tile and direction, which share one
-// operand) and brings every operand tile in with 512-byte bulk row copies (TMA
-// engine) that complete on the slot's mbarrier.  Slots are handed out in the
-// order the consumers free them, so a chunk's shared operand is fetched while
-// the previous chunk still runs.  The consumers wait for a descriptor and its
-// slots, run the 64x64x64 DMMA product, free the slots, and add the product into
-// P or E by reductions in L2 (red_add: each element gets one contribution per
-// launch, so the sum equals a load, add and store).  Several launches on one plan
-// (one beside the next sweep, one on the SMs that sweep frees) share the
-// dispenser.  Every wait gives up after kWaitLimitNs, sets *a.err and leaves the
-// kernel (the call then reports GPTQ2D_ERR_TIMEOUT); a producer that gives up
-// first waits, again bounded, for the copies it has in flight.
+// four consumer warps.  The producer walks its list of groups (FarPlan), claims
+// the group's tasks one at a time from the group's counter (a task is one
+// 64x64x64 product; the tasks of a group share one operand, loaded once per
+// group and stream) and brings every operand tile in with 512-byte bulk row
+// copies (TMA engine) that complete on the slot's mbarrier.  Slots are handed out
+// in the order the consumers free them, so the next group's shared operand is
+// fetched while the current one runs.  The consumers wait for a descriptor and
+// its slots, run the DMMA product, free the slots, and add the product into P or
+// E by reductions in L2 (red_add: each element gets one contribution per launch,
+// so the sum equals a load, add and store).  Both launches on one plan (one
+// beside the next sweep, one on the SMs that sweep frees) share the counters.
+// Every wait gives up after kWaitLimitNs, sets *a.err and leaves the kernel (the
+// call then reports GPTQ2D_ERR_TIMEOUT); a producer that gives up first waits,
+// again bounded, for the copies it has in flight.
 __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl) {
   extern __shared__ __align__(128) double sm[];
   __shared__ FarSync sync[2];
@@ -639,7 +651,6 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
 
   if (producer) {
     const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
-    const int nchunks = pl.start[2 * pl.nt];
     int fills[FAR_SLOTS] = {0, 0, 0};  // fills issued per slot
     int fifo[4] = {0, 1, 2, 0};        // slots in the order the consumers free them
     int fh = 0, ft = FAR_SLOTS, nd = 0;
@@ -678,32 +689,74 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
       ++nd;
       return true;
     };
-    while (ok) {
-      int ch = 0;
-      if (lane == 0) ch = atomicAdd(pl.counter, 1);
-      ch = __shfl_sync(0xffffffffu, ch, 0);
-      if (ch >= nchunks) break;
-      int g;
-      {
-        int lo = 0, hi = 2 * pl.nt;  // largest g with start[g] <= ch
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (pl.start[mid] <= ch) lo = mid; else hi = mid;
+    const int G = 2 * pl.nt;
+    const int sid = pl.stream_base + 2 * blockIdx.x + h;  // this stream
+    int own_k = 0;
+    // the next group on this stream's own list, -1 when the list is done
+    auto next_group = [&]() -> int {
+      if (sid < pl.nstreams) {
+        if (pl.rr_a > 0) {
+          const int base = sid < pl.rr_a ? sid : sid - pl.rr_a;
+          const int stride = sid < pl.rr_a ? pl.rr_a : pl.rr_b;
+          const int g = base + own_k * stride;
+          if (stride > 0 && g < G) {
+            ++own_k;
+            return g;
+          }
+        } else if (own_k == 0) {
+          ++own_k;
+          return pl.own[sid];
         }
-        g = lo;
+      }
+      return -1;
+    };
+    // claims the next FAR_CLAIM tasks of group g for this stream; returns the first
+    auto claim = [&](int g) -> int {
+      int x = 0;
+      if (lane == 0) x = atomicAdd(pl.gcnt + g, FAR_CLAIM);
+      return __shfl_sync(0xffffffffu, x, 0);
+    };
+    auto group_count = [&](int g) -> int {
+      const bool dn = g >= pl.nt;
+      const int I = pl.I0 + (dn ? g - pl.nt : g), J = pl.D - I;
+      return min(pl.cap, dn ? a.Tm - I - pl.dist0 : a.Tn - J - pl.dist0);
+    };
+    unsigned help_done = 0;  // help groups found empty
+    for (int g = next_group(); ok; g = next_group()) {
+      if (g < 0) {
+        // own list done: look at every help group at once and join one with tasks left
+        bool left = false;
+        if (lane < pl.nhelp && !((help_done >> lane) & 1u)) {
+          const int hg = pl.help[lane];
+          left = *(volatile const int*)(pl.gcnt + hg) < group_count(hg);
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, left);
+        help_done |= ~m & ((pl.nhelp >= 32 ? 0u : (1u << pl.nhelp)) - 1u);
+        if (m == 0) break;
+        const int q = __ffs(m) - 1;
+        help_done |= 1u << q;
+        g = pl.help[q];
       }
       const bool down = g >= pl.nt;
       const int I = pl.I0 + (down ? g - pl.nt : g), J = pl.D - I;
-      const int count = min(pl.cap, down ? a.Tm - I - pl.dist0 : a.Tn - J - pl.dist0);
-      const int first = (ch - pl.start[g]) * pl.per_chunk;
-      const int last = min(first + pl.per_chunk, count);
+      const int count = group_count(g);
+      if (count <= 0) continue;
+      int x = claim(g), xe = min(x + FAR_CLAIM, count);
+      if (x >= count) continue;  // nothing left: no operand load
       // shared operand: right -> dW[I,J] as [a][k]; down -> P_final[I,J] as [k][c]
       int shs;
       ok = acquire(shs);
       if (!ok) break;
       fill(shs, (down ? a.P : a.Dl) + (int64_t)I * TB * np + J * TB, np, stream);
       const int64_t opld = down ? a.mp : np;
-      for (int x = first; x < last && ok; ++x) {
+      bool first = true;
+      while (ok) {
+        int xn = xe;
+        bool lastx = false;
+        if (x + 1 >= xe) {  // last of the claimed run: claim more before publishing it
+          xn = claim(g);
+          lastx = xn >= count;
+        }
         int ts;
         ok = acquire(ts);
         if (!ok) break;
@@ -713,12 +766,19 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
                   : a.Rh + (int64_t)(J + pl.dist0 + x) * TB * np + J * TB,
              opld, keep);
         release_later(ts);
-        if (x + 1 == last) release_later(shs);
+        if (lastx) release_later(shs);
         double* C = down ? a.E + (int64_t)(I + pl.dist0 + x) * TB * np + J * TB
                          : a.P + (int64_t)I * TB * np + (J + pl.dist0 + x) * TB;
         ok = put_desc(C, ts, shs,
-                      (down ? FD_DOWN : 0) | (x == first ? FD_FIRST : 0) |
-                          (x + 1 == last ? FD_LAST : 0));
+                      (down ? FD_DOWN : 0) | (first ? FD_FIRST : 0) | (lastx ? FD_LAST : 0));
+        first = false;
+        if (lastx) break;
+        if (x + 1 >= xe) {
+          x = xn;
+          xe = min(xn + FAR_CLAIM, count);
+        } else {
+          ++x;
+        }
       }
     }
     if (ok) ok = put_desc(nullptr, 0, 0, FD_END);
@@ -837,7 +897,7 @@ struct WsLayout {
   int64_t mp, np;
   int Tm, Tn;
   size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_part, off_cnt, total;
-  int n_cnt;  // chunk dispensers, one per far-field plan
+  int n_cnt;  // far-field plans (MAX_GROUPS group counters each)
 };
 
 // Tiles of wavefront D, and the first of them.
@@ -866,7 +926,7 @@ WsLayout layout(int64_t m, int64_t n) {
   L.n_cnt = 0;
   for (int D = 0; D < L.Tm + L.Tn - 1; ++D)  // one far-field plan per MAX_GROUPS/2 tiles
     L.n_cnt += (wave_tiles(D, L.Tm, L.Tn) + MAX_GROUPS / 2 - 1) / (MAX_GROUPS / 2);
-  L.off_cnt = o; o += align256((size_t)(L.n_cnt + 1) * sizeof(int));  // error word + dispensers
+  L.off_cnt = o; o += align256((1 + (size_t)L.n_cnt * MAX_GROUPS) * sizeof(int));  // error word + group counters
   L.total = o;
   return L;
 }
@@ -899,16 +959,17 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
        cudaStreamWaitEvent(lo, ds->setup, 0) == cudaSuccess;
 
   int* counters = a.err + 1;
-  ok = ok && cudaMemsetAsync(a.err, 0, (size_t)(L.n_cnt + 1) * sizeof(int), hi) == cudaSuccess;
+  ok = ok && cudaMemsetAsync(a.err, 0, (1 + (size_t)L.n_cnt * MAX_GROUPS) * sizeof(int), hi) ==
+                  cudaSuccess;
   const int nd = a.Tm + a.Tn - 1;
   const int sms = ds->sms;
   int next_cnt = 0;
   // far(D) = one launch on the low-priority stream beside sweep(D+1), on the SMs that
   // sweep leaves free, plus (when the work outlasts that sweep) one on the
   // high-priority stream after sweep(D+1), on the SMs it frees; both draw chunks from
-  // the same dispenser.  sweep(D+2) waits for both.
+  // the same group counters.  sweep(D+2) waits for both.
   std::vector<FarPlan> prev_plans;  // far(D-1), still to get its second launch
-  int prev_b_ctas = 0;
+  std::vector<int> prev_b;          // and its CTA counts
   bool far_recorded[RING] = {};
   for (int D = 0; D < nd && ok; ++D) {
     const int I0 = wave_i0(D, a.Tn);
@@ -919,10 +980,11 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
     GPTQ2D_LAUNCH(KC_SWEEP, hi,
                   sweep_kernel<TW><<<nt, SWEEP_THREADS, SW_SMEM, hi>>>(a, D, I0));
     const bool b_launched = !prev_plans.empty();
-    for (const FarPlan& pl : prev_plans)
+    for (size_t q = 0; q < prev_plans.size(); ++q)
       GPTQ2D_LAUNCH(KC_PROPAGATE, hi,
-                    far_kernel<<<prev_b_ctas, FAR_THREADS, FAR_SMEM, hi>>>(a, pl));
+                    far_kernel<<<prev_b[q], FAR_THREADS, FAR_SMEM, hi>>>(a, prev_plans[q]));
     prev_plans.clear();
+    prev_b.clear();
 
     // band products of wavefront D to tiles two or more tiles away
     long long total = 0;
@@ -936,8 +998,6 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
     // a second launch pays when the work outlasts the next sweep on a_ctas SMs
     // (about 24 tasks per CTA fit in one sweep's time)
     const bool want_b = nt_next > 0 && total > 24LL * a_ctas;
-    const long long streams = 2LL * (a_ctas + (want_b ? nt_next : 0));
-    const int per_chunk = (int)std::min<long long>(8, std::max<long long>(1, total / (4 * streams)));
     ok = ok && cudaEventRecord(b_launched ? ds->farb[(D - 1) % RING] : ds->sw[D % RING], hi) ==
                    cudaSuccess &&
          cudaStreamWaitEvent(lo, b_launched ? ds->farb[(D - 1) % RING] : ds->sw[D % RING], 0) ==
@@ -949,22 +1009,63 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
       pl.nt = std::min(nt - tb, MAX_GROUPS / 2);
       pl.dist0 = 2;
       pl.cap = 1 << 30;
-      pl.per_chunk = per_chunk;
-      pl.counter = counters + next_cnt++;
-      int chunks = 0;
-      for (int gidx = 0; gidx < 2 * pl.nt; ++gidx) {
+      pl.gcnt = counters + (size_t)(next_cnt++) * MAX_GROUPS;
+      const int G = 2 * pl.nt;
+      int cnt[MAX_GROUPS];
+      long long tasks = 0;
+      int nonempty = 0;
+      for (int gidx = 0; gidx < G; ++gidx) {
         const int I = pl.I0 + (gidx < pl.nt ? gidx : gidx - pl.nt), J = D - I;
-        const int cnt = gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
-        pl.start[gidx] = chunks;
-        chunks += (cnt + per_chunk - 1) / per_chunk;
+        cnt[gidx] = gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
+        tasks += cnt[gidx];
+        nonempty += cnt[gidx] > 0;
       }
-      pl.start[2 * pl.nt] = chunks;
-      if (chunks == 0) continue;
-      const int ctas = std::min(a_ctas, (chunks + 1) / 2);
+      if (tasks == 0) continue;
+      const int ctas = (int)std::min<long long>(std::min(a_ctas, MAX_STREAMS / 4), (tasks + 1) / 2);
+      const int b_ctas = want_b ? std::min(nt_next, MAX_STREAMS / 2 - ctas) : 0;
+      const int sa = 2 * ctas, sb = 2 * b_ctas;
+      pl.stream_base = 0;
+      pl.nstreams = sa + sb;
+      // streams of the first launch cover every group; the others join the groups
+      // with the most tasks per stream (those of the second launch arrive later)
+      if (sa >= nonempty) {
+        pl.rr_a = pl.rr_b = 0;
+        int k[MAX_GROUPS];
+        int s2 = 0;
+        for (int gidx = 0; gidx < G; ++gidx) {
+          k[gidx] = 0;
+          if (cnt[gidx] > 0) {
+            pl.own[s2++] = (short)gidx;
+            k[gidx] = 1;
+          }
+        }
+        for (; s2 < sa + sb; ++s2) {
+          int best = -1;
+          for (int gidx = 0; gidx < G; ++gidx)
+            if (cnt[gidx] > 0 && (best < 0 || (long long)cnt[gidx] * k[best] >
+                                                  (long long)cnt[best] * k[gidx]))
+              best = gidx;
+          pl.own[s2] = (short)best;
+          ++k[best];
+        }
+      } else {
+        pl.rr_a = sa;
+        pl.rr_b = sb;
+      }
+      // idle streams help the largest groups
+      int order[MAX_GROUPS];
+      for (int gidx = 0; gidx < G; ++gidx) order[gidx] = gidx;
+      std::stable_sort(order, order + G, [&](int x, int y) { return cnt[x] > cnt[y]; });
+      pl.nhelp = 0;
+      for (int q = 0; q < G && pl.nhelp < FAR_HELP && cnt[order[q]] > 0; ++q)
+        pl.help[pl.nhelp++] = (short)order[q];
       GPTQ2D_LAUNCH(KC_PROPAGATE, lo, far_kernel<<<ctas, FAR_THREADS, FAR_SMEM, lo>>>(a, pl));
-      if (want_b && chunks > 2 * ctas) prev_plans.push_back(pl);
+      if (b_ctas > 0) {
+        pl.stream_base = sa;
+        prev_plans.push_back(pl);
+        prev_b.push_back(b_ctas);
+      }
     }
-    prev_b_ctas = nt_next;
     ok = ok && cudaEventRecord(ds->far[D % RING], lo) == cudaSuccess;
     far_recorded[D % RING] = true;
   }
