@@ -628,6 +628,7 @@ struct FarSync {
 __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl) {
   extern __shared__ __align__(128) double sm[];
   __shared__ FarSync sync[2];
+  __shared__ __align__(16) double stage[8][8 * 40];  // per consumer warp: one 8x32 strip (row stride 40)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool producer = warp >= 8;
   const int h = producer ? warp - 8 : warp >> 2;  // task stream
@@ -833,14 +834,20 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
       mbar_arrive(&S.empty[d.task_slot]);
       if (d.flags & FD_LAST) mbar_arrive(&S.empty[d.sh_slot]);
     }
+    // reductions of whole 256-byte rows: each 8x32 strip goes through shared memory
+    double* st = stage[warp];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        double* p = d.C + (int64_t)(wr + i * 8 + g8) * np + wc + j * 8 + 2 * t4;
-        red_add(p, acc[i][j][0]);
-        red_add(p + 1, acc[i][j][1]);
-      }
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<double2*>(st + g8 * 40 + j * 8 + 2 * t4) =
+            make_double2(acc[i][j][0], acc[i][j][1]);
+      __syncwarp();
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        red_add(d.C + (int64_t)(wr + i * 8 + r) * np + wc + lane, st[r * 40 + lane]);
+      __syncwarp();
+    }
   }
   if (lane == 0) atomicExch(a.err, 1);  // a wait gave up
 }
