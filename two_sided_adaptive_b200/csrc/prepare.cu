@@ -29,7 +29,8 @@ namespace {
 
 constexpr int OLD = TB + 4;  // 68: row stride of shared 64x64 tiles (conflict-free DMMA fragments)
 constexpr int TR_THREADS = 128;
-constexpr int PANEL_THREADS = 256;
+constexpr int PANEL_THREADS = 384;   // 8 factor warps + 4 warps for the block-row lookahead
+constexpr int FACTOR_THREADS = 256;
 constexpr int MAX_TR_GROUPS = 512;
 
 template <typename TH>
@@ -68,34 +69,57 @@ __device__ __forceinline__ void load_block(double* dst, const double* M, int64_t
   }
 }
 
-// Subtracts Xs^T Ys from the 64x64 shared tile Cs, all [r][c] with stride OLD:
-// Cs[i][j] -= sum_r Xs[r][i] Ys[r][j].  8 warps; warp w owns rows (w>>1)*16..+16
-// and columns (w&1)*32..+32 of Cs, so every element has one owner.
-__device__ __forceinline__ void sub_xty_8w(double* Cs, const double* Xs, const double* Ys) {
+// The lower 8x8 blocks (bi >= bj) of Cs -= Xs^T Xs on `nw` warps, one block at a time
+// per warp (K = 64 in 16 DMMA steps).  The blocks above the diagonal are not used.
+__device__ __forceinline__ void sub_xtx_lower(double* Cs, const double* Xs, int nw) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int wr = (warp >> 1) * 16, wc = (warp & 1) * 32;
-  double acc[2][4][2] = {};
+  for (int x = warp; x < 36; x += nw) {
+    int bi = 0;
+    while ((bi + 1) * (bi + 2) / 2 <= x) ++bi;
+    const int bj = x - bi * (bi + 1) / 2;
+    double c0 = 0.0, c1 = 0.0;
+#pragma unroll
+    for (int kk = 0; kk < TB; kk += 4)
+      dmma_m8n8k4(c0, c1, Xs[(kk + t) * OLD + 8 * bi + g], Xs[(kk + t) * OLD + 8 * bj + g]);
+    double* c = Cs + (8 * bi + g) * OLD + 8 * bj + 2 * t;
+    c[0] -= c0;
+    c[1] -= c1;
+  }
+}
+
+// Cs -= Xs^T Ys (64x64, K = 64) on 4 warps, warp w owning the quadrant (w>>1, w&1);
+// `warp` is the warp's index inside the group.
+__device__ __forceinline__ void sub_xty_4w(double* Cs, const double* Xs, const double* Ys,
+                                           int warp) {
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
+  double acc[4][4][2] = {};
 #pragma unroll 4
   for (int kk = 0; kk < TB; kk += 4) {
-    double a[2], b[4];
+    double a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) a[i] = Xs[(kk + t) * OLD + wr + i * 8 + g];
+    for (int i = 0; i < 4; ++i) a[i] = Xs[(kk + t) * OLD + wr + i * 8 + g];
 #pragma unroll
     for (int j = 0; j < 4; ++j) b[j] = Ys[(kk + t) * OLD + wc + j * 8 + g];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
   }
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       double* c = Cs + (wr + i * 8 + g) * OLD + wc + j * 8 + 2 * t;
       c[0] -= acc[i][j][0];
       c[1] -= acc[i][j][1];
     }
+}
+
+__device__ __forceinline__ void factor_group_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(FACTOR_THREADS) : "memory");
 }
 
 constexpr int PANEL_SMEM = 4 * TB * OLD * (int)sizeof(double);
@@ -217,45 +241,62 @@ __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict
   cp_async_commit_group();
   cp_async_wait_group<0>();
   __syncthreads();
-  if (nn > 0) {
-    sub_xty_8w(Ad, Mn, Mn);
-    if (b < K) sub_xty_8w(Ab, Mn, Mb);
-  }
+  if (nn > 0) sub_xtx_lower(Ad, Mn, PANEL_THREADS / 32);  // the factor needs it first
   // unit diagonal past a ragged edge (only the last block row is ragged, and it
   // has no lookahead update, so no other thread writes these elements)
   if (tid < TB && tid >= nb) Ad[tid * OLD + tid] = 1.0;
   __syncthreads();
 
-  // factor A_KK in place, strips s = 7..0
-#pragma unroll 1
-  for (int s = TB / 8 - 1; s >= 0; --s) {
+  if (warp >= FACTOR_THREADS / 32) {
+    // warps 8..11: the block-row lookahead A_Kb -= M_{K+1,K}^T M_{K+1,b}, needed only
+    // by the solve below, while warps 0..7 factor the diagonal block
+    if (nn > 0 && b < K) sub_xty_4w(Ab, Mn, Mb, warp - FACTOR_THREADS / 32);
+  } else {
+  // factor A_KK in place, strips s = 7..0.  Threads <= 8s factor strip s's 8x8
+  // diagonal block in registers; threads < 8s then solve one column of the strip
+  // each, and thread 8s stores the block.
+  auto factor_strip = [&](int s) {
     const int R0 = 8 * s;
-    if (tid <= R0) {  // threads < R0 solve a column of the strip, thread R0 stores M_D
-      double L[8][8], inv[8];
-      const int bp = factor_diag8_regs(Ad, R0, L, inv);
-      if (tid < R0) {
-        solve_col8_regs(Ad, L, inv, R0, tid);
-      } else {
+    double L[8][8], inv[8];
+    const int bp = factor_diag8_regs(Ad, R0, L, inv);
+    if (tid < R0) {
+      solve_col8_regs(Ad, L, inv, R0, tid);
+    } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          invd[R0 + i] = inv[i];
+      for (int i = 0; i < 8; ++i) {
+        invd[R0 + i] = inv[i];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) Ad[(R0 + i) * OLD + R0 + j] = j <= i ? L[i][j] : 0.0;
-        }
-        if (bp >= 0 && bad < 0) bad = rb + R0 + bp;
+        for (int j = 0; j < 8; ++j) Ad[(R0 + i) * OLD + R0 + j] = j <= i ? L[i][j] : 0.0;
+      }
+      if (bp >= 0 && bad < 0) bad = rb + R0 + bp;
+    }
+  };
+  if (tid <= TB - 8) factor_strip(TB / 8 - 1);
+  factor_group_sync();
+#pragma unroll 1
+  for (int s = TB / 8 - 1; s >= 1; --s) {
+    // strip s is done.  First its update of the next strip's row of blocks
+    // (s-1, 0..s-1), one block per warp ...
+    if (warp < s) rank8_block(Ad, Ad, Ad, 8 * s, s - 1, warp);
+    factor_group_sync();
+    // ... then strip s-1 is factored on warps 0..1 while warps 2..7 apply strip s's
+    // update to the rows above it: A[i][j] -= sum_a M[8s+a][i] M[8s+a][j], lower
+    // 8x8 blocks (bi >= bj) with bi < s-1
+    if (tid <= 8 * (s - 1)) {
+      factor_strip(s - 1);
+    } else if (warp >= 2) {
+      const int nblk = (s - 1) * s / 2;
+      for (int x = warp - 2; x < nblk; x += FACTOR_THREADS / 32 - 2) {
+        int bi = 0;
+        while ((bi + 1) * (bi + 2) / 2 <= x) ++bi;
+        rank8_block(Ad, Ad, Ad, 8 * s, bi, x - bi * (bi + 1) / 2);
       }
     }
-    __syncthreads();
-    // A_lead[i][j] -= sum_a M[R0+a][i] M[R0+a][j], lower 8x8 blocks (bi >= bj) of the lead
-    const int nblk = s * (s + 1) / 2;
-    for (int x = warp; x < nblk; x += PANEL_THREADS / 32) {
-      int bi = 0;
-      while ((bi + 1) * (bi + 2) / 2 <= x) ++bi;
-      rank8_block(Ad, Ad, Ad, R0, bi, x - bi * (bi + 1) / 2);
-    }
-    __syncthreads();
+    factor_group_sync();
   }
-  if (bad >= 0) {  // uniform: read after the last barrier
+  }
+  __syncthreads();
+  if (bad >= 0) {  // uniform: read after the barrier
     if (tid == 0) *info = bad;
     return;
   }
