@@ -94,16 +94,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
   return p;
 }
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint64_t pol) {
-  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
-               "l"(pol));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
-}
 // C += v without reading C back: each C element gets one contribution per
 // far-field launch and launches on one plan are stream-ordered, so the sum is
 // the same as a load, add and store.
@@ -159,57 +149,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       " [%0], [%1], %2, [%3], %4;\n" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
-}
-
-// Copies a 64x64 fp64 tile (row stride `ld` elements, 16-byte aligned rows) into
-// shared memory with row stride `sld`, 16 bytes per cp.async.
-template <int NT>
-__device__ __forceinline__ void tile_cp_async(double* dst, int sld, const double* src, int64_t ld,
-                                              uint64_t pol, int tix) {
-  for (int x = tix; x < TB * TB / 2; x += NT) {
-    const int r = x >> 5, c2 = (x & 31) * 2;
-    cp_async16(dst + r * sld + c2, src + (int64_t)r * ld + c2, pol);
-  }
-}
-
-// 64x64x64 product on 8 warps: warp w owns rows (w>>1)*16..+16, cols (w&1)*32..+32.
-template <typename FA, typename FB>
-__device__ __forceinline__ void mma8w(double (&acc)[2][4][2], FA fa, FB fb) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int wr = (warp >> 1) * 16, wc = (warp & 1) * 32;
-#pragma unroll 4
-  for (int kk = 0; kk < TB; kk += 4) {
-    double av[2], bv[4];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) av[i] = fa(wr + i * 8 + g, kk + t);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) bv[j] = fb(kk + t, wc + j * 8 + g);
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
-  }
-}
-
-// 64x64x64 product on 16 warps: warp w owns rows (w>>2)*16..+16, cols (w&3)*16..+16.
-template <typename FA, typename FB>
-__device__ __forceinline__ void mma16w(double (&acc)[2][2][2], FA fa, FB fb) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int wr = (warp >> 2) * 16, wc = (warp & 3) * 16;
-#pragma unroll 4
-  for (int kk = 0; kk < TB; kk += 4) {
-    double av[2], bv[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) av[i] = fa(wr + i * 8 + g, kk + t);
-#pragma unroll
-    for (int j = 0; j < 2; ++j) bv[j] = fb(kk + t, wc + j * 8 + g);
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -270,7 +209,7 @@ constexpr int NSUB = TB / SUB;     // sub-tiles per tile edge
 // per target sub-tile.
 template <typename TW>
 __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D, int I0) {
-  extern __shared__ __align__(16) double sm[];
+  extern __shared__ __align__(128) double sm[];
   double* Pt = sm;                 // P of the tile
   double* Vt = Pt + TB * SLD;      // V of the tile
   double* Dt = Vt + TB * SLD;      // W, overwritten by dW entry by entry
@@ -283,7 +222,6 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   const int rows = min(TB, a.m - r0), cols = min(TB, a.n - c0);
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
-  const int wr = (warp >> 2) * 16, wc = (warp & 3) * 16;
   const int64_t np = a.np;
   const int64_t ts = (int64_t)r0 * np + c0;  // tile origin in the workspace matrices
 
