@@ -282,15 +282,32 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(ws);
   const size_t hs = elem_size(h_dtype);
-  if (cudaMemcpyAsync(b + L.off_W, W, (size_t)m * n * elem_size(w_dtype), cudaMemcpyHostToDevice, s) ||
-      cudaMemcpyAsync(b + L.off_HL, H_L, (size_t)m * m * hs, cudaMemcpyHostToDevice, s) ||
-      cudaMemcpyAsync(b + L.off_HR, H_R, (size_t)n * n * hs, cudaMemcpyHostToDevice, s) ||
-      cudaMemcpyAsync(b + L.off_s, scales, (size_t)m * sizeof(float), cudaMemcpyHostToDevice, s))
+  DevStreams* ds = nullptr;
+  int rc = dev_streams(&ds);
+  if (rc != GPTQ2D_OK) return rc;
+  // Inputs go over one copy stream in the order they are needed: H_L, then H_R,
+  // then W and the scales.  Factor L starts once H_L is in, factor R once H_R is,
+  // and the rounding once both factors and W are done, so the later copies run
+  // under the factorizations.
+  std::lock_guard<std::recursive_mutex> lk(ds->mu);
+  if (cudaEventRecord(ds->fork, s) != cudaSuccess ||
+      cudaStreamWaitEvent(ds->cp, ds->fork, 0) != cudaSuccess ||
+      cudaMemcpyAsync(b + L.off_HL, H_L, (size_t)m * m * hs, cudaMemcpyHostToDevice, ds->cp) ||
+      cudaEventRecord(ds->cp_ev[0], ds->cp) != cudaSuccess ||
+      cudaMemcpyAsync(b + L.off_HR, H_R, (size_t)n * n * hs, cudaMemcpyHostToDevice, ds->cp) ||
+      cudaEventRecord(ds->cp_ev[1], ds->cp) != cudaSuccess ||
+      cudaMemcpyAsync(b + L.off_W, W, (size_t)m * n * elem_size(w_dtype), cudaMemcpyHostToDevice,
+                      ds->cp) ||
+      cudaMemcpyAsync(b + L.off_s, scales, (size_t)m * sizeof(float), cudaMemcpyHostToDevice,
+                      ds->cp) ||
+      cudaEventRecord(ds->cp_ev[2], ds->cp) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
   double* ML = reinterpret_cast<double*>(b + L.off_ML);
   double* MR = reinterpret_cast<double*>(b + L.off_MR);
-  int rc = prepare_pair_launch(b + L.off_HL, m, m, b + L.off_HR, n, n, h_dtype, ML, m, MR, n,
-                               b + L.off_pl, b + L.off_pr, s);
+  rc = prepare_pair_launch(b + L.off_HL, m, m, b + L.off_HR, n, n, h_dtype, ML, m, MR, n,
+                           b + L.off_pl, b + L.off_pr, s, ds->cp_ev[0], ds->cp_ev[1]);
+  if (rc == GPTQ2D_OK && cudaStreamWaitEvent(s, ds->cp_ev[2], 0) != cudaSuccess)
+    rc = GPTQ2D_ERR_CUDA;
   if (rc == GPTQ2D_OK)
     rc = quantize_launch(b + L.off_W, w_dtype, (int)m, (int)n, n, ML, m, MR, n,
                          reinterpret_cast<const float*>(b + L.off_s), bits, clamp,

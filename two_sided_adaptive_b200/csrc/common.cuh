@@ -142,12 +142,14 @@ struct TileStat {
 // ---------------------------------------------------------------------------
 constexpr int RING = 4;
 struct DevStreams {
-  std::mutex mu;
+  std::recursive_mutex mu;  // held across nested enqueues (round_host -> prepare, quantize)
   bool ready = false;
   int sms = 148;
   cudaStream_t hi = nullptr, lo = nullptr, hi2 = nullptr, lo2 = nullptr;
+  cudaStream_t cp = nullptr;  // host<->device copies of round_host
   cudaEvent_t fork = nullptr, setup = nullptr, join_hi = nullptr, join_lo = nullptr;
   cudaEvent_t join_hi2 = nullptr, join_lo2 = nullptr;
+  cudaEvent_t cp_ev[3] = {};  // H_L, H_R, W + scales copied
   cudaEvent_t sw[RING] = {}, far[RING] = {}, farb[RING] = {};
   cudaEvent_t panel_done[2][RING] = {}, rest_done[2][RING] = {};  // factor preparation
 };
@@ -163,9 +165,11 @@ int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
 // Both factors at once, interleaved step by step on the internal streams
 // (panels on the high-priority ones, trailing updates on the low-priority
 // ones), forked from and joined back to `s`.
+// ready_l / ready_r (may be null): events that H_L / H_R wait for beyond `s`.
 int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
-                        int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s);
+                        int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s,
+                        cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr);
 
 size_t quantize_ws_bytes(int64_t m, int64_t n);
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,

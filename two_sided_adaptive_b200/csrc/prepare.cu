@@ -442,6 +442,7 @@ struct FactorJob {
   long long* info;
   bool v16;
   cudaStream_t ps, us;
+  cudaEvent_t ready;        // H is in place once this has completed (may be null)
   cudaEvent_t* panel_done;  // [RING]
   cudaEvent_t* rest_done;   // [RING]
 };
@@ -530,6 +531,7 @@ FactorJob make_job(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
   f.us = us;
   f.panel_done = pd;
   f.rest_done = rd;
+  f.ready = nullptr;
   return f;
 }
 
@@ -538,9 +540,12 @@ int enqueue_factors(FactorJob* jobs, int nj, cudaStream_t s, DevStreams* ds) {
   int rc = ensure_prepare_smem();
   if (rc != GPTQ2D_OK) return rc;
   bool ok = cudaEventRecord(ds->fork, s) == cudaSuccess;
-  for (int j = 0; j < nj && ok; ++j)
+  for (int j = 0; j < nj && ok; ++j) {
     ok = cudaStreamWaitEvent(jobs[j].ps, ds->fork, 0) == cudaSuccess &&
          cudaStreamWaitEvent(jobs[j].us, ds->fork, 0) == cudaSuccess;
+    if (ok && jobs[j].ready)
+      ok = cudaStreamWaitEvent(jobs[j].ps, jobs[j].ready, 0) == cudaSuccess;
+  }
   if (!ok) return GPTQ2D_ERR_CUDA;
   for (int j = 0; j < nj && rc == GPTQ2D_OK; ++j) rc = enqueue_convert(jobs[j], ds->sms);
   int steps = 0;
@@ -567,7 +572,7 @@ int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
   DevStreams* ds = nullptr;
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
-  std::lock_guard<std::mutex> lk(ds->mu);
+  std::lock_guard<std::recursive_mutex> lk(ds->mu);
   FactorJob f = make_job(H, h_dtype, k, ldh, M, ldm, ws, ds->hi, ds->lo, ds->panel_done[0],
                          ds->rest_done[0]);
   return enqueue_factors(&f, 1, s, ds);
@@ -575,20 +580,23 @@ int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
 
 int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
-                        int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s) {
+                        int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s,
+                        cudaEvent_t ready_l, cudaEvent_t ready_r) {
   DevStreams* ds = nullptr;
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
-  std::lock_guard<std::mutex> lk(ds->mu);
+  std::lock_guard<std::recursive_mutex> lk(ds->mu);
   FactorJob jobs[2];
   int nj = 0;
-  if (m > 0)
-    jobs[nj++] = make_job(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ds->hi, ds->lo,
-                          ds->panel_done[0], ds->rest_done[0]);
+  if (m > 0) {
+    jobs[nj] = make_job(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ds->hi, ds->lo,
+                        ds->panel_done[0], ds->rest_done[0]);
+    jobs[nj++].ready = ready_l;
+  }
   if (n > 0) {
     jobs[nj] = make_job(H_R, h_dtype, (int)n, ldhr, M_R, ldmr, ws_r, nj ? ds->hi2 : ds->hi,
                         nj ? ds->lo2 : ds->lo, ds->panel_done[nj], ds->rest_done[nj]);
-    ++nj;
+    jobs[nj++].ready = ready_r;
   }
   if (nj == 0) return GPTQ2D_OK;
   return enqueue_factors(jobs, nj, s, ds);

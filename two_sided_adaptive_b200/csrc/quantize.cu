@@ -888,7 +888,7 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
   DevStreams* ds = nullptr;
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
-  std::lock_guard<std::mutex> lk(ds->mu);
+  std::lock_guard<std::recursive_mutex> lk(ds->mu);
   cudaStream_t hi = ds->hi, lo = ds->lo;
   bool ok = cudaEventRecord(ds->fork, s) == cudaSuccess &&
             cudaStreamWaitEvent(hi, ds->fork, 0) == cudaSuccess &&

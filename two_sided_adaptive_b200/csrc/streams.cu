@@ -12,16 +12,18 @@ int dev_streams(DevStreams** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GPTQ2D_ERR_CUDA;
   DevStreams& d = g_dev[dev];
-  std::lock_guard<std::mutex> lk(d.mu);
+  std::lock_guard<std::recursive_mutex> lk(d.mu);
   if (!d.ready) {
     int least = 0, greatest = 0;
     if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ2D_ERR_CUDA;
     if (cudaStreamCreateWithPriority(&d.hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
         cudaStreamCreateWithPriority(&d.lo, cudaStreamNonBlocking, least) != cudaSuccess ||
         cudaStreamCreateWithPriority(&d.hi2, cudaStreamNonBlocking, greatest) != cudaSuccess ||
-        cudaStreamCreateWithPriority(&d.lo2, cudaStreamNonBlocking, least) != cudaSuccess)
+        cudaStreamCreateWithPriority(&d.lo2, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&d.cp, cudaStreamNonBlocking) != cudaSuccess)
       return GPTQ2D_ERR_CUDA;
-    cudaEvent_t* evs[] = {&d.fork, &d.setup, &d.join_hi, &d.join_lo, &d.join_hi2, &d.join_lo2};
+    cudaEvent_t* evs[] = {&d.fork,     &d.setup,    &d.join_hi,  &d.join_lo,  &d.join_hi2,
+                          &d.join_lo2, &d.cp_ev[0], &d.cp_ev[1], &d.cp_ev[2]};
     for (auto* e : evs)
       if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GPTQ2D_ERR_CUDA;
     for (int r = 0; r < RING; ++r)
