@@ -365,7 +365,10 @@ def run_ours(args, rank, world, local_rank):
         f1.record()
         torch.cuda.synchronize()
         ems = max_over_ranks(f0.elapsed_time(f1) / ke, dev)
-        h2d = Wh.numel() * Wh.element_size() + (HLh.numel() + HRh.numel() + sh.numel()) * 4
+        def lower_bytes(k, esz):  # round_host copies each 64-row block of a Gram up to its diagonal
+            return sum(min(64, k - r0) * min(k, r0 + 64) for r0 in range(0, k, 64)) * esz
+        h2d = (Wh.numel() * Wh.element_size() + lower_bytes(m, HLh.element_size())
+               + lower_bytes(n, HRh.element_size()) + sh.numel() * sh.element_size())
         d2h = Qh.numel() + sth.numel() * 8
         e2e = {"value": aggregate_value(m, n, world, ems), "unit": "entries/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),

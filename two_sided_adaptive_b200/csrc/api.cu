@@ -289,12 +289,23 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
   // then W and the scales.  Factor L starts once H_L is in, factor R once H_R is,
   // and the rounding once both factors and W are done, so the later copies run
   // under the factorizations.
+  // Only the lower triangle of a Gram is read, so each 64-row block is copied up to
+  // the end of its diagonal block (about half of the matrix).
+  auto copy_lower = [&](char* dst, const void* src, int64_t k) -> bool {
+    for (int64_t r0 = 0; r0 < k; r0 += 64) {
+      const int64_t rows = std::min<int64_t>(64, k - r0), cols = std::min<int64_t>(k, r0 + 64);
+      if (cudaMemcpy2DAsync(dst + (size_t)r0 * k * hs, (size_t)k * hs,
+                            static_cast<const char*>(src) + (size_t)r0 * k * hs, (size_t)k * hs,
+                            (size_t)cols * hs, (size_t)rows, cudaMemcpyHostToDevice,
+                            ds->cp) != cudaSuccess)
+        return false;
+    }
+    return true;
+  };
   std::lock_guard<std::recursive_mutex> lk(ds->mu);
   if (cudaEventRecord(ds->fork, s) != cudaSuccess ||
-      cudaStreamWaitEvent(ds->cp, ds->fork, 0) != cudaSuccess ||
-      cudaMemcpyAsync(b + L.off_HL, H_L, (size_t)m * m * hs, cudaMemcpyHostToDevice, ds->cp) ||
-      cudaEventRecord(ds->cp_ev[0], ds->cp) != cudaSuccess ||
-      cudaMemcpyAsync(b + L.off_HR, H_R, (size_t)n * n * hs, cudaMemcpyHostToDevice, ds->cp) ||
+      cudaStreamWaitEvent(ds->cp, ds->fork, 0) != cudaSuccess || !copy_lower(b + L.off_HL, H_L, m) ||
+      cudaEventRecord(ds->cp_ev[0], ds->cp) != cudaSuccess || !copy_lower(b + L.off_HR, H_R, n) ||
       cudaEventRecord(ds->cp_ev[1], ds->cp) != cudaSuccess ||
       cudaMemcpyAsync(b + L.off_W, W, (size_t)m * n * elem_size(w_dtype), cudaMemcpyHostToDevice,
                       ds->cp) ||
