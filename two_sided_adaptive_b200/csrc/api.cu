@@ -319,14 +319,31 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
                            b + L.off_pl, b + L.off_pr, s, ds->cp_ev[0], ds->cp_ev[1]);
   if (rc == GPTQ2D_OK && cudaStreamWaitEvent(s, ds->cp_ev[2], 0) != cudaSuccess)
     rc = GPTQ2D_ERR_CUDA;
+  // Q goes back in up to four bands of tile rows, each as soon as its rows are final
+  const int Tm = (int)((m + 63) / 64);
+  int row_tile[4], nband = 0;
+  for (int k = 0; k < 4; ++k) {
+    const int last = (int)(((int64_t)(k + 1) * Tm + 3) / 4) - 1;
+    if (last >= 0 && (nband == 0 || last > row_tile[nband - 1])) row_tile[nband++] = last;
+  }
   if (rc == GPTQ2D_OK)
     rc = quantize_launch(b + L.off_W, w_dtype, (int)m, (int)n, n, ML, m, MR, n,
                          reinterpret_cast<const float*>(b + L.off_s), bits, clamp,
                          reinterpret_cast<int8_t*>(b + L.off_Q), n,
-                         reinterpret_cast<gptq2d_stats*>(b + L.off_stats), b + L.off_q, s);
+                         reinterpret_cast<gptq2d_stats*>(b + L.off_stats), b + L.off_q, s, nband,
+                         row_tile, ds->q_ev);
   if (rc != GPTQ2D_OK) return rc;
+  for (int k = 0, r0 = 0; k < nband; ++k) {
+    const int r1 = (int)std::min<int64_t>(m, (int64_t)(row_tile[k] + 1) * 64);
+    if (cudaStreamWaitEvent(ds->cp, ds->q_ev[k], 0) != cudaSuccess ||
+        cudaMemcpyAsync(Q + (size_t)r0 * n, b + L.off_Q + (size_t)r0 * n, (size_t)(r1 - r0) * n,
+                        cudaMemcpyDeviceToHost, ds->cp) != cudaSuccess)
+      return GPTQ2D_ERR_CUDA;
+    r0 = r1;
+  }
   long long piv[2] = {-1, -1};
-  if (cudaMemcpyAsync(Q, b + L.off_Q, (size_t)m * n, cudaMemcpyDeviceToHost, s) ||
+  if (cudaEventRecord(ds->cp_ev[2], ds->cp) != cudaSuccess ||
+      cudaStreamWaitEvent(s, ds->cp_ev[2], 0) != cudaSuccess ||
       cudaMemcpyAsync(stats, b + L.off_stats, sizeof(gptq2d_stats), cudaMemcpyDeviceToHost, s) ||
       cudaMemcpyAsync(&piv[0], b + L.off_pl, sizeof(long long), cudaMemcpyDeviceToHost, s) ||
       cudaMemcpyAsync(&piv[1], b + L.off_pr, sizeof(long long), cudaMemcpyDeviceToHost, s))

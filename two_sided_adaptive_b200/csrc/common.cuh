@@ -150,6 +150,7 @@ struct DevStreams {
   cudaEvent_t fork = nullptr, setup = nullptr, join_hi = nullptr, join_lo = nullptr;
   cudaEvent_t join_hi2 = nullptr, join_lo2 = nullptr;
   cudaEvent_t cp_ev[3] = {};  // H_L, H_R, W + scales copied
+  cudaEvent_t q_ev[4] = {};   // rows of Q final (round_host copies them out early)
   cudaEvent_t sw[RING] = {}, far[RING] = {}, farb[RING] = {};
   cudaEvent_t panel_done[2][RING] = {}, rest_done[2][RING] = {};  // factor preparation
 };
@@ -172,9 +173,12 @@ int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_
                         cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr);
 
 size_t quantize_ws_bytes(int64_t m, int64_t n);
+// Optional row events: row_ev[k] is recorded once the tile rows 0..row_tile[k] of
+// Q are final (row_tile ascending), so a caller can copy them out early.
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
                     int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
-                    cudaStream_t s);
+                    cudaStream_t s, int n_row_ev = 0, const int* row_tile = nullptr,
+                    cudaEvent_t* row_ev = nullptr);
 
 }  // namespace gptq2d

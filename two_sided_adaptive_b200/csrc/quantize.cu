@@ -880,7 +880,8 @@ std::atomic<uint64_t> g_sweep_smem_set[3];
 std::atomic<uint64_t> g_far_smem_set{0};
 
 template <typename TW>
-int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s, int wslot) {
+int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s, int wslot,
+               int n_row_ev, const int* row_tile, cudaEvent_t* row_ev) {
   constexpr int SW_SMEM = sweep_smem_bytes<TW>();
   if (ensure_smem(sweep_kernel<TW>, SW_SMEM, g_sweep_smem_set[wslot]) != cudaSuccess ||
       ensure_smem(far_kernel, FAR_SMEM, g_far_smem_set) != cudaSuccess)
@@ -924,6 +925,9 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
     far_recorded[D % RING] = false;
     GPTQ2D_LAUNCH(KC_SWEEP, hi,
                   sweep_kernel<TW><<<nt, SWEEP_THREADS, SW_SMEM, hi>>>(a, D, I0));
+    // tile row I is final after the sweep of its last tile, on wavefront I + Tn - 1
+    for (int k = 0; k < n_row_ev && ok; ++k)
+      if (D == row_tile[k] + a.Tn - 1) ok = cudaEventRecord(row_ev[k], hi) == cudaSuccess;
     const bool b_launched = !prev_plans.empty();
     for (size_t q = 0; q < prev_plans.size(); ++q)
       GPTQ2D_LAUNCH(KC_PROPAGATE, hi,
@@ -1029,7 +1033,7 @@ size_t quantize_ws_bytes(int64_t m, int64_t n) { return layout(m, n).total; }
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
                     int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
-                    cudaStream_t s) {
+                    cudaStream_t s, int n_row_ev, const int* row_tile, cudaEvent_t* row_ev) {
   if (m == 0 || n == 0) {
     GPTQ2D_LAUNCH(KC_OTHER, s, zero_stats_kernel<<<1, 1, 0, s>>>(stats));
     return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
@@ -1066,9 +1070,11 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
   a.Tn = L.Tn;
   int rc;
   switch (w_dtype) {
-    case GPTQ2D_F32: rc = launch_all<float>(a, L, stats, s, 0); break;
-    case GPTQ2D_BF16: rc = launch_all<__nv_bfloat16>(a, L, stats, s, 1); break;
-    default: rc = launch_all<double>(a, L, stats, s, 2); break;
+    case GPTQ2D_F32: rc = launch_all<float>(a, L, stats, s, 0, n_row_ev, row_tile, row_ev); break;
+    case GPTQ2D_BF16:
+      rc = launch_all<__nv_bfloat16>(a, L, stats, s, 1, n_row_ev, row_tile, row_ev);
+      break;
+    default: rc = launch_all<double>(a, L, stats, s, 2, n_row_ev, row_tile, row_ev); break;
   }
   if (rc != GPTQ2D_OK) return rc;
   return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;

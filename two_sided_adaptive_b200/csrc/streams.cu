@@ -23,7 +23,8 @@ int dev_streams(DevStreams** out) {
         cudaStreamCreateWithFlags(&d.cp, cudaStreamNonBlocking) != cudaSuccess)
       return GPTQ2D_ERR_CUDA;
     cudaEvent_t* evs[] = {&d.fork,     &d.setup,    &d.join_hi,  &d.join_lo,  &d.join_hi2,
-                          &d.join_lo2, &d.cp_ev[0], &d.cp_ev[1], &d.cp_ev[2]};
+                          &d.join_lo2, &d.cp_ev[0], &d.cp_ev[1], &d.cp_ev[2], &d.q_ev[0],
+                          &d.q_ev[1],  &d.q_ev[2],  &d.q_ev[3]};
     for (auto* e : evs)
       if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GPTQ2D_ERR_CUDA;
     for (int r = 0; r < RING; ++r)
