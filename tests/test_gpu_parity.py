@@ -262,6 +262,37 @@ def test_attention_layer_4096(g):
     assert st["proxy_loss"] < rtn_loss
 
 
+@pytest.mark.slow
+def test_mlp_layer_4096x14336_int3(g):
+    """The rectangular MLP shape (m = 4096 < n = 14336) on the INT3 grid: factor rows
+    against LAPACK, the leading prefix against the oracle, sampled entries against the
+    definition, and the in-kernel loss against the direct trace."""
+    pb = WL.mlp(0, bits=3, matmul=_gpu_gram)
+    m, n = pb.shape
+    ML, MR = g.prepare_pair(dev(pb.H_L), dev(pb.H_R))
+    Q, st = g.quantize(dev(pb.W).to(torch.bfloat16), ML, MR, dev(pb.scales), pb.bits, pb.clamp)
+    Qg, st = Q.cpu().numpy(), g.stats_dict(st)
+    assert st["status"] == 0
+    MLo, MRo = O.reverse_cholesky(pb.H_L), O.reverse_cholesky(pb.H_R)
+    for M, Mo, rows in ((ML.cpu().numpy(), MLo, np.r_[0:3, 2047, 4093:4096]),
+                        (MR.cpu().numpy(), MRo, np.r_[0:3, 7000, 14333:14336])):
+        np.testing.assert_allclose(M[rows], Mo[rows], rtol=1e-8, atol=1e-10 * np.abs(Mo).max())
+    # W reaches the kernels as bf16: the oracle rounds the same bf16 values
+    W64 = torch.from_numpy(pb.W).to(torch.bfloat16).double().numpy()
+    s64 = pb.scales.astype(np.float64)
+    k, l = 320, 384
+    check_against_oracle(W64[:k, :l], MLo[:k, :k], MRo[:l, :l], s64[:k], pb.bits, pb.clamp,
+                         Qg[:k, :l])
+    rng = np.random.default_rng(1)
+    lo, hi = O.grid_bounds(pb.bits, pb.clamp)
+    for i, j in zip(rng.integers(0, m, 16), rng.integers(0, n, 16)):
+        t = O.entry_value(W64, Qg, s64, MLo, MRo, int(i), int(j)) / s64[i]
+        if not O.near_tie(np.array([t]), lo, hi)[0]:
+            assert Qg[i, j] == O.round_to_grid(t, lo, hi), (i, j, t)
+    direct = O.proxy_loss(W64, Qg, s64, pb.H_L, pb.H_R)
+    assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
+
+
 # --------------------------------------------------------------------------- #
 # both factors in one call
 # --------------------------------------------------------------------------- #

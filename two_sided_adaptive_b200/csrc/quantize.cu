@@ -749,24 +749,29 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
     const bool down = (d.flags & FD_DOWN) != 0;
     const double* Ts = slot_ptr(d.task_slot);
     const double* Hs = slot_ptr(d.sh_slot);
-    const double* As = down ? Ts : Hs;  // A(r, k) = As[r * SLD + k]
-    const double* Bs = down ? Hs : Ts;  // B(k, c) = down ? Bs[k * SLD + c] : Bs[c * SLD + k]
+    // A(r, k) = Ap[i * 8 * SLD + kk] for r = wr + 8i + g8, k = kk + t4 (both layouts);
+    // B(k, c) for c = wc + 8j + g8: down [k][c] -> Bp[kk * SLD + 8j], right [c][k] ->
+    // Bp[8j * SLD + kk].  Two loops with fixed strides, no per-load layout choice.
+    const double* Ap = (down ? Ts : Hs) + (wr + g8) * SLD + t4;
     double acc[4][4][2] = {};
+    auto product = [&](const double* Bp, int bk, int bj) {
 #pragma unroll 4
-    for (int kk = 0; kk < TB; kk += 4) {
-      double av[4], bv[4];
+      for (int kk = 0; kk < TB; kk += 4) {
+        double av[4], bv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[(wr + i * 8 + g8) * SLD + kk + t4];
+        for (int i = 0; i < 4; ++i) av[i] = Ap[i * 8 * SLD + kk];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = wc + j * 8 + g8;
-        bv[j] = down ? Bs[(kk + t4) * SLD + c] : Bs[c * SLD + kk + t4];
+        for (int j = 0; j < 4; ++j) bv[j] = Bp[kk * bk + j * bj];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], av[i], bv[j]);
-    }
+    };
+    if (down)
+      product(Hs + t4 * SLD + wc + g8, SLD, 8);
+    else
+      product(Ts + (wc + g8) * SLD + t4, 1, 8 * SLD);
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(&S.empty[d.task_slot]);
