@@ -69,6 +69,11 @@ __device__ __forceinline__ void load_block(double* dst, const double* M, int64_t
   }
 }
 
+// C += v by a reduction in L2, without reading C back.
+__device__ __forceinline__ void red_add(double* p, double v) {
+  asm volatile("red.global.add.f64 [%0], %1;\n" ::"l"(p), "d"(v) : "memory");
+}
+
 // The lower 8x8 blocks (bi >= bj) of Cs -= Xs^T Xs on `nw` warps, one block at a time
 // per warp (K = 64 in 16 DMMA steps).  The blocks above the diagonal are not used.
 __device__ __forceinline__ void sub_xtx_lower(double* Cs, const double* Xs, int nw) {
@@ -336,13 +341,13 @@ struct TrailPlan {
   int start[MAX_TR_GROUPS + 1];  // first CTA of each group; group g updates A[I0+g][0..I0+g]
 };
 
-constexpr int TR_SMEM = 3 * TB * OLD * (int)sizeof(double);
+constexpr int TR_SMEM = (3 * TB * OLD + 4 * 8 * 40) * (int)sizeof(double);
 
 // A_IJ -= M_KI^T M_KJ for J <= I, over a range of J of one block row I.  Each
 // CTA keeps M_KI in shared memory and streams the M_KJ blocks through a double
-// buffer; the A_IJ block is loaded into registers before the product so that
-// its latency overlaps the tensor-core work.  Only the lower part of A_II is
-// written.
+// buffer; the product goes into A_IJ by reductions in L2 (no read of the block),
+// one whole 256-byte row at a time through a shared strip.  Only the lower part
+// of A_II is touched.
 template <bool V16>
 __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restrict__ M,
                                                                  int64_t ldm, int k,
@@ -352,6 +357,7 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
   extern __shared__ __align__(16) double sm[];
   double* Xs = sm;  // Xs[r][i] = M[rb + r][64 I + i]
   double* const Y0 = sm + TB * OLD;
+  double* const stage = sm + 3 * TB * OLD;  // 4 warps x one 8x32 strip (row stride 40)
   auto ybuf = [&](int bsel) { return Y0 + bsel * (TB * OLD); };
   const int cta = blockIdx.x;
   int g;
@@ -383,22 +389,6 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
       load_block<V16, TR_THREADS>(ybuf(bsel ^ 1), M, ldm, rb, (J + 1) * TB, nb, TB);
       cp_async_commit_group();
     }
-    double* Cg = M + (int64_t)(I * TB + wr + g8) * ldm + (int64_t)J * TB + wc + 2 * t4;
-    double cv[4][4][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const double* src = Cg + (int64_t)i * 8 * ldm + j * 8;
-        if (V16) {
-          const double2 x = *reinterpret_cast<const double2*>(src);
-          cv[i][j][0] = x.x;
-          cv[i][j][1] = x.y;
-        } else {
-          cv[i][j][0] = src[0];
-          cv[i][j][1] = src[1];
-        }
-      }
     if (J + 1 < last) cp_async_wait_group<1>(); else cp_async_wait_group<0>();
     __syncthreads();
     const double* Ys = ybuf(bsel);
@@ -406,25 +396,24 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
     mma_64x64x64(
         acc, [&](int row, int kk) { return Xs[kk * OLD + row]; },
         [&](int kk, int col) { return Ys[kk * OLD + col]; }, kmax);
+    // A_IJ -= product by reductions in L2 (each element of the block gets exactly
+    // one contribution per launch): whole 256-byte rows through a shared strip
+    double* st = stage + warp * (8 * 40);
+    double* Cw = M + (int64_t)(I * TB + wr) * ldm + (int64_t)J * TB + wc;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = wr + i * 8 + g8, c = wc + j * 8 + 2 * t4;
-        double* dst = Cg + (int64_t)i * 8 * ldm + j * 8;
-        const double x0 = cv[i][j][0] - acc[i][j][0], x1 = cv[i][j][1] - acc[i][j][1];
-        if (I != J) {
-          if (V16) {
-            *reinterpret_cast<double2*>(dst) = make_double2(x0, x1);
-          } else {
-            dst[0] = x0;
-            dst[1] = x1;
-          }
-        } else {
-          if (c <= r) dst[0] = x0;
-          if (c + 1 <= r) dst[1] = x1;
-        }
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<double2*>(st + g8 * 40 + j * 8 + 2 * t4) =
+            make_double2(-acc[i][j][0], -acc[i][j][1]);
+      __syncwarp();
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int row = wr + i * 8 + r, col = wc + lane;
+        if (I != J || col <= row) red_add(Cw + (int64_t)(i * 8 + r) * ldm + lane, st[r * 40 + lane]);
       }
+      __syncwarp();
+    }
     __syncthreads();
   }
 }
