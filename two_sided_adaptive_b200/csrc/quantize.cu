@@ -154,24 +154,26 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
 // ---------------------------------------------------------------------------
 // set-up: normalised, tile-padded factors and their diagonals
 // ---------------------------------------------------------------------------
-__global__ void normalize_kernel(QArgs a) {
-  const int64_t nl = a.mp * a.mp, nr = a.np * a.np;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nl + nr;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    if (e < nl) {
-      const int i = (int)(e / a.mp), k = (int)(e % a.mp);
-      double v = 0.0;
-      if (i < a.m && k < i) v = a.ML[(int64_t)i * a.ldl + k] / a.ML[(int64_t)i * a.ldl + i];
-      a.Lh[e] = v;
-      if (k == 0) a.dL[i] = (i < a.m) ? a.ML[(int64_t)i * a.ldl + i] : 0.0;
-    } else {
-      const int64_t f = e - nl;
-      const int j = (int)(f / a.np), k = (int)(f % a.np);
-      double v = 0.0;
-      if (j < a.n && k < j) v = a.MR[(int64_t)j * a.ldr + k] / a.MR[(int64_t)j * a.ldr + j];
-      a.Rh[f] = v;
-      if (k == 0) a.dR[j] = (j < a.n) ? a.MR[(int64_t)j * a.ldr + j] : 0.0;
-    }
+// Normalised factors Lh = diag(M_L)^-1 M_L and Rh = diag(M_R)^-1 M_R, strictly
+// lower (the unit diagonal is implied), and the diagonals dL, dR.  Only the blocks
+// on or below the 64-block diagonal are written: no kernel reads the others.  One
+// CTA per row i (rows of Lh first, then rows of Rh); the threads take the columns
+// k < 64 (i / 64 + 1), two at a time.
+__global__ void __launch_bounds__(256) normalize_kernel(QArgs a) {
+  const bool left = blockIdx.x < a.mp;
+  const int i = left ? blockIdx.x : blockIdx.x - (int)a.mp;
+  const int64_t ldo = left ? a.mp : a.np;
+  const int dim = left ? a.m : a.n;
+  const double* Mrow = (left ? a.ML + (int64_t)i * a.ldl : a.MR + (int64_t)i * a.ldr);
+  double* out = (left ? a.Lh : a.Rh) + (int64_t)i * ldo;
+  const double d = i < dim ? Mrow[i] : 0.0;
+  if (threadIdx.x == 0) (left ? a.dL : a.dR)[i] = d;
+  const int kend = (i / TB + 1) * TB;  // end of the diagonal block
+  for (int k = 2 * threadIdx.x; k < kend; k += 2 * blockDim.x) {
+    double2 v;
+    v.x = (i < dim && k < i) ? Mrow[k] / d : 0.0;
+    v.y = (i < dim && k + 1 < i) ? Mrow[k + 1] / d : 0.0;
+    *reinterpret_cast<double2*>(out + k) = v;
   }
 }
 
@@ -243,10 +245,12 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
     }
   }
   cp_async_commit_group();
+  // far-field feedback reaches a tile only from two or more tiles away: P needs
+  // J >= 2 and E needs I >= 2 (else zero; those buffers may not be zeroed yet)
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
     const int r = x >> 5, c2 = (x & 31) * 2;
-    cp_async16_zfill(Pt + r * SLD + c2, a.P + ts + (int64_t)r * np + c2, true);
-    cp_async16_zfill(Vt + r * SLD + c2, a.E + ts + (int64_t)r * np + c2, true);
+    cp_async16_zfill(Pt + r * SLD + c2, J >= 2 ? a.P + ts + (int64_t)r * np + c2 : a.P, J >= 2);
+    cp_async16_zfill(Vt + r * SLD + c2, I >= 2 ? a.E + ts + (int64_t)r * np + c2 : a.E, I >= 2);
   }
   cp_async_commit_group();
   // row scales, their reciprocals and the factor diagonals of the tile
@@ -901,17 +905,17 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
             cudaStreamWaitEvent(lo, ds->fork, 0) == cudaSuccess;
   if (!ok) return GPTQ2D_ERR_CUDA;
 
-  // set-up on the high-priority stream: zero P and E, normalised factors
-  ok = cudaMemsetAsync(a.P, 0, (size_t)(L.off_D - L.off_P), hi) == cudaSuccess;
-  const int64_t nnorm = L.mp * L.mp + L.np * L.np;
-  const int nblk = (int)std::min<int64_t>((nnorm + 255) / 256, (int64_t)ds->sms * 8);
-  GPTQ2D_LAUNCH(KC_OTHER, hi, normalize_kernel<<<nblk, 256, 0, hi>>>(a));
+  // set-up: normalised factors on the high-priority stream (the first sweeps need
+  // them); zero P and E and the counters on the low-priority one, where only the
+  // far-field launches, which run after it, write them (the sweeps of tiles with
+  // I < 2 or J < 2, which get no far-field feedback, do not read them)
+  GPTQ2D_LAUNCH(KC_OTHER, hi, normalize_kernel<<<(int)(L.mp + L.np), 256, 0, hi>>>(a));
+  ok = ok && cudaMemsetAsync(a.P, 0, (size_t)(L.off_D - L.off_P), lo) == cudaSuccess;
+  int* counters = a.err + 1;
+  ok = ok && cudaMemsetAsync(a.err, 0, (1 + (size_t)L.n_cnt * MAX_GROUPS) * sizeof(int), lo) ==
+                  cudaSuccess;
   ok = ok && cudaEventRecord(ds->setup, hi) == cudaSuccess &&
        cudaStreamWaitEvent(lo, ds->setup, 0) == cudaSuccess;
-
-  int* counters = a.err + 1;
-  ok = ok && cudaMemsetAsync(a.err, 0, (1 + (size_t)L.n_cnt * MAX_GROUPS) * sizeof(int), hi) ==
-                  cudaSuccess;
   const int nd = a.Tm + a.Tn - 1;
   const int sms = ds->sms;
   int next_cnt = 0;
