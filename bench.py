@@ -478,13 +478,78 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_block70b(args):
+    """Seconds per layer and for the whole block: the seven linear layers of one
+    70B-class block (q, o: 8192x8192; k, v: 1024x8192; gate, up: 8192x28672; down:
+    28672x8192), INT4 per-row absmax scales, W ~ N(0, 0.015^2) in bf16, Grams from
+    Student-t(4) activations times U(0.1, 10) column scales with rows = width, plus 1%
+    mean-diagonal damping.  The inputs are generated on the GPU (torch, seeded per
+    layer) because the largest Gram is 28672^2; each layer is timed with CUDA events
+    over prepare_pair + quantize with its inputs resident in HBM."""
+    import torch
+    import two_sided_adaptive_b200 as g
+    from two_sided_adaptive_b200 import build as gbuild
+    import workloads as WL
+    gbuild.build()
+    dev = torch.device("cuda", 0)
+    layers, total = [], 0.0
+    for li, (name, m, n, _) in enumerate(WL.block70b_shapes()):
+        torch.manual_seed(1000 + li)
+
+        def gram(width):
+            z = torch.randn(width, width, device=dev, dtype=torch.float64)
+            chi2 = torch.distributions.Chi2(torch.tensor(4.0, device=dev, dtype=torch.float64))
+            X = z / torch.sqrt(chi2.sample((width, width)) / 4.0)
+            del z
+            X *= torch.empty(width, device=dev, dtype=torch.float64).uniform_(0.1, 10.0)[None, :]
+            G = X.T @ X / width
+            del X
+            G = 0.5 * (G + G.T)
+            G.diagonal().add_(0.01 * G.diagonal().mean())
+            return G.float()
+        HL, HR = gram(m), gram(n)
+        W = (torch.randn(m, n, device=dev, dtype=torch.float32) * 0.015).to(torch.bfloat16)
+        s = (W.float().abs().amax(dim=1) / 7.0).clamp_min(1e-30).contiguous()
+        ML = torch.empty((m, m), dtype=torch.float64, device=dev)
+        MR = torch.empty((n, n), dtype=torch.float64, device=dev)
+        wsP = torch.empty(512, dtype=torch.uint8, device=dev)
+        wsQ = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
+        Q = torch.empty((m, n), dtype=torch.int8, device=dev)
+        st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for rep in range(2):  # the first pass warms up
+            torch.cuda.synchronize()
+            e[0].record()
+            g.prepare_pair(HL, HR, out_l=ML, out_r=MR, workspace=wsP, check=False)
+            e[1].record()
+            g.quantize(W, ML, MR, s, 4, True, out=Q, stats=st, workspace=wsQ)
+            e[2].record()
+            torch.cuda.synchronize()
+        sd = g.stats_dict(st)
+        tp, tq = e[0].elapsed_time(e[1]) / 1e3, e[1].elapsed_time(e[2]) / 1e3
+        total += tp + tq
+        layers.append({"layer": name, "m": m, "n": n, "prepare_s": tp, "quantize_s": tq,
+                       "entries_per_s": m * n / (tp + tq),
+                       "quantize_fp64_tflops": m * n * (m + n) / tq / 1e12,
+                       "status": sd["status"], "n_near_tie": sd["n_near_tie"]})
+        del HL, HR, W, s, ML, MR, wsP, wsQ, Q, st
+        torch.cuda.empty_cache()
+    return {"metric": "70B-class block: seconds for its 7 linear layers (INT4, 1 B200)",
+            "value": total, "unit": "s", "n_gpus": 1, "higher_is_better": False,
+            "dtype": "f64", "data": "synthetic (generated on the GPU, see run_block70b)",
+            "config": {"workload": "block70b", "step": "prepare_pair + quantize per layer"},
+            "layers": layers}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("attn", "mlp", "small"), default="attn")
+    ap.add_argument("--workload", choices=("attn", "mlp", "small", "block70b"), default="attn",
+                    help="block70b: seconds per layer for one 70B-class block (a report, not the "
+                         "headline metric)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=768)
@@ -506,6 +571,10 @@ def main():
 
     import torch
     torch.cuda.set_device(local_rank)
+    if args.workload == "block70b":
+        if rank == 0:
+            print(json.dumps(run_block70b(args)), flush=True)
+        return
     if world > 1:
         import datetime
         import torch.distributed as dist
