@@ -83,6 +83,15 @@ int gptq2d_version(void);
  * devices, all threads).  Lets a caller count launches inside a timed region. */
 int64_t gptq2d_launch_count(void);
 
+/* Self-check of the device-side bounded waits: runs the wait the far-field
+ * kernel uses on an mbarrier that nothing completes, with a limit of `limit_ns`
+ * nanoseconds (1000 .. 10^10), on `stream`, and synchronizes it (no allocation:
+ * the status goes through a static device word).  Returns
+ * GPTQ2D_ERR_TIMEOUT when the wait gave up as it must (the device stays usable),
+ * GPTQ2D_ERR_INVALID_ARG for a limit out of range, GPTQ2D_ERR_CUDA on a launch
+ * error; GPTQ2D_OK would mean the wait did not time out. */
+int gptq2d_check_wait_timeout(int64_t limit_ns, void* stream);
+
 /* Optional per-launch timing (off by default).  While enabled, every kernel the
  * library launches is bracketed by a pair of CUDA events recorded on the
  * launching stream; events are created on first use and recycled.  Kernel

@@ -104,6 +104,12 @@ def test_round_host_rejects_invalid_arguments(L):
     assert R(*args[:12], 256, 10, *args[14:]) == g.Status.WORKSPACE
 
 
+def test_wait_timeout_check_rejects_limits_out_of_range(L):
+    # argument checks come before any CUDA call
+    for bad in (0, 999, 10_000_000_001, -5):
+        assert L.gptq2d_check_wait_timeout(ctypes.c_int64(bad), None) == 1  # INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(g, "library_path", str(tmp_path / "missing.so"))
     monkeypatch.setattr(g, "_LIB", None)

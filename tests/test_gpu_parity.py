@@ -314,3 +314,20 @@ def test_prepare_pair_reports_which_factor(g, bad_side):
         g.prepare_pair(dev(H_L), dev(H_R))
     assert ei.value.status == g.Status.NOT_SPD
     assert f"factor {bad_side} pivot 33" in str(ei.value)
+
+
+# --------------------------------------------------------------------------- #
+# failure detection without a fault: a bounded device wait that must give up
+# --------------------------------------------------------------------------- #
+def test_bounded_wait_times_out_and_device_stays_usable(g):
+    import time
+    t0 = time.perf_counter()
+    assert g.check_wait_timeout(50_000_000) == g.Status.TIMEOUT  # 50 ms on a barrier nobody completes
+    assert time.perf_counter() - t0 >= 0.05
+    pb = WL.small(0, 96, 80)
+    ML, MR = g.prepare(dev(pb.H_L)), g.prepare(dev(pb.H_R))
+    Q, st = g.quantize(dev(pb.W), ML, MR, dev(pb.scales), pb.bits, pb.clamp)
+    assert g.stats_dict(st)["status"] == 0
+    check_against_oracle(pb.W.astype(np.float64), O.reverse_cholesky(pb.H_L),
+                         O.reverse_cholesky(pb.H_R), pb.scales.astype(np.float64), pb.bits,
+                         pb.clamp, Q.cpu().numpy())

@@ -19,7 +19,8 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
-    "round_host_workspace_size", "quantize_noalloc", "profile_enable", "profile_reset", "profile_read", "profile_timeline",
+    "round_host_workspace_size", "quantize_noalloc", "check_wait_timeout", "profile_enable",
+    "profile_reset", "profile_read", "profile_timeline",
     "KERNEL_CLASSES", "STATS_WORDS", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F64",
 ]
 
@@ -64,6 +65,8 @@ def lib():
         L.gptq2d_status_string.argtypes = [ctypes.c_int]
         L.gptq2d_version.restype = ctypes.c_int
         L.gptq2d_launch_count.restype = _c_i64
+        L.gptq2d_check_wait_timeout.restype = ctypes.c_int
+        L.gptq2d_check_wait_timeout.argtypes = [_c_i64, _c_p]
         L.gptq2d_profile_enable.restype = None
         L.gptq2d_profile_enable.argtypes = [ctypes.c_int]
         L.gptq2d_profile_read.restype = ctypes.c_int
@@ -107,6 +110,13 @@ def lib():
 def launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(lib().gptq2d_launch_count())
+
+
+def check_wait_timeout(limit_ns: int, stream=None) -> int:
+    """Runs the device-side bounded wait on an mbarrier that nothing completes
+    (gptq2d_check_wait_timeout); returns the status, Status.TIMEOUT when the wait
+    gave up as it must."""
+    return int(lib().gptq2d_check_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 KERNEL_CLASSES = ("prep_panel", "prep_trailing", "sweep", "propagate", "other")

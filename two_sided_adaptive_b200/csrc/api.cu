@@ -123,6 +123,11 @@ int gptq2d_version(void) { return (1 << 16) | 0; }
 
 int64_t gptq2d_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int gptq2d_check_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return GPTQ2D_ERR_INVALID_ARG;
+  return check_wait_timeout(limit_ns, static_cast<cudaStream_t>(stream));
+}
+
 void gptq2d_profile_enable(int on) { g_prof_on.store(on != 0); }
 
 int gptq2d_profile_read(int kernel_class, int64_t* launches, double* total_ms) {

@@ -173,6 +173,7 @@ int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_
                         cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr);
 
 size_t quantize_ws_bytes(int64_t m, int64_t n);
+int check_wait_timeout(long long limit_ns, cudaStream_t s);  // synchronizes s
 // Optional row events: row_ev[k] is recorded once the tile rows 0..row_tile[k] of
 // Q are final (row_tile ascending), so a caller can copy them out early.
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,

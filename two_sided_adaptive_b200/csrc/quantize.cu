@@ -134,12 +134,26 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // Waits for the phase of `bar` with the given parity to complete; gives up after
 // kWaitLimitNs and returns false (the caller reports a timeout).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (!mbar_try_wait(bar, parity))
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   return true;
+}
+
+// The bounded wait above on an mbarrier that nothing completes: the check behind
+// gptq2d_check_wait_timeout.  *status = GPTQ2D_ERR_TIMEOUT once the wait has
+// given up (GPTQ2D_OK would mean the barrier completed).
+__global__ void wait_timeout_kernel(unsigned long long limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  __syncthreads();
+  const bool done = mbar_wait(&bar, 0, limit_ns);
+  __syncwarp();
+  if (threadIdx.x == 0) *status = done ? GPTQ2D_OK : GPTQ2D_ERR_TIMEOUT;
 }
 // One bulk copy global -> shared (TMA engine, no multicast), completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar,
@@ -1038,6 +1052,24 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
 }  // namespace
 
 size_t quantize_ws_bytes(int64_t m, int64_t n) { return layout(m, n).total; }
+
+namespace {
+__device__ int g_wait_status;
+}  // namespace
+
+int check_wait_timeout(long long limit_ns, cudaStream_t s) {
+  int* st = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st), g_wait_status) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  GPTQ2D_LAUNCH(KC_OTHER, s,
+                wait_timeout_kernel<<<1, 32, 0, s>>>((unsigned long long)limit_ns, st));
+  int host = GPTQ2D_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpyAsync(&host, st, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  return host;
+}
 
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
