@@ -245,9 +245,9 @@ size_t gptq2d_round_host_workspace_size(int64_t m, int64_t n, int w_dtype, int h
  * triangles of H_L (m x m) and H_R (n x n) (each 64-row block up to the end of
  * its diagonal block; the rest is never read) and scales to the device
  * workspace, factors both Kronecker factors, rounds, and copies Q (m x n int8,
- * dense) and the statistics back.  The copies go over an internal stream in the
- * order H_L, H_R, W: each factorization starts when its Gram is in, and the
- * later copies run under it.  Host buffers should be pinned for asynchronous
+ * dense) and the statistics back.  The copies go over an internal stream, the
+ * larger Gram first, then the other, then W: each factorization starts when its
+ * Gram is in, and the later copies run under it.  Host buffers should be pinned for asynchronous
  * copies.  Synchronizes `stream` before returning.  Returns GPTQ2D_ERR_NOT_SPD if either factor is
  * not positive definite (the left factor is checked first; *bad_pivot, if
  * non-NULL, receives the pivot, and *which_factor, if non-NULL, 0 for H_L and

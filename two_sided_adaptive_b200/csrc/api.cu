@@ -290,10 +290,9 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
   DevStreams* ds = nullptr;
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
-  // Inputs go over one copy stream in the order they are needed: H_L, then H_R,
-  // then W and the scales.  Factor L starts once H_L is in, factor R once H_R is,
-  // and the rounding once both factors and W are done, so the later copies run
-  // under the factorizations.
+  // Inputs go over one copy stream in the order they are needed: the Grams, then W
+  // and the scales.  Each factor starts once its Gram is in, and the rounding once
+  // both factors and W are done, so the later copies run under the factorizations.
   // Only the lower triangle of a Gram is read, so each 64-row block is copied up to
   // the end of its diagonal block (about half of the matrix).
   auto copy_lower = [&](char* dst, const void* src, int64_t k) -> bool {
@@ -308,10 +307,14 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
     return true;
   };
   std::lock_guard<std::recursive_mutex> lk(ds->mu);
+  // the larger Gram first: its factorization takes longer
+  const bool r_first = n > m;
   if (cudaEventRecord(ds->fork, s) != cudaSuccess ||
-      cudaStreamWaitEvent(ds->cp, ds->fork, 0) != cudaSuccess || !copy_lower(b + L.off_HL, H_L, m) ||
-      cudaEventRecord(ds->cp_ev[0], ds->cp) != cudaSuccess || !copy_lower(b + L.off_HR, H_R, n) ||
-      cudaEventRecord(ds->cp_ev[1], ds->cp) != cudaSuccess ||
+      cudaStreamWaitEvent(ds->cp, ds->fork, 0) != cudaSuccess ||
+      !(r_first ? copy_lower(b + L.off_HR, H_R, n) : copy_lower(b + L.off_HL, H_L, m)) ||
+      cudaEventRecord(ds->cp_ev[r_first ? 1 : 0], ds->cp) != cudaSuccess ||
+      !(r_first ? copy_lower(b + L.off_HL, H_L, m) : copy_lower(b + L.off_HR, H_R, n)) ||
+      cudaEventRecord(ds->cp_ev[r_first ? 0 : 1], ds->cp) != cudaSuccess ||
       cudaMemcpyAsync(b + L.off_W, W, (size_t)m * n * elem_size(w_dtype), cudaMemcpyHostToDevice,
                       ds->cp) ||
       cudaMemcpyAsync(b + L.off_s, scales, (size_t)m * sizeof(float), cudaMemcpyHostToDevice,
