@@ -206,6 +206,50 @@ def test_round_host_matches_device_path(g):
     assert g.stats_dict(sth) == g.stats_dict(std)
 
 
+def test_round_host_wide_layer_copies_right_gram_first(g):
+    # n > m: the right Gram goes over first; the result must not depend on the order
+    pb = WL.small(5, 96, 300)
+    Wh = torch.from_numpy(pb.W).pin_memory()
+    HLh = torch.from_numpy(pb.H_L).pin_memory()
+    HRh = torch.from_numpy(pb.H_R).pin_memory()
+    sh = torch.from_numpy(pb.scales).pin_memory()
+    Qh, sth = g.round_host(Wh, HLh, HRh, sh, pb.bits, pb.clamp)
+    ML, MR = g.prepare(dev(pb.H_L)), g.prepare(dev(pb.H_R))
+    Qd, std = g.quantize(dev(pb.W), ML, MR, dev(pb.scales), pb.bits, pb.clamp)
+    assert torch.equal(Qh, Qd.cpu())
+    assert g.stats_dict(sth) == g.stats_dict(std)
+
+
+def test_concurrent_callers_share_the_internal_streams(g):
+    # two host threads round different problems at once on their own streams: the
+    # enqueues on the library's internal streams are serialised, the results are the
+    # serial ones
+    import threading
+    probs = [WL.small(10 + k, 160 + 32 * k, 200 - 24 * k) for k in range(2)]
+    inputs = []
+    for pb in probs:
+        ML, MR = g.prepare(dev(pb.H_L)), g.prepare(dev(pb.H_R))
+        inputs.append((dev(pb.W), ML, MR, dev(pb.scales), pb.bits, pb.clamp))
+    serial = [g.quantize(*x) for x in inputs]
+    torch.cuda.synchronize()
+    out = [None, None]
+
+    def work(k):
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            for _ in range(3):
+                out[k] = g.quantize(*inputs[k], stream=st)
+        st.synchronize()
+    th = [threading.Thread(target=work, args=(k,)) for k in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    for k in range(2):
+        assert torch.equal(out[k][0], serial[k][0])
+        assert g.stats_dict(out[k][1]) == g.stats_dict(serial[k][1])
+
+
 def test_round_host_reports_non_spd(g):
     m, n = 16, 12
     W = torch.zeros((m, n), dtype=torch.float32).pin_memory()
