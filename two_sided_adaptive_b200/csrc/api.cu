@@ -93,13 +93,16 @@ HostWs host_layout(int64_t m, int64_t n, int w_dtype, int h_dtype) {
   return L;
 }
 
+// The pivot word of a factorization: -1 fine, >= 0 the first bad pivot.
+int pivot_status(long long info) { return info >= 0 ? GPTQ2D_ERR_NOT_SPD : GPTQ2D_OK; }
+
 int read_pivot(const void* ws, cudaStream_t s, int64_t* bad_pivot) {
   long long info = -1;
   if (cudaMemcpyAsync(&info, ws, sizeof(info), cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
-  if (bad_pivot) *bad_pivot = info;
-  return info >= 0 ? GPTQ2D_ERR_NOT_SPD : GPTQ2D_OK;
+  if (bad_pivot) *bad_pivot = info >= 0 ? info : -1;
+  return pivot_status(info);
 }
 
 }  // namespace
@@ -227,10 +230,10 @@ int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl, const void* H_
     return GPTQ2D_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
   for (int f = 0; f < 2; ++f)
-    if (piv[f] >= 0) {
-      if (bad_pivot) *bad_pivot = piv[f];
+    if (pivot_status(piv[f]) != GPTQ2D_OK) {
+      if (bad_pivot) *bad_pivot = piv[f] >= 0 ? piv[f] : -1;
       if (which_factor) *which_factor = f;
-      return GPTQ2D_ERR_NOT_SPD;
+      return pivot_status(piv[f]);
     }
   if (bad_pivot) *bad_pivot = -1;
   if (which_factor) *which_factor = -1;
@@ -358,10 +361,10 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
     return GPTQ2D_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
   for (int f = 0; f < 2; ++f)
-    if (piv[f] >= 0) {
-      if (bad_pivot) *bad_pivot = piv[f];
+    if (pivot_status(piv[f]) != GPTQ2D_OK) {
+      if (bad_pivot) *bad_pivot = piv[f] >= 0 ? piv[f] : -1;
       if (which_factor) *which_factor = f;
-      return GPTQ2D_ERR_NOT_SPD;
+      return pivot_status(piv[f]);
     }
   if (bad_pivot) *bad_pivot = -1;
   if (which_factor) *which_factor = -1;

@@ -22,6 +22,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "pipeline.cuh"
 
 namespace gptq2d {
 
@@ -67,11 +68,6 @@ __device__ __forceinline__ void load_block(double* dst, const double* M, int64_t
       cp_async8_zfill(dst + r * OLD + c, src, ok);
     }
   }
-}
-
-// C += v by a reduction in L2, without reading C back.
-__device__ __forceinline__ void red_add(double* p, double v) {
-  asm volatile("red.global.add.f64 [%0], %1;\n" ::"l"(p), "d"(v) : "memory");
 }
 
 // The lower 8x8 blocks (bi >= bj) of Cs -= Xs^T Xs on `nw` warps, one block at a time
@@ -224,7 +220,7 @@ template <bool V16>
 __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict__ M, int64_t ldm,
                                                               int k, int K, long long* info) {
   if (*(volatile long long*)info >= 0) return;
-  extern __shared__ __align__(16) double sm[];
+  extern __shared__ __align__(128) double sm[];
   double* Ad = sm;              // A_KK, then M_KK
   double* Ab = Ad + TB * OLD;   // A_Kb, then M_Kb
   double* Mn = Ab + TB * OLD;   // M_{K+1,K}
@@ -354,7 +350,7 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
                                                                  const long long* info,
                                                                  TrailPlan pl) {
   if (*(volatile const long long*)info >= 0) return;
-  extern __shared__ __align__(16) double sm[];
+  extern __shared__ __align__(128) double sm[];
   double* Xs = sm;  // Xs[r][i] = M[rb + r][64 I + i]
   double* const Y0 = sm + TB * OLD;
   double* const stage = sm + 3 * TB * OLD;  // 4 warps x one 8x32 strip (row stride 40)

@@ -47,6 +47,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "pipeline.cuh"
 
 namespace gptq2d {
 
@@ -84,65 +85,6 @@ struct QArgs {
 // ---------------------------------------------------------------------------
 // small PTX helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
-  return p;
-}
-// C += v without reading C back: each C element gets one contribution per
-// far-field launch and launches on one plan are stream-ordered, so the sum is
-// the same as a load, add and store.
-__device__ __forceinline__ void red_add(double* p, double v) {
-  asm volatile("red.global.add.f64 [%0], %1;\n" ::"l"(p), "d"(v) : "memory");
-}
-
-// ---- mbarriers and bulk copies (the far-field kernel's producer/consumer pipeline)
-__device__ __forceinline__ unsigned smem_u32(const void* p) {
-  return static_cast<unsigned>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
-  return t;
-}
-// Waits for the phase of `bar` with the given parity to complete; gives up after
-// kWaitLimitNs and returns false (the caller reports a timeout).
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity,
-                                          unsigned long long limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (global_ns() - t0 > limit_ns) return false;
-  return true;
-}
-
 // The bounded wait above on an mbarrier that nothing completes: the check behind
 // gptq2d_check_wait_timeout.  *status = GPTQ2D_ERR_TIMEOUT once the wait has
 // given up (GPTQ2D_OK would mean the barrier completed).
@@ -154,15 +96,6 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns, int* status) {
   const bool done = mbar_wait(&bar, 0, limit_ns);
   __syncwarp();
   if (threadIdx.x == 0) *status = done ? GPTQ2D_OK : GPTQ2D_ERR_TIMEOUT;
-}
-// One bulk copy global -> shared (TMA engine, no multicast), completing on `bar`.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar,
-                                         uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;\n" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
 }
 
 // ---------------------------------------------------------------------------
