@@ -33,6 +33,11 @@ Functions, from most literal to fastest:
   O2  gptq2d_antidiagonal           the cubic anti-diagonal algorithm
 and the special cases used as pins: RTN, 1-D GPTQ in OBS form, exhaustive
 closest-vector search on tiny problems.
+
+Hessians with k > 2 Kronecker factors (arxivlens, Abstract), W a k-way tensor:
+  O1k babai_tensor_sweep            1-D GPTQ over the C-order flattening, explicit Gram
+  O2k gptq_kron_hyperplane          hyperplane order, per-mode factors applied separately
+      gptq_kron_via_2d              the same problem as a 2-D one with H_R = H_2 kron ... kron H_k
 """
 from __future__ import annotations
 
@@ -370,3 +375,135 @@ def sphere_decode(W, H_L, H_R, s, bits, clamp):
     rec(0, 0.0)
     to_q = lambda v: (v / sv).reshape((m, n), order="F")
     return to_q(best[1]), best[0], to_q(first[0])
+
+
+# --------------------------------------------------------------------------- #
+# Hessians with more than two Kronecker factors (arxivlens, Abstract: the
+# algorithm extends to any number of Kronecker factors)
+# --------------------------------------------------------------------------- #
+# Reading: W is a k-way tensor of shape (m_1, ..., m_k), stored in C order (last
+# index fastest); H_j (m_j x m_j) acts on mode j, so the proxy loss is
+#     L(Q) = sum_{i, i'} dW[i] dW[i'] prod_j H_j[i_j, i'_j]
+# and on the C-order flattening the Gram is H_1 kron H_2 kron ... kron H_k.  Scales
+# are per index of mode 1 (the output channel), as the per-row scales of the 2-D
+# case.  With two factors this is the 2-D problem with H_L = H_1, H_R = H_2.
+
+
+def kron_gram(Hs):
+    """G = H_1 kron ... kron H_k: the Gram of the C-order flattening."""
+    G = np.ones((1, 1))
+    for H in Hs:
+        G = np.kron(G, np.asarray(H, np.float64))
+    return G
+
+
+def babai_tensor_sweep(W, Hs, s, bits, clamp):
+    """1-D GPTQ over all coordinates of the tensor in C order (a linear extension
+    of the product order on multi-indices), on the explicit Gram kron_gram(Hs):
+    the same form as babai_kron_sweep (upper Cholesky factor of G^{-1}, each
+    rounding error divided by the pivot and pushed along its row).  Returns (Q, T)
+    shaped like W.  Tiny problems only (the Gram is N x N, N = W.size).
+    """
+    W = np.asarray(W, np.float64)
+    lo, hi = grid_bounds(bits, clamp)
+    G = kron_gram(Hs)
+    U = np.linalg.cholesky(np.linalg.inv(G)).T
+    x = W.reshape(-1).copy()
+    N = x.size
+    sv = np.repeat(np.asarray(s, np.float64), N // W.shape[0])   # mode 1 is the slowest index
+    Q = np.zeros(N)
+    T = np.zeros(N)
+    for p in range(N):
+        T[p] = x[p] / sv[p]
+        Q[p] = round_to_grid(T[p], lo, hi)
+        e = (x[p] - sv[p] * Q[p]) / U[p, p]
+        x[p + 1:] -= e * U[p, p + 1:]
+    return Q.reshape(W.shape), T.reshape(W.shape)
+
+
+def mode_product(X, M, j):
+    """(X x_j M)[..., a, ...] = sum_b M[a, b] X[..., b, ...] (mode-j product)."""
+    return np.moveaxis(np.tensordot(M, X, axes=([1], [j])), 0, j)
+
+
+def gptq_kron_hyperplane(W, Ms, s, bits, clamp):
+    """GPTQ with a k-factor Kronecker Hessian, hyperplane by hyperplane.
+
+    With lower factors M_j (M_j^T M_j = H_j), the triangular factor of the
+    flattened problem is M_1 kron ... kron M_k, so the value rounded at entry i
+    is
+        y_i = W_i + (dW x_1 M_1 x_2 M_2 ... x_k M_k)_i / prod_j M_j[i_j, i_j]
+    with dW = 0 on the entries not rounded yet (i itself included): each mode's
+    factor applied separately (the separable feedback), and only the dominated
+    orthant {i' <= i} contributes because every M_j is lower triangular.  The
+    entries of one hyperplane i_1 + ... + i_k = d depend only on earlier
+    hyperplanes, so each hyperplane is rounded as one vector.  Evaluated from
+    scratch for every hyperplane: small tensors only.
+
+    Returns a Result (Q, T = y/s, loss by the nearest-plane identity, clamp count,
+    near-tie mask), arrays shaped like W.
+    """
+    W = np.asarray(W, np.float64)
+    Ms = [np.asarray(M, np.float64) for M in Ms]
+    if len(Ms) != W.ndim or any(M.shape != (d, d) for M, d in zip(Ms, W.shape)):
+        raise ValueError("one square factor per mode")
+    s = np.asarray(s, np.float64)
+    lo, hi = grid_bounds(bits, clamp)
+    idx = np.indices(W.shape)
+    level = idx.sum(axis=0)
+    diag = np.ones(W.shape)
+    for j, M in enumerate(Ms):
+        diag = diag * np.diag(M)[idx[j]]
+    srow = s[idx[0]]
+    D = np.zeros(W.shape)
+    Q = np.zeros(W.shape)
+    T = np.zeros(W.shape)
+    tie = np.zeros(W.shape, bool)
+    loss = 0.0
+    n_clamped = 0
+    for d in range(int(level.max()) + 1 if W.size else 0):
+        F = D
+        for j, M in enumerate(Ms):
+            F = mode_product(F, M, j)
+        sel = level == d
+        y = W[sel] + F[sel] / diag[sel]
+        t = y / srow[sel]
+        q_raw = np.rint(t)
+        q = np.clip(q_raw, lo, hi)
+        n_clamped += int(np.count_nonzero(q != q_raw))
+        D[sel] = W[sel] - srow[sel] * q
+        loss += float(np.sum((diag[sel] * (y - srow[sel] * q)) ** 2))
+        Q[sel] = q
+        T[sel] = t
+        tie[sel] = near_tie(t, lo, hi)
+    return Result(Q, T, loss, n_clamped, tie, set())
+
+
+def proxy_loss_tensor(W, Q, s, Hs):
+    """L(Q) = sum dW[i] dW[i'] prod_j H_j[i_j, i'_j], dW = W - s Q (s along mode 1)."""
+    W = np.asarray(W, np.float64)
+    D = W - np.asarray(s, np.float64).reshape((-1,) + (1,) * (W.ndim - 1)) * np.asarray(Q, np.float64)
+    HD = D
+    for j, H in enumerate(Hs):
+        HD = mode_product(HD, np.asarray(H, np.float64), j)
+    return float(np.sum(D * HD))
+
+
+def kron_factor(Ms):
+    """M_1 kron ... kron M_k of lower factors: lower triangular, and the reverse
+    Cholesky factor of H_1 kron ... kron H_k (uniqueness of the factor with a
+    positive diagonal)."""
+    return kron_gram(Ms)
+
+
+def gptq_kron_via_2d(W, Ms, s, bits, clamp, **kw):
+    """The k-factor problem as a 2-D one: rows = mode 1 (H_L = H_1), columns = modes
+    2..k flattened in C order (H_R = H_2 kron ... kron H_k, factor M_2 kron ... kron
+    M_k).  Column-major vec of that m_1 x (m_2...m_k) matrix orders the coordinates
+    by a linear extension of the k-way product order, and its factor has the
+    k-way dominated-orthant sparsity, so the anti-diagonal algorithm computes the
+    same rounding.  Returns the 2-D Result (arrays m_1 x N/m_1)."""
+    W = np.asarray(W, np.float64)
+    W2 = W.reshape(W.shape[0], -1)
+    M_R = kron_factor(Ms[1:]) if len(Ms) > 1 else np.ones((1, 1))
+    return gptq2d_antidiagonal(W2, Ms[0], M_R, s, bits, clamp, **kw)
