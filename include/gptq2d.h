@@ -171,6 +171,38 @@ int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl,
 int gptq2d_prepare_info(const void* ws, void* stream, int64_t* bad_pivot);
 
 /* ------------------------------------------------------------------------- */
+/* Hessians with more than two Kronecker factors (arxivlens "GPTQ-2D: Cubic-   */
+/* Time Two-Sided Adaptive Rounding", Abstract: the algorithm extends to any   */
+/* number of Kronecker factors).                                               */
+/* ------------------------------------------------------------------------- */
+
+/* Largest number of factors gptq2d_kron_factor combines. */
+#define GPTQ2D_MAX_KRON_FACTORS 8
+
+/* Kronecker product of lower factors.  A k-way tensor W of shape (m_1, ..., m_k),
+ * row-major (C order), under H = H_1 (x) H_2 (x) ... (x) H_k (H_j acting on mode
+ * j) is rounded as the m_1 x (m_2 ... m_k) matrix with H_L = H_1 and
+ * H_R = H_2 (x) ... (x) H_k.  The reverse Cholesky factor of that H_R is
+ * M_R = M_2 (x) ... (x) M_k (M_j from gptq2d_prepare of H_j), which this call
+ * forms; gptq2d_quantize with M_L = M_1 then gives the k-way rounding: every
+ * entry sees only its dominated orthant {i' : i'_j <= i_j for all j}, and the
+ * result equals the 1-D sweep over the tensor's coordinates in any order that
+ * respects that product order.  Scales are per index of mode 1.
+ *
+ *   nf           : number of factors, 1 <= nf <= GPTQ2D_MAX_KRON_FACTORS.
+ *   M, dims, ldm : HOST arrays of nf entries.  M[f] is a DEVICE pointer to a
+ *                  dims[f] x dims[f] fp64 lower factor, row-major with leading
+ *                  dimension ldm[f] >= dims[f]; its strict upper triangle is not read.
+ *   out, ldo     : DEVICE fp64 output, n x n row-major, n = prod dims <= 2^20,
+ *                  ldo >= n.  With r = (r_1, ..., r_nf) and c the mixed-radix digits
+ *                  of the row and column (last factor fastest),
+ *                  out[r][c] = prod_f M[f][r_f][c_f] when every c_f <= r_f, and an
+ *                  exact zero otherwise.  Must not overlap a factor.
+ * n == 0 (a zero dimension) writes nothing and returns GPTQ2D_OK. */
+int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
+                       double* out, int64_t ldo, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Rounding                                                                    */
 /* ------------------------------------------------------------------------- */
 

@@ -115,3 +115,25 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(g, "_LIB", None)
     with pytest.raises(RuntimeError, match="not built"):
         g.lib()
+
+
+def _kron(L, nf=2, ptrs=(4096, 8192), dims=(4, 4), lds=(4, 4), out=1 << 20, ldo=16):
+    P = (ctypes.c_void_p * len(ptrs))(*ptrs) if ptrs is not None else None
+    D = (ctypes.c_int64 * len(dims))(*dims) if dims is not None else None
+    S = (ctypes.c_int64 * len(lds))(*lds) if lds is not None else None
+    return L.gptq2d_kron_factor(nf, P, D, S, out, ldo, None)
+
+
+@pytest.mark.parametrize("bad", [dict(nf=0), dict(nf=9), dict(ptrs=None), dict(dims=None),
+                                 dict(lds=None), dict(dims=(4, -1)), dict(lds=(3, 4)),
+                                 dict(ldo=15), dict(out=None), dict(dims=(1 << 11, 1 << 10)),
+                                 dict(ptrs=(4096, 0)), dict(out=4096 + 8)])
+def test_kron_factor_rejects_invalid_arguments(L, bad):
+    """Checked on the host before anything is enqueued (no GPU needed): factor count,
+    null arrays, sizes, leading dimensions, n = prod dims <= 2^20, an output that
+    overlaps a factor."""
+    assert _kron(L, **bad) == g.Status.INVALID_ARG
+
+
+def test_kron_factor_with_a_zero_dimension_is_a_no_op(L):
+    assert _kron(L, dims=(4, 0), out=None) == g.Status.OK

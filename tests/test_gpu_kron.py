@@ -1,0 +1,138 @@
+"""GPU parity for Hessians with more than two Kronecker factors (arxivlens
+"GPTQ-2D: Cubic-Time Two-Sided Adaptive Rounding", Abstract: the algorithm
+extends to any number of Kronecker factors), through the C ABI.
+
+The k-way tensor (m_1, ..., m_k) is rounded as the m_1 x (m_2...m_k) problem with
+M_R = M_2 kron ... kron M_k (gptq2d_kron_factor).  Bar:
+  * the Kronecker factor equals the oracle's (np.kron of the same factors) to
+    fp64 rounding of a product of nf doubles (relative 1e-14), with exact zeros
+    wherever a column digit exceeds the row digit;
+  * Q is bit-exact against the k-way oracle (the reduced 2-D oracle with the
+    near-tie replay of tests/parity.py; the CPU pins tie it to the hyperplane
+    and naive-sweep oracles), the proxy loss within 1e-5 relative.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as WL
+from tests.parity import check_against_oracle
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    from two_sided_adaptive_b200 import build as gbuild
+    gbuild.build()
+    import two_sided_adaptive_b200 as g
+    return g
+
+
+def _spd(rng, k):
+    X = WL.student_t_activations(rng, 4 * k, k)
+    return WL.damped_gram(X).astype(np.float64)
+
+
+def _case(seed, shape):
+    rng = np.random.default_rng(5000 + 31 * seed + sum(shape) * 7 + len(shape))
+    W = rng.normal(0, 0.02, shape).astype(np.float32)
+    Hs = [_spd(rng, d) for d in shape]
+    s = WL.absmax_scales(W.reshape(shape[0], -1).astype(np.float64), 4).astype(np.float32)
+    return W, Hs, s
+
+
+def _digits(x, dims):
+    out = []
+    for d in reversed(dims):
+        out.append(x % d)
+        x //= d
+    return np.stack(out[::-1])
+
+
+@pytest.mark.parametrize("dims", [(3, 4), (5, 2, 3), (2,) * 8, (64, 64), (1, 7), (13,)],
+                         ids=lambda d: "x".join(map(str, d)))
+def test_kron_factor_matches_oracle(g, dims):
+    rng = np.random.default_rng(sum(dims))
+    Ms = [O.reverse_cholesky(_spd(rng, d)) for d in dims]
+    # fill the strict upper triangles with garbage: the kernel must not read them
+    Mg = []
+    for M in Ms:
+        G = M + np.triu(rng.normal(0, 1, M.shape), 1)
+        Mg.append(torch.from_numpy(G).cuda())
+    K = g.kron_factor(Mg).cpu().numpy()
+    Kref = O.kron_factor(Ms)
+    n = Kref.shape[0]
+    rd = _digits(np.arange(n)[:, None].repeat(n, 1), dims)
+    cd = _digits(np.arange(n)[None, :].repeat(n, 0), dims)
+    zero = np.any(cd > rd, axis=0)
+    assert np.all(K[zero] == 0.0)
+    np.testing.assert_allclose(K[~zero], Kref[~zero], rtol=1e-14, atol=0)
+
+
+def test_kron_factor_rejects_bad_arguments(g):
+    L = g.lib()
+    import ctypes
+    M = torch.eye(4, dtype=torch.float64, device="cuda")
+    ptrs = (ctypes.c_void_p * 2)(M.data_ptr(), M.data_ptr())
+    dims = (ctypes.c_int64 * 2)(4, 4)
+    lds = (ctypes.c_int64 * 2)(4, 4)
+    out = torch.empty((16, 16), dtype=torch.float64, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert L.gptq2d_kron_factor(2, ptrs, dims, lds, out.data_ptr(), 15, s) == g.Status.INVALID_ARG
+    assert L.gptq2d_kron_factor(9, ptrs, dims, lds, out.data_ptr(), 16, s) == g.Status.INVALID_ARG
+    # the output may not overlap a factor
+    ptrs_alias = (ctypes.c_void_p * 2)(out.data_ptr(), M.data_ptr())
+    assert L.gptq2d_kron_factor(2, ptrs_alias, dims, lds, out.data_ptr(), 16, s) == g.Status.INVALID_ARG
+    assert L.gptq2d_kron_factor(2, ptrs, dims, lds, out.data_ptr(), 16, s) == g.Status.OK
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy(), np.eye(16))
+
+
+SHAPES = [(70, 9, 13), (33, 5, 7, 3), (130, 8, 8, 2), (1, 64, 3), (64, 1, 70),
+          (40, 2, 2, 2, 2, 2, 2, 2), (97, 3, 41)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("bits,clamp", [(4, True), (3, True), (4, False)])
+def test_kway_rounding_matches_oracle(g, shape, bits, clamp):
+    W, Hs, s = _case(bits + 3 * clamp, shape)
+    s = s if clamp else (s * 4).astype(np.float32)
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    # the k-way problem through the library: GPU Kronecker factor, GPU rounding
+    MR = g.kron_factor([torch.from_numpy(M).cuda() for M in Ms[1:]]) if len(Ms) > 2 \
+        else torch.from_numpy(Ms[1]).cuda()
+    W2 = torch.from_numpy(W.reshape(shape[0], -1)).cuda()
+    Q, st = g.quantize(W2, torch.from_numpy(Ms[0]).cuda(), MR,
+                       torch.from_numpy(s).cuda(), bits, clamp)
+    torch.cuda.synchronize()
+    Qg = Q.cpu().numpy()
+    st = g.stats_dict(st)
+    s64 = s.astype(np.float64)
+    rep = check_against_oracle(W.reshape(shape[0], -1).astype(np.float64), Ms[0],
+                               O.kron_factor(Ms[1:]), s64, bits, clamp, Qg)
+    assert st["status"] == 0
+    assert st["n_clamped"] == rep.result.n_clamped
+    assert st["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+    if not rep.flips:
+        # the k-way hyperplane oracle gives the same rounding
+        rk = O.gptq_kron_hyperplane(W.astype(np.float64), Ms, s64, bits, clamp)
+        np.testing.assert_array_equal(rk.Q.reshape(shape[0], -1), Qg)
+
+
+def test_quantize_tensor_end_to_end(g):
+    """prepare each mode's factor on the GPU, form M_R, round: the k-way tensor result."""
+    shape = (96, 6, 11, 2)
+    W, Hs, s = _case(11, shape)
+    Q, st = g.quantize_tensor(torch.from_numpy(W).cuda(), [torch.from_numpy(H).cuda() for H in Hs],
+                              torch.from_numpy(s).cuda(), 4, True)
+    torch.cuda.synchronize()
+    assert tuple(Q.shape) == shape
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    rep = check_against_oracle(W.reshape(shape[0], -1).astype(np.float64), Ms[0],
+                               O.kron_factor(Ms[1:]), s.astype(np.float64), 4, True,
+                               Q.cpu().numpy().reshape(shape[0], -1))
+    assert g.stats_dict(st)["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+    assert O.proxy_loss_tensor(W.astype(np.float64), Q.cpu().numpy(), s.astype(np.float64), Hs) == \
+        pytest.approx(rep.result.loss_identity, rel=1e-6)

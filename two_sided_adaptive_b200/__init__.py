@@ -18,6 +18,7 @@ import numpy as np
 
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
+    "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
     "round_host_workspace_size", "quantize_noalloc", "check_wait_timeout", "profile_enable",
     "profile_reset", "profile_read", "profile_timeline",
@@ -29,6 +30,7 @@ library_path = os.path.join(_PKG, "libgptq2d.so")
 
 DTYPE_F32, DTYPE_BF16, DTYPE_F64 = 0, 1, 2
 STATS_WORDS = 5  # gptq2d_stats: double + 4 x int64
+MAX_KRON_FACTORS = 8  # GPTQ2D_MAX_KRON_FACTORS
 
 
 class Status:
@@ -86,6 +88,8 @@ def lib():
                                           ctypes.POINTER(_c_i64), ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_prepare_info.restype = ctypes.c_int
         L.gptq2d_prepare_info.argtypes = [_c_p, _c_p, ctypes.POINTER(_c_i64)]
+        L.gptq2d_kron_factor.restype = ctypes.c_int
+        L.gptq2d_kron_factor.argtypes = [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p]
         L.gptq2d_quantize_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_quantize_workspace_size.argtypes = [_c_i64, _c_i64]
         L.gptq2d_quantize.restype = ctypes.c_int
@@ -255,6 +259,52 @@ def prepare_pair(H_L, H_R, *, out_l=None, out_r=None, workspace=None, stream=Non
         raise GPTQ2DError(rc, "gptq2d_prepare_pair",
                           f"factor {which.value} pivot {piv.value}" if rc == Status.NOT_SPD else "")
     return ML, MR
+
+
+def kron_factor(Ms, *, out=None, stream=None):
+    """M_1 kron M_2 kron ... of lower fp64 factors (gptq2d_kron_factor): the reverse Cholesky
+    factor of H_1 kron H_2 kron ... when M_j = prepare(H_j).  Entries where some column
+    digit exceeds the row digit are exact zeros."""
+    torch = _torch()
+    if not 1 <= len(Ms) <= MAX_KRON_FACTORS:
+        raise ValueError(f"1 to {MAX_KRON_FACTORS} factors")
+    _check_device(*Ms)
+    for M in Ms:
+        if M.dtype != torch.float64 or M.dim() != 2 or M.shape[0] != M.shape[1]:
+            raise ValueError("factors must be square fp64 matrices")
+    n = int(np.prod([M.shape[0] for M in Ms]))
+    K = out if out is not None else torch.empty((n, n), dtype=torch.float64, device=Ms[0].device)
+    nf = len(Ms)
+    ptrs = (ctypes.c_void_p * nf)(*[M.data_ptr() for M in Ms])
+    dims = (_c_i64 * nf)(*[M.shape[0] for M in Ms])
+    lds = (_c_i64 * nf)(*[_ld(M) for M in Ms])
+    rc = lib().gptq2d_kron_factor(nf, ptrs, dims, lds, K.data_ptr(), _ld(K) if n else n,
+                                  _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_kron_factor")
+    return K
+
+
+def prepare_kron(Hs, *, stream=None, check: bool = True):
+    """Factors of a k-factor Kronecker Hessian H_1 kron ... kron H_k (H_j on mode j of a
+    k-way tensor) for the 2-D rounding: returns (M_L, M_R) with M_L = prepare(H_1) and
+    M_R = kron_factor([prepare(H_2), ..., prepare(H_k)])."""
+    if len(Hs) < 2:
+        raise ValueError("at least two factors")
+    Ms = [prepare(H, stream=stream, check=check) for H in Hs]
+    return Ms[0], (Ms[1] if len(Ms) == 2 else kron_factor(Ms[1:], stream=stream))
+
+
+def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, stream=None):
+    """GPTQ-2D rounding of a k-way tensor W (m_1 x ... x m_k, C order) under
+    H_1 kron ... kron H_k with per-mode-1 scales: the m_1 x (m_2 ... m_k) problem with
+    M_L = prepare(H_1), M_R = M_2 kron ... kron M_k.  Returns (Q shaped like W, stats)."""
+    if W.dim() != len(Hs) or W.dim() < 2:
+        raise ValueError("one Hessian factor per mode, at least two modes")
+    M_L, M_R = prepare_kron(Hs, stream=stream)
+    W2 = W.reshape(W.shape[0], -1)
+    Q, st = quantize(W2, M_L, M_R, scales, bits, clamp, stream=stream)
+    return Q.reshape(W.shape), st
 
 
 def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None, stats=None,

@@ -206,6 +206,28 @@ int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh, double* M
   return GPTQ2D_OK;
 }
 
+int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
+                       double* out, int64_t ldo, void* stream) {
+  if (nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !M || !dims || !ldm) return GPTQ2D_ERR_INVALID_ARG;
+  int64_t n = 1;
+  for (int f = 0; f < nf; ++f) {
+    if (dims[f] < 0 || dims[f] > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+    n *= dims[f];
+    if (n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  }
+  if (n == 0) return GPTQ2D_OK;
+  if (!out || ldo < n) return GPTQ2D_ERR_INVALID_ARG;
+  const char* o0 = reinterpret_cast<const char*>(out);
+  const char* o1 = o0 + (size_t)((n - 1) * ldo + n) * sizeof(double);
+  for (int f = 0; f < nf; ++f) {
+    if (!M[f] || ldm[f] < dims[f]) return GPTQ2D_ERR_INVALID_ARG;
+    const char* m0 = reinterpret_cast<const char*>(M[f]);
+    const char* m1 = m0 + (size_t)((dims[f] - 1) * ldm[f] + dims[f]) * sizeof(double);
+    if (m0 < o1 && o0 < m1) return GPTQ2D_ERR_INVALID_ARG;  // overlaps the output
+  }
+  return kron_factor_launch(nf, M, dims, ldm, out, ldo, static_cast<cudaStream_t>(stream));
+}
+
 int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
                         int64_t ldmr, void* ws, size_t ws_bytes, void* stream,

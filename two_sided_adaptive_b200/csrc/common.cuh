@@ -157,7 +157,7 @@ struct DevStreams {
 int dev_streams(DevStreams** out);
 
 // ---------------------------------------------------------------------------
-// Host-side launchers (defined in prepare.cu / quantize.cu)
+// Host-side launchers (defined in prepare.cu / quantize.cu / kron.cu)
 // ---------------------------------------------------------------------------
 size_t prepare_ws_bytes(int64_t k);
 int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, int64_t ldm,
@@ -171,6 +171,10 @@ int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
                         int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s,
                         cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr);
+
+// Kronecker product of nf lower factors into out (defined in kron.cu).
+int kron_factor_launch(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
+                       double* out, int64_t ldo, cudaStream_t s);
 
 size_t quantize_ws_bytes(int64_t m, int64_t n);
 int check_wait_timeout(long long limit_ns, cudaStream_t s);  // synchronizes s
