@@ -34,6 +34,11 @@ Functions, from most literal to fastest:
 and the special cases used as pins: RTN, 1-D GPTQ in OBS form, exhaustive
 closest-vector search on tiny problems.
 
+Grid variants (the pages fix only a 4-bit integer grid; these are GPTQ's usual
+ones): expand_grid turns group-wise scales and integer zero points into a
+per-entry step and admissible range that O0, O1 and O2 take as ``grid``;
+stored_codes / packed_codes / pack_nibbles give the bytes of the outputs.
+
 Hessians with k > 2 Kronecker factors (arxivlens, Abstract), W a k-way tensor:
   O1k babai_tensor_sweep            1-D GPTQ over the C-order flattening, explicit Gram
   O2k gptq_kron_hyperplane          hyperplane order, per-mode factors applied separately
@@ -62,10 +67,76 @@ def round_to_grid(t, lo, hi):
     return np.clip(np.rint(t), lo, hi)
 
 
+def expand_grid(m, n, scales, bits, clamp, group_size=0, zeros=None):
+    """Per-entry grid of GPTQ's grid variants: returns (S, LO, HI), each m x n, so
+    that entry (i, j) rounds to S[i,j] * q with q an integer in [LO[i,j], HI[i,j]].
+
+      * group_size 0: one scale per row (scales has m entries); else the columns
+        form groups of group_size and scales is m x ceil(n / group_size).
+      * zeros None: symmetric grid, q in [-2^(bits-1), 2^(bits-1)-1].
+      * zeros given (integers, shaped like the scales): asymmetric grid, code
+        c = q + z in [0, 2^bits - 1] and value S (c - z); for the integer q this
+        is the range [-z, 2^bits - 1 - z].  With an integer z,
+        clamp(rint(t + z)) - z = clamp(rint(t), -z, 2^bits - 1 - z), so the
+        rounding is the same nearest admissible integer along the coordinate.
+      * clamp False: every integer is admissible (zeros only shift the code).
+    """
+    sc = np.asarray(scales, np.float64).reshape(m, -1)
+    col = np.arange(n) // group_size if group_size else np.zeros(n, np.int64)
+    S = sc[:, col] if n else np.zeros((m, 0))
+    if zeros is None:
+        lo, hi = grid_bounds(bits, clamp)
+        LO = np.full((m, n), lo)
+        HI = np.full((m, n), hi)
+    else:
+        Z = np.asarray(zeros, np.float64).reshape(m, -1)[:, col] if n else np.zeros((m, 0))
+        if clamp:
+            LO = -Z
+            HI = float((1 << bits) - 1) - Z
+        else:
+            LO = np.full((m, n), -np.inf)
+            HI = np.full((m, n), np.inf)
+    return S, LO, HI
+
+
+def stored_codes(Q, m, n, bits, group_size=0, zeros=None):
+    """The byte a caller receives for each entry: q itself on the symmetric grid,
+    the unsigned code q + z on the asymmetric one."""
+    Q = np.asarray(Q, np.float64)
+    if zeros is None:
+        return Q
+    col = np.arange(n) // group_size if group_size else np.zeros(n, np.int64)
+    return Q + np.asarray(zeros, np.float64).reshape(m, -1)[:, col]
+
+
+def pack_nibbles(codes):
+    """Two unsigned 4-bit codes per byte, row by row: byte k of a row holds the
+    entry of column 2k in its low nibble and that of column 2k+1 in its high
+    nibble (zero past the last column)."""
+    c = np.asarray(codes, np.int64)
+    m, n = c.shape
+    if np.any((c < 0) | (c > 15)):
+        raise ValueError("codes must lie in [0, 15]")
+    out = np.zeros((m, (n + 1) // 2), np.uint8)
+    out[:, :] = c[:, 0::2]
+    out[:, : n // 2] |= (c[:, 1::2] << 4).astype(np.uint8)
+    return out
+
+
+def packed_codes(Q, m, n, bits, group_size=0, zeros=None):
+    """Unsigned 4-bit code of every entry for packed output: q - lo on the symmetric
+    grid (offset binary, lo = -2^(bits-1)), q + z on the asymmetric one."""
+    if zeros is None:
+        return np.asarray(Q, np.float64) + float(1 << (bits - 1))
+    return stored_codes(Q, m, n, bits, group_size, zeros)
+
+
 def proxy_loss(W, Q, s, H_L, H_R) -> float:
-    """L(Q) = tr(dW^T H_L dW H_R), dW = W - diag(s) Q (the two-sided quadratic metric)."""
+    """L(Q) = tr(dW^T H_L dW H_R), dW = W - S Q (the two-sided quadratic metric), with
+    S = diag(s) for per-row scales or the per-entry grid steps (an m x n array)."""
     W = np.asarray(W, np.float64)
-    D = W - np.asarray(s, np.float64)[:, None] * np.asarray(Q, np.float64)
+    s = np.asarray(s, np.float64)
+    D = W - (s if s.ndim == 2 else s[:, None]) * np.asarray(Q, np.float64)
     return float(np.sum(D * (np.asarray(H_L, np.float64) @ D @ np.asarray(H_R, np.float64))))
 
 
@@ -107,7 +178,7 @@ def reverse_cholesky(H):
 # --------------------------------------------------------------------------- #
 # O0: the definition
 # --------------------------------------------------------------------------- #
-def nearest_plane_by_definition(W, H_L, H_R, s, bits, clamp, order="row"):
+def nearest_plane_by_definition(W, H_L, H_R, s, bits, clamp, order="row", grid=None):
     """Sequential nearest-plane rounding of vec(W) under G = H_R kron H_L, written
     as its definition (mind-verse.de, "Geometrische Grundlagen ..."): coordinates
     are fixed one at a time; the value rounded for coordinate p is the p-th
@@ -115,15 +186,17 @@ def nearest_plane_by_definition(W, H_L, H_R, s, bits, clamp, order="row"):
     not yet fixed, with the fixed ones held at s*q.
 
     ``order`` is any linear extension of the product order on (i, j):
-    "row" (row-major) or "col" (column-major).  Returns (Q, T) with T = y / s.
-    Dense solves of size mn: tiny problems only.
+    "row" (row-major) or "col" (column-major).  ``grid`` = (S, LO, HI) from
+    expand_grid replaces the per-row scales s and the bits/clamp range.
+    Returns (Q, T) with T = y / s.  Dense solves of size mn: tiny problems only.
     """
     W = np.asarray(W, np.float64)
     m, n = W.shape
-    lo, hi = grid_bounds(bits, clamp)
+    S, LO, HI = grid if grid is not None else expand_grid(m, n, s, bits, clamp)
     G = np.kron(np.asarray(H_R, np.float64), np.asarray(H_L, np.float64))
     x = W.reshape(-1, order="F")                         # p = i + m j
-    sv = np.tile(np.asarray(s, np.float64), n)
+    sv = S.reshape(-1, order="F")
+    lov, hiv = LO.reshape(-1, order="F"), HI.reshape(-1, order="F")
     if order == "row":
         seq = [i + m * j for i in range(m) for j in range(n)]
     elif order == "col":
@@ -143,7 +216,7 @@ def nearest_plane_by_definition(W, H_L, H_R, s, bits, clamp, order="row"):
             zr = x[r] - np.linalg.solve(G[np.ix_(r, r)], G[np.ix_(r, f)] @ (z[f] - x[f]))
         y = zr[np.searchsorted(r, p)]
         T[p] = y / sv[p]
-        Q[p] = round_to_grid(T[p], lo, hi)
+        Q[p] = round_to_grid(T[p], lov[p], hiv[p])
         z[p] = sv[p] * Q[p]
         fixed[p] = True
     return Q.reshape((m, n), order="F"), T.reshape((m, n), order="F")
@@ -152,28 +225,30 @@ def nearest_plane_by_definition(W, H_L, H_R, s, bits, clamp, order="row"):
 # --------------------------------------------------------------------------- #
 # O1: naive vectorised Babai / 1-D GPTQ sweep on the full Kronecker Gram
 # --------------------------------------------------------------------------- #
-def babai_kron_sweep(W, H_L, H_R, s, bits, clamp):
+def babai_kron_sweep(W, H_L, H_R, s, bits, clamp, grid=None):
     """The naive vectorised sweep whose trajectory GPTQ-2D reproduces (arxivlens,
     Analysis > Results; mind-verse.de, "Die algorithmische Neuerung"): one-sided
     GPTQ over all mn coordinates of vec(W) (column-major), with the Gram
     G = H_R kron H_L.  GPTQ form: U = upper Cholesky factor of G^{-1}; coordinate
     p is rounded, and its error, divided by U_pp, is propagated to the later
-    coordinates along row p of U.  Quartic work; 64 x 64 at most.
+    coordinates along row p of U.  Quartic work; 64 x 64 at most.  ``grid`` =
+    (S, LO, HI) from expand_grid replaces per-row scales and the bits/clamp range.
     Returns (Q, T) with T = (updated x_p) / s_p.
     """
     W = np.asarray(W, np.float64)
     m, n = W.shape
-    lo, hi = grid_bounds(bits, clamp)
+    S, LO, HI = grid if grid is not None else expand_grid(m, n, s, bits, clamp)
     G = np.kron(np.asarray(H_R, np.float64), np.asarray(H_L, np.float64))
     U = np.linalg.cholesky(np.linalg.inv(G)).T            # U^T U = G^{-1}, upper
     x = W.reshape(-1, order="F").copy()
-    sv = np.tile(np.asarray(s, np.float64), n)
+    sv = S.reshape(-1, order="F")
+    lov, hiv = LO.reshape(-1, order="F"), HI.reshape(-1, order="F")
     N = m * n
     Q = np.zeros(N)
     T = np.zeros(N)
     for p in range(N):
         T[p] = x[p] / sv[p]
-        Q[p] = round_to_grid(T[p], lo, hi)
+        Q[p] = round_to_grid(T[p], lov[p], hiv[p])
         e = (x[p] - sv[p] * Q[p]) / U[p, p]
         x[p + 1:] -= e * U[p, p + 1:]
     return Q.reshape((m, n), order="F"), T.reshape((m, n), order="F")
@@ -194,7 +269,7 @@ class Result:
         self.flipped = flipped
 
 
-def gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=None, band=NEAR_TIE_BAND):
+def gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=None, band=NEAR_TIE_BAND, grid=None):
     """GPTQ-2D: round W anti-diagonal by anti-diagonal (arxivlens Abstract;
     mind-verse.de "Die algorithmische Neuerung") with the rank-one separable
     feedback kept in an accumulated buffer (arxivlens, Analysis > Results and
@@ -214,15 +289,18 @@ def gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=None, band=NEAR_TIE_BA
     run's own trajectory, else ValueError: the flip set only selects among the
     roundings that the near-tie rule admits.
 
+    ``grid``: optional (S, LO, HI) from expand_grid (group-wise scales, zero
+    points): entry (i, j) then rounds to S[i,j] * q, q in [LO[i,j], HI[i,j]], in
+    place of the per-row scales s and the bits/clamp range.
+
     Returns a Result with Q, T = y/s, the loss via the Babai identity
     sum d_ij^2 (y_ij - s_i q_ij)^2, the clamp count and the near-tie mask.
     """
     W = np.asarray(W, np.float64)
     M_L = np.asarray(M_L, np.float64)
     M_R = np.asarray(M_R, np.float64)
-    s = np.asarray(s, np.float64)
     m, n = W.shape
-    lo, hi = grid_bounds(bits, clamp)
+    S, LO, HI = grid if grid is not None else expand_grid(m, n, s, bits, clamp)
     flip = set() if flip is None else set(flip)
     P = np.zeros((m, n))
     Q = np.zeros((m, n))
@@ -238,7 +316,8 @@ def gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=None, band=NEAR_TIE_BA
         fb = np.einsum("ek,ke->e", M_L[i, :], P[:, j])
         dij = M_L[i, i] * M_R[j, j]
         y = W[i, j] + fb / dij
-        t = y / s[i]
+        sd, lo, hi = S[i, j], LO[i, j], HI[i, j]
+        t = y / sd
         q_raw = np.rint(t)
         q = np.clip(q_raw, lo, hi)
         nt = near_tie(t, lo, hi, band)
@@ -252,10 +331,10 @@ def gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=None, band=NEAR_TIE_BA
                     q[e] = h + 0.5 if q[e] == h - 0.5 else h - 0.5
                     done_flips.add(key)
         n_clamped += int(np.count_nonzero(q != q_raw))
-        delta = W[i, j] - s[i] * q
+        delta = W[i, j] - sd * q
         # right feedback: P[i, j'] += delta * M_R[j', j]; zero for j' < j (M_R lower)
         P[i, :] += delta[:, None] * M_R[:, j].T
-        loss += float(np.sum((dij * (y - s[i] * q)) ** 2))
+        loss += float(np.sum((dij * (y - sd * q)) ** 2))
         Q[i, j] = q
         T[i, j] = t
         tie[i, j] = nt
@@ -272,10 +351,12 @@ def gptq2d(W, H_L, H_R, s, bits, clamp, **kw):
 def entry_value(W, Q, s, M_L, M_R, i, j):
     """y_ij computed directly from its definition, given the integers already chosen
     for the dominated quadrant {i' <= i, j' <= j} minus (i, j) itself.  O(ij) work;
-    used to check single sampled entries of large outputs."""
+    used to check single sampled entries of large outputs.  s: per-row scales or
+    the m x n per-entry grid steps."""
     W = np.asarray(W, np.float64)
     s = np.asarray(s, np.float64)
-    D = W[: i + 1, : j + 1] - s[: i + 1, None] * np.asarray(Q[: i + 1, : j + 1], np.float64)
+    S = s[: i + 1, : j + 1] if s.ndim == 2 else s[: i + 1, None]   # per-entry or per-row steps
+    D = W[: i + 1, : j + 1] - S * np.asarray(Q[: i + 1, : j + 1], np.float64)
     D[i, j] = 0.0
     fb = np.asarray(M_L[i, : i + 1], np.float64) @ D @ np.asarray(M_R[j, : j + 1], np.float64)
     return W[i, j] + fb / (float(M_L[i, i]) * float(M_R[j, j]))
@@ -284,7 +365,7 @@ def entry_value(W, Q, s, M_L, M_R, i, j):
 # --------------------------------------------------------------------------- #
 # Special cases used as pins
 # --------------------------------------------------------------------------- #
-def gptq_1d_obs(w, H, s, bits, clamp):
+def gptq_1d_obs(w, H, s, bits, clamp, bounds=None):
     """Textbook one-sided GPTQ on a vector (mind-verse.de, "GPTQ-2D: Eine
     Weiterentwicklung ...": one-sided rounding with triangular feedback), in the
     optimal-brain-surgeon form rather than the Cholesky form: round coordinate
@@ -293,12 +374,16 @@ def gptq_1d_obs(w, H, s, bits, clamp):
     Index 0 first.  Returns q."""
     w = np.asarray(w, np.float64).copy()
     s = np.broadcast_to(np.asarray(s, np.float64), w.shape)
-    lo, hi = grid_bounds(bits, clamp)
+    if bounds is None:
+        lo, hi = grid_bounds(bits, clamp)
+        lo, hi = np.full(w.shape, lo), np.full(w.shape, hi)
+    else:
+        lo, hi = (np.broadcast_to(np.asarray(b, np.float64), w.shape) for b in bounds)
     Hinv = np.linalg.inv(np.asarray(H, np.float64))
     k = w.size
     q = np.zeros(k)
     for p in range(k):
-        q[p] = round_to_grid(w[p] / s[p], lo, hi)
+        q[p] = round_to_grid(w[p] / s[p], lo[p], hi[p])
         err = w[p] - s[p] * q[p]
         w -= err * Hinv[p, :] / Hinv[p, p]
         Hinv = Hinv - np.outer(Hinv[:, p], Hinv[p, :]) / Hinv[p, p]

@@ -66,6 +66,43 @@ def absmax_scales(W: np.ndarray, bits: int) -> np.ndarray:
     return s.astype(np.float32)
 
 
+def group_absmax_scales(W: np.ndarray, bits: int, group_size: int) -> np.ndarray:
+    """Symmetric group-wise scales: s[i, g] = max |W[i, group g]| / hi, shape
+    m x ceil(n / group_size); all-zero groups get 1."""
+    m, n = W.shape
+    _, hi = grid_limits(bits)
+    ng = -(-n // group_size)
+    A = np.zeros((m, ng))
+    for g in range(ng):
+        A[:, g] = np.max(np.abs(W[:, g * group_size:(g + 1) * group_size].astype(np.float64)), axis=1)
+    s = A / hi
+    s[s == 0] = 1.0
+    return s.astype(np.float32)
+
+
+def group_minmax_grid(W: np.ndarray, bits: int, group_size: int):
+    """Asymmetric group-wise grid in the usual GPTQ convention: the range of each
+    (row, group) is widened to include 0, s = (max - min) / (2^bits - 1) and the
+    integer zero point z = round(-min / s) in [0, 2^bits - 1], so that code c
+    stands for s (c - z).  group_size 0 means one group per row.  Returns
+    (scales fp32, zeros uint8), each m x ceil(n / group_size)."""
+    m, n = W.shape
+    G = group_size or n
+    ng = -(-n // G) if n else 0
+    top = float((1 << bits) - 1)
+    S = np.ones((m, ng), np.float32)
+    Z = np.zeros((m, ng), np.uint8)
+    for g in range(ng):
+        blk = W[:, g * G:(g + 1) * G].astype(np.float64)
+        lo = np.minimum(blk.min(axis=1), 0.0)
+        hi = np.maximum(blk.max(axis=1), 0.0)
+        sc = ((hi - lo) / top).astype(np.float32).astype(np.float64)
+        sc[sc == 0] = 1.0
+        S[:, g] = sc
+        Z[:, g] = np.clip(np.rint(-lo / sc), 0, top).astype(np.uint8)
+    return S, Z
+
+
 def student_t_activations(rng: np.random.Generator, rows: int, width: int,
                           nu: float = 4.0) -> np.ndarray:
     """rows x width activations: Student-t(nu) entries times a per-column scale U(0.1, 10)."""
