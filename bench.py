@@ -618,16 +618,79 @@ def run_kron3(args):
             "status": sd["status"], "n_near_tie": sd["n_near_tie"]}
 
 
+def run_grid128(args):
+    """The 4096 x 4096 INT4 attention layer of the headline metric on a grid variant:
+    128-column groups, asymmetric (integer zero points from each group's min/max, the
+    usual GPTQ convention), packed 4-bit output, through gptq2d_quantize_grid.  Inputs as
+    for the headline line (workloads.attn, Grams formed on the GPU); one step =
+    prepare_pair + quantize_grid, timed with CUDA events over K steps after W warm-ups."""
+    import torch
+    import two_sided_adaptive_b200 as g
+    from two_sided_adaptive_b200 import build as gbuild
+    import workloads as WL
+    gbuild.build()
+    pb = make_problem("attn", seed=0, device_gram=True)
+    m, n = pb.W.shape
+    dev = torch.device("cuda", 0)
+    W = torch.from_numpy(pb.W).to(dev).to(torch.bfloat16)
+    S, Z = WL.group_minmax_grid(W.double().cpu().numpy(), 4, 128)
+    S, Z = torch.from_numpy(S).to(dev), torch.from_numpy(Z).to(dev)
+    HL, HR = torch.from_numpy(pb.H_L).to(dev), torch.from_numpy(pb.H_R).to(dev)
+    ML = torch.empty((m, m), dtype=torch.float64, device=dev)
+    MR = torch.empty((n, n), dtype=torch.float64, device=dev)
+    wsP = torch.empty(512, dtype=torch.uint8, device=dev)
+    wsQ = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
+    Q = torch.empty((m, (n + 1) // 2), dtype=torch.uint8, device=dev)
+    st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        g.prepare_pair(HL, HR, out_l=ML, out_r=MR, workspace=wsP, check=False)
+        if ev:
+            ev[1].record()
+        g.quantize_grid(W, ML, MR, S, 4, True, group_size=128, zeros=Z, packed=True, out=Q,
+                        stats=st, workspace=wsQ)
+        if ev:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    tp = tq = 0.0
+    for _ in range(args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        step(ev)
+        torch.cuda.synchronize()
+        tp += ev[0].elapsed_time(ev[1])
+        tq += ev[1].elapsed_time(ev[2])
+    tp /= args.steps
+    tq /= args.steps
+    sd = g.stats_dict(st)
+    return {"metric": "weight entries rounded per second, INT4 asymmetric g128 packed (1 B200)",
+            "value": m * n / ((tp + tq) * 1e-3), "unit": "entries/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tp + tq,
+            "higher_is_better": True, "dtype": "f64", "data": "synthetic (workloads.attn)",
+            "config": {"workload": "grid128", "m": m, "n": n, "bits": 4, "group_size": 128,
+                       "zero_points": True, "packed": True,
+                       "step": "prepare_pair + quantize_grid, inputs resident in HBM"},
+            "phases": {"prepare_pair_ms": tp, "quantize_ms": tq,
+                       "quantize_fp64_tflops": m * n * (m + n) / (tq * 1e-3) / 1e12},
+            "status": sd["status"], "n_near_tie": sd["n_near_tie"], "n_clamped": sd["n_clamped"]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("attn", "mlp", "small", "block70b", "kron3"),
+    ap.add_argument("--workload", choices=("attn", "mlp", "small", "block70b", "kron3", "grid128"),
                     default="attn",
                     help="block70b: seconds per layer for one 70B-class block; kron3: a "
-                         "three-factor Kronecker Hessian (reports, not the headline metric)")
+                         "three-factor Kronecker Hessian; grid128: the attention layer on an "
+                         "asymmetric 128-column-group packed INT4 grid (reports, not the "
+                         "headline metric)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=768)
@@ -649,9 +712,9 @@ def main():
 
     import torch
     torch.cuda.set_device(local_rank)
-    if args.workload in ("block70b", "kron3"):
+    if args.workload in ("block70b", "kron3", "grid128"):
         if rank == 0:
-            run = run_block70b if args.workload == "block70b" else run_kron3
+            run = {"block70b": run_block70b, "kron3": run_kron3, "grid128": run_grid128}[args.workload]
             print(json.dumps(run(args)), flush=True)
         return
     if world > 1:

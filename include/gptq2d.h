@@ -234,6 +234,54 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
                     void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* Grid variants (the pages fix only a 4-bit integer grid: mind-verse.de       */
+/* "Neue Ansätze ...", section "Quantisierung von Large Language Models";      */
+/* these are GPTQ's usual variants of it)                                      */
+/* ------------------------------------------------------------------------- */
+
+/* The grid of gptq2d_quantize_grid.  Entry (i, j) lies in column group
+ * g = j / group_size (g = 0 when group_size is 0) and rounds to s q with
+ * s = scales[i * ld_scales + g] and q an integer:
+ *   symmetric (zeros NULL): q in [-2^(bits-1), 2^(bits-1) - 1];
+ *   asymmetric: z = zeros[i * ld_scales + g], code c = q + z in [0, 2^bits - 1],
+ *     the value s (c - z): q in [-z, 2^bits - 1 - z].  With an integer z the
+ *     nearest code to y / s + z is the nearest admissible q to y / s plus z, so
+ *     the rounding is the same one-coordinate nearest-plane step;
+ *   clamp = 0: any integer q (symmetric grid only: zero points need clamp = 1,
+ *     since an unclamped code need not fit its byte).
+ * Storage of Q:
+ *   packed = 0: one byte per entry, row stride ldq >= n bytes: int8 q on the
+ *     symmetric grid, uint8 code c on the asymmetric one;
+ *   packed = 1 (bits <= 4, clamp = 1): two entries per byte, row stride
+ *     ldq >= ceil(n / 2) bytes; byte k of a row holds the code of column 2k in
+ *     its low nibble and that of column 2k + 1 in its high nibble (0 past the
+ *     last column); the code is q + 2^(bits-1) (offset binary) on the symmetric
+ *     grid and c on the asymmetric one. */
+typedef struct {
+  int bits;               /* 2..8 */
+  int clamp;              /* 0 or 1 */
+  int64_t group_size;     /* 0: one scale per row; else a multiple of 8, or >= n (one group) */
+  const float* scales;    /* DEVICE fp32, m rows of ceil(n / group_size) groups (1 if
+                             group_size is 0), row stride ld_scales; finite and > 0 */
+  int64_t ld_scales;      /* >= groups per row */
+  const uint8_t* zeros;   /* DEVICE, NULL for the symmetric grid; else integer zero points
+                             in the layout of scales (requires clamp = 1) */
+  int packed;             /* 0 or 1 (see above) */
+} gptq2d_grid;
+
+/* gptq2d_quantize with a grid variant: group-wise scales, integer zero points,
+ * packed 4-bit output.  Arguments other than `grid` (a HOST pointer), Q (bytes)
+ * and ldq (bytes) are those of gptq2d_quantize, as are the rounding, the
+ * statistics (the loss uses each entry's own step) and the determinism; with
+ * group_size 0, zeros NULL and packed 0 the result is gptq2d_quantize's.
+ * A scale that is not finite and > 0 is counted once per group in
+ * stats->n_nonfinite. */
+int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                         const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                         const gptq2d_grid* grid, void* Q, int64_t ldq, gptq2d_stats* stats,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Rounding without any allocation                                             */
 /* (no counterpart in the GPTQ-2D pages: an interface for callers of this     */
 /* library that may not allocate device memory)                               */

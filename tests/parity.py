@@ -22,11 +22,13 @@ class ParityReport:
         self.n_near_tie = n_near_tie
 
 
-def check_against_oracle(W, M_L, M_R, s, bits, clamp, Q_candidate, max_flips=64):
+def check_against_oracle(W, M_L, M_R, s, bits, clamp, Q_candidate, max_flips=64, grid=None):
+    """``Q_candidate``: the candidate's integers q (for a grid variant, codes already
+    converted back to q); ``grid``: the per-entry grid (oracle.expand_grid), if any."""
     Qc = np.asarray(Q_candidate, np.float64)
     flips = set()
     for _ in range(max_flips + 1):
-        r = O.gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=flips)
+        r = O.gptq2d_antidiagonal(W, M_L, M_R, s, bits, clamp, flip=flips, grid=grid)
         mism = np.argwhere(r.Q != Qc)
         if mism.size == 0:
             return ParityReport(r, flips, int(r.near_tie.sum()))

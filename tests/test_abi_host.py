@@ -137,3 +137,37 @@ def test_kron_factor_rejects_invalid_arguments(L, bad):
 
 def test_kron_factor_with_a_zero_dimension_is_a_no_op(L):
     assert _kron(L, dims=(4, 0), out=None) == g.Status.OK
+
+
+def _qg(L, grid=None, **kw):
+    gr = dict(bits=4, clamp=1, group_size=0, scales=16, ld_scales=1, zeros=None, packed=0)
+    gr.update(grid or {})
+    a = dict(W=16, wdt=0, m=4, n=20, ldw=20, ML=16, ldl=4, MR=16, ldr=20, Q=16, ldq=20, st=16,
+             ws=256, wsb=1 << 30)
+    a.update(kw)
+    G = g._Grid(**gr)  # the binding's gptq2d_grid layout
+    return L.gptq2d_quantize_grid(a["W"], a["wdt"], a["m"], a["n"], a["ldw"], a["ML"], a["ldl"],
+                                  a["MR"], a["ldr"], ctypes.byref(G), a["Q"], a["ldq"], a["st"],
+                                  a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("grid,kw", [
+    (dict(bits=5, packed=1), {}),                 # packed needs bits <= 4
+    (dict(clamp=0, packed=1), {}),                # and a clamped grid
+    (dict(packed=2), {}),
+    (dict(group_size=12), {}),                    # groups: multiples of 8 (or >= n)
+    (dict(group_size=-8), {}),
+    (dict(group_size=8, ld_scales=2), {}),        # 20 columns in groups of 8: 3 per row
+    (dict(scales=None), {}),
+    (dict(packed=1), dict(ldq=9)),                # packed rows need ceil(20 / 2) bytes
+    (dict(), dict(ldq=19)),
+    (dict(bits=1), {}),
+    (dict(zeros=4096, clamp=0), {}),              # zero points need a clamped grid
+])
+def test_quantize_grid_rejects_invalid_arguments(L, grid, kw):
+    assert _qg(L, grid, **kw) == g.Status.INVALID_ARG
+
+
+def test_quantize_grid_rejects_a_null_grid(L):
+    assert L.gptq2d_quantize_grid(16, 0, 4, 4, 4, 16, 4, 16, 4, None, 16, 4, 16, 256, 1 << 30,
+                                  None) == g.Status.INVALID_ARG

@@ -18,7 +18,7 @@ import numpy as np
 
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
-    "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS",
+    "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS", "quantize_grid",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
     "round_host_workspace_size", "quantize_noalloc", "check_wait_timeout", "profile_enable",
     "profile_reset", "profile_read", "profile_timeline",
@@ -53,6 +53,12 @@ class GPTQ2DError(RuntimeError):
 _LIB = None
 _c_i64 = ctypes.c_int64
 _c_p = ctypes.c_void_p
+
+
+class _Grid(ctypes.Structure):
+    """gptq2d_grid"""
+    _fields_ = [("bits", ctypes.c_int), ("clamp", ctypes.c_int), ("group_size", _c_i64),
+                ("scales", _c_p), ("ld_scales", _c_i64), ("zeros", _c_p), ("packed", ctypes.c_int)]
 
 
 def lib():
@@ -90,6 +96,10 @@ def lib():
         L.gptq2d_prepare_info.argtypes = [_c_p, _c_p, ctypes.POINTER(_c_i64)]
         L.gptq2d_kron_factor.restype = ctypes.c_int
         L.gptq2d_kron_factor.argtypes = [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p]
+        L.gptq2d_quantize_grid.restype = ctypes.c_int
+        L.gptq2d_quantize_grid.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
+                                           _c_p, _c_i64, ctypes.POINTER(_Grid), _c_p, _c_i64, _c_p,
+                                           _c_p, ctypes.c_size_t, _c_p]
         L.gptq2d_quantize_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_quantize_workspace_size.argtypes = [_c_i64, _c_i64]
         L.gptq2d_quantize.restype = ctypes.c_int
@@ -327,6 +337,46 @@ def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None
                                _stream(stream))
     if rc != Status.OK:
         raise GPTQ2DError(rc, "gptq2d_quantize")
+    return Q, st
+
+
+def quantize_grid(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, group_size: int = 0,
+                  zeros=None, packed: bool = False, out=None, stats=None, workspace=None, stream=None):
+    """GPTQ-2D rounding on a grid variant (gptq2d_quantize_grid).  ``scales``: fp32 m x groups
+    (or a length-m vector when group_size is 0); ``zeros``: optional uint8 integer zero points
+    of the same shape (asymmetric grid, codes in [0, 2^bits - 1]; needs clamp); ``packed``: two 4-bit codes
+    per byte (bits <= 4).  Returns (Q bytes: int8 q on the symmetric grid, uint8 codes on the
+    asymmetric one, packed codes m x ceil(n/2) when packed; stats on the device)."""
+    torch = _torch()
+    _check_device(W, M_L, M_R, scales)
+    m, n = W.shape
+    if scales.dtype != torch.float32:
+        raise ValueError("scales must be fp32")
+    S = scales.reshape(m, -1) if scales.dim() == 1 else scales
+    if S.shape[0] != m or S.stride(1) != 1:
+        raise ValueError("scales must have m rows with unit column stride")
+    if zeros is not None:
+        _check_device(zeros)
+        if zeros.dtype != torch.uint8 or tuple(zeros.reshape(m, -1).shape) != tuple(S.shape):
+            raise ValueError("zeros must be uint8, shaped like the scales")
+        Z = zeros.reshape(m, -1)
+        if Z.stride(0) != S.stride(0) or Z.stride(1) != 1:
+            raise ValueError("zeros must share the scales' layout")
+    if M_L.dtype != torch.float64 or M_R.dtype != torch.float64:
+        raise ValueError("factors must be fp64")
+    qdt = torch.uint8 if (zeros is not None or packed) else torch.int8
+    ncol = (n + 1) // 2 if packed else n
+    Q = out if out is not None else torch.empty((m, ncol), dtype=qdt, device=W.device)
+    st = stats if stats is not None else torch.empty(STATS_WORDS, dtype=torch.int64, device=W.device)
+    ws = _workspace(quantize_workspace_size(m, n), W.device, workspace)
+    gr = _Grid(int(bits), int(clamp), int(group_size), S.data_ptr(), S.stride(0) if m else 1,
+               zeros.data_ptr() if zeros is not None else None, int(bool(packed)))
+    rc = lib().gptq2d_quantize_grid(W.data_ptr(), _dtype_code(W), m, n, _ld(W), M_L.data_ptr(),
+                                    _ld(M_L), M_R.data_ptr(), _ld(M_R), ctypes.byref(gr),
+                                    Q.data_ptr(), _ld(Q) if Q.numel() else ncol, st.data_ptr(),
+                                    ws.data_ptr(), ws.numel(), _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_quantize_grid")
     return Q, st
 
 

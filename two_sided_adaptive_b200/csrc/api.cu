@@ -292,6 +292,40 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
                          Q, ldq, stats, ws, s);
 }
 
+int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                         const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                         const gptq2d_grid* grid, void* Q, int64_t ldq, gptq2d_stats* stats,
+                         void* ws, size_t ws_bytes, void* stream) {
+  if (m < 0 || n < 0 || m > kMaxDim || n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  if (elem_size(w_dtype) == 0 || !grid || !stats) return GPTQ2D_ERR_INVALID_ARG;
+  const int bits = grid->bits, clamp = grid->clamp;
+  if (bits < 2 || bits > 8 || (clamp != 0 && clamp != 1)) return GPTQ2D_ERR_INVALID_ARG;
+  if (grid->packed != 0 && grid->packed != 1) return GPTQ2D_ERR_INVALID_ARG;
+  if (grid->packed && (bits > 4 || !clamp)) return GPTQ2D_ERR_INVALID_ARG;
+  if (grid->zeros && !clamp) return GPTQ2D_ERR_INVALID_ARG;  // codes must fit their byte
+  const int64_t G = grid->group_size;
+  if (G < 0 || (G > 0 && G % 8 != 0 && G < n)) return GPTQ2D_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GridSpec gs;
+  gs.group = G;
+  gs.lds = grid->ld_scales;
+  gs.zero = grid->zeros;
+  gs.packed = grid->packed;
+  if (m == 0 || n == 0)
+    return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales,
+                           bits, clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0, nullptr,
+                           nullptr, &gs);
+  const int64_t groups = (G == 0 || G >= n) ? 1 : (n + G - 1) / G;
+  if (!W || !M_L || !M_R || !grid->scales || !Q) return GPTQ2D_ERR_INVALID_ARG;
+  if (grid->ld_scales < groups) return GPTQ2D_ERR_INVALID_ARG;
+  if (ldw < n || ldl < m || ldr < n || ldq < (grid->packed ? (n + 1) / 2 : n))
+    return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(m, n)) return GPTQ2D_ERR_WORKSPACE;
+  return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales, bits,
+                         clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0, nullptr, nullptr,
+                         &gs);
+}
+
 size_t gptq2d_round_host_workspace_size(int64_t m, int64_t n, int w_dtype, int h_dtype) {
   if (m <= 0 || n <= 0 || m > kMaxDim || n > kMaxDim) return 0;
   if (elem_size(w_dtype) == 0 || (h_dtype != GPTQ2D_F32 && h_dtype != GPTQ2D_F64)) return 0;

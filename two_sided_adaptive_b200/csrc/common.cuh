@@ -178,12 +178,22 @@ int kron_factor_launch(int nf, const double* const* M, const int64_t* dims, cons
 
 size_t quantize_ws_bytes(int64_t m, int64_t n);
 int check_wait_timeout(long long limit_ns, cudaStream_t s);  // synchronizes s
+
+// Grid of a rounding call beyond bits/clamp (default: one scale per row, symmetric,
+// one byte per entry).
+struct GridSpec {
+  int64_t group = 0;              // columns per scale group (multiple of 8, or >= n); 0: per row
+  int64_t lds = 1;                // row stride of scales and zeros, in groups
+  const uint8_t* zero = nullptr;  // integer zero points (asymmetric grid), or null
+  int packed = 0;                 // two 4-bit codes per byte
+};
+
 // Optional row events: row_ev[k] is recorded once the tile rows 0..row_tile[k] of
 // Q are final (row_tile ascending), so a caller can copy them out early.
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
                     int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
                     cudaStream_t s, int n_row_ev = 0, const int* row_tile = nullptr,
-                    cudaEvent_t* row_ev = nullptr);
+                    cudaEvent_t* row_ev = nullptr, const GridSpec* grid = nullptr);
 
 }  // namespace gptq2d

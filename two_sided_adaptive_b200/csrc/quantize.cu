@@ -65,10 +65,16 @@ struct QArgs {
   const double* MR;
   int64_t ldr;
   const float* scales;
-  double lo, hi;
+  int64_t lds;           // row stride of scales / zero in groups
+  int64_t group;         // columns per scale group; 0: one scale per row
+  const uint8_t* zero;   // integer zero points (asymmetric grid), or null
+  double lo, hi;         // symmetric grid range (infinite without clamp)
+  double top;            // 2^bits - 1: top of the asymmetric code range
+  double code_off;       // added to q + z for the stored code (offset binary when packed)
   int clamp;
-  int8_t* Q;
-  int64_t ldq;
+  int packed;            // two 4-bit codes per byte
+  uint8_t* Q;
+  int64_t ldq;           // bytes
   int* err;       // nonzero: a bounded wait in a kernel timed out
   double* Lh;     // mp x mp
   double* Rh;     // np x np
@@ -200,14 +206,30 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
     cp_async16_zfill(Vt + r * SLD + c2, I >= 2 ? a.E + ts + (int64_t)r * np + c2 : a.E, I >= 2);
   }
   cp_async_commit_group();
-  // row scales, their reciprocals and the factor diagonals of the tile
-  __shared__ double Ss[TB], Si[TB], Sdl[TB], Sdr[TB];
-  if (tid < TB) {
-    const double sv = tid < rows ? (double)a.scales[r0 + tid] : 1.0;
-    Ss[tid] = sv;
-    Si[tid] = 1.0 / sv;
-    Sdl[tid] = a.dL[r0 + tid];
-    Sdr[tid] = a.dR[c0 + tid];
+  // grid of every (row, 8-column sub-tile): step, its reciprocal, integer zero point
+  // (a scale group holds a multiple of 8 columns, so a sub-tile lies in one group);
+  // the factor diagonals of the tile
+  __shared__ double Ss[TB][NSUB], Si[TB][NSUB];
+  __shared__ float Sz[TB][NSUB];
+  __shared__ double Sdl[TB], Sdr[TB];
+  static_assert(SWEEP_THREADS == TB * NSUB, "one thread per (row, sub-tile column)");
+  {
+    const int r = tid / NSUB, qs = tid % NSUB;
+    const int64_t col = c0 + SUB * qs;
+    double sv = 1.0;
+    float z = 0.f;
+    if (r < rows && col < a.n) {
+      const int64_t gi = (int64_t)(r0 + r) * a.lds + (a.group ? col / a.group : 0);
+      sv = (double)a.scales[gi];
+      if (a.zero) z = (float)a.zero[gi];
+    }
+    Ss[r][qs] = sv;
+    Si[r][qs] = 1.0 / sv;
+    Sz[r][qs] = z;
+    if (tid < TB) {
+      Sdl[tid] = a.dL[r0 + tid];
+      Sdr[tid] = a.dR[c0 + tid];
+    }
   }
   // W of the tile (zero outside the matrix)
   constexpr int WPT = TB * TB / SWEEP_THREADS;
@@ -307,7 +329,12 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       if (R0 < rows && C0 < cols) {
         const int ar = R0 + sa;
         const bool rok = ar < rows;
-        const double s = Ss[ar], inv_s = Si[ar];
+        const double s = Ss[ar][q], inv_s = Si[ar][q];
+        // admissible range of this sub-tile's entries: the symmetric grid, or the
+        // codes [0, 2^bits - 1] shifted by the zero point
+        const double zq = Sz[ar][q];
+        const double lo = a.zero ? (a.clamp ? -zq : -HUGE_VAL) : a.lo;
+        const double hi = a.zero ? (a.clamp ? a.top - zq : HUGE_VAL) : a.hi;
         double P[2], V[2], Wd[2];
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
@@ -326,7 +353,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
           const double y = (o1 ? V[1] : V[0]) + Px;
           const double tq = y * inv_s;
           const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;  // rint, |t| <= 2^51
-          const double qv = qr < a.lo ? a.lo : (qr > a.hi ? a.hi : qr);  // lo/hi infinite: no clamp
+          const double qv = qr < lo ? lo : (qr > hi ? hi : qr);  // lo/hi infinite: no clamp
           const double delta = fma(-s, qv, o1 ? Wd[1] : Wd[0]);
           const double pf = Px + delta;
           const double dO = mine ? delta : 0.0, pO = mine ? pf : 0.0;
@@ -400,22 +427,39 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
         make_double2(Dt[r * SLD + c2], Dt[r * SLD + c2 + 1]);
   }
   // Q and the statistics of every rounded entry, from its t = y / s:
-  // loss term (M_L[i,i] M_R[j,j] s_i (t - q))^2 (the nearest-plane residual identity)
-  for (int x = tid; x < TB * TB; x += SWEEP_THREADS) {
-    const int r = x >> 6, c = x & 63;
-    if (r < rows && c < cols) {
-      const double sr = Ss[r];
-      const double tq = Tq[r * SLD + c];
+  // loss term (M_L[i,i] M_R[j,j] s (t - q))^2 (the nearest-plane residual identity).
+  // Two adjacent columns per thread (one byte of packed output; both in one sub-tile).
+  for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+    const int r = x >> 5, c = (x & 31) * 2;
+    if (r >= rows || c >= cols) continue;
+    const double sr = Ss[r][c / SUB], zq = Sz[r][c / SUB];
+    const double lo = a.zero ? (a.clamp ? -zq : -HUGE_VAL) : a.lo;
+    const double hi = a.zero ? (a.clamp ? a.top - zq : HUGE_VAL) : a.hi;
+    int code[2] = {0, 0};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int cc = c + k;
+      if (cc >= cols) break;
+      const double tq = Tq[r * SLD + cc];
       const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;
-      const double qv = qr < a.lo ? a.lo : (qr > a.hi ? a.hi : qr);
-      a.Q[(int64_t)(r0 + r) * a.ldq + c0 + c] = (int8_t)(int)qv;
-      const double res = Sdl[r] * Sdr[c] * sr * (tq - qv);
+      const double qv = qr < lo ? lo : (qr > hi ? hi : qr);
+      code[k] = (int)(qv + zq + a.code_off);
+      const double res = Sdl[r] * Sdr[cc] * sr * (tq - qv);
       loss += res * res;
       ncl += (qv != qr);
       const double qn = qr + (tq >= qr ? 1.0 : -1.0);
-      nnt += (0.5 - fabs(tq - qr) < 1e-6) && (fmin(qr, qn) >= a.lo) && (fmax(qr, qn) <= a.hi);
+      nnt += (0.5 - fabs(tq - qr) < 1e-6) && (fmin(qr, qn) >= lo) && (fmax(qr, qn) <= hi);
       nnf += !isfinite(tq);
-      if (c == 0 && J == 0 && !(sr > 0.0 && isfinite(sr))) ++nnf;
+      // a bad step counts once per group (at the group's first column)
+      const int64_t col = (int64_t)c0 + cc;
+      if ((a.group ? col % a.group == 0 : col == 0) && !(sr > 0.0 && isfinite(sr))) ++nnf;
+    }
+    uint8_t* qrow = a.Q + (int64_t)(r0 + r) * a.ldq;
+    if (a.packed) {
+      qrow[(c0 + c) / 2] = (uint8_t)((code[0] & 15) | ((code[1] & 15) << 4));
+    } else {
+      qrow[c0 + c] = (uint8_t)code[0];
+      if (c + 1 < cols) qrow[c0 + c + 1] = (uint8_t)code[1];
     }
   }
 
@@ -1007,7 +1051,8 @@ int check_wait_timeout(long long limit_ns, cudaStream_t s) {
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
                     int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
-                    cudaStream_t s, int n_row_ev, const int* row_tile, cudaEvent_t* row_ev) {
+                    cudaStream_t s, int n_row_ev, const int* row_tile, cudaEvent_t* row_ev,
+                    const GridSpec* grid) {
   if (m == 0 || n == 0) {
     GPTQ2D_LAUNCH(KC_OTHER, s, zero_stats_kernel<<<1, 1, 0, s>>>(stats));
     return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
@@ -1023,11 +1068,18 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
   a.ldl = ldl;
   a.MR = MR;
   a.ldr = ldr;
+  const GridSpec gs = grid ? *grid : GridSpec{};
   a.scales = scales;
+  a.lds = gs.lds;
+  a.group = gs.group >= n ? 0 : gs.group;  // one group per row
+  a.zero = gs.zero;
   a.lo = clamp ? -(double)(1 << (bits - 1)) : -HUGE_VAL;
   a.hi = clamp ? (double)((1 << (bits - 1)) - 1) : HUGE_VAL;
+  a.top = (double)((1 << bits) - 1);
+  a.code_off = (gs.packed && !gs.zero) ? (double)(1 << (bits - 1)) : 0.0;
   a.clamp = clamp;
-  a.Q = Q;
+  a.packed = gs.packed;
+  a.Q = reinterpret_cast<uint8_t*>(Q);
   a.ldq = ldq;
   a.Lh = reinterpret_cast<double*>(base + L.off_Lh);
   a.Rh = reinterpret_cast<double*>(base + L.off_Rh);
