@@ -72,6 +72,42 @@ def test_prepare_matches_lapack(g, k, hdtype):
     np.testing.assert_allclose(M, Mref, rtol=1e-9, atol=1e-11 * scale)
 
 
+def _gpu_spd(k, seed):
+    """Damped Student-t Gram of k + 64 rows (workloads recipe), formed with a GPU matmul."""
+    rng = np.random.default_rng(seed)
+    X = torch.from_numpy(WL.student_t_activations(rng, k + 64, k).astype(np.float64)).cuda()
+    G = (X.T @ X / (k + 64)).cpu().numpy()
+    G = 0.5 * (G + G.T)
+    G[np.diag_indices(k)] += 0.01 * np.mean(np.diag(G))
+    return G
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("k", [6000, 8256, 10305, 12032])
+def test_prepare_strips_match_lapack(g, k):
+    """Sizes on both sides of the switch from one-row to four-row strips (more than 128
+    block rows): 6000 (94 block rows, ragged last row of 48), 8256 (129 block rows: 32
+    strips of 4 and a single-row strip), 10305 (ragged last row of 1), 12032 (47 strips
+    of 4): every row against LAPACK's reverse Cholesky."""
+    H = _gpu_spd(k, k)
+    M = g.prepare(dev(H)).cpu().numpy()
+    Mref = O.reverse_cholesky(H)
+    assert np.all(np.triu(M, 1) == 0.0)
+    scale = np.abs(Mref).max()
+    np.testing.assert_allclose(M, Mref, rtol=1e-9, atol=1e-11 * scale)
+
+
+@pytest.mark.parametrize("k,bad", [(9000, 8999), (9000, 8930), (9000, 17), (11000, 10990),
+                                   (11000, 6001), (11000, 3)])
+def test_prepare_reports_first_bad_pivot_in_strips(g, k, bad):
+    H = np.eye(k)
+    H[bad, bad] = -1.0
+    with pytest.raises(g.GPTQ2DError) as ei:
+        g.prepare(dev(H))
+    assert ei.value.status == g.Status.NOT_SPD
+    assert f"pivot {bad}" in str(ei.value)
+
+
 def test_prepare_strided_input(g):
     rng = np.random.default_rng(3)
     H = WL.random_spd(rng, 100)

@@ -13,10 +13,13 @@
 //   1. M_KK^T M_KK = A_KK            (in-SM factorization of one 64x64 block)
 //   2. M_Kb = M_KK^{-T} A_Kb, b < K  (triangular solve of the block row)
 //   3. A_IJ -= M_KI^T M_KJ, J<=I<K   (rank-64 trailing update on FP64 tensor cores)
-// Step 3 is split with a lookahead of one block row: the update of row K-1 by
-// M row K is done inside panel(K-1) itself, and the rest (rows I <= K-2) runs
-// on a second stream beside panel(K-1).  panel(K-1) therefore waits only for
-// the rest-update of step K+1.  Everything is fp64.  A pivot that is not
+// Step 3 is organised in strips of r block rows (r = 1 for up to 128 block rows,
+// 4 beyond): each panel applies the factored rows of its own strip
+// and of the strip below it left-looking, and one rank-64r trailing update per
+// strip applies the strip to the rows below the next strip, on a second stream
+// beside the next strip's panels.  With r = 1 this is the lookahead of one block
+// row (panel(K-1) applies row K; rows I <= K-2 get row K from the trailing
+// update).  Everything is fp64.  A pivot that is not
 // positive and finite stops the factorization and is reported through a pivot
 // word in the workspace.
 #include <algorithm>
@@ -29,7 +32,6 @@ namespace gptq2d {
 namespace {
 
 constexpr int OLD = TB + 4;  // 68: row stride of shared 64x64 tiles (conflict-free DMMA fragments)
-constexpr int TR_THREADS = 128;
 constexpr int PANEL_THREADS = 384;   // 8 factor warps + 4 warps for the block-row lookahead
 constexpr int FACTOR_THREADS = 256;
 constexpr int MAX_TR_GROUPS = 512;
@@ -123,7 +125,7 @@ __device__ __forceinline__ void factor_group_sync() {
   asm volatile("bar.sync 1, %0;\n" ::"n"(FACTOR_THREADS) : "memory");
 }
 
-constexpr int PANEL_SMEM = 4 * TB * OLD * (int)sizeof(double);
+constexpr int PANEL_SMEM = 6 * TB * OLD * (int)sizeof(double);
 
 // Reverse Cholesky of the 8x8 block D = A[R0..R0+8)^2 of the shared tile A into
 // registers: L (lower) = M_D and inv[p] = 1/M_D[p][p].  Every calling thread
@@ -206,9 +208,12 @@ __device__ __forceinline__ void rank8_block(double* C, const double* S, const do
 
 // One launch per block row K.  CTA K factors the diagonal block and writes it;
 // CTAs b < K factor the same block redundantly (cheaper than a separate launch)
-// and solve their block M_Kb = M_KK^{-T} A_Kb.  When a factored block row K+1
-// exists, each CTA first applies its update to the blocks it reads:
-// A_KK -= M_{K+1,K}^T M_{K+1,K} and A_Kb -= M_{K+1,K}^T M_{K+1,b}.
+// and solve their block M_Kb = M_KK^{-T} A_Kb.  Each CTA first applies, left-
+// looking, the updates of the factored block rows j = K+1 .. whi (the window that
+// the trailing updates have not applied) to the blocks it reads:
+// A_KK -= M_jK^T M_jK and A_Kb -= M_jK^T M_jb, streaming the window's blocks
+// through a double buffer; the last row's update of A_Kb runs beside the
+// factorization of the diagonal block.
 //
 // The 64x64 factorization runs in 8-row strips from the bottom: warp 0 factors
 // the strip's 8x8 diagonal block (factor_diag8); one thread per column solves
@@ -218,40 +223,56 @@ __device__ __forceinline__ void rank8_block(double* C, const double* S, const do
 // leaves the factor of the leading part unchanged.
 template <bool V16>
 __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict__ M, int64_t ldm,
-                                                              int k, int K, long long* info) {
+                                                              int k, int K, int whi,
+                                                              long long* info) {
   if (*(volatile long long*)info >= 0) return;
   extern __shared__ __align__(128) double sm[];
   double* Ad = sm;              // A_KK, then M_KK
   double* Ab = Ad + TB * OLD;   // A_Kb, then M_Kb
-  double* Mn = Ab + TB * OLD;   // M_{K+1,K}
-  double* Mb = Mn + TB * OLD;   // M_{K+1,b}
+  // window row j in stage (j - K - 1) & 1: M_jK, then M_jb
+  auto mn = [&](int st) { return Ab + (1 + 2 * st) * (TB * OLD); };
+  auto mb = [&](int st) { return Ab + (2 + 2 * st) * (TB * OLD); };
   __shared__ double invd[TB];
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int rb = K * TB, nb = min(TB, k - rb);
-  const int rn = rb + TB, nn = max(0, min(TB, k - rn));  // block row K+1, if any
   const int b = blockIdx.x;
   if (tid == 0) bad = -1;
+  auto load_row = [&](int j, int st) {  // window row j (only the last block row is ragged)
+    const int rj = j * TB, nj = min(TB, k - rj);
+    load_block<V16, PANEL_THREADS>(mn(st), M, ldm, rj, rb, nj, nb);
+    if (b < K) load_block<V16, PANEL_THREADS>(mb(st), M, ldm, rj, b * TB, nj, TB);
+  };
 
   load_block<V16, PANEL_THREADS>(Ad, M, ldm, rb, rb, nb, nb);
   if (b < K) load_block<V16, PANEL_THREADS>(Ab, M, ldm, rb, b * TB, nb, TB);
-  if (nn > 0) {
-    load_block<V16, PANEL_THREADS>(Mn, M, ldm, rn, rb, nn, nb);
-    if (b < K) load_block<V16, PANEL_THREADS>(Mb, M, ldm, rn, b * TB, nn, TB);
-  }
+  if (whi > K) load_row(K + 1, 0);
   cp_async_commit_group();
+  // every window row but the last: A_KK on warps 0..7, A_Kb on warps 8..11
+#pragma unroll 1
+  for (int j = K + 1; j < whi; ++j) {
+    const int st = (j - K - 1) & 1;
+    load_row(j + 1, st ^ 1);
+    cp_async_commit_group();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    if (warp < FACTOR_THREADS / 32) sub_xtx_lower(Ad, mn(st), FACTOR_THREADS / 32);
+    else if (b < K) sub_xty_4w(Ab, mn(st), mb(st), warp - FACTOR_THREADS / 32);
+    __syncthreads();
+  }
   cp_async_wait_group<0>();
   __syncthreads();
-  if (nn > 0) sub_xtx_lower(Ad, Mn, PANEL_THREADS / 32);  // the factor needs it first
+  const int st_last = (whi - K - 1) & 1;
+  if (whi > K) sub_xtx_lower(Ad, mn(st_last), PANEL_THREADS / 32);  // the factor needs it first
   // unit diagonal past a ragged edge (only the last block row is ragged, and it
-  // has no lookahead update, so no other thread writes these elements)
+  // has no window, so no other thread writes these elements)
   if (tid < TB && tid >= nb) Ad[tid * OLD + tid] = 1.0;
   __syncthreads();
 
   if (warp >= FACTOR_THREADS / 32) {
-    // warps 8..11: the block-row lookahead A_Kb -= M_{K+1,K}^T M_{K+1,b}, needed only
-    // by the solve below, while warps 0..7 factor the diagonal block
-    if (nn > 0 && b < K) sub_xty_4w(Ab, Mn, Mb, warp - FACTOR_THREADS / 32);
+    // warps 8..11: the last window row's A_Kb -= M_jK^T M_jb, needed only by the
+    // solve below, while warps 0..7 factor the diagonal block
+    if (whi > K && b < K) sub_xty_4w(Ab, mn(st_last), mb(st_last), warp - FACTOR_THREADS / 32);
   } else {
   // factor A_KK in place, strips s = 7..0.  Threads <= 8s factor strip s's 8x8
   // diagonal block in registers; threads < 8s then solve one column of the strip
@@ -331,29 +352,40 @@ __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict
   }
 }
 
+constexpr int MAX_STRIP = 4;  // block rows per strip (rank of a trailing update: 64 x strip)
+
 struct TrailPlan {
-  int K, I0, ng;                 // factored block row, first group, number of groups
+  int k0, nk;                    // the strip: factored block rows k0 .. k0 + nk - 1
+  int I0, ng;                    // first group, number of groups
   int per_cta;                   // blocks J per CTA
   int start[MAX_TR_GROUPS + 1];  // first CTA of each group; group g updates A[I0+g][0..I0+g]
 };
 
-constexpr int TR_SMEM = (3 * TB * OLD + 4 * 8 * 40) * (int)sizeof(double);
+constexpr int TR_STAGE = 8 * 40;  // per warp: one 8x32 strip of the product (row stride 40)
+// Shared memory of a trailing CTA of nw warps for a strip of nk rows: the strip's
+// blocks of column I, two stream buffers, one staging strip per warp.
+constexpr int tr_smem(int nk, int nw) { return ((nk + 2) * TB * OLD + nw * TR_STAGE) * (int)sizeof(double); }
 
-// A_IJ -= M_KI^T M_KJ for J <= I, over a range of J of one block row I.  Each
-// CTA keeps M_KI in shared memory and streams the M_KJ blocks through a double
-// buffer; the product goes into A_IJ by reductions in L2 (no read of the block),
-// one whole 256-byte row at a time through a shared strip.  Only the lower part
-// of A_II is touched.
-template <bool V16>
-__global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restrict__ M,
+// A_IJ -= sum_{q < nk} M_{k0+q,I}^T M_{k0+q,J} for J <= I, over a range of J of one
+// block row I: the rank-64 nk update of one strip.  Each CTA keeps the strip's
+// blocks of column I in shared memory and streams the blocks M_{k0+q,J} through a
+// double buffer (q fastest); the sum over the strip stays in registers, and goes
+// into A_IJ by reductions in L2 (no read of the block), one whole 256-byte row at a
+// time through a shared strip.  NW warps (4: two CTAs per SM, for strips of one row;
+// 8: one CTA per SM with room for four rows), warp w owning rows (64 / (NW/2)) (w>>1)..
+// and columns 32 (w&1).. of the 64x64 block.  Only the lower part of A_II is touched.
+template <bool V16, int NW>
+__global__ void __launch_bounds__(NW * 32, NW == 4 ? 2 : 1) trailing_kernel(double* __restrict__ M,
                                                                  int64_t ldm, int k,
                                                                  const long long* info,
                                                                  TrailPlan pl) {
+  constexpr int NT = NW * 32;
+  constexpr int RF = 64 / (NW / 2) / 8;  // 8-row fragments per warp
   if (*(volatile const long long*)info >= 0) return;
   extern __shared__ __align__(128) double sm[];
-  double* Xs = sm;  // Xs[r][i] = M[rb + r][64 I + i]
-  double* const Y0 = sm + TB * OLD;
-  double* const stage = sm + 3 * TB * OLD;  // 4 warps x one 8x32 strip (row stride 40)
+  double* const Xs = sm;                        // Xs[q][r][i] = M[64 (k0+q) + r][64 I + i]
+  double* const Y0 = sm + pl.nk * TB * OLD;     // two stream buffers
+  double* const stage = Y0 + 2 * TB * OLD;
   auto ybuf = [&](int bsel) { return Y0 + bsel * (TB * OLD); };
   const int cta = blockIdx.x;
   int g;
@@ -369,52 +401,73 @@ __global__ void __launch_bounds__(TR_THREADS, 2) trailing_kernel(double* __restr
   const int first = (cta - pl.start[g]) * pl.per_cta;
   const int last = min(first + pl.per_cta, I + 1);
   if (first >= last) return;
-  const int rb = pl.K * TB, nb = min(TB, k - rb);
+  const int nk = pl.nk;
+  auto rows_of = [&](int q) { return min(TB, k - (pl.k0 + q) * TB); };  // only the last block row is ragged
 
-  load_block<V16, TR_THREADS>(Xs, M, ldm, rb, I * TB, nb, TB);
-  load_block<V16, TR_THREADS>(ybuf(0), M, ldm, rb, first * TB, nb, TB);
+  for (int q = 0; q < nk; ++q)
+    load_block<V16, NT>(Xs + q * (TB * OLD), M, ldm, (pl.k0 + q) * TB, I * TB, rows_of(q), TB);
+  load_block<V16, NT>(ybuf(0), M, ldm, pl.k0 * TB, first * TB, rows_of(0), TB);
   cp_async_commit_group();
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, t4 = lane & 3;
-  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
-  const int kmax = (nb + 3) & ~3;
-  for (int J = first; J < last; ++J) {
-    const int bsel = (J - first) & 1;
-    if (J + 1 < last) {
-      load_block<V16, TR_THREADS>(ybuf(bsel ^ 1), M, ldm, rb, (J + 1) * TB, nb, TB);
+  const int wr = (warp >> 1) * (8 * RF), wc = (warp & 1) * 32;
+  const int nsteps = (last - first) * nk;
+  double acc[RF][4][2] = {};
+  for (int step = 0; step < nsteps; ++step) {
+    const int J = first + step / nk, q = step % nk;
+    const int bsel = step & 1;
+    if (step + 1 < nsteps) {
+      const int J1 = first + (step + 1) / nk, q1 = (step + 1) % nk;
+      load_block<V16, NT>(ybuf(bsel ^ 1), M, ldm, (pl.k0 + q1) * TB, J1 * TB, rows_of(q1), TB);
       cp_async_commit_group();
+      cp_async_wait_group<1>();
+    } else {
+      cp_async_wait_group<0>();
     }
-    if (J + 1 < last) cp_async_wait_group<1>(); else cp_async_wait_group<0>();
     __syncthreads();
+    const double* Xq = Xs + q * (TB * OLD);
     const double* Ys = ybuf(bsel);
-    double acc[4][4][2] = {};
-    mma_64x64x64(
-        acc, [&](int row, int kk) { return Xs[kk * OLD + row]; },
-        [&](int kk, int col) { return Ys[kk * OLD + col]; }, kmax);
-    // A_IJ -= product by reductions in L2 (each element of the block gets exactly
-    // one contribution per launch): whole 256-byte rows through a shared strip
-    double* st = stage + warp * (8 * 40);
-    double* Cw = M + (int64_t)(I * TB + wr) * ldm + (int64_t)J * TB + wc;
+#pragma unroll 4
+    for (int kk = 0; kk < TB; kk += 4) {
+      double a[RF], bv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < RF; ++i) a[i] = Xq[(kk + t4) * OLD + wr + i * 8 + g8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        *reinterpret_cast<double2*>(st + g8 * 40 + j * 8 + 2 * t4) =
-            make_double2(-acc[i][j][0], -acc[i][j][1]);
-      __syncwarp();
+      for (int j = 0; j < 4; ++j) bv[j] = Ys[(kk + t4) * OLD + wc + j * 8 + g8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int row = wr + i * 8 + r, col = wc + lane;
-        if (I != J || col <= row) red_add(Cw + (int64_t)(i * 8 + r) * ldm + lane, st[r * 40 + lane]);
+      for (int i = 0; i < RF; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j][0], acc[i][j][1], a[i], bv[j]);
+    }
+    if (q == nk - 1) {
+      // A_IJ -= the strip's product by reductions in L2 (each element of the block
+      // gets exactly one contribution per launch): whole 256-byte rows through a
+      // shared strip
+      double* st = stage + warp * TR_STAGE;
+      double* Cw = M + (int64_t)(I * TB + wr) * ldm + (int64_t)J * TB + wc;
+#pragma unroll
+      for (int i = 0; i < RF; ++i) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          *reinterpret_cast<double2*>(st + g8 * 40 + j * 8 + 2 * t4) =
+              make_double2(-acc[i][j][0], -acc[i][j][1]);
+          acc[i][j][0] = acc[i][j][1] = 0.0;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int row = wr + i * 8 + r, col = wc + lane;
+          if (I != J || col <= row) red_add(Cw + (int64_t)(i * 8 + r) * ldm + lane, st[r * 40 + lane]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     __syncthreads();
   }
 }
 
-std::atomic<uint64_t> g_trailing_smem_set[2];
+std::atomic<uint64_t> g_trailing_smem_set[4];
 std::atomic<uint64_t> g_panel_smem_set[2];
 
 
@@ -445,29 +498,54 @@ int enqueue_convert(const FactorJob& f, int sms) {
   return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
-// Step K of one factor: panel(K) after the trailing update of step K+2, then the
-// trailing update of rows I <= K-2 by M row K.
+// Block rows per strip: one row (a lookahead of one row, as in the classic
+// right-looking scheme) up to 128 block rows, where the panels set the pace; four
+// beyond, where the trailing updates dominate: each pass over the trailing matrix
+// then carries a rank-256 update, with a quarter of the launches (measured on a
+// B200: 16384^2 in 82 ms instead of 103, 28672^2 in 418 ms instead of 502; two
+// equal factors at once gain nothing, the GPU being full either way).
+inline int strip_rows(int T) { return T <= 128 ? 1 : MAX_STRIP; }
+
+// Step K of one factor.  The block rows are grouped into strips of r rows from the
+// bottom (strip s: rows lo_s .. hi_s, hi_s = T-1 - s r).  panel(K) applies the rows
+// K+1 .. hi_{s-1} (its own strip and the one below it) left-looking; the strip's
+// trailing update, launched after its last panel, applies it to the rows below the
+// next strip (I < lo_s - r).  So every row K sees each factored row exactly once,
+// and the first panel of strip s waits only for the trailing update of strip s-2,
+// which leaves strip s-1's trailing update running beside strip s's panels.  The
+// trailing updates of one factor run in order on one stream (a fixed order of the
+// reductions into each block: deterministic).
 int enqueue_step(const FactorJob& f, int K, int sms) {
+  const int r = strip_rows(f.T);
+  const int sidx = (f.T - 1 - K) / r;
+  const int hi_s = f.T - 1 - sidx * r, lo_s = std::max(0, hi_s - r + 1);
+  const int whi = std::min(f.T - 1, hi_s + r);
   bool ok = true;
-  if (K + 2 < f.T) ok = cudaStreamWaitEvent(f.ps, f.rest_done[(K + 2) % RING], 0) == cudaSuccess;
+  if (K == hi_s && sidx >= 2)
+    ok = cudaStreamWaitEvent(f.ps, f.rest_done[(sidx - 2) % RING], 0) == cudaSuccess;
   if (f.v16)
     GPTQ2D_LAUNCH(KC_PREP_PANEL, f.ps,
                   panel_kernel<true><<<K + 1, PANEL_THREADS, PANEL_SMEM, f.ps>>>(f.M, f.ldm, f.k,
-                                                                                   K, f.info));
+                                                                                   K, whi, f.info));
   else
     GPTQ2D_LAUNCH(KC_PREP_PANEL, f.ps,
                   panel_kernel<false><<<K + 1, PANEL_THREADS, PANEL_SMEM, f.ps>>>(f.M, f.ldm, f.k,
-                                                                                    K, f.info));
-  if (K < 2) return ok && cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
-  ok = ok && cudaEventRecord(f.panel_done[K % RING], f.ps) == cudaSuccess &&
-       cudaStreamWaitEvent(f.us, f.panel_done[K % RING], 0) == cudaSuccess;
-  const int rows = K - 1;  // block rows I = 0..K-2
+                                                                                    K, whi, f.info));
+  const int rows = lo_s - r;  // block rows I = 0 .. lo_s - r - 1
+  if (K != lo_s || rows <= 0)
+    return ok && cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
+  ok = ok && cudaEventRecord(f.panel_done[sidx % RING], f.ps) == cudaSuccess &&
+       cudaStreamWaitEvent(f.us, f.panel_done[sidx % RING], 0) == cudaSuccess;
   const long long total = (long long)rows * (rows + 1) / 2;
   const int target = 2 * sms;
   const int per_cta = (int)std::max<long long>(1, (total + target - 1) / target);
+  const int nk = hi_s - lo_s + 1;
+  const bool wide = nk > 1;  // 8 warps, one CTA per SM; else 4 warps, two per SM
+  const int smem = tr_smem(nk, wide ? 8 : 4);
   for (int g0 = 0; g0 < rows && ok; g0 += MAX_TR_GROUPS) {
     TrailPlan pl;
-    pl.K = K;
+    pl.k0 = lo_s;
+    pl.nk = hi_s - lo_s + 1;
     pl.I0 = g0;
     pl.ng = std::min(rows - g0, MAX_TR_GROUPS);
     pl.per_cta = per_cta;
@@ -477,22 +555,20 @@ int enqueue_step(const FactorJob& f, int K, int sms) {
       ctas += (g0 + gi + 1 + per_cta - 1) / per_cta;
     }
     pl.start[pl.ng] = ctas;
-    if (f.v16)
-      GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
-                    trailing_kernel<true><<<ctas, TR_THREADS, TR_SMEM, f.us>>>(f.M, f.ldm, f.k,
-                                                                                 f.info, pl));
-    else
-      GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
-                    trailing_kernel<false><<<ctas, TR_THREADS, TR_SMEM, f.us>>>(f.M, f.ldm, f.k,
-                                                                                  f.info, pl));
+    auto kern = f.v16 ? (wide ? trailing_kernel<true, 8> : trailing_kernel<true, 4>)
+                      : (wide ? trailing_kernel<false, 8> : trailing_kernel<false, 4>);
+    GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
+                  kern<<<ctas, wide ? 256 : 128, smem, f.us>>>(f.M, f.ldm, f.k, f.info, pl));
   }
-  ok = ok && cudaEventRecord(f.rest_done[K % RING], f.us) == cudaSuccess;
+  ok = ok && cudaEventRecord(f.rest_done[sidx % RING], f.us) == cudaSuccess;
   return ok && cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
 int ensure_prepare_smem() {
-  if (ensure_smem(trailing_kernel<true>, TR_SMEM, g_trailing_smem_set[0]) != cudaSuccess ||
-      ensure_smem(trailing_kernel<false>, TR_SMEM, g_trailing_smem_set[1]) != cudaSuccess ||
+  if (ensure_smem(trailing_kernel<true, 8>, tr_smem(MAX_STRIP, 8), g_trailing_smem_set[0]) != cudaSuccess ||
+      ensure_smem(trailing_kernel<false, 8>, tr_smem(MAX_STRIP, 8), g_trailing_smem_set[1]) != cudaSuccess ||
+      ensure_smem(trailing_kernel<true, 4>, tr_smem(1, 4), g_trailing_smem_set[2]) != cudaSuccess ||
+      ensure_smem(trailing_kernel<false, 4>, tr_smem(1, 4), g_trailing_smem_set[3]) != cudaSuccess ||
       ensure_smem(panel_kernel<true>, PANEL_SMEM, g_panel_smem_set[0]) != cudaSuccess ||
       ensure_smem(panel_kernel<false>, PANEL_SMEM, g_panel_smem_set[1]) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
