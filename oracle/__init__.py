@@ -7,3 +7,4 @@ from .gptq2d_oracle import (NEAR_TIE_BAND, Result, babai_kron_sweep, closest_vec
 from .gptq2d_oracle import (babai_tensor_sweep, gptq_kron_hyperplane, gptq_kron_via_2d,
                             kron_factor, kron_gram, mode_product, proxy_loss_tensor)
 from .gptq2d_oracle import expand_grid, pack_nibbles, packed_codes, stored_codes
+from .gptq2d_oracle import gram, gram_batches

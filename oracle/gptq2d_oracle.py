@@ -39,6 +39,9 @@ ones): expand_grid turns group-wise scales and integer zero points into a
 per-entry step and admissible range that O0, O1 and O2 take as ``grid``;
 stored_codes / packed_codes / pack_nibbles give the bytes of the outputs.
 
+The step before the path: gram / gram_batches form a Kronecker factor
+H = X^T X / N (+ damping) from N rows of activations.
+
 Hessians with k > 2 Kronecker factors (arxivlens, Abstract), W a k-way tensor:
   O1k babai_tensor_sweep            1-D GPTQ over the C-order flattening, explicit Gram
   O2k gptq_kron_hyperplane          hyperplane order, per-mode factors applied separately
@@ -592,3 +595,37 @@ def gptq_kron_via_2d(W, Ms, s, bits, clamp, **kw):
     W2 = W.reshape(W.shape[0], -1)
     M_R = kron_factor(Ms[1:]) if len(Ms) > 1 else np.ones((1, 1))
     return gptq2d_antidiagonal(W2, Ms[0], M_R, s, bits, clamp, **kw)
+
+
+# --------------------------------------------------------------------------- #
+# The Kronecker factors from calibration activations (the step before the
+# path: arxivlens, Analysis > Limitations, fixed bases A, B whose Grams are
+# factored; Future work, "Gram factorizations")
+# --------------------------------------------------------------------------- #
+# Reading: a factor is the Gram of its basis, H = A^T A, with A = X / sqrt(N) for N
+# rows of activations X (N x k), i.e. H = X^T X / N, plus GPTQ's usual damping of
+# the diagonal by a fraction of its mean (the pages give no damping; it keeps a
+# rank-deficient Gram positive definite).
+
+
+def gram(X, damp=0.0):
+    """H = X^T X / N + damp * mean(diag(X^T X / N)) * I, in fp64 (X upcast exactly)."""
+    X = np.asarray(X, np.float64)
+    N = X.shape[0]
+    H = X.T @ X / N
+    H[np.diag_indices_from(H)] += damp * float(np.mean(np.diag(H))) if H.size else 0.0
+    return H
+
+
+def gram_batches(batches, damp=0.0):
+    """The same Gram accumulated over batches of rows: sum of X_b^T X_b over all
+    batches, divided by the total row count, then damped."""
+    S = None
+    N = 0
+    for X in batches:
+        X = np.asarray(X, np.float64)
+        S = X.T @ X if S is None else S + X.T @ X
+        N += X.shape[0]
+    H = S / N
+    H[np.diag_indices_from(H)] += damp * float(np.mean(np.diag(H)))
+    return H
