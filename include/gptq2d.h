@@ -171,6 +171,47 @@ int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl,
 int gptq2d_prepare_info(const void* ws, void* stream, int64_t* bad_pivot);
 
 /* ------------------------------------------------------------------------- */
+/* The Kronecker factors from calibration activations (the step before the     */
+/* path; arxivlens "GPTQ-2D: Cubic-Time Two-Sided Adaptive Rounding",          */
+/* Analysis > Limitations and Future work: fixed bases whose Grams are formed   */
+/* and factored once).  A factor is the Gram of its basis A = X / sqrt(N):      */
+/* H = X^T X / N for N rows of activations X, plus GPTQ's usual damping of the  */
+/* diagonal (a reading: the pages give none).  Runs on the tcgen05 tensor cores */
+/* with bf16 operands and fp32 accumulation.                                    */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace the Gram calls need (a diagonal sum and an error word). */
+size_t gptq2d_gram_workspace_size(void);
+
+/* Accumulate the Gram of a batch of activation rows.
+ *   X, x_dtype, rows, k, ldx : DEVICE, rows x k, GPTQ2D_BF16 only, row-major;
+ *                              k and ldx multiples of 8, X 16-byte aligned.
+ *   H, ldh                   : DEVICE fp32 k x k.  The lower 128-block triangle
+ *                              (every 128 x 128 block on or below the diagonal, so
+ *                              every j <= i and a few j > i near the diagonal) is
+ *                              written: accumulate = 0 sets it to X^T X and clears
+ *                              the workspace's error word (a new Gram);
+ *                              accumulate = 1 adds X^T X.  Other entries are untouched.
+ *   ws, ws_bytes             : DEVICE workspace >= gptq2d_gram_workspace_size(),
+ *                              256-byte aligned, kept from the first batch to finalize.
+ * Products of bf16 values are exact in fp32; the sums are fp32 (tensor-core order).
+ * rows == 0 with accumulate = 0 writes zeros.  k == 0 is a no-op.  A bounded
+ * device-side wait that gives up sets the error word (read by gptq2d_gram_finalize
+ * when it is given a HOST status pointer). */
+int gptq2d_gram_accumulate(const void* X, int x_dtype, int64_t rows, int64_t k, int64_t ldx,
+                           float* H, int64_t ldh, int accumulate, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Finish a Gram: H <- H / total_rows on the lower 128-block triangle, then
+ * H_ii += damp * mean_i(H_ii), the mean of the scaled diagonal (damp >= 0; GPTQ's
+ * usual value is 0.01).  The result is ready for gptq2d_prepare (which reads only
+ * the lower triangle).  status (HOST, may be NULL): if non-NULL the call
+ * synchronizes `stream` and returns GPTQ2D_ERR_TIMEOUT if a bounded wait of an
+ * accumulate call gave up, else GPTQ2D_OK (also written to *status). */
+int gptq2d_gram_finalize(float* H, int64_t k, int64_t ldh, int64_t total_rows, double damp,
+                         void* ws, size_t ws_bytes, void* stream, int* status);
+
+/* ------------------------------------------------------------------------- */
 /* Hessians with more than two Kronecker factors (arxivlens "GPTQ-2D: Cubic-   */
 /* Time Two-Sided Adaptive Rounding", Abstract: the algorithm extends to any   */
 /* number of Kronecker factors).                                               */

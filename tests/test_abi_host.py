@@ -171,3 +171,33 @@ def test_quantize_grid_rejects_invalid_arguments(L, grid, kw):
 def test_quantize_grid_rejects_a_null_grid(L):
     assert L.gptq2d_quantize_grid(16, 0, 4, 4, 4, 16, 4, 16, 4, None, 16, 4, 16, 256, 1 << 30,
                                   None) == g.Status.INVALID_ARG
+
+
+def _ga(L, **kw):
+    a = dict(X=4096, dt=g.DTYPE_BF16, rows=16, k=64, ldx=64, H=8192, ldh=64, acc=0, ws=256, wsb=256)
+    a.update(kw)
+    return L.gptq2d_gram_accumulate(a["X"], a["dt"], a["rows"], a["k"], a["ldx"], a["H"], a["ldh"],
+                                    a["acc"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("bad", [dict(dt=g.DTYPE_F32), dict(k=60, ldx=64, ldh=64), dict(ldx=68),
+                                 dict(ldx=60), dict(X=4096 + 8), dict(H=None), dict(ldh=63),
+                                 dict(acc=2), dict(rows=-1), dict(X=None)])
+def test_gram_accumulate_rejects_invalid_arguments(L, bad):
+    """Checked on the host: bf16 only, k and ldx multiples of 8, a 16-byte aligned X."""
+    assert _ga(L, **bad) == g.Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("bad,code", [(dict(ws=None), "WORKSPACE"), (dict(wsb=255), "WORKSPACE"),
+                                      (dict(ws=272), "WORKSPACE")])
+def test_gram_accumulate_rejects_bad_workspace(L, bad, code):
+    assert _ga(L, **bad) == getattr(g.Status, code)
+
+
+def test_gram_finalize_rejects_invalid_arguments(L):
+    f = L.gptq2d_gram_finalize
+    assert f(8192, 64, 64, 0, 0.01, 256, 256, None, None) == g.Status.INVALID_ARG     # no rows
+    assert f(8192, 64, 64, 10, -0.5, 256, 256, None, None) == g.Status.INVALID_ARG    # damp < 0
+    assert f(8192, 64, 63, 10, 0.01, 256, 256, None, None) == g.Status.INVALID_ARG    # ldh < k
+    assert f(8192, 64, 64, 10, 0.01, 0, 256, None, None) == g.Status.WORKSPACE
+    assert L.gptq2d_gram_workspace_size() >= 12

@@ -19,6 +19,7 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS", "quantize_grid",
+    "gram_accumulate", "gram_finalize", "gram",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
     "round_host_workspace_size", "quantize_noalloc", "check_wait_timeout", "profile_enable",
     "profile_reset", "profile_read", "profile_timeline",
@@ -94,6 +95,13 @@ def lib():
                                           ctypes.POINTER(_c_i64), ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_prepare_info.restype = ctypes.c_int
         L.gptq2d_prepare_info.argtypes = [_c_p, _c_p, ctypes.POINTER(_c_i64)]
+        L.gptq2d_gram_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_gram_accumulate.restype = ctypes.c_int
+        L.gptq2d_gram_accumulate.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
+                                             ctypes.c_int, _c_p, ctypes.c_size_t, _c_p]
+        L.gptq2d_gram_finalize.restype = ctypes.c_int
+        L.gptq2d_gram_finalize.argtypes = [_c_p, _c_i64, _c_i64, _c_i64, ctypes.c_double, _c_p,
+                                           ctypes.c_size_t, _c_p, ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_kron_factor.restype = ctypes.c_int
         L.gptq2d_kron_factor.argtypes = [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p]
         L.gptq2d_quantize_grid.restype = ctypes.c_int
@@ -269,6 +277,54 @@ def prepare_pair(H_L, H_R, *, out_l=None, out_r=None, workspace=None, stream=Non
         raise GPTQ2DError(rc, "gptq2d_prepare_pair",
                           f"factor {which.value} pivot {piv.value}" if rc == Status.NOT_SPD else "")
     return ML, MR
+
+
+def gram_accumulate(X, H, *, accumulate: bool, workspace, stream=None):
+    """gptq2d_gram_accumulate: H's lower 128-block triangle (+)= X^T X for a bf16 batch X
+    (rows x k on the GPU; k a multiple of 8) on the tensor cores.  ``workspace``: a device
+    uint8 tensor of at least gptq2d_gram_workspace_size() bytes, kept until finalize."""
+    torch = _torch()
+    _check_device(X, H, workspace)
+    if X.dtype != torch.bfloat16 or H.dtype != torch.float32:
+        raise ValueError("X must be bf16 and H fp32")
+    rows, k = X.shape
+    rc = lib().gptq2d_gram_accumulate(X.data_ptr(), DTYPE_BF16, rows, k, _ld(X) if rows else k,
+                                      H.data_ptr(), _ld(H), int(bool(accumulate)),
+                                      workspace.data_ptr(), workspace.numel(), _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_gram_accumulate")
+    return H
+
+
+def gram_finalize(H, total_rows: int, damp: float = 0.01, *, workspace, stream=None,
+                  check: bool = True):
+    """gptq2d_gram_finalize: H <- H / total_rows with damp * mean(diag) added to the
+    diagonal.  ``check`` synchronizes and raises if a bounded wait gave up."""
+    _check_device(H, workspace)
+    st = ctypes.c_int(0)
+    rc = lib().gptq2d_gram_finalize(H.data_ptr(), H.shape[0], _ld(H), int(total_rows), float(damp),
+                                    workspace.data_ptr(), workspace.numel(), _stream(stream),
+                                    ctypes.byref(st) if check else None)
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_gram_finalize")
+    return H
+
+
+def gram(batches, damp: float = 0.01, *, out=None, stream=None):
+    """The damped Gram X^T X / N + damp * mean(diag) I of bf16 activation batches (each
+    rows x k on the GPU), accumulated on the tensor cores.  Returns H (fp32 k x k; its
+    lower triangle is the Gram, ready for prepare)."""
+    torch = _torch()
+    batches = list(batches)
+    k = batches[0].shape[1]
+    dev_ = batches[0].device
+    H = out if out is not None else torch.empty((k, k), dtype=torch.float32, device=dev_)
+    ws = torch.empty(max(lib().gptq2d_gram_workspace_size(), 256), dtype=torch.uint8, device=dev_)
+    total = 0
+    for b, X in enumerate(batches):
+        gram_accumulate(X, H, accumulate=b > 0, workspace=ws, stream=stream)
+        total += X.shape[0]
+    return gram_finalize(H, total, damp, workspace=ws, stream=stream)
 
 
 def kron_factor(Ms, *, out=None, stream=None):

@@ -206,6 +206,46 @@ int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh, double* M
   return GPTQ2D_OK;
 }
 
+size_t gptq2d_gram_workspace_size(void) { return 256; }
+
+int gptq2d_gram_accumulate(const void* X, int x_dtype, int64_t rows, int64_t k, int64_t ldx,
+                           float* H, int64_t ldh, int accumulate, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (x_dtype != GPTQ2D_BF16 || rows < 0 || k < 0 || k > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return GPTQ2D_ERR_INVALID_ARG;
+  if (k == 0) return GPTQ2D_OK;
+  if (!H || ldh < k || k % 8 != 0) return GPTQ2D_ERR_INVALID_ARG;
+  if (rows > 0 && (!X || ldx < k || ldx % 8 != 0 ||
+                   (reinterpret_cast<uintptr_t>(X) & 15u) != 0))
+    return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < 256) return GPTQ2D_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = reinterpret_cast<int*>(static_cast<char*>(ws) + 8);
+  if (!accumulate && cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+  return gram_accumulate_launch(X, rows, (int)k, ldx, H, ldh, accumulate, err, s);
+}
+
+int gptq2d_gram_finalize(float* H, int64_t k, int64_t ldh, int64_t total_rows, double damp,
+                         void* ws, size_t ws_bytes, void* stream, int* status) {
+  if (k < 0 || k > kMaxDim || total_rows < 1 || !(damp >= 0.0)) return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < 256) return GPTQ2D_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k > 0) {
+    if (!H || ldh < k) return GPTQ2D_ERR_INVALID_ARG;
+    const int rc = gram_finalize_launch(H, (int)k, ldh, total_rows, damp,
+                                        reinterpret_cast<double*>(ws), s);
+    if (rc != GPTQ2D_OK) return rc;
+  }
+  if (!status) return GPTQ2D_OK;
+  int err = 0;
+  if (cudaMemcpyAsync(&err, static_cast<char*>(ws) + 8, sizeof(int), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  *status = err ? GPTQ2D_ERR_TIMEOUT : GPTQ2D_OK;
+  return *status;
+}
+
 int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
                        double* out, int64_t ldo, void* stream) {
   if (nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !M || !dims || !ldm) return GPTQ2D_ERR_INVALID_ARG;

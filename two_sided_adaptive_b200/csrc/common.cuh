@@ -172,6 +172,14 @@ int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_
                         int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s,
                         cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr);
 
+// Gram of activations on the tcgen05 tensor cores (defined in gram.cu): H's lower
+// 128-block triangle (+)= X^T X (X bf16, N x k, k and ldx multiples of 8); then
+// H <- H / total_rows with diagonal damping.
+int gram_accumulate_launch(const void* X, int64_t N, int k, int64_t ldx, float* H, int64_t ldh,
+                           int beta, int* err, cudaStream_t s);
+int gram_finalize_launch(float* H, int k, int64_t ldh, int64_t total_rows, double damp,
+                         double* diag_sum, cudaStream_t s);
+
 // Kronecker product of nf lower factors into out (defined in kron.cu).
 int kron_factor_launch(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
                        double* out, int64_t ldo, cudaStream_t s);
