@@ -679,17 +679,88 @@ def run_grid128(args):
             "status": sd["status"], "n_near_tie": sd["n_near_tie"], "n_clamped": sd["n_clamped"]}
 
 
+def run_gram(args):
+    """The step before the path: the Kronecker factors from activations on the tensor
+    cores (gram_accumulate + gram_finalize, bf16 activations, fp32 accumulation).  For
+    each width k the activations are k rows of the workloads recipe (Student-t(4) times
+    U(0.1, 10) column scales; the 70B block's recipe uses rows = width), generated on the
+    GPU.  Algorithmic work: the lower block triangle, rows * k * (k + 128) flops (the
+    128-wide diagonal blocks are computed whole).  Timed with CUDA events, best of K steps
+    after W warm-ups, against MEASURED_PEAKS.json's bf16 burst figure; the fp64 matmul that
+    forms the same Gram (torch, cuBLAS DGEMM) is timed beside it for context."""
+    import torch
+    import two_sided_adaptive_b200 as g
+    from two_sided_adaptive_b200 import build as gbuild
+    gbuild.build()
+    dev = torch.device("cuda", 0)
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = peaks.get("bf16_tflops", 1590.0)
+    out = []
+    for k in (4096, 8192, 28672):
+        torch.manual_seed(k)
+        rows = k
+        z = torch.randn(rows, k, device=dev, dtype=torch.float32)
+        chi2 = torch.distributions.Chi2(torch.tensor(4.0, device=dev))
+        X = (z / torch.sqrt(chi2.sample((rows, k)) / 4.0)) * \
+            torch.empty(k, device=dev).uniform_(0.1, 10.0)[None, :]
+        del z
+        Xb = X.to(torch.bfloat16)
+        del X
+        H = torch.empty((k, k), dtype=torch.float32, device=dev)
+        ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+
+        def step():
+            g.gram_accumulate(Xb, H, accumulate=False, workspace=ws)
+            g.gram_finalize(H, rows, 0.01, workspace=ws, check=False)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        best = 1e30
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            step()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        fl = float(rows) * k * (k + 128)
+        Xd = Xb.double()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.matmul(Xd.T, Xd)
+        torch.cuda.synchronize()
+        e0.record()
+        torch.matmul(Xd.T, Xd)
+        e1.record()
+        torch.cuda.synchronize()
+        t64 = e0.elapsed_time(e1)
+        del Xd, Xb, H
+        torch.cuda.empty_cache()
+        out.append({"k": k, "rows": rows, "ms": best, "tflops": fl / (best * 1e-3) / 1e12,
+                    "frac_of_bf16_peak": fl / (best * 1e-3) / 1e12 / peak,
+                    "fp64_matmul_ms": t64})
+    return {"metric": "Gram X^T X / N + damping from bf16 activations (tensor cores), TFLOP/s",
+            "value": out[-1]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16 operands, f32 accumulation",
+            "data": "synthetic (generated on the GPU, see run_gram)",
+            "peak": {"bf16_tflops": peak, "source": "MEASURED_PEAKS.json bf16_tflops (burst)"},
+            "config": {"workload": "gram", "widths": [o["k"] for o in out]}, "sizes": out}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("attn", "mlp", "small", "block70b", "kron3", "grid128"),
+    ap.add_argument("--workload", choices=("attn", "mlp", "small", "block70b", "kron3", "grid128",
+                                           "gram"),
                     default="attn",
                     help="block70b: seconds per layer for one 70B-class block; kron3: a "
                          "three-factor Kronecker Hessian; grid128: the attention layer on an "
-                         "asymmetric 128-column-group packed INT4 grid (reports, not the "
+                         "asymmetric 128-column-group packed INT4 grid; gram: the Kronecker "
+                         "factors from activations on the tensor cores (reports, not the "
                          "headline metric)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -712,9 +783,10 @@ def main():
 
     import torch
     torch.cuda.set_device(local_rank)
-    if args.workload in ("block70b", "kron3", "grid128"):
+    if args.workload in ("block70b", "kron3", "grid128", "gram"):
         if rank == 0:
-            run = {"block70b": run_block70b, "kron3": run_kron3, "grid128": run_grid128}[args.workload]
+            run = {"block70b": run_block70b, "kron3": run_kron3, "grid128": run_grid128,
+                   "gram": run_gram}[args.workload]
             print(json.dumps(run(args)), flush=True)
         return
     if world > 1:

@@ -11,18 +11,19 @@
 // fp32 in tensor memory by tcgen05.mma (kind::f16, bf16 operands, M = N = 128,
 // K = 16 per instruction).  Both operands are chunks of 64 rows of X, and X is
 // row-major (features contiguous), so A (128 features x 64 rows) and B are
-// "MN-major": element (feature f, row r) of a chunk sits at byte
-//     (f / 8) * 128 + (r / 8) * 2048 + (r % 8) * 16 + (f % 8) * 2
-// of its shared-memory tile: 8 x 8 core matrices of 128 contiguous bytes, the
-// canonical layout without swizzle of the operand descriptor (stride byte offset
-// 128 between feature groups, leading byte offset 2048 between row groups).
-//   warps 1..3  fill a 4-stage ring with 16-byte cp.async copies (zero past the
-//               last row or column) and signal each stage's full barrier with
-//               cp.async.mbarrier.arrive.noinc;
-//   warp 0      allocates 128 columns of tensor memory; its elected thread waits
-//               for a full stage, fences the copies into the async proxy, issues
-//               the stage's four MMAs and frees the stage with tcgen05.commit on
-//               its empty barrier.  A last commit signals the end.
+// "MN-major".  Each operand is two TMA boxes of 64 features x 64 rows
+// (cp.async.bulk.tensor, 128-byte swizzle; zero fill past the last row or
+// column): a box holds the rows as 128-byte lines, swizzled in groups of 8 lines,
+// which is the canonical 128B-swizzled MN-major layout of the operand descriptor
+// (stride byte offset 1024 between 8-row groups, leading byte offset 8192 between
+// the two 64-feature boxes).
+//   warp 1, one thread  fills a 4-stage ring: it waits for the stage's empty
+//                       barrier, arms the full barrier with the stage's bytes and
+//                       issues the 2 (diagonal block) or 4 box loads;
+//   warp 0              allocates 128 columns of tensor memory; its elected thread
+//                       waits for a full stage, issues the stage's four MMAs and
+//                       frees the stage with tcgen05.commit on its empty barrier.
+//                       A last commit signals the end.
 // Then each warp reads its 32 lanes (rows) of the accumulator with tcgen05.ld and
 // writes (or adds) the fp32 block into H.  Every wait is bounded (%globaltimer);
 // a wait that gives up sets the error word, and the CTA still waits (bounded) for
@@ -31,6 +32,9 @@
 // gram_diag_kernel + gram_finalize_kernel: the diagonal's sum (one CTA, fixed order:
 // deterministic) into the workspace, then H <- H / N on the lower block triangle
 // and H_ii += damp * mean_i(H_ii / N).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "pipeline.cuh"
 
@@ -42,22 +46,34 @@ constexpr int GB = 128;                      // block edge (MMA M = N)
 constexpr int GK = 64;                       // rows of X per stage
 constexpr int GSTAGES = 4;
 constexpr int GTHREADS = 128;
-constexpr int GPRODUCERS = GTHREADS - 32;    // warps 1..3
-constexpr int G_TILE = GB * GK * 2;          // one bf16 operand tile: 16 KB
+constexpr int G_BOX = 64 * GK * 2;           // one TMA box: 64 features x 64 rows, 8 KB
+constexpr int G_TILE = 2 * G_BOX;            // one bf16 operand tile: 16 KB
 constexpr int G_STAGE = 2 * G_TILE;          // A and B
-constexpr int G_SMEM = GSTAGES * G_STAGE;
-constexpr uint32_t G_SBO = 128;              // between 8-feature groups
-constexpr uint32_t G_LBO = 2048;             // between 8-row groups
+constexpr int G_SMEM = GSTAGES * G_STAGE + 1024;  // + room to align the ring to 1024 bytes
+constexpr uint32_t G_SBO = 1024;             // between 8-row groups
+constexpr uint32_t G_LBO = G_BOX;            // between the two 64-feature boxes
 constexpr uint32_t G_TMEM_COLS = GB;         // fp32 accumulator: 128 lanes x 128 columns
 
 // Shared-memory operand descriptor: start address, leading and stride byte offsets
-// (all in 16-byte units), descriptor version 1, no swizzle.
+// (all in 16-byte units), descriptor version 1, 128-byte swizzle (layout type 2).
 __device__ __forceinline__ uint64_t g_desc(uint32_t saddr) {
   uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((G_LBO >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((G_SBO >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
   return d;
+}
+
+// One TMA box (x = feature, y = row) into shared memory, completing on `bar`.
+// x is a multiple of 64 (a 128-byte boundary of a row).  No multicast.
+__device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x, int y,
+                                        uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];\n" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // Instruction descriptor (kind::f16): fp32 accumulator (bit 4), bf16 A (bit 7) and
@@ -84,10 +100,6 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 }
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar))
-               : "memory");
-}
 
 struct GramArgs {
   const __nv_bfloat16* X;
@@ -100,11 +112,15 @@ struct GramArgs {
   int* err;
 };
 
-__global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a) {
-  extern __shared__ __align__(128) uint8_t gsm[];
+__global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a,
+                                                          const __grid_constant__ CUtensorMap tmap) {
+  extern __shared__ __align__(1024) uint8_t gsm_raw[];
+  // the 128-byte swizzle repeats every 1024 bytes: align the ring to that
+  uint8_t* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
   __shared__ __align__(8) uint64_t full_bar[GSTAGES], empty_bar[GSTAGES], done_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ long long issued;  // chunks whose loads were issued
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // block (bi, bj), bj <= bi, of the lower block triangle
@@ -118,11 +134,12 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a) {
 
   if (tid == 0) {
     for (int s = 0; s < GSTAGES; ++s) {
-      mbar_init(&full_bar[s], GPRODUCERS);
+      mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&done_bar, 1);
     abort_flag = 0;
+    issued = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == 0) {
@@ -138,11 +155,11 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a) {
   const uint32_t tmem = tmem_base;
   const int64_t nchunks = (a.N + GK - 1) / GK;
 
-  if (warp >= 1) {
-    // ---- producers: chunk c into stage c % GSTAGES, after the MMAs of chunk c - GSTAGES
-    const int ptid = tid - 32;
-    const int pieces = (diag ? 1 : 2) * (GB * GK / 8);  // 16-byte pieces per stage
-    for (int64_t c = 0; c < nchunks; ++c) {
+  if (warp == 1 && lane == 0) {
+    // ---- producer: chunk c into stage c % GSTAGES, after the MMAs of chunk c - GSTAGES
+    const unsigned bytes = (diag ? 1 : 2) * G_TILE;
+    long long c = 0;
+    for (; c < nchunks; ++c) {
       const int st = (int)(c % GSTAGES);
       if (c >= GSTAGES &&
           !mbar_wait(&empty_bar[st], (uint32_t)(((c / GSTAGES) - 1) & 1))) {
@@ -151,22 +168,18 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a) {
       }
       if (*(volatile int*)&abort_flag) break;
       uint8_t* sA = gsm + st * G_STAGE;
-      const int64_t r0 = c * GK;
-      for (int p = ptid; p < pieces; p += GPRODUCERS) {
-        const int op = p / (GB * GK / 8), q = p % (GB * GK / 8);
-        const int r8 = q & 7, fg = (q >> 3) & 15, rg = q >> 7;  // row % 8, feature group, row group
-        const int64_t row = r0 + rg * 8 + r8;
-        const int f = (op ? j0 : i0) + fg * 8;
-        const bool ok = row < a.N && f < a.k;
-        const void* src = ok ? (const void*)(a.X + row * a.ldx + f) : (const void*)a.X;
-        cp_async16_zfill(sA + op * G_TILE + fg * 128 + rg * 2048 + r8 * 16, src, ok);
+      const int y = (int)(c * GK);
+      mbar_arrive_expect_tx(&full_bar[st], bytes);
+      tma_box(sA, &tmap, i0, y, &full_bar[st]);
+      tma_box(sA + G_BOX, &tmap, i0 + 64, y, &full_bar[st]);
+      if (!diag) {
+        tma_box(sA + G_TILE, &tmap, j0, y, &full_bar[st]);
+        tma_box(sA + G_TILE + G_BOX, &tmap, j0 + 64, y, &full_bar[st]);
       }
-      cp_async_arrive_noinc(&full_bar[st]);
     }
-    cp_async_wait_group<0>();
-    asm volatile("cp.async.wait_all;\n" ::: "memory");
-  } else if (lane == 0) {
-    // ---- MMA issuer
+    issued = c;
+  } else if (warp == 0 && lane == 0) {
+    // ---- MMA issuer (one thread)
     for (int64_t c = 0; c < nchunks; ++c) {
       const int st = (int)(c % GSTAGES);
       if (!mbar_wait(&full_bar[st], (uint32_t)((c / GSTAGES) & 1))) {
@@ -174,13 +187,13 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a) {
         break;
       }
       if (*(volatile int*)&abort_flag) break;
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       tc_fence_after();
       const uint32_t aaddr = smem_u32(gsm + st * G_STAGE);
       const uint32_t baddr = diag ? aaddr : aaddr + G_TILE;
+      // K step s16 = rows 16 s16 .. 16 s16 + 15: two 8-row groups further (2 * SBO)
 #pragma unroll
       for (int s16 = 0; s16 < GK / 16; ++s16)
-        tc_mma(tmem, g_desc(aaddr + s16 * 2 * G_LBO), g_desc(baddr + s16 * 2 * G_LBO), G_IDESC,
+        tc_mma(tmem, g_desc(aaddr + s16 * 2 * G_SBO), g_desc(baddr + s16 * 2 * G_SBO), G_IDESC,
                (c > 0 || s16 > 0) ? 1u : 0u);
       tc_commit(&empty_bar[st]);
     }
@@ -188,6 +201,11 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a) {
   }
   __syncwarp();
   __syncthreads();
+  if (abort_flag && warp == 1 && lane == 0) {
+    // a wait gave up: let the box loads still in flight land before the CTA exits
+    for (long long c = issued - GSTAGES > 0 ? issued - GSTAGES : 0; c < issued; ++c)
+      mbar_wait(&full_bar[c % GSTAGES], (uint32_t)((c / GSTAGES) & 1));
+  }
   // every thread: the accumulator is final once done_bar completes
   const bool done = mbar_wait(&done_bar, 0);
   if (!done) atomicExch(&abort_flag, 1);
@@ -269,6 +287,21 @@ __global__ void __launch_bounds__(256) gram_finalize_kernel(float* H, int k, int
 
 std::atomic<uint64_t> g_gram_smem_set{0};
 
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<void*> fn{nullptr};
+  void* p = fn.load(std::memory_order_acquire);
+  if (!p) {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn.store(p, std::memory_order_release);
+  }
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+}
+
 }  // namespace
 
 int gram_accumulate_launch(const void* X, int64_t N, int k, int64_t ldx, float* H, int64_t ldh,
@@ -276,8 +309,24 @@ int gram_accumulate_launch(const void* X, int64_t N, int k, int64_t ldx, float* 
   if (ensure_smem(gram_kernel, G_SMEM, g_gram_smem_set) != cudaSuccess) return GPTQ2D_ERR_CUDA;
   const int nb = (k + GB - 1) / GB;
   GramArgs a{static_cast<const __nv_bfloat16*>(X), N, k, ldx, H, ldh, beta, err};
+  // X as a 2-D tensor (features fastest) in boxes of 64 x 64, 128-byte swizzle, zero
+  // fill outside; not built when there are no rows (the kernel then loads nothing)
+  CUtensorMap tmap;
+  memset(&tmap, 0, sizeof(tmap));
+  if (N > 0) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return GPTQ2D_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)GK};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTQ2D_ERR_CUDA;
+  }
   const int blocks = nb * (nb + 1) / 2;
-  GPTQ2D_LAUNCH(KC_OTHER, s, gram_kernel<<<blocks, GTHREADS, G_SMEM, s>>>(a));
+  GPTQ2D_LAUNCH(KC_OTHER, s, gram_kernel<<<blocks, GTHREADS, G_SMEM, s>>>(a, tmap));
   return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
