@@ -697,7 +697,7 @@ def run_gram(args):
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     peak = peaks.get("bf16_tflops", 1590.0)
     out = []
-    for k in (4096, 8192, 28672):
+    for k in ((8192,) if args.profile_step else (4096, 8192, 28672)):
         torch.manual_seed(k)
         rows = k
         z = torch.randn(rows, k, device=dev, dtype=torch.float32)
@@ -714,6 +714,10 @@ def run_gram(args):
             g.gram_accumulate(Xb, H, accumulate=False, workspace=ws)
             g.gram_finalize(H, rows, 0.01, workspace=ws, check=False)
 
+        if args.profile_step:  # one Gram of the 8192-wide case, nothing else (ncu input)
+            step()
+            torch.cuda.synchronize()
+            return None
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
@@ -787,7 +791,9 @@ def main():
         if rank == 0:
             run = {"block70b": run_block70b, "kron3": run_kron3, "grid128": run_grid128,
                    "gram": run_gram}[args.workload]
-            print(json.dumps(run(args)), flush=True)
+            res = run(args)
+            if res is not None:
+                print(json.dumps(res), flush=True)
         return
     if world > 1:
         import datetime
