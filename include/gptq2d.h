@@ -323,6 +323,56 @@ int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64
                          void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* A block of layers (the pages quantize whole models, block by block:         */
+/* arxivlens, Abstract, Llama-3.1-70B-Instruct on one GPU)                     */
+/* ------------------------------------------------------------------------- */
+
+/* One linear layer of a block.  All pointers are DEVICE pointers except that the
+ * grid is held by value (its scales and zeros are device pointers).
+ *   W, w_dtype, m, n, ldw  : as in gptq2d_quantize.
+ *   H_L, ldhl, H_R, ldhr, h_dtype : the layer's Grams (m x m and n x n, GPTQ2D_F32
+ *                            or GPTQ2D_F64, lower triangles read), e.g. from
+ *                            gptq2d_gram_accumulate / gptq2d_gram_finalize.
+ *   grid                   : as in gptq2d_quantize_grid.
+ *   Q, ldq, stats          : outputs, as in gptq2d_quantize_grid. */
+typedef struct {
+  const void* W;
+  int w_dtype;
+  int64_t m, n, ldw;
+  const void* H_L;
+  int64_t ldhl;
+  const void* H_R;
+  int64_t ldhr;
+  int h_dtype;
+  gptq2d_grid grid;
+  void* Q;
+  int64_t ldq;
+  gptq2d_stats* stats;
+} gptq2d_layer;
+
+/* Bytes of device workspace gptq2d_quantize_block needs for these layers (two factor
+ * slots for the largest layer, 512 bytes per layer, one rounding workspace for the
+ * largest layer); 0 for invalid sizes. */
+size_t gptq2d_block_workspace_size(const gptq2d_layer* layers, int nl);
+
+/* Factors and rounds nl layers, overlapping the factor preparation of layer i + 1
+ * with the rounding of layer i: the factors go to library-internal streams of their
+ * own, the roundings run one after another in the given order (largest first keeps
+ * the GPU busiest), and each of the two factor slots is reused once the layer that
+ * read it is rounded.  Every layer's result is exactly what gptq2d_prepare_pair +
+ * gptq2d_quantize_grid give it alone.  Waits for `stream` before it starts; later
+ * work on `stream` sees every output.  Synchronizes `stream` at the end to read
+ * the factors' pivot words: returns GPTQ2D_ERR_NOT_SPD for the first layer with a
+ * factor that is not positive definite (*bad_layer, *bad_pivot and *which_factor,
+ * each a HOST pointer or NULL, receive the layer, the pivot and 0 for H_L / 1 for
+ * H_R; -1 when all are positive definite); that layer's rounding ran on a failed
+ * factor and its statistics are not meaningful.  Arguments of every layer are
+ * checked before anything is enqueued. */
+int gptq2d_quantize_block(const gptq2d_layer* layers, int nl, void* ws, size_t ws_bytes,
+                          void* stream, int64_t* bad_layer, int64_t* bad_pivot,
+                          int* which_factor);
+
+/* ------------------------------------------------------------------------- */
 /* Rounding without any allocation                                             */
 /* (no counterpart in the GPTQ-2D pages: an interface for callers of this     */
 /* library that may not allocate device memory)                               */

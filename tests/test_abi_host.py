@@ -201,3 +201,23 @@ def test_gram_finalize_rejects_invalid_arguments(L):
     assert f(8192, 64, 63, 10, 0.01, 256, 256, None, None) == g.Status.INVALID_ARG    # ldh < k
     assert f(8192, 64, 64, 10, 0.01, 0, 256, None, None) == g.Status.WORKSPACE
     assert L.gptq2d_gram_workspace_size() >= 12
+
+
+def test_block_rejects_invalid_arguments(L):
+    """Checked on the host before anything is enqueued."""
+    assert L.gptq2d_quantize_block(None, -1, None, 0, None, None, None, None) == g.Status.INVALID_ARG
+    assert L.gptq2d_quantize_block(None, 2, None, 0, None, None, None, None) == g.Status.INVALID_ARG
+    assert L.gptq2d_quantize_block(None, 0, None, 0, None, None, None, None) == g.Status.OK
+    lay = (g._Layer * 1)()
+    lay[0] = g._Layer(4096, g.DTYPE_BF16, 64, 64, 64, 8192, 64, 8192, 64, 7,   # bad Gram dtype
+                      g._Grid(4, 1, 0, 16, 1, None, 0), 16, 64, 16)
+    assert L.gptq2d_quantize_block(lay, 1, 256, 1 << 40, None, None, None, None) == g.Status.INVALID_ARG
+    lay[0].h_dtype = g.DTYPE_F32
+    lay[0].ldhl = 63
+    assert L.gptq2d_quantize_block(lay, 1, 256, 1 << 40, None, None, None, None) == g.Status.INVALID_ARG
+    lay[0].ldhl = 64
+    lay[0].grid.bits = 9
+    assert L.gptq2d_quantize_block(lay, 1, 256, 1 << 40, None, None, None, None) == g.Status.INVALID_ARG
+    lay[0].grid.bits = 4
+    assert L.gptq2d_quantize_block(lay, 1, 256, 10, None, None, None, None) == g.Status.WORKSPACE
+    assert L.gptq2d_block_workspace_size(lay, 1) >= 2 * 2 * 64 * 64 * 8

@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS", "quantize_grid",
-    "gram_accumulate", "gram_finalize", "gram",
+    "gram_accumulate", "gram_finalize", "gram", "quantize_block", "block_workspace_size",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
     "round_host_workspace_size", "quantize_noalloc", "check_wait_timeout", "profile_enable",
     "profile_reset", "profile_read", "profile_timeline",
@@ -62,6 +62,14 @@ class _Grid(ctypes.Structure):
                 ("scales", _c_p), ("ld_scales", _c_i64), ("zeros", _c_p), ("packed", ctypes.c_int)]
 
 
+class _Layer(ctypes.Structure):
+    """gptq2d_layer"""
+    _fields_ = [("W", _c_p), ("w_dtype", ctypes.c_int), ("m", _c_i64), ("n", _c_i64),
+                ("ldw", _c_i64), ("H_L", _c_p), ("ldhl", _c_i64), ("H_R", _c_p), ("ldhr", _c_i64),
+                ("h_dtype", ctypes.c_int), ("grid", _Grid), ("Q", _c_p), ("ldq", _c_i64),
+                ("stats", _c_p)]
+
+
 def lib():
     """The loaded shared library (built in-tree by two_sided_adaptive_b200.build)."""
     global _LIB
@@ -95,6 +103,12 @@ def lib():
                                           ctypes.POINTER(_c_i64), ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_prepare_info.restype = ctypes.c_int
         L.gptq2d_prepare_info.argtypes = [_c_p, _c_p, ctypes.POINTER(_c_i64)]
+        L.gptq2d_block_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_block_workspace_size.argtypes = [ctypes.POINTER(_Layer), ctypes.c_int]
+        L.gptq2d_quantize_block.restype = ctypes.c_int
+        L.gptq2d_quantize_block.argtypes = [ctypes.POINTER(_Layer), ctypes.c_int, _c_p,
+                                            ctypes.c_size_t, _c_p, ctypes.POINTER(_c_i64),
+                                            ctypes.POINTER(_c_i64), ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_gram_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_gram_accumulate.restype = ctypes.c_int
         L.gptq2d_gram_accumulate.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
@@ -434,6 +448,68 @@ def quantize_grid(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, gro
     if rc != Status.OK:
         raise GPTQ2DError(rc, "gptq2d_quantize_grid")
     return Q, st
+
+
+def _layers(specs, outs, stats):
+    torch = _torch()
+    arr = (_Layer * len(specs))()
+    keep = []
+    for i, sp in enumerate(specs):
+        W, H_L, H_R, sc = sp["W"], sp["H_L"], sp["H_R"], sp["scales"]
+        m, n = W.shape
+        S = sc.reshape(m, -1) if sc.dim() == 1 else sc
+        Z = sp.get("zeros")
+        if Z is not None:
+            Z = Z.reshape(m, -1)
+        packed = bool(sp.get("packed", False))
+        keep += [S, Z]
+        gr = _Grid(int(sp.get("bits", 4)), int(sp.get("clamp", True)), int(sp.get("group_size", 0)),
+                   S.data_ptr(), S.stride(0) if m else 1, Z.data_ptr() if Z is not None else None,
+                   int(packed))
+        if H_L.dtype != H_R.dtype:
+            raise ValueError("H_L and H_R must share a dtype")
+        arr[i] = _Layer(W.data_ptr(), _dtype_code(W), m, n, _ld(W), H_L.data_ptr(), _ld(H_L),
+                        H_R.data_ptr(), _ld(H_R), _dtype_code(H_L), gr,
+                        outs[i].data_ptr() if outs is not None else None,
+                        _ld(outs[i]) if outs is not None and outs[i].numel() else 1,
+                        stats[i].data_ptr() if stats is not None else None)
+    return arr, keep
+
+
+def block_workspace_size(specs) -> int:
+    """gptq2d_block_workspace_size for layer specs (dicts with W, H_L, H_R, scales, ...)."""
+    arr, _ = _layers(specs, None, None)
+    return int(lib().gptq2d_block_workspace_size(arr, len(specs)))
+
+
+def quantize_block(specs, *, workspace=None, stream=None):
+    """gptq2d_quantize_block: factors and rounds a block of layers, the factor preparation
+    of the next layer overlapping the rounding of the current one.  ``specs``: dicts with
+    W (m x n), H_L (m x m), H_R (n x n) Grams on the GPU, scales (m or m x groups fp32),
+    and optionally bits, clamp, group_size, zeros (uint8), packed.  Returns (list of Q,
+    list of stats)."""
+    torch = _torch()
+    if not specs:
+        return [], []
+    dev_ = specs[0]["W"].device
+    outs, stats = [], []
+    for sp in specs:
+        m, n = sp["W"].shape
+        packed = bool(sp.get("packed", False))
+        qdt = torch.uint8 if (sp.get("zeros") is not None or packed) else torch.int8
+        outs.append(torch.empty((m, (n + 1) // 2 if packed else n), dtype=qdt, device=dev_))
+        stats.append(torch.empty(STATS_WORDS, dtype=torch.int64, device=dev_))
+    arr, keep = _layers(specs, outs, stats)
+    nbytes = int(lib().gptq2d_block_workspace_size(arr, len(specs)))
+    ws = _workspace(nbytes, dev_, workspace)
+    bl, bp, wf = _c_i64(-1), _c_i64(-1), ctypes.c_int(-1)
+    rc = lib().gptq2d_quantize_block(arr, len(specs), ws.data_ptr(), ws.numel(), _stream(stream),
+                                     ctypes.byref(bl), ctypes.byref(bp), ctypes.byref(wf))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_quantize_block",
+                          f"layer {bl.value} factor {wf.value} pivot {bp.value}"
+                          if rc == Status.NOT_SPD else "")
+    return outs, stats
 
 
 def quantize_noalloc(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None,

@@ -332,10 +332,12 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
                          Q, ldq, stats, ws, s);
 }
 
-int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
-                         const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
-                         const gptq2d_grid* grid, void* Q, int64_t ldq, gptq2d_stats* stats,
-                         void* ws, size_t ws_bytes, void* stream) {
+namespace {
+// Host checks of a rounding call on a grid (everything but the factors and the
+// workspace); fills `gs`.  m == 0 or n == 0 passes (nothing to round).
+int check_grid_call(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                    const gptq2d_grid* grid, const void* Q, int64_t ldq, const gptq2d_stats* stats,
+                    GridSpec* gs) {
   if (m < 0 || n < 0 || m > kMaxDim || n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
   if (elem_size(w_dtype) == 0 || !grid || !stats) return GPTQ2D_ERR_INVALID_ARG;
   const int bits = grid->bits, clamp = grid->clamp;
@@ -345,25 +347,159 @@ int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64
   if (grid->zeros && !clamp) return GPTQ2D_ERR_INVALID_ARG;  // codes must fit their byte
   const int64_t G = grid->group_size;
   if (G < 0 || (G > 0 && G % 8 != 0 && G < n)) return GPTQ2D_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gs->group = G;
+  gs->lds = grid->ld_scales;
+  gs->zero = grid->zeros;
+  gs->packed = grid->packed;
+  if (m == 0 || n == 0) return GPTQ2D_OK;
+  const int64_t groups = (G == 0 || G >= n) ? 1 : (n + G - 1) / G;
+  if (!W || !grid->scales || !Q) return GPTQ2D_ERR_INVALID_ARG;
+  if (grid->ld_scales < groups) return GPTQ2D_ERR_INVALID_ARG;
+  if (ldw < n || ldq < (grid->packed ? (n + 1) / 2 : n)) return GPTQ2D_ERR_INVALID_ARG;
+  return GPTQ2D_OK;
+}
+}  // namespace
+
+int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                         const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                         const gptq2d_grid* grid, void* Q, int64_t ldq, gptq2d_stats* stats,
+                         void* ws, size_t ws_bytes, void* stream) {
   GridSpec gs;
-  gs.group = G;
-  gs.lds = grid->ld_scales;
-  gs.zero = grid->zeros;
-  gs.packed = grid->packed;
+  const int rc = check_grid_call(W, w_dtype, m, n, ldw, grid, Q, ldq, stats, &gs);
+  if (rc != GPTQ2D_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (m == 0 || n == 0)
     return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales,
-                           bits, clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0, nullptr,
-                           nullptr, &gs);
-  const int64_t groups = (G == 0 || G >= n) ? 1 : (n + G - 1) / G;
-  if (!W || !M_L || !M_R || !grid->scales || !Q) return GPTQ2D_ERR_INVALID_ARG;
-  if (grid->ld_scales < groups) return GPTQ2D_ERR_INVALID_ARG;
-  if (ldw < n || ldl < m || ldr < n || ldq < (grid->packed ? (n + 1) / 2 : n))
-    return GPTQ2D_ERR_INVALID_ARG;
+                           grid->bits, grid->clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0,
+                           nullptr, nullptr, &gs);
+  if (!M_L || !M_R || ldl < m || ldr < n) return GPTQ2D_ERR_INVALID_ARG;
   if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(m, n)) return GPTQ2D_ERR_WORKSPACE;
-  return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales, bits,
-                         clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0, nullptr, nullptr,
-                         &gs);
+  return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales,
+                         grid->bits, grid->clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0,
+                         nullptr, nullptr, &gs);
+}
+
+// ---------------------------------------------------------------------------
+// A block of layers (gptq2d_quantize_block)
+// ---------------------------------------------------------------------------
+namespace {
+struct BlockLayout {
+  size_t slot, off_piv, off_q, total;
+};
+// Two factor slots (each holds one layer's M_L then M_R, both dense with ld = m, n),
+// 512 bytes of pivot words per layer, one rounding workspace for the largest layer.
+BlockLayout block_layout(const gptq2d_layer* L, int nl) {
+  BlockLayout B{0, 0, 0, 0};
+  size_t q = 256;
+  for (int i = 0; i < nl; ++i) {
+    const size_t fl = align256((size_t)L[i].m * L[i].m * sizeof(double)) +
+                      align256((size_t)L[i].n * L[i].n * sizeof(double));
+    B.slot = std::max(B.slot, fl);
+    if (L[i].m > 0 && L[i].n > 0) q = std::max(q, quantize_ws_bytes(L[i].m, L[i].n));
+  }
+  B.off_piv = 2 * B.slot;
+  B.off_q = B.off_piv + align256((size_t)nl * 512);
+  B.total = B.off_q + align256(q);
+  return B;
+}
+}  // namespace
+
+size_t gptq2d_block_workspace_size(const gptq2d_layer* layers, int nl) {
+  if (nl < 0 || (nl > 0 && !layers)) return 0;
+  for (int i = 0; i < nl; ++i)
+    if (layers[i].m < 0 || layers[i].n < 0 || layers[i].m > kMaxDim || layers[i].n > kMaxDim)
+      return 0;
+  return block_layout(layers, nl).total;
+}
+
+int gptq2d_quantize_block(const gptq2d_layer* L, int nl, void* ws, size_t ws_bytes, void* stream,
+                          int64_t* bad_layer, int64_t* bad_pivot, int* which_factor) {
+  if (bad_layer) *bad_layer = -1;
+  if (bad_pivot) *bad_pivot = -1;
+  if (which_factor) *which_factor = -1;
+  if (nl < 0 || (nl > 0 && !L)) return GPTQ2D_ERR_INVALID_ARG;
+  if (nl == 0) return GPTQ2D_OK;
+  std::vector<GridSpec> gs(nl);
+  for (int i = 0; i < nl; ++i) {
+    const gptq2d_layer& l = L[i];
+    const int rc = check_grid_call(l.W, l.w_dtype, l.m, l.n, l.ldw, &l.grid, l.Q, l.ldq, l.stats,
+                                   &gs[i]);
+    if (rc != GPTQ2D_OK) return rc;
+    if (l.h_dtype != GPTQ2D_F32 && l.h_dtype != GPTQ2D_F64) return GPTQ2D_ERR_INVALID_ARG;
+    if (l.m > 0 && (!l.H_L || l.ldhl < l.m)) return GPTQ2D_ERR_INVALID_ARG;
+    if (l.n > 0 && (!l.H_R || l.ldhr < l.n)) return GPTQ2D_ERR_INVALID_ARG;
+  }
+  const BlockLayout B = block_layout(L, nl);
+  if (!ws || !aligned256(ws) || ws_bytes < B.total) return GPTQ2D_ERR_WORKSPACE;
+  DevStreams* ds = nullptr;
+  int rc = dev_streams(&ds);
+  if (rc != GPTQ2D_OK) return rc;
+  std::lock_guard<std::recursive_mutex> lk(ds->mu);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(ws);
+  bool ok = cudaEventRecord(ds->blk_start, s) == cudaSuccess &&
+            cudaStreamWaitEvent(ds->blk_p, ds->blk_start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(ds->blk_q, ds->blk_start, 0) == cudaSuccess;
+  if (!ok) return GPTQ2D_ERR_CUDA;
+  auto ML = [&](int i) { return reinterpret_cast<double*>(base + (i & 1) * B.slot); };
+  auto MR = [&](int i) {
+    return reinterpret_cast<double*>(base + (i & 1) * B.slot +
+                                     align256((size_t)L[i].m * L[i].m * sizeof(double)));
+  };
+  // The factors of layer i on the second factor pairs, beside the rounding of layer
+  // i - 1; slot i & 1 is free once layer i - 2 is rounded.
+  auto prep = [&](int i) -> int {
+    const gptq2d_layer& l = L[i];
+    if (i >= 2 && cudaStreamWaitEvent(ds->blk_p, ds->blk_quant[i & 1], 0) != cudaSuccess)
+      return GPTQ2D_ERR_CUDA;
+    char* pv = base + B.off_piv + (size_t)i * 512;
+    if (cudaMemsetAsync(pv, 0xFF, 512, ds->blk_p) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+    const int r = prepare_pair_launch(l.H_L, l.m, l.ldhl, l.H_R, l.n, l.ldhr, l.h_dtype, ML(i), l.m,
+                                      MR(i), l.n, pv, pv + 256, ds->blk_p, nullptr, nullptr, true);
+    if (r != GPTQ2D_OK) return r;
+    return cudaEventRecord(ds->blk_prep[i & 1], ds->blk_p) == cudaSuccess ? GPTQ2D_OK
+                                                                           : GPTQ2D_ERR_CUDA;
+  };
+  auto quant = [&](int i) -> int {
+    const gptq2d_layer& l = L[i];
+    if (cudaStreamWaitEvent(ds->blk_q, ds->blk_prep[i & 1], 0) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+    const int r = quantize_launch(l.W, l.w_dtype, (int)l.m, (int)l.n, l.ldw, ML(i), l.m, MR(i), l.n,
+                                  l.grid.scales, l.grid.bits, l.grid.clamp,
+                                  static_cast<int8_t*>(l.Q), l.ldq, l.stats, base + B.off_q,
+                                  ds->blk_q, 0, nullptr, nullptr, &gs[i]);
+    if (r != GPTQ2D_OK) return r;
+    return cudaEventRecord(ds->blk_quant[i & 1], ds->blk_q) == cudaSuccess ? GPTQ2D_OK
+                                                                            : GPTQ2D_ERR_CUDA;
+  };
+  rc = prep(0);
+  if (rc == GPTQ2D_OK && nl > 1) rc = prep(1);
+  for (int i = 0; i < nl && rc == GPTQ2D_OK; ++i) {
+    rc = quant(i);
+    if (rc == GPTQ2D_OK && i + 2 < nl) rc = prep(i + 2);
+  }
+  ok = cudaEventRecord(ds->blk_end[0], ds->blk_p) == cudaSuccess &&
+       cudaEventRecord(ds->blk_end[1], ds->blk_q) == cudaSuccess &&
+       cudaStreamWaitEvent(s, ds->blk_end[0], 0) == cudaSuccess &&
+       cudaStreamWaitEvent(s, ds->blk_end[1], 0) == cudaSuccess;
+  if (rc != GPTQ2D_OK) return rc;
+  if (!ok) return GPTQ2D_ERR_CUDA;
+  // pivot words of every layer (two per layer: left, right)
+  std::vector<long long> piv((size_t)nl * 64);
+  if (cudaMemcpyAsync(piv.data(), base + B.off_piv, (size_t)nl * 512, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return GPTQ2D_ERR_CUDA;
+  for (int i = 0; i < nl; ++i)
+    for (int side = 0; side < 2; ++side) {
+      const long long p = piv[(size_t)i * 64 + side * 32];
+      if (p >= 0 && ((side == 0 && L[i].m > 0) || (side == 1 && L[i].n > 0))) {
+        if (bad_layer) *bad_layer = i;
+        if (bad_pivot) *bad_pivot = p;
+        if (which_factor) *which_factor = side;
+        return GPTQ2D_ERR_NOT_SPD;
+      }
+    }
+  return GPTQ2D_OK;
 }
 
 size_t gptq2d_round_host_workspace_size(int64_t m, int64_t n, int w_dtype, int h_dtype) {

@@ -146,9 +146,12 @@ struct DevStreams {
   bool ready = false;
   int sms = 148;
   cudaStream_t hi = nullptr, lo = nullptr, hi2 = nullptr, lo2 = nullptr;
+  cudaStream_t hi3 = nullptr, lo3 = nullptr;  // a second factor pair, beside a rounding
   cudaStream_t cp = nullptr;  // host<->device copies of round_host
+  cudaStream_t blk_p = nullptr, blk_q = nullptr;  // block scheduler: factor and rounding lanes
   cudaEvent_t fork = nullptr, setup = nullptr, join_hi = nullptr, join_lo = nullptr;
-  cudaEvent_t join_hi2 = nullptr, join_lo2 = nullptr;
+  cudaEvent_t join_hi2 = nullptr, join_lo2 = nullptr, join_hi3 = nullptr, join_lo3 = nullptr;
+  cudaEvent_t blk_start = nullptr, blk_prep[2] = {}, blk_quant[2] = {}, blk_end[2] = {};
   cudaEvent_t cp_ev[3] = {};  // H_L, H_R, W + scales copied
   cudaEvent_t q_ev[4] = {};   // rows of Q final (round_host copies them out early)
   cudaEvent_t sw[RING] = {}, far[RING] = {}, farb[RING] = {};
@@ -167,10 +170,13 @@ int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
 // (panels on the high-priority ones, trailing updates on the low-priority
 // ones), forked from and joined back to `s`.
 // ready_l / ready_r (may be null): events that H_L / H_R wait for beyond `s`.
+// alt: run on the second factor pairs (hi2/lo2 and hi3/lo3), leaving hi/lo to a
+// rounding that runs beside it.
 int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
                         int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s,
-                        cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr);
+                        cudaEvent_t ready_l = nullptr, cudaEvent_t ready_r = nullptr,
+                        bool alt = false);
 
 // Gram of activations on the tcgen05 tensor cores (defined in gram.cu): H's lower
 // 128-block triangle (+)= X^T X (X bf16, N x k, k and ldx multiples of 8); then

@@ -597,7 +597,8 @@ FactorJob make_job(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
 }
 
 // Enqueues the factorizations of `jobs` (1 or 2), forked from and joined back to s.
-int enqueue_factors(FactorJob* jobs, int nj, cudaStream_t s, DevStreams* ds) {
+// alt: the jobs run on hi2/lo2 and hi3/lo3 (join events to match).
+int enqueue_factors(FactorJob* jobs, int nj, cudaStream_t s, DevStreams* ds, bool alt = false) {
   int rc = ensure_prepare_smem();
   if (rc != GPTQ2D_OK) return rc;
   bool ok = cudaEventRecord(ds->fork, s) == cudaSuccess;
@@ -614,7 +615,8 @@ int enqueue_factors(FactorJob* jobs, int nj, cudaStream_t s, DevStreams* ds) {
   for (int st = 0; st < steps && rc == GPTQ2D_OK; ++st)
     for (int j = 0; j < nj && rc == GPTQ2D_OK; ++j)
       if (st < jobs[j].T) rc = enqueue_step(jobs[j], jobs[j].T - 1 - st, ds->sms);
-  cudaEvent_t joins[4] = {ds->join_hi, ds->join_lo, ds->join_hi2, ds->join_lo2};
+  cudaEvent_t joins[4] = {alt ? ds->join_hi3 : ds->join_hi, alt ? ds->join_lo3 : ds->join_lo,
+                          ds->join_hi2, ds->join_lo2};
   for (int j = 0; j < nj && ok; ++j)
     ok = cudaEventRecord(joins[2 * j], jobs[j].ps) == cudaSuccess &&
          cudaEventRecord(joins[2 * j + 1], jobs[j].us) == cudaSuccess &&
@@ -642,25 +644,28 @@ int prepare_launch(const void* H, int h_dtype, int k, int64_t ldh, double* M, in
 int prepare_pair_launch(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
                         int64_t ldmr, void* ws_l, void* ws_r, cudaStream_t s,
-                        cudaEvent_t ready_l, cudaEvent_t ready_r) {
+                        cudaEvent_t ready_l, cudaEvent_t ready_r, bool alt) {
   DevStreams* ds = nullptr;
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
   std::lock_guard<std::recursive_mutex> lk(ds->mu);
+  // stream pairs: (hi, lo) then (hi2, lo2); alt: (hi3, lo3) then (hi2, lo2)
+  cudaStream_t ph[2] = {alt ? ds->hi3 : ds->hi, ds->hi2};
+  cudaStream_t pl[2] = {alt ? ds->lo3 : ds->lo, ds->lo2};
   FactorJob jobs[2];
   int nj = 0;
   if (m > 0) {
-    jobs[nj] = make_job(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ds->hi, ds->lo,
+    jobs[nj] = make_job(H_L, h_dtype, (int)m, ldhl, M_L, ldml, ws_l, ph[0], pl[0],
                         ds->panel_done[0], ds->rest_done[0]);
     jobs[nj++].ready = ready_l;
   }
   if (n > 0) {
-    jobs[nj] = make_job(H_R, h_dtype, (int)n, ldhr, M_R, ldmr, ws_r, nj ? ds->hi2 : ds->hi,
-                        nj ? ds->lo2 : ds->lo, ds->panel_done[nj], ds->rest_done[nj]);
+    jobs[nj] = make_job(H_R, h_dtype, (int)n, ldhr, M_R, ldmr, ws_r, ph[nj], pl[nj],
+                        ds->panel_done[nj], ds->rest_done[nj]);
     jobs[nj++].ready = ready_r;
   }
   if (nj == 0) return GPTQ2D_OK;
-  return enqueue_factors(jobs, nj, s, ds);
+  return enqueue_factors(jobs, nj, s, ds, alt);
 }
 
 }  // namespace gptq2d
