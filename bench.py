@@ -234,6 +234,20 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
+def lpt_assign(costs, world: int):
+    """Longest-processing-time-first assignment of independent layers to ranks: layers in
+    descending cost (ties: lower index first), each to the least-loaded rank (ties: lower
+    rank).  Every rank computes the same assignment; no collective is needed."""
+    order = sorted(range(len(costs)), key=lambda i: (-costs[i], i))
+    load = [0.0] * world
+    owner = [0] * len(costs)
+    for i in order:
+        r = min(range(world), key=lambda q: (load[q], q))
+        owner[i] = r
+        load[r] += costs[i]
+    return owner
+
+
 def rank_seed(rank: int) -> int:
     """Each rank rounds its own independent layer: the workload seed is the rank."""
     return rank
@@ -478,7 +492,7 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
-def run_block70b(args):
+def run_block70b(args, rank: int = 0, world: int = 1):
     """Seconds per layer and for the whole block: the seven linear layers of one
     70B-class block (q, o: 8192x8192; k, v: 1024x8192; gate, up: 8192x28672; down:
     28672x8192), INT4 per-row absmax scales, W ~ N(0, 0.015^2) in bf16, Grams from
@@ -488,15 +502,23 @@ def run_block70b(args):
     each timed with CUDA events on its second pass:
       sequential  prepare_pair + quantize per layer, one after another;
       pipelined   one quantize_block call (the factors of the next layer prepared
-                  beside the rounding of the current one), largest layers first."""
+                  beside the rounding of the current one), largest layers first.
+    Under torchrun the layers are spread over the ranks by LPT on mn(m + n) (no
+    collective on the data path); each rank times quantize_block on its share between
+    barriers, and the block's time is the slowest rank's (the sequential schedule is
+    then not timed)."""
     import torch
     import two_sided_adaptive_b200 as g
     from two_sided_adaptive_b200 import build as gbuild
     import workloads as WL
     gbuild.build()
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shapes = WL.block70b_shapes()
+    owner = lpt_assign([m * n * (m + n) for _, m, n, _ in shapes], world)
     specs, names = [], []
-    for li, (name, m, n, _) in enumerate(WL.block70b_shapes()):
+    for li, (name, m, n, _) in enumerate(shapes):
+        if owner[li] != rank:
+            continue
         torch.manual_seed(1000 + li)
 
         def gram(width):
@@ -518,7 +540,7 @@ def run_block70b(args):
         torch.cuda.empty_cache()
     # sequential
     layers, total = [], 0.0
-    for name, sp in zip(names, specs):
+    for name, sp in zip(names, specs if world == 1 else []):
         m, n = sp["W"].shape
         ML = torch.empty((m, m), dtype=torch.float64, device=dev)
         MR = torch.empty((n, n), dtype=torch.float64, device=dev)
@@ -550,23 +572,33 @@ def run_block70b(args):
     bspecs = [specs[i] for i in order]
     ws = torch.empty(g.block_workspace_size(bspecs), dtype=torch.uint8, device=dev)
     tb = None
+    import torch.distributed as dist
+    multi = world > 1 and dist.is_initialized()
     for rep in range(2):
+        if multi:
+            dist.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         Qs, sts = g.quantize_block(bspecs, workspace=ws)
         e1.record()
         torch.cuda.synchronize()
+        if multi:
+            dist.barrier()
         tb = e0.elapsed_time(e1) / 1e3
+    tb = max_over_ranks(tb, device=dev)
     bstat = [g.stats_dict(st)["status"] for st in sts]
-    return {"metric": "70B-class block: seconds for its 7 linear layers (INT4, 1 B200)",
-            "value": tb, "unit": "s", "n_gpus": 1, "higher_is_better": False,
+    return {"metric": "70B-class block: seconds for its 7 linear layers (INT4, %d B200)" % world,
+            "value": tb, "unit": "s", "n_gpus": world, "higher_is_better": False,
             "dtype": "f64", "data": "synthetic (generated on the GPU, see run_block70b)",
             "config": {"workload": "block70b",
                        "step": "quantize_block (factors of the next layer beside the rounding "
                                "of the current one), largest first",
-                       "order": [names[i] for i in order]},
-            "sequential_s": total, "pipelined_s": tb, "pipelined_status": bstat,
+                       "order": [names[i] for i in order],
+                       "parallelism": "layers by LPT over ranks" if world > 1 else "single GPU",
+                       "owner": [shapes[i][0] + ":%d" % owner[i] for i in range(len(shapes))]},
+            "sequential_s": total if world == 1 else None, "pipelined_s": tb,
+            "pipelined_status": bstat,
             "block_workspace_gb": ws.numel() / 1e9, "layers": layers}
 
 
@@ -816,6 +848,18 @@ def main():
 
     import torch
     torch.cuda.set_device(local_rank)
+    if args.workload == "block70b" and world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+        try:
+            res = run_block70b(args, rank, world)
+        finally:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     if args.workload in ("block70b", "kron3", "grid128", "gram"):
         if rank == 0:
             run = {"block70b": run_block70b, "kron3": run_kron3, "grid128": run_grid128,
