@@ -63,7 +63,7 @@ def test_real_activations_within_fp32_bound(g):
     X = WL.student_t_activations(rng, rows, k)
     Xb = torch.from_numpy(X.astype(np.float32)).cuda().to(torch.bfloat16)
     Xd = Xb.double().cpu().numpy()
-    H = torch.empty((k, k), dtype=torch.float32, device="cuda")
+    H = torch.zeros((k, k), dtype=torch.float32, device="cuda")  # entries above the block triangle stay untouched
     g.gram_accumulate(Xb, H, accumulate=False, workspace=_ws(g))
     torch.cuda.synchronize()
     Hg = H.cpu().numpy().astype(np.float64)
