@@ -34,7 +34,6 @@ namespace {
 constexpr int OLD = TB + 4;  // 68: row stride of shared 64x64 tiles (conflict-free DMMA fragments)
 constexpr int PANEL_THREADS = 384;   // 8 factor warps + 4 warps for the block-row lookahead
 constexpr int FACTOR_THREADS = 256;
-constexpr int MAX_TR_GROUPS = 512;
 
 template <typename TH>
 __global__ void __launch_bounds__(256) convert_lower_kernel(const TH* __restrict__ H, int64_t ldh,
@@ -355,10 +354,9 @@ __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict
 constexpr int MAX_STRIP = 4;  // block rows per strip (rank of a trailing update: 64 x strip)
 
 struct TrailPlan {
-  int k0, nk;                    // the strip: factored block rows k0 .. k0 + nk - 1
-  int I0, ng;                    // first group, number of groups
-  int per_cta;                   // blocks J per CTA
-  int start[MAX_TR_GROUPS + 1];  // first CTA of each group; group g updates A[I0+g][0..I0+g]
+  int k0, nk;    // the strip: factored block rows k0 .. k0 + nk - 1
+  int rows;      // block rows I = 0 .. rows - 1 are updated (J <= I)
+  int per_cta;   // block pairs per CTA
 };
 
 constexpr int TR_STAGE = 8 * 40;  // per warp: one 8x32 strip of the product (row stride 40)
@@ -366,9 +364,11 @@ constexpr int TR_STAGE = 8 * 40;  // per warp: one 8x32 strip of the product (ro
 // blocks of column I, two stream buffers, one staging strip per warp.
 constexpr int tr_smem(int nk, int nw) { return ((nk + 2) * TB * OLD + nw * TR_STAGE) * (int)sizeof(double); }
 
-// A_IJ -= sum_{q < nk} M_{k0+q,I}^T M_{k0+q,J} for J <= I, over a range of J of one
-// block row I: the rank-64 nk update of one strip.  Each CTA keeps the strip's
-// blocks of column I in shared memory and streams the blocks M_{k0+q,J} through a
+// A_IJ -= sum_{q < nk} M_{k0+q,I}^T M_{k0+q,J} for J <= I: the rank-64 nk update of
+// one strip.  The block pairs (I, J) are numbered row by row and every CTA takes an
+// equal run of them (no CTA waits for a longer one at the end of the launch).  A
+// CTA keeps the strip's blocks of its current column I in shared memory (reloaded
+// when its run enters the next row) and streams the blocks M_{k0+q,J} through a
 // double buffer (q fastest); the sum over the strip stays in registers, and goes
 // into A_IJ by reductions in L2 (no read of the block), one whole 256-byte row at a
 // time through a shared strip.  NW warps (4: two CTAs per SM, for strips of one row;
@@ -387,39 +387,56 @@ __global__ void __launch_bounds__(NW * 32, NW == 4 ? 2 : 1) trailing_kernel(doub
   double* const Y0 = sm + pl.nk * TB * OLD;     // two stream buffers
   double* const stage = Y0 + 2 * TB * OLD;
   auto ybuf = [&](int bsel) { return Y0 + bsel * (TB * OLD); };
-  const int cta = blockIdx.x;
-  int g;
-  {
-    int lo = 0, hi = pl.ng;  // largest g with start[g] <= cta
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (pl.start[mid] <= cta) lo = mid; else hi = mid;
-    }
-    g = lo;
-  }
-  const int I = pl.I0 + g;
-  const int first = (cta - pl.start[g]) * pl.per_cta;
-  const int last = min(first + pl.per_cta, I + 1);
-  if (first >= last) return;
+  const long long total = (long long)pl.rows * (pl.rows + 1) / 2;
+  const long long p0 = (long long)blockIdx.x * pl.per_cta;
+  const long long p1 = min(p0 + pl.per_cta, total);
+  if (p0 >= p1) return;
   const int nk = pl.nk;
   auto rows_of = [&](int q) { return min(TB, k - (pl.k0 + q) * TB); };  // only the last block row is ragged
-
-  for (int q = 0; q < nk; ++q)
-    load_block<V16, NT>(Xs + q * (TB * OLD), M, ldm, (pl.k0 + q) * TB, I * TB, rows_of(q), TB);
-  load_block<V16, NT>(ybuf(0), M, ldm, pl.k0 * TB, first * TB, rows_of(0), TB);
+  // (I, J) of the first pair: row I holds pairs I (I + 1) / 2 .. I (I + 1) / 2 + I
+  int I = (int)((sqrt(8.0 * (double)p0 + 1.0) - 1.0) * 0.5);
+  while ((long long)(I + 1) * (I + 2) / 2 <= p0) ++I;
+  while ((long long)I * (I + 1) / 2 > p0) --I;
+  int J = (int)(p0 - (long long)I * (I + 1) / 2);
+  auto load_x = [&](int col) {
+    for (int q = 0; q < nk; ++q)
+      load_block<V16, NT>(Xs + q * (TB * OLD), M, ldm, (pl.k0 + q) * TB, col * TB, rows_of(q), TB);
+  };
+  load_x(I);
+  load_block<V16, NT>(ybuf(0), M, ldm, pl.k0 * TB, J * TB, rows_of(0), TB);
   cp_async_commit_group();
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int wr = (warp >> 1) * (8 * RF), wc = (warp & 1) * 32;
-  const int nsteps = (last - first) * nk;
+  const long long nsteps = (p1 - p0) * nk;
   double acc[RF][4][2] = {};
-  for (int step = 0; step < nsteps; ++step) {
-    const int J = first + step / nk, q = step % nk;
-    const int bsel = step & 1;
+  int Jn = J, In = I;  // the pair of the next step's block
+  for (long long step = 0; step < nsteps; ++step) {
+    const int q = (int)(step % nk);
+    if (q == 0 && step > 0) {
+      // next pair; entering a new row reloads the strip's blocks of column I (every
+      // warp finished with the old ones at the end of the previous step)
+      const int Iprev = I;
+      I = In;
+      J = Jn;
+      if (I != Iprev) {
+        load_x(I);
+        cp_async_commit_group();
+      }
+    }
+    const int bsel = (int)(step & 1);
     if (step + 1 < nsteps) {
-      const int J1 = first + (step + 1) / nk, q1 = (step + 1) % nk;
-      load_block<V16, NT>(ybuf(bsel ^ 1), M, ldm, (pl.k0 + q1) * TB, J1 * TB, rows_of(q1), TB);
+      const int q1 = (int)((step + 1) % nk);
+      if (q1 == 0) {  // the following pair
+        Jn = J + 1;
+        In = I;
+        if (Jn > In) {
+          ++In;
+          Jn = 0;
+        }
+      }
+      load_block<V16, NT>(ybuf(bsel ^ 1), M, ldm, (pl.k0 + q1) * TB, (q1 == 0 ? Jn : J) * TB, rows_of(q1), TB);
       cp_async_commit_group();
       cp_async_wait_group<1>();
     } else {
@@ -537,29 +554,20 @@ int enqueue_step(const FactorJob& f, int K, int sms) {
   ok = ok && cudaEventRecord(f.panel_done[sidx % RING], f.ps) == cudaSuccess &&
        cudaStreamWaitEvent(f.us, f.panel_done[sidx % RING], 0) == cudaSuccess;
   const long long total = (long long)rows * (rows + 1) / 2;
-  const int target = 2 * sms;
-  const int per_cta = (int)std::max<long long>(1, (total + target - 1) / target);
   const int nk = hi_s - lo_s + 1;
   const bool wide = nk > 1;  // 8 warps, one CTA per SM; else 4 warps, two per SM
   const int smem = tr_smem(nk, wide ? 8 : 4);
-  for (int g0 = 0; g0 < rows && ok; g0 += MAX_TR_GROUPS) {
-    TrailPlan pl;
-    pl.k0 = lo_s;
-    pl.nk = hi_s - lo_s + 1;
-    pl.I0 = g0;
-    pl.ng = std::min(rows - g0, MAX_TR_GROUPS);
-    pl.per_cta = per_cta;
-    int ctas = 0;
-    for (int gi = 0; gi < pl.ng; ++gi) {
-      pl.start[gi] = ctas;
-      ctas += (g0 + gi + 1 + per_cta - 1) / per_cta;
-    }
-    pl.start[pl.ng] = ctas;
-    auto kern = f.v16 ? (wide ? trailing_kernel<true, 8> : trailing_kernel<true, 4>)
-                      : (wide ? trailing_kernel<false, 8> : trailing_kernel<false, 4>);
-    GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
-                  kern<<<ctas, wide ? 256 : 128, smem, f.us>>>(f.M, f.ldm, f.k, f.info, pl));
-  }
+  const int target = (wide ? 1 : 2) * sms;  // one wave of CTAs
+  TrailPlan pl;
+  pl.k0 = lo_s;
+  pl.nk = nk;
+  pl.rows = rows;
+  pl.per_cta = (int)std::max<long long>(1, (total + target - 1) / target);
+  const int ctas = (int)((total + pl.per_cta - 1) / pl.per_cta);
+  auto kern = f.v16 ? (wide ? trailing_kernel<true, 8> : trailing_kernel<true, 4>)
+                    : (wide ? trailing_kernel<false, 8> : trailing_kernel<false, 4>);
+  GPTQ2D_LAUNCH(KC_PREP_TRAILING, f.us,
+                kern<<<ctas, wide ? 256 : 128, smem, f.us>>>(f.M, f.ldm, f.k, f.info, pl));
   ok = ok && cudaEventRecord(f.rest_done[sidx % RING], f.us) == cudaSuccess;
   return ok && cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
