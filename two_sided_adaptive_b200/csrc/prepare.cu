@@ -205,9 +205,14 @@ __device__ __forceinline__ void rank8_block(double* C, const double* S, const do
   dst[1] -= c1;
 }
 
-// One launch per block row K.  CTA K factors the diagonal block and writes it;
-// CTAs b < K factor the same block redundantly (cheaper than a separate launch)
-// and solve their block M_Kb = M_KK^{-T} A_Kb.  Each CTA first applies, left-
+// One launch per block row K.  CTA K factors the diagonal block; CTAs b < K
+// factor the same block redundantly (cheaper than a separate launch) and solve
+// their block M_Kb = M_KK^{-T} A_Kb.  Those CTAs read A_KK from M, and the order in
+// which the CTAs of a launch are dispatched is not fixed, so CTA K must not
+// overwrite A_KK in this launch: it leaves M_KK in the block above the diagonal,
+// (K-1, K), which is zero and read by no step of the factorization, and CTA K-1 of
+// the next launch moves it to (K, K) and zeroes (K-1, K) again.  The last launch
+// (K = 0) has one CTA and writes its block in place.  Each CTA first applies, left-
 // looking, the updates of the factored block rows j = K+1 .. whi (the window that
 // the trailing updates have not applied) to the blocks it reads:
 // A_KK -= M_jK^T M_jK and A_Kb -= M_jK^T M_jb, streaming the window's blocks
@@ -237,6 +242,19 @@ __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict
   const int rb = K * TB, nb = min(TB, k - rb);
   const int b = blockIdx.x;
   if (tid == 0) bad = -1;
+  if (b == K && rb + TB < k) {
+    // the previous launch's diagonal factor, from (K, K + 1) to (K + 1, K + 1);
+    // no CTA of this launch reads either block
+    const int r1 = rb + TB, n1 = min(TB, k - r1);
+    for (int e = tid; e < n1 * TB; e += PANEL_THREADS) {
+      const int r = e >> 6, c = e & 63;
+      if (c < n1) {
+        double* src = M + (int64_t)(rb + r) * ldm + r1 + c;
+        M[(int64_t)(r1 + r) * ldm + r1 + c] = *src;
+        *src = 0.0;
+      }
+    }
+  }
   auto load_row = [&](int j, int st) {  // window row j (only the last block row is ragged)
     const int rj = j * TB, nj = min(TB, k - rj);
     load_block<V16, PANEL_THREADS>(mn(st), M, ldm, rj, rb, nj, nb);
@@ -327,10 +345,11 @@ __global__ void __launch_bounds__(PANEL_THREADS) panel_kernel(double* __restrict
     if (c > r) Ad[r * OLD + c] = 0.0;
   }
   __syncthreads();
-  if (b == K) {
+  if (b == K) {  // in place for K = 0, else parked in (K - 1, K)
+    const int r0 = K > 0 ? rb - TB : rb;
     for (int e = tid; e < nb * TB; e += PANEL_THREADS) {
       const int r = e >> 6, c = e & 63;
-      if (c < nb) M[(int64_t)(rb + r) * ldm + rb + c] = Ad[r * OLD + c];
+      if (c < nb) M[(int64_t)(r0 + r) * ldm + rb + c] = Ad[r * OLD + c];
     }
     return;
   }
