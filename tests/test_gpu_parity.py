@@ -373,6 +373,65 @@ def test_mlp_layer_4096x14336_int3(g):
     assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
 
 
+def _device_t4_gram(width, gen):
+    """The 70B-block Gram recipe on the GPU (input generation only): width rows of
+    Student-t(4) activations times U(0.1, 10) column scales, X^T X / width in fp64, 1%
+    mean-diagonal damping, stored fp32.  Rows are drawn in chunks to bound memory."""
+    G = torch.zeros(width, width, dtype=torch.float64, device="cuda")
+    c = torch.empty(width, dtype=torch.float64, device="cuda").uniform_(0.1, 10.0, generator=gen)
+    for r0 in range(0, width, 4096):
+        rows = min(4096, width - r0)
+        z = torch.randn(rows, width, dtype=torch.float64, device="cuda", generator=gen)
+        chi2 = torch.randn(4, rows, width, dtype=torch.float64, device="cuda",
+                           generator=gen).square_().sum(0)
+        X = z / torch.sqrt(chi2 / 4.0) * c
+        del z, chi2
+        G.addmm_(X.T, X)
+        del X
+    G /= width
+    G = 0.5 * (G + G.T)
+    G.diagonal().add_(0.01 * G.diagonal().mean())
+    return G.float()
+
+
+@pytest.mark.slow
+def test_block70b_gate_layer_8192x28672(g):
+    """The largest shape of the 70B block (gate/up: 8192 x 28672, INT4 per-row absmax, bf16
+    W ~ N(0, 0.015^2)), where a factor passes 2^31 bytes: factor rows against LAPACK, the
+    leading prefix against the oracle, sampled entries against the definition, and the
+    in-kernel loss against the direct trace.  The oracle factors its own copies of the
+    Grams on the host."""
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    m, n = 8192, 28672
+    HL, HR = _device_t4_gram(m, gen), _device_t4_gram(n, gen)
+    W = (torch.randn(m, n, device="cuda", generator=gen) * 0.015).to(torch.bfloat16)
+    W64 = W.double().cpu().numpy()
+    s = torch.from_numpy(WL.absmax_scales(W64, 4)).cuda()
+    ML, MR = g.prepare_pair(HL, HR)
+    Q, st = g.quantize(W, ML, MR, s, 4, True)
+    Qg, st = Q.cpu().numpy(), g.stats_dict(st)
+    assert st["status"] == 0 and st["n_nonfinite"] == 0
+    HLh, HRh = HL.double().cpu().numpy(), HR.double().cpu().numpy()
+    del HL, HR, Q
+    MLo, MRo = O.reverse_cholesky(HLh), O.reverse_cholesky(HRh)
+    for M, Mo, rows in ((ML, MLo, [0, 1, 2, 4095, 8189, 8190, 8191]),
+                        (MR, MRo, [0, 1, 2, 14335, 28669, 28670, 28671])):
+        np.testing.assert_allclose(M[rows].cpu().numpy(), Mo[rows], rtol=1e-8,
+                                   atol=1e-10 * np.abs(Mo).max())
+    del ML, MR
+    s64 = s.double().cpu().numpy()
+    k, l = 320, 384
+    check_against_oracle(W64[:k, :l], MLo[:k, :k], MRo[:l, :l], s64[:k], 4, True, Qg[:k, :l])
+    rng = np.random.default_rng(5)
+    lo, hi = O.grid_bounds(4, True)
+    for i, j in zip(rng.integers(0, m, 8), rng.integers(0, n, 8)):
+        t = O.entry_value(W64, Qg, s64, MLo, MRo, int(i), int(j)) / s64[i]
+        if not O.near_tie(np.array([t]), lo, hi)[0]:
+            assert Qg[i, j] == O.round_to_grid(t, lo, hi), (i, j, t)
+    direct = O.proxy_loss(W64, Qg, s64, HLh, HRh)
+    assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
+
+
 # --------------------------------------------------------------------------- #
 # both factors in one call
 # --------------------------------------------------------------------------- #
