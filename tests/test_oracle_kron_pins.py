@@ -125,3 +125,28 @@ def test_loss_identity_and_bound(clamp):
         for j, M in enumerate(Ms):
             d2 = d2 * np.diag(M)[idx[j]] ** 2
         assert r.loss_identity <= 0.25 * float(np.sum(d2 * s[idx[0]] ** 2)) * (1 + 1e-12)
+
+
+def test_mode_product_on_a_matrix_is_left_and_right_multiplication():
+    """On a matrix, the mode-0 product is A X and the mode-1 product is X B^T."""
+    rng = np.random.default_rng(7)
+    X, A, B = rng.normal(size=(3, 5)), rng.normal(size=(3, 3)), rng.normal(size=(5, 5))
+    np.testing.assert_allclose(O.mode_product(X, A, 0), A @ X, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(O.mode_product(X, B, 1), X @ B.T, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("shape", [(3, 4), (2, 3, 4), (2, 2, 3, 2)])
+def test_mode_products_are_the_kronecker_matrix_on_the_flattening(shape):
+    """Applying M_j along every mode j is M_1 kron ... kron M_k acting on the C-order
+    flattening (mode 1 slowest), the identity behind the separable feedback; checked
+    against numpy's Kronecker product of the explicit matrices."""
+    rng = np.random.default_rng(sum(shape) + len(shape))
+    X = rng.normal(size=shape)
+    Ms = [rng.normal(size=(d, d)) for d in shape]
+    Y = X
+    for j, M in enumerate(Ms):
+        Y = O.mode_product(Y, M, j)
+    K = Ms[0]
+    for M in Ms[1:]:
+        K = np.kron(K, M)
+    np.testing.assert_allclose(Y.reshape(-1), K @ X.reshape(-1), rtol=1e-12, atol=1e-12)

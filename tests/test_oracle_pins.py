@@ -342,3 +342,30 @@ def test_near_tie_detection_and_flip():
     assert alt.Q[0, 0] == 0
     with pytest.raises(ValueError):
         O.gptq2d(W, H, H, np.ones(2), 4, False, flip={(1, 1)})
+
+
+# --------------------------------------------------------------------------- #
+# the rounding step along one coordinate
+# --------------------------------------------------------------------------- #
+def test_round_to_grid_ties_go_to_even():
+    """IEEE round-half-to-even at exact ties (the reading of the tie rule), with no clamp."""
+    t = np.array([0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5, -3.5])
+    np.testing.assert_array_equal(O.round_to_grid(t, -np.inf, np.inf),
+                                  [0.0, 2.0, 2.0, 0.0, -2.0, -2.0, 4.0, -4.0])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_round_to_grid_is_the_nearest_admissible_integer(bits):
+    """Brute force over the admissible integers: clamp(rint(t)) is the nearest one
+    (GPTQ's rounding along one coordinate), for values inside, at and past the range."""
+    lo, hi = O.grid_bounds(bits, True)
+    rng = np.random.default_rng(bits)
+    t = np.concatenate([rng.uniform(lo - 3, hi + 3, 400), [lo - 0.5, hi + 0.5, lo, hi]])
+    q = O.round_to_grid(t, lo, hi)
+    grid = np.arange(lo, hi + 1)
+    for tv, qv in zip(t, q):
+        dist = np.abs(grid - tv)
+        best = grid[dist == dist.min()]
+        # a tie inside the range has two nearest points; the rule picks the even one
+        expect = best[0] if len(best) == 1 else best[best % 2 == 0][0]
+        assert qv == expect, (tv, qv, best)
