@@ -17,7 +17,7 @@ What it computes (sources are the two on-topic pages):
     one anti-diagonal rounded in parallel) and Analysis > Results / Methodology
     (exact 1-D GPTQ trajectory; rank-one separable feedback kept in a buffer).
 
-Conventions (readings where the pages are silent; each is listed in the design doc):
+Conventions (readings where the pages are silent):
   * W is m x n.  H_L (m x m) acts on the row index i, H_R (n x n) on the column
     index j.  Proxy loss  L(Q) = tr(dW^T H_L dW H_R),  dW = W - diag(s) Q, which
     is vec(dW)^T (H_R kron H_L) vec(dW) with column-major vec.
@@ -32,7 +32,9 @@ Functions, from most literal to fastest:
   O1  babai_kron_sweep              1-D GPTQ sweep over vec(W) on the mn x mn Gram
   O2  gptq2d_antidiagonal           the cubic anti-diagonal algorithm
 and the special cases used as pins: RTN, 1-D GPTQ in OBS form, exhaustive
-closest-vector search on tiny problems.
+closest-vector search on tiny problems.  For checking large candidate outputs
+entry by entry: entry_value (one entry) and entry_values_all (every entry, from
+the candidate's own integers, by two matrix products).
 
 Grid variants (the pages fix only a 4-bit integer grid; these are GPTQ's usual
 ones): expand_grid turns group-wise scales and integer zero points into a
@@ -363,6 +365,38 @@ def entry_value(W, Q, s, M_L, M_R, i, j):
     D[i, j] = 0.0
     fb = np.asarray(M_L[i, : i + 1], np.float64) @ D @ np.asarray(M_R[j, : j + 1], np.float64)
     return W[i, j] + fb / (float(M_L[i, i]) * float(M_R[j, j]))
+
+
+def entry_values_all(W, Q, s, M_L, M_R, rows=None):
+    """y_ij of every entry (of rows r0..r1-1 when ``rows`` = (r0, r1)), each from its
+    definition, given a candidate's integers Q everywhere.
+
+    With D = W - S Q and d_ij = M_L[i,i] M_R[j,j], the feedback sum of entry (i, j)
+    over its dominated quadrant minus (i, j) itself is (M_L D M_R^T)_ij - d_ij D_ij:
+    M_L and M_R are lower triangular, so the product only reaches i' <= i and
+    j' <= j (arxivlens, Analysis > Results: row (i, j) of the Kronecker triangular
+    factor applied to the errors).  Hence
+        y = W + (M_L D M_R^T - d * D) / d
+    for all entries at once: two matrix products.  This is entry_value for every
+    (i, j); for rows r0..r1-1 only M_L[r0:r1, :r1] and D[:r1] are needed.
+
+    A candidate Q is the trajectory of the sweep (up to the near-tie choices) iff
+    every entry satisfies q_ij = clamp(rint(y_ij / s_ij)) with y from Q itself:
+    y_ij depends only on entries rounded before (i, j), so the first entry, in any
+    linear extension of the product order, that breaks the equality is where Q
+    leaves the trajectory.
+    """
+    W = np.asarray(W, np.float64)
+    s = np.asarray(s, np.float64)
+    m, n = W.shape
+    r0, r1 = (0, m) if rows is None else (int(rows[0]), int(rows[1]))
+    S = s if s.ndim == 2 else np.broadcast_to(s[:, None], (m, n))
+    D = W[:r1] - S[:r1] * np.asarray(Q[:r1], np.float64)
+    ML = np.asarray(M_L, np.float64)
+    MR = np.asarray(M_R, np.float64)
+    F = (ML[r0:r1, :r1] @ D) @ MR.T
+    d = np.diag(ML)[r0:r1, None] * np.diag(MR)[None, :]
+    return W[r0:r1] + (F - d * D[r0:r1]) / d
 
 
 # --------------------------------------------------------------------------- #

@@ -285,6 +285,69 @@ def test_entry_value_matches_sweep():
         assert O.entry_value(W, r.Q, s, ML, MR, i, j) / s[i] == pytest.approx(r.T[i, j], abs=1e-12)
 
 
+def _kron_feedback_values(W, Q, S, ML, MR):
+    """y of every entry through the explicit Kronecker factor: with column-major vec,
+    M = M_R kron M_L is lower triangular and row p of M vec(D), minus its diagonal
+    term, divided by M[p, p], is the feedback of coordinate p (an independent route)."""
+    m, n = W.shape
+    D = (W - S * Q).flatten(order="F")
+    M = np.kron(MR, ML)
+    fb = M @ D - np.diag(M) * D
+    return W + (fb / np.diag(M)).reshape((m, n), order="F")
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (1, 7), (6, 1), (5, 9), (11, 4), (13, 13)])
+def test_entry_values_all_is_the_definition(shape):
+    """entry_values_all equals, for any integers Q (not only a trajectory), entry_value
+    at every entry and the explicit mn x mn Kronecker factor's rows; per-row scales and
+    per-entry grid steps; a row band equals the same rows of the whole."""
+    m, n = shape
+    rng = np.random.default_rng(m * 100 + n)
+    W = rng.normal(0, 0.5, (m, n))
+    ML, MR = O.reverse_cholesky(_heavy_spd(rng, m)), O.reverse_cholesky(_heavy_spd(rng, n))
+    Q = rng.integers(-8, 8, (m, n)).astype(float)
+    for s in (rng.uniform(0.1, 1.0, m), rng.uniform(0.1, 1.0, (m, n))):
+        Y = O.entry_values_all(W, Q, s, ML, MR)
+        S = s if s.ndim == 2 else np.broadcast_to(s[:, None], (m, n))
+        np.testing.assert_allclose(Y, _kron_feedback_values(W, Q, S, ML, MR), rtol=1e-12,
+                                   atol=1e-12)
+        for i in range(m):
+            for j in range(n):
+                assert Y[i, j] == pytest.approx(O.entry_value(W, Q, s, ML, MR, i, j), abs=1e-12)
+        r0, r1 = m // 3, max(m // 3 + 1, (2 * m) // 3)
+        np.testing.assert_allclose(O.entry_values_all(W, Q, s, ML, MR, rows=(r0, r1)), Y[r0:r1],
+                                   rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("clamp", [True, False])
+def test_entry_values_all_fixed_point_characterises_the_trajectory(clamp):
+    """On the sweep's own Q, y / s from entry_values_all is the sweep's T, and every
+    entry rounds to itself; the naive Kronecker sweep's Q (another route) is a fixed
+    point too; changing one integer of the trajectory breaks the fixed point exactly
+    there (y_ij does not depend on q_ij)."""
+    rng = np.random.default_rng(41 + clamp)
+    m, n = 12, 10
+    W = rng.normal(0, 0.05, (m, n))
+    H_L, H_R = _heavy_spd(rng, m), _heavy_spd(rng, n)
+    s = WL.absmax_scales(W, 4).astype(np.float64) * (1.0 if clamp else 0.3)
+    ML, MR = O.reverse_cholesky(H_L), O.reverse_cholesky(H_R)
+    lo, hi = O.grid_bounds(4, clamp)
+    r = O.gptq2d_antidiagonal(W, ML, MR, s, 4, clamp)
+    T = O.entry_values_all(W, r.Q, s, ML, MR) / s[:, None]
+    np.testing.assert_allclose(T, r.T, rtol=0, atol=1e-11)
+    np.testing.assert_array_equal(O.round_to_grid(T, lo, hi), r.Q)
+    Q1, _ = O.babai_kron_sweep(W, H_L, H_R, s, 4, clamp)
+    np.testing.assert_array_equal(
+        O.round_to_grid(O.entry_values_all(W, Q1, s, ML, MR) / s[:, None], lo, hi), Q1)
+    for i, j in ((0, 0), (5, 3), (11, 9)):
+        Qb = r.Q.copy()
+        Qb[i, j] += 1.0 if Qb[i, j] < hi else -1.0
+        bad = O.round_to_grid(O.entry_values_all(W, Qb, s, ML, MR) / s[:, None], lo, hi) != Qb
+        assert bad[i, j]
+        # nothing before (i, j) in the product order is disturbed
+        assert not bad[: i + 1, : j + 1].ravel()[:-1].any()
+
+
 # --------------------------------------------------------------------------- #
 # brute force
 # --------------------------------------------------------------------------- #
@@ -369,3 +432,23 @@ def test_round_to_grid_is_the_nearest_admissible_integer(bits):
         # a tie inside the range has two nearest points; the rule picks the even one
         expect = best[0] if len(best) == 1 else best[best % 2 == 0][0]
         assert qv == expect, (tv, qv, best)
+
+
+def test_fixed_point_checker_accepts_the_trajectory_and_rejects_a_wrong_entry():
+    """The every-entry check of the full-size GPU tests: it passes the oracle's own
+    trajectory in row chunks of any size and fails a single wrong integer."""
+    from tests.parity import check_fixed_point
+    rng = np.random.default_rng(77)
+    m, n = 37, 29
+    W = rng.normal(0, 0.05, (m, n))
+    ML = O.reverse_cholesky(_heavy_spd(rng, m))
+    MR = O.reverse_cholesky(_heavy_spd(rng, n))
+    s = WL.absmax_scales(W, 4).astype(np.float64)
+    r = O.gptq2d_antidiagonal(W, ML, MR, s, 4, True)
+    for chunk in (1, 8, 64):
+        rep = check_fixed_point(W, ML, MR, s, 4, True, r.Q, row_chunk=chunk)
+        assert rep.n_entries == m * n and rep.n_other_neighbour == 0
+    Qb = r.Q.copy()
+    Qb[30, 20] = Qb[30, 20] - 1 if Qb[30, 20] > -8 else Qb[30, 20] + 1
+    with pytest.raises(AssertionError, match=r"\(30,20\)"):
+        check_fixed_point(W, ML, MR, s, 4, True, Qb, row_chunk=8)
