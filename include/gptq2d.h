@@ -51,7 +51,9 @@ typedef enum {
   GPTQ2D_ERR_NONFINITE = 3,   /* NaN/Inf in W or a scale <= 0 / non-finite (reported in stats) */
   GPTQ2D_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
   GPTQ2D_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
-  GPTQ2D_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed */
+  GPTQ2D_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
+  GPTQ2D_ERR_RANGE = 7        /* an unclamped integer does not fit its output byte (reported in
+                                 stats; the byte holds the integer saturated to [-128, 127]) */
 } gptq2d_status;
 
 typedef enum {
@@ -70,7 +72,11 @@ typedef struct {
   int64_t n_near_tie;  /* entries whose y/s lies within 1e-6 of a boundary k + 1/2
                           between two admissible integers */
   int64_t n_nonfinite; /* entries with non-finite W or y, or rows with an invalid scale */
-  int64_t status;      /* GPTQ2D_OK, or GPTQ2D_ERR_NONFINITE if n_nonfinite > 0 */
+  int64_t status;      /* GPTQ2D_OK; else, in this order of precedence, GPTQ2D_ERR_TIMEOUT
+                          (a bounded device wait gave up), GPTQ2D_ERR_NONFINITE
+                          (n_nonfinite > 0), GPTQ2D_ERR_RANGE (n_out_of_range > 0) */
+  int64_t n_out_of_range; /* clamp = 0 only: entries whose integer lies outside [-128, 127]
+                             and so does not fit its int8 byte; the byte is saturated */
 } gptq2d_stats;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -259,7 +265,10 @@ size_t gptq2d_quantize_workspace_size(int64_t m, int64_t n);
  *   M_R, ldr        : device fp64, n x n lower factor of H_R (upper triangle ignored).
  *   scales          : device fp32 [m], grid step of each row; must be finite and > 0.
  *   bits, clamp     : grid [-2^(bits-1), 2^(bits-1)-1] when clamp = 1 (2 <= bits <= 8);
- *                     clamp = 0 rounds to any integer (results must fit int8).
+ *                     clamp = 0 rounds to any integer; an integer outside [-128, 127]
+ *                     is stored saturated, counted in stats->n_out_of_range and
+ *                     reported as GPTQ2D_ERR_RANGE in stats->status (the rounding
+ *                     itself, and every later entry, use the true integer).
  *   Q, ldq          : device int8 output, m x n.
  *   stats           : device pointer to one gptq2d_stats, written at the end.
  *   ws, ws_bytes    : device workspace, >= gptq2d_quantize_workspace_size(m, n).

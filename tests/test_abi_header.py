@@ -22,13 +22,15 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "gptq2d.h")
 
 STRUCTS = {
-    "gptq2d_stats": ["proxy_loss", "n_clamped", "n_near_tie", "n_nonfinite", "status"],
+    "gptq2d_stats": ["proxy_loss", "n_clamped", "n_near_tie", "n_nonfinite", "status",
+                     "n_out_of_range"],
     "gptq2d_grid": ["bits", "clamp", "group_size", "scales", "ld_scales", "zeros", "packed"],
     "gptq2d_layer": ["W", "w_dtype", "m", "n", "ldw", "H_L", "ldhl", "H_R", "ldhr", "h_dtype",
                      "grid", "Q", "ldq", "stats"],
 }
 CONSTANTS = ["GPTQ2D_OK", "GPTQ2D_ERR_INVALID_ARG", "GPTQ2D_ERR_NOT_SPD", "GPTQ2D_ERR_NONFINITE",
-             "GPTQ2D_ERR_WORKSPACE", "GPTQ2D_ERR_TIMEOUT", "GPTQ2D_ERR_CUDA", "GPTQ2D_F32",
+             "GPTQ2D_ERR_WORKSPACE", "GPTQ2D_ERR_TIMEOUT", "GPTQ2D_ERR_CUDA", "GPTQ2D_ERR_RANGE",
+             "GPTQ2D_F32",
              "GPTQ2D_BF16", "GPTQ2D_F64", "GPTQ2D_MAX_KRON_FACTORS"]
 
 
@@ -78,14 +80,15 @@ def test_struct_layouts_match_the_header(header_facts, g):
     for k, f in enumerate(STRUCTS["gptq2d_stats"]):
         assert header_facts[f"gptq2d_stats.{f}"] == 8 * k, f
     words = [0] * g.STATS_WORDS
-    words[1:] = [11, 22, 33, 44]
+    words[1:] = [11, 22, 33, 44, 55]
     assert list(g.stats_dict(words).keys())[1:] == ["n_clamped", "n_near_tie", "n_nonfinite",
-                                                    "status"]
-    assert [g.stats_dict(words)[k] for k in STRUCTS["gptq2d_stats"][1:]] == [11, 22, 33, 44]
+                                                    "status", "n_out_of_range"]
+    assert [g.stats_dict(words)[k] for k in STRUCTS["gptq2d_stats"][1:]] == [11, 22, 33, 44, 55]
 
 
 def test_constants_match_the_header(header_facts, g):
-    for name in ("OK", "INVALID_ARG", "NOT_SPD", "NONFINITE", "WORKSPACE", "TIMEOUT", "CUDA"):
+    for name in ("OK", "INVALID_ARG", "NOT_SPD", "NONFINITE", "WORKSPACE", "TIMEOUT", "CUDA",
+                 "RANGE"):
         key = "GPTQ2D_OK" if name == "OK" else f"GPTQ2D_ERR_{name}"
         assert getattr(g.Status, name) == header_facts[key], name
     assert (g.DTYPE_F32, g.DTYPE_BF16, g.DTYPE_F64) == (

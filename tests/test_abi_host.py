@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for code in range(0, 7):
+    for code in range(0, 8):
         assert L.gptq2d_status_string(code).startswith(b"GPTQ2D_")
     assert b"unknown" in L.gptq2d_status_string(99)
 

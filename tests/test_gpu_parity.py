@@ -15,7 +15,7 @@ import pytest
 
 import oracle as O
 import workloads as WL
-from tests.parity import check_against_oracle
+from tests.parity import check_against_oracle, check_fixed_point
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -301,7 +301,7 @@ def test_round_host_reports_non_spd(g):
 
 # --------------------------------------------------------------------------- #
 # full size: the 4096 x 4096 attention projection in the benchmark's launch
-# configuration (prefix property, sampled entries, loss identity)
+# configuration (prefix property, every entry against its definition, loss identity)
 # --------------------------------------------------------------------------- #
 def _gpu_gram(X):
     Xt = torch.from_numpy(X).cuda()
@@ -327,14 +327,10 @@ def test_attention_layer_4096(g):
     k, l = 384, 320
     check_against_oracle(W64[:k, :l], MLo[:k, :k], MRo[:l, :l], s64[:k], pb.bits, pb.clamp,
                          Qg[:k, :l])
-    # sampled entries anywhere: q_ij must be the rounding of y_ij computed from the GPU's own
-    # dominated quadrant (a fixed point that, over all entries, characterises the output)
-    rng = np.random.default_rng(0)
-    lo, hi = O.grid_bounds(pb.bits, pb.clamp)
-    for i, j in zip(rng.integers(0, m, 24), rng.integers(0, n, 24)):
-        t = O.entry_value(W64, Qg, s64, MLo, MRo, int(i), int(j)) / s64[i]
-        if not O.near_tie(np.array([t]), lo, hi)[0]:
-            assert Qg[i, j] == O.round_to_grid(t, lo, hi), (i, j, t)
+    # every entry: q_ij must be the rounding of y_ij computed from the GPU's own integers
+    rep = check_fixed_point(W64, MLo, MRo, s64, pb.bits, pb.clamp, Qg)
+    print(f"attn 4096^2: {rep.n_entries} entries checked, near-ties {rep.n_near_tie} "
+          f"(GPU counted {st['n_near_tie']}), other neighbour taken at {rep.n_other_neighbour}")
     # loss: in-kernel identity against the direct trace
     direct = O.proxy_loss(W64, Qg, s64, pb.H_L, pb.H_R)
     assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
@@ -343,11 +339,12 @@ def test_attention_layer_4096(g):
 
 
 @pytest.mark.slow
-def test_mlp_layer_4096x14336_int3(g):
-    """The rectangular MLP shape (m = 4096 < n = 14336) on the INT3 grid: factor rows
-    against LAPACK, the leading prefix against the oracle, sampled entries against the
-    definition, and the in-kernel loss against the direct trace."""
-    pb = WL.mlp(0, bits=3, matmul=_gpu_gram)
+@pytest.mark.parametrize("bits", [4, 3], ids=["int4", "int3"])
+def test_mlp_layer_4096x14336(g, bits):
+    """The rectangular MLP shape (m = 4096 < n = 14336) on the INT4 and INT3 grids:
+    factor rows against LAPACK, the leading prefix against the oracle, every entry
+    against its definition, and the in-kernel loss against the direct trace."""
+    pb = WL.mlp(0, bits=bits, matmul=_gpu_gram)
     m, n = pb.shape
     ML, MR = g.prepare_pair(dev(pb.H_L), dev(pb.H_R))
     Q, st = g.quantize(dev(pb.W).to(torch.bfloat16), ML, MR, dev(pb.scales), pb.bits, pb.clamp)
@@ -363,12 +360,10 @@ def test_mlp_layer_4096x14336_int3(g):
     k, l = 320, 384
     check_against_oracle(W64[:k, :l], MLo[:k, :k], MRo[:l, :l], s64[:k], pb.bits, pb.clamp,
                          Qg[:k, :l])
-    rng = np.random.default_rng(1)
-    lo, hi = O.grid_bounds(pb.bits, pb.clamp)
-    for i, j in zip(rng.integers(0, m, 16), rng.integers(0, n, 16)):
-        t = O.entry_value(W64, Qg, s64, MLo, MRo, int(i), int(j)) / s64[i]
-        if not O.near_tie(np.array([t]), lo, hi)[0]:
-            assert Qg[i, j] == O.round_to_grid(t, lo, hi), (i, j, t)
+    rep = check_fixed_point(W64, MLo, MRo, s64, pb.bits, pb.clamp, Qg)
+    print(f"mlp 4096x14336 int{bits}: {rep.n_entries} entries checked, near-ties "
+          f"{rep.n_near_tie} (GPU counted {st['n_near_tie']}), other neighbour taken at "
+          f"{rep.n_other_neighbour}")
     direct = O.proxy_loss(W64, Qg, s64, pb.H_L, pb.H_R)
     assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
 
@@ -398,7 +393,7 @@ def _device_t4_gram(width, gen):
 def test_block70b_gate_layer_8192x28672(g):
     """The largest shape of the 70B block (gate/up: 8192 x 28672, INT4 per-row absmax, bf16
     W ~ N(0, 0.015^2)), where a factor passes 2^31 bytes: factor rows against LAPACK, the
-    leading prefix against the oracle, sampled entries against the definition, and the
+    leading prefix against the oracle, every entry against its definition, and the
     in-kernel loss against the direct trace.  The oracle factors its own copies of the
     Grams on the host."""
     gen = torch.Generator(device="cuda").manual_seed(5)
@@ -422,12 +417,10 @@ def test_block70b_gate_layer_8192x28672(g):
     s64 = s.double().cpu().numpy()
     k, l = 320, 384
     check_against_oracle(W64[:k, :l], MLo[:k, :k], MRo[:l, :l], s64[:k], 4, True, Qg[:k, :l])
-    rng = np.random.default_rng(5)
-    lo, hi = O.grid_bounds(4, True)
-    for i, j in zip(rng.integers(0, m, 8), rng.integers(0, n, 8)):
-        t = O.entry_value(W64, Qg, s64, MLo, MRo, int(i), int(j)) / s64[i]
-        if not O.near_tie(np.array([t]), lo, hi)[0]:
-            assert Qg[i, j] == O.round_to_grid(t, lo, hi), (i, j, t)
+    # every entry, the 6.6 GB right factor's rows past 2^31 bytes included
+    rep = check_fixed_point(W64, MLo, MRo, s64, 4, True, Qg)
+    print(f"gate 8192x28672: {rep.n_entries} entries checked, near-ties {rep.n_near_tie} "
+          f"(GPU counted {st['n_near_tie']}), other neighbour taken at {rep.n_other_neighbour}")
     direct = O.proxy_loss(W64, Qg, s64, HLh, HRh)
     assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
 
@@ -453,6 +446,60 @@ def test_prepare_pair_reports_which_factor(g, bad_side):
         g.prepare_pair(dev(H_L), dev(H_R))
     assert ei.value.status == g.Status.NOT_SPD
     assert f"factor {bad_side} pivot 33" in str(ei.value)
+
+
+def test_unclamped_integers_beyond_int8_are_saturated_and_reported(g):
+    """clamp = 0 with a tiny scale on a few rows: integers beyond [-128, 127] are stored
+    saturated, counted and reported as GPTQ2D_ERR_RANGE; every other entry (and the
+    feedback, which uses the true integers) still matches the oracle."""
+    pb = WL.small(4, 96, 72)
+    s = pb.scales.astype(np.float64).copy()
+    s[[5, 40]] *= 1e-3
+    W64 = pb.W.astype(np.float64)
+    ML, MR = g.prepare(dev(pb.H_L)), g.prepare(dev(pb.H_R))
+    Q, st = g.quantize(dev(pb.W), ML, MR, dev(s.astype(np.float32)), 4, False)
+    Qg, st = Q.cpu().numpy().astype(np.float64), g.stats_dict(st)
+    r = O.gptq2d_antidiagonal(W64, O.reverse_cholesky(pb.H_L), O.reverse_cholesky(pb.H_R),
+                              s.astype(np.float32).astype(np.float64), 4, False)
+    big = (r.Q < -128) | (r.Q > 127)
+    assert big.sum() > 0 and st["n_out_of_range"] == int(big.sum())
+    assert st["status"] == g.Status.RANGE
+    np.testing.assert_array_equal(Qg, np.clip(r.Q, -128, 127))
+
+
+# --------------------------------------------------------------------------- #
+# pointers the device cannot dereference are rejected on the host
+# --------------------------------------------------------------------------- #
+def test_pageable_host_pointers_are_rejected_before_any_launch(g):
+    """A pageable host buffer handed to a device entry point is refused with
+    INVALID_ARG by the host-side pointer check (no kernel is launched for it); the
+    same call with device buffers then succeeds."""
+    import ctypes
+    pb = WL.small(3, 70, 90)
+    W, s = dev(pb.W), dev(pb.scales)
+    ML, MR = g.prepare(dev(pb.H_L)), g.prepare(dev(pb.H_R))
+    m, n = pb.shape
+    Q = torch.empty((m, n), dtype=torch.int8, device="cuda")
+    st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device="cuda")
+    ws = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device="cuda")
+    Wh = torch.from_numpy(np.array(pb.W, copy=True))        # pageable host memory
+    Qh = torch.empty((m, n), dtype=torch.int8)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    L = g.lib()
+
+    def call(Wp, Qp):
+        return L.gptq2d_quantize(Wp, g.DTYPE_F32, m, n, n, ML.data_ptr(), m, MR.data_ptr(), n,
+                                 s.data_ptr(), 4, 1, Qp, n, st.data_ptr(), ws.data_ptr(),
+                                 ws.numel(), stream)
+    launches = g.launch_count()
+    assert call(Wh.data_ptr(), Q.data_ptr()) == g.Status.INVALID_ARG
+    assert call(W.data_ptr(), Qh.data_ptr()) == g.Status.INVALID_ARG
+    assert g.launch_count() == launches
+    assert call(W.data_ptr(), Q.data_ptr()) == g.Status.OK
+    torch.cuda.synchronize()
+    assert g.stats_dict(st)["status"] == 0
+    with pytest.raises(ValueError):
+        g.quantize(Wh, ML, MR, s, 4, True)
 
 
 # --------------------------------------------------------------------------- #

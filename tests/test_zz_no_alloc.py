@@ -67,6 +67,38 @@ def test_noalloc_matches_workspace_entry_point(g):
                          pb.clamp, Qn.cpu().numpy())
 
 
+def test_noalloc_call_allocates_no_device_memory(g):
+    """After a first call on the device (which resolves the scratch address and loads the
+    library's kernels), further calls leave both torch's allocator and the device's free
+    memory untouched: the scratch is the static array, the outputs are the caller's."""
+    pb = WL.small(2, 200, 136)
+    W, s = _dev(pb.W), _dev(pb.scales)
+    ML, MR = g.prepare(_dev(pb.H_L)), g.prepare(_dev(pb.H_R))
+    m, n = W.shape
+    Q = torch.empty((m, n), dtype=torch.int8, device="cuda")
+    st = torch.empty((g.STATS_WORDS,), dtype=torch.int64, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
+        rc = g.lib().gptq2d_quantize_noalloc(
+            W.data_ptr(), g._dtype_code(W), m, n, W.stride(0), ML.data_ptr(), ML.stride(0),
+            MR.data_ptr(), MR.stride(0), s.data_ptr(), pb.bits, int(pb.clamp), Q.data_ptr(), n,
+            st.data_ptr(), stream)
+        assert rc == g.Status.OK, g.lib().gptq2d_status_string(rc)
+
+    call()
+    torch.cuda.synchronize()
+    Q0 = Q.clone()
+    before_torch = torch.cuda.memory_stats()["allocation.all.allocated"]
+    before_free = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_stats()["allocation.all.allocated"] == before_torch
+    assert torch.cuda.mem_get_info()[0] == before_free
+    assert torch.equal(Q, Q0)
+
+
 def test_noalloc_rejects_problems_beyond_the_static_scratch(g):
     cap = 48 << 20
     assert g.quantize_workspace_size(1024, 1024) <= cap < g.quantize_workspace_size(2048, 2048)

@@ -12,6 +12,7 @@ call fails loudly when the compiled library is missing.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import numpy as np
@@ -30,7 +31,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libgptq2d.so")
 
 DTYPE_F32, DTYPE_BF16, DTYPE_F64 = 0, 1, 2
-STATS_WORDS = 5  # gptq2d_stats: double + 4 x int64
+STATS_WORDS = 6  # gptq2d_stats: double + 5 x int64
 MAX_KRON_FACTORS = 8  # GPTQ2D_MAX_KRON_FACTORS
 
 
@@ -42,6 +43,7 @@ class Status:
     WORKSPACE = 4
     TIMEOUT = 5
     CUDA = 6
+    RANGE = 7
 
 
 class GPTQ2DError(RuntimeError):
@@ -229,15 +231,62 @@ def _ld(t) -> int:
 
 
 def _stream(stream):
+    """The stream to enqueue on: the current device's current stream, or ``stream``,
+    which must belong to the current device (the library launches on the current
+    device, and every wrapper makes its tensors' device current first)."""
     torch = _torch()
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if stream.device.index != torch.cuda.current_device():
+        raise ValueError(f"stream is on {stream.device}, the tensors on cuda:"
+                         f"{torch.cuda.current_device()}")
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _check_device(*ts):
+    """Every given tensor (None skipped) must live on the current CUDA device, which the
+    wrapper has made the tensors' own (see _device_scoped)."""
+    torch = _torch()
+    cur = torch.cuda.current_device() if torch.cuda.is_available() else None
     for t in ts:
+        if t is None:
+            continue
         if not t.is_cuda:
             raise ValueError("tensors must be on a CUDA device")
+        if t.device.index != cur:
+            raise ValueError(f"all tensors of a call must share one device: {t.device} "
+                             f"is not cuda:{cur}")
+
+
+def _first_cuda_device(objs):
+    for o in objs:
+        if hasattr(o, "is_cuda") and hasattr(o, "device"):
+            if o.is_cuda:
+                return o.device
+        elif isinstance(o, dict):
+            d = _first_cuda_device(o.values())
+            if d is not None:
+                return d
+        elif isinstance(o, (list, tuple)):
+            d = _first_cuda_device(o)
+            if d is not None:
+                return d
+    return None
+
+
+def _device_scoped(fn):
+    """Runs the wrapper with the device of its first CUDA tensor argument current, so
+    that the library's kernels, its per-device streams and its static scratch all
+    belong to the device that holds the data (a tensor on another device is then
+    rejected by _check_device instead of being dereferenced by the wrong GPU)."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kw):
+        dev = _first_cuda_device(list(args) + list(kw.values()))
+        if dev is None:
+            return fn(*args, **kw)
+        with _torch().cuda.device(dev):
+            return fn(*args, **kw)
+    return wrapper
 
 
 def _workspace(nbytes, device, workspace):
@@ -250,11 +299,12 @@ def _workspace(nbytes, device, workspace):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+@_device_scoped
 def prepare(H, *, out=None, workspace=None, stream=None, check: bool = True):
     """Lower-triangular M with M^T M = H (fp64), by gptq2d_prepare.  H: k x k fp32/fp64 on
     the GPU (lower triangle read).  ``check`` synchronizes and raises on a non-SPD H."""
     torch = _torch()
-    _check_device(H)
+    _check_device(H, out, workspace)
     k = H.shape[0]
     if H.dim() != 2 or H.shape[1] != k:
         raise ValueError("H must be square")
@@ -269,12 +319,13 @@ def prepare(H, *, out=None, workspace=None, stream=None, check: bool = True):
     return M
 
 
+@_device_scoped
 def prepare_pair(H_L, H_R, *, out_l=None, out_r=None, workspace=None, stream=None,
                  check: bool = True):
     """Both factors at once (gptq2d_prepare_pair): the two factorizations run concurrently
     on library-internal streams joined back to ``stream``.  Returns (M_L, M_R)."""
     torch = _torch()
-    _check_device(H_L, H_R)
+    _check_device(H_L, H_R, out_l, out_r, workspace)
     if H_L.dtype != H_R.dtype:
         raise ValueError("H_L and H_R must share a dtype")
     m, n = H_L.shape[0], H_R.shape[0]
@@ -293,6 +344,7 @@ def prepare_pair(H_L, H_R, *, out_l=None, out_r=None, workspace=None, stream=Non
     return ML, MR
 
 
+@_device_scoped
 def gram_accumulate(X, H, *, accumulate: bool, workspace, stream=None):
     """gptq2d_gram_accumulate: H's lower 128-block triangle (+)= X^T X for a bf16 batch X
     (rows x k on the GPU; k a multiple of 8) on the tensor cores.  ``workspace``: a device
@@ -310,6 +362,7 @@ def gram_accumulate(X, H, *, accumulate: bool, workspace, stream=None):
     return H
 
 
+@_device_scoped
 def gram_finalize(H, total_rows: int, damp: float = 0.01, *, workspace, stream=None,
                   check: bool = True):
     """gptq2d_gram_finalize: H <- H / total_rows with damp * mean(diag) added to the
@@ -324,6 +377,7 @@ def gram_finalize(H, total_rows: int, damp: float = 0.01, *, workspace, stream=N
     return H
 
 
+@_device_scoped
 def gram(batches, damp: float = 0.01, *, out=None, stream=None):
     """The damped Gram X^T X / N + damp * mean(diag) I of bf16 activation batches (each
     rows x k on the GPU), accumulated on the tensor cores.  Returns H (fp32 k x k; its
@@ -341,6 +395,7 @@ def gram(batches, damp: float = 0.01, *, out=None, stream=None):
     return gram_finalize(H, total, damp, workspace=ws, stream=stream)
 
 
+@_device_scoped
 def kron_factor(Ms, *, out=None, stream=None):
     """M_1 kron M_2 kron ... of lower fp64 factors (gptq2d_kron_factor): the reverse Cholesky
     factor of H_1 kron H_2 kron ... when M_j = prepare(H_j).  Entries where some column
@@ -348,7 +403,7 @@ def kron_factor(Ms, *, out=None, stream=None):
     torch = _torch()
     if not 1 <= len(Ms) <= MAX_KRON_FACTORS:
         raise ValueError(f"1 to {MAX_KRON_FACTORS} factors")
-    _check_device(*Ms)
+    _check_device(*Ms, out)
     for M in Ms:
         if M.dtype != torch.float64 or M.dim() != 2 or M.shape[0] != M.shape[1]:
             raise ValueError("factors must be square fp64 matrices")
@@ -365,6 +420,7 @@ def kron_factor(Ms, *, out=None, stream=None):
     return K
 
 
+@_device_scoped
 def prepare_kron(Hs, *, stream=None, check: bool = True):
     """Factors of a k-factor Kronecker Hessian H_1 kron ... kron H_k (H_j on mode j of a
     k-way tensor) for the 2-D rounding: returns (M_L, M_R) with M_L = prepare(H_1) and
@@ -375,6 +431,7 @@ def prepare_kron(Hs, *, stream=None, check: bool = True):
     return Ms[0], (Ms[1] if len(Ms) == 2 else kron_factor(Ms[1:], stream=stream))
 
 
+@_device_scoped
 def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, stream=None):
     """GPTQ-2D rounding of a k-way tensor W (m_1 x ... x m_k, C order) under
     H_1 kron ... kron H_k with per-mode-1 scales: the m_1 x (m_2 ... m_k) problem with
@@ -387,12 +444,13 @@ def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, stream=
     return Q.reshape(W.shape), st
 
 
+@_device_scoped
 def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None, stats=None,
              workspace=None, stream=None):
     """GPTQ-2D rounding by gptq2d_quantize.  Returns (Q int8 m x n, stats int64[5] on the
     device; decode with stats_dict)."""
     torch = _torch()
-    _check_device(W, M_L, M_R, scales)
+    _check_device(W, M_L, M_R, scales, out, stats, workspace)
     m, n = W.shape
     if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
         raise ValueError("scales must be a contiguous fp32 vector of length m")
@@ -410,6 +468,7 @@ def quantize(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None
     return Q, st
 
 
+@_device_scoped
 def quantize_grid(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, group_size: int = 0,
                   zeros=None, packed: bool = False, out=None, stats=None, workspace=None, stream=None):
     """GPTQ-2D rounding on a grid variant (gptq2d_quantize_grid).  ``scales``: fp32 m x groups
@@ -418,7 +477,7 @@ def quantize_grid(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, gro
     per byte (bits <= 4).  Returns (Q bytes: int8 q on the symmetric grid, uint8 codes on the
     asymmetric one, packed codes m x ceil(n/2) when packed; stats on the device)."""
     torch = _torch()
-    _check_device(W, M_L, M_R, scales)
+    _check_device(W, M_L, M_R, scales, out, stats, workspace)
     m, n = W.shape
     if scales.dtype != torch.float32:
         raise ValueError("scales must be fp32")
@@ -482,6 +541,7 @@ def block_workspace_size(specs) -> int:
     return int(lib().gptq2d_block_workspace_size(arr, len(specs)))
 
 
+@_device_scoped
 def quantize_block(specs, *, workspace=None, stream=None):
     """gptq2d_quantize_block: factors and rounds a block of layers, the factor preparation
     of the next layer overlapping the rounding of the current one.  ``specs``: dicts with
@@ -491,6 +551,8 @@ def quantize_block(specs, *, workspace=None, stream=None):
     torch = _torch()
     if not specs:
         return [], []
+    _check_device(*[sp.get(k) for sp in specs for k in ("W", "H_L", "H_R", "scales", "zeros")],
+                  workspace)
     dev_ = specs[0]["W"].device
     outs, stats = [], []
     for sp in specs:
@@ -512,13 +574,14 @@ def quantize_block(specs, *, workspace=None, stream=None):
     return outs, stats
 
 
+@_device_scoped
 def quantize_noalloc(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, out=None,
                      stats=None, stream=None):
     """gptq2d_quantize_noalloc: the same rounding with the library's static device scratch
     (no workspace; for callers that cannot allocate).  Problems must fit
     GPTQ2D_NOALLOC_SCRATCH_BYTES; calls that overlap on the GPU race on the shared scratch."""
     torch = _torch()
-    _check_device(W, M_L, M_R, scales)
+    _check_device(W, M_L, M_R, scales, out, stats)
     m, n = W.shape
     if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
         raise ValueError("scales must be a contiguous fp32 vector of length m")
@@ -536,12 +599,14 @@ def quantize_noalloc(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, 
 
 
 def stats_dict(st) -> dict:
-    """Decodes a gptq2d_stats (int64[5] tensor or array) into a dict."""
+    """Decodes a gptq2d_stats (int64[STATS_WORDS] tensor or array) into a dict."""
     a = np.asarray(st.cpu() if hasattr(st, "cpu") else st, dtype=np.int64).copy()
     return {"proxy_loss": float(a[:1].view(np.float64)[0]), "n_clamped": int(a[1]),
-            "n_near_tie": int(a[2]), "n_nonfinite": int(a[3]), "status": int(a[4])}
+            "n_near_tie": int(a[2]), "n_nonfinite": int(a[3]), "status": int(a[4]),
+            "n_out_of_range": int(a[5])}
 
 
+@_device_scoped
 def round_host(W, H_L, H_R, scales, bits: int = 4, clamp: bool = True, *, workspace=None,
                stream=None, Q_out=None, stats_out=None):
     """The whole path from HOST tensors through gptq2d_round_host: copies in, factors both
@@ -554,6 +619,7 @@ def round_host(W, H_L, H_R, scales, bits: int = 4, clamp: bool = True, *, worksp
             raise ValueError("round_host takes contiguous host tensors")
     if H_L.dtype != H_R.dtype:
         raise ValueError("H_L and H_R must share a dtype")
+    _check_device(workspace)
     wdt, hdt = _dtype_code(W), _dtype_code(H_L)
     need = round_host_workspace_size(m, n, wdt, hdt)
     if workspace is None:
@@ -566,7 +632,7 @@ def round_host(W, H_L, H_R, scales, bits: int = 4, clamp: bool = True, *, worksp
                                  scales.data_ptr(), int(bits), int(clamp), Q.data_ptr(),
                                  st.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                  _stream(stream), ctypes.byref(piv), ctypes.byref(which))
-    if rc not in (Status.OK, Status.NONFINITE):
+    if rc not in (Status.OK, Status.NONFINITE, Status.RANGE):
         raise GPTQ2DError(rc, "gptq2d_round_host",
                           f"factor {which.value} pivot {piv.value}" if rc == Status.NOT_SPD else "")
     return Q, st

@@ -50,6 +50,21 @@ ProfScope::~ProfScope() {
   else
     g_prof_pool.push_back(e0);
 }
+int check_device_pointers(std::initializer_list<const void*> ps) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ2D_ERR_CUDA;
+  for (const void* p : ps) {
+    if (!p) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      cudaGetLastError();  // not sticky: clear it
+      return GPTQ2D_ERR_INVALID_ARG;
+    }
+    if (at.type == cudaMemoryTypeUnregistered) return GPTQ2D_ERR_INVALID_ARG;
+    if (at.type == cudaMemoryTypeDevice && at.device != dev) return GPTQ2D_ERR_INVALID_ARG;
+  }
+  return GPTQ2D_OK;
+}
 }  // namespace gptq2d
 
 using namespace gptq2d;
@@ -118,6 +133,7 @@ const char* gptq2d_status_string(int status) {
     case GPTQ2D_ERR_WORKSPACE: return "GPTQ2D_ERR_WORKSPACE: workspace too small or misaligned";
     case GPTQ2D_ERR_TIMEOUT: return "GPTQ2D_ERR_TIMEOUT: bounded device wait gave up";
     case GPTQ2D_ERR_CUDA: return "GPTQ2D_ERR_CUDA: CUDA runtime error";
+    case GPTQ2D_ERR_RANGE: return "GPTQ2D_ERR_RANGE: an unclamped integer does not fit its byte";
     default: return "GPTQ2D: unknown status";
   }
 }
@@ -199,8 +215,10 @@ int gptq2d_prepare(const void* H, int h_dtype, int64_t k, int64_t ldh, double* M
   if (!H || !M || ldh < k || ldm < k) return GPTQ2D_ERR_INVALID_ARG;
   if (static_cast<const void*>(M) == H) return GPTQ2D_ERR_INVALID_ARG;
   if (!ws || !aligned256(ws) || ws_bytes < prepare_ws_bytes(k)) return GPTQ2D_ERR_WORKSPACE;
+  int rc = check_device_pointers({H, M, ws});
+  if (rc != GPTQ2D_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int rc = prepare_launch(H, h_dtype, (int)k, ldh, M, ldm, ws, s);
+  rc = prepare_launch(H, h_dtype, (int)k, ldh, M, ldm, ws, s);
   if (rc != GPTQ2D_OK) return rc;
   if (bad_pivot) return read_pivot(ws, s, bad_pivot);
   return GPTQ2D_OK;
@@ -219,6 +237,8 @@ int gptq2d_gram_accumulate(const void* X, int x_dtype, int64_t rows, int64_t k, 
                    (reinterpret_cast<uintptr_t>(X) & 15u) != 0))
     return GPTQ2D_ERR_INVALID_ARG;
   if (!ws || !aligned256(ws) || ws_bytes < 256) return GPTQ2D_ERR_WORKSPACE;
+  const int rc = check_device_pointers({rows > 0 ? X : nullptr, H, ws});
+  if (rc != GPTQ2D_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* err = reinterpret_cast<int*>(static_cast<char*>(ws) + 8);
   if (!accumulate && cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return GPTQ2D_ERR_CUDA;
@@ -232,6 +252,7 @@ int gptq2d_gram_finalize(float* H, int64_t k, int64_t ldh, int64_t total_rows, d
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (k > 0) {
     if (!H || ldh < k) return GPTQ2D_ERR_INVALID_ARG;
+    if (check_device_pointers({H, ws}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
     const int rc = gram_finalize_launch(H, (int)k, ldh, total_rows, damp,
                                         reinterpret_cast<double*>(ws), s);
     if (rc != GPTQ2D_OK) return rc;
@@ -264,7 +285,9 @@ int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, cons
     const char* m0 = reinterpret_cast<const char*>(M[f]);
     const char* m1 = m0 + (size_t)((dims[f] - 1) * ldm[f] + dims[f]) * sizeof(double);
     if (m0 < o1 && o0 < m1) return GPTQ2D_ERR_INVALID_ARG;  // overlaps the output
+    if (check_device_pointers({M[f]}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
   }
+  if (check_device_pointers({out}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
   return kron_factor_launch(nf, M, dims, ldm, out, ldo, static_cast<cudaStream_t>(stream));
 }
 
@@ -279,6 +302,9 @@ int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl, const void* H_
   if (n > 0 && (!H_R || !M_R || ldhr < n || ldmr < n || static_cast<const void*>(M_R) == H_R))
     return GPTQ2D_ERR_INVALID_ARG;
   if (!ws || !aligned256(ws) || ws_bytes < 512) return GPTQ2D_ERR_WORKSPACE;
+  if (check_device_pointers({m > 0 ? H_L : nullptr, m > 0 ? M_L : nullptr,
+                             n > 0 ? H_R : nullptr, n > 0 ? M_R : nullptr, ws}) != GPTQ2D_OK)
+    return GPTQ2D_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(ws);
   const int rc = prepare_pair_launch(H_L, m, ldhl, H_R, n, ldhr, h_dtype, M_L, ldml, M_R, ldmr,
@@ -328,6 +354,8 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
   if (!W || !M_L || !M_R || !scales || !Q) return GPTQ2D_ERR_INVALID_ARG;
   if (ldw < n || ldl < m || ldr < n || ldq < n) return GPTQ2D_ERR_INVALID_ARG;
   if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(m, n)) return GPTQ2D_ERR_WORKSPACE;
+  if (check_device_pointers({W, M_L, M_R, scales, Q, stats, ws}) != GPTQ2D_OK)
+    return GPTQ2D_ERR_INVALID_ARG;
   return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, scales, bits, clamp,
                          Q, ldq, stats, ws, s);
 }
@@ -374,6 +402,8 @@ int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64
                            nullptr, nullptr, &gs);
   if (!M_L || !M_R || ldl < m || ldr < n) return GPTQ2D_ERR_INVALID_ARG;
   if (!ws || !aligned256(ws) || ws_bytes < quantize_ws_bytes(m, n)) return GPTQ2D_ERR_WORKSPACE;
+  if (check_device_pointers({W, M_L, M_R, grid->scales, grid->zeros, Q, stats, ws}) != GPTQ2D_OK)
+    return GPTQ2D_ERR_INVALID_ARG;
   return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales,
                          grid->bits, grid->clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0,
                          nullptr, nullptr, &gs);
@@ -431,6 +461,14 @@ int gptq2d_quantize_block(const gptq2d_layer* L, int nl, void* ws, size_t ws_byt
   }
   const BlockLayout B = block_layout(L, nl);
   if (!ws || !aligned256(ws) || ws_bytes < B.total) return GPTQ2D_ERR_WORKSPACE;
+  for (int i = 0; i < nl; ++i) {
+    const gptq2d_layer& l = L[i];
+    if (l.m == 0 || l.n == 0) continue;
+    if (check_device_pointers({l.W, l.H_L, l.H_R, l.grid.scales, l.grid.zeros, l.Q, l.stats}) !=
+        GPTQ2D_OK)
+      return GPTQ2D_ERR_INVALID_ARG;
+  }
+  if (check_device_pointers({ws}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
   DevStreams* ds = nullptr;
   int rc = dev_streams(&ds);
   if (rc != GPTQ2D_OK) return rc;
@@ -519,6 +557,7 @@ int gptq2d_round_host(const void* W, int w_dtype, int64_t m, int64_t n, const vo
   if (!W || !H_L || !H_R || !scales || !Q || !stats) return GPTQ2D_ERR_INVALID_ARG;
   const HostWs L = host_layout(m, n, w_dtype, h_dtype);
   if (!ws || !aligned256(ws) || ws_bytes < L.total) return GPTQ2D_ERR_WORKSPACE;
+  if (check_device_pointers({ws}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(ws);
   const size_t hs = elem_size(h_dtype);

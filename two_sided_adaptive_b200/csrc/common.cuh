@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 #include <atomic>
+#include <initializer_list>
 #include <mutex>
 
 #include "gptq2d.h"
@@ -41,6 +42,16 @@ struct ProfScope {
     __VA_ARGS__;                                    \
     ::gptq2d::count_launch();                       \
   } while (0)
+
+// Most devices the library keeps per-device state for (internal streams, the
+// no-allocation scratch address).
+constexpr int kMaxDevices = 64;
+
+// GPTQ2D_OK when every non-null pointer is memory the current device may
+// dereference: device memory of the current device, managed memory, or
+// page-locked host memory; GPTQ2D_ERR_INVALID_ARG for another device's memory or
+// pageable host memory (a kernel given either would fault or read the wrong GPU).
+int check_device_pointers(std::initializer_list<const void*> ps);
 
 inline int64_t round_up(int64_t x, int64_t r) { return (x + r - 1) / r * r; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -132,7 +143,7 @@ __device__ __forceinline__ void cp_async_wait_group() {
 // Per-tile partial statistics of one rounding sweep.
 struct TileStat {
   double loss;
-  long long clamped, near_tie, nonfinite;
+  long long clamped, near_tie, nonfinite, out_of_range;
 };
 
 // ---------------------------------------------------------------------------

@@ -32,7 +32,7 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GPTQ2D_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 256;
+using gptq2d::kMaxDevices;
 constexpr int64_t kMaxDim = (int64_t)1 << 20;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
@@ -72,6 +72,8 @@ extern "C" int gptq2d_quantize_noalloc(const void* W, int w_dtype, int64_t m, in
   // the problem's scratch need must fit the static array
   if (gptq2d::quantize_ws_bytes(m, n) > (size_t)GPTQ2D_NOALLOC_SCRATCH_BYTES)
     return GPTQ2D_ERR_WORKSPACE;
+  if (gptq2d::check_device_pointers({W, M_L, M_R, scales, Q, stats}) != GPTQ2D_OK)
+    return GPTQ2D_ERR_INVALID_ARG;
   void* ws = nullptr;
   const int rc = scratch_address(&ws);
   if (rc != GPTQ2D_OK) return rc;

@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   };
 
   double loss = 0.0;
-  long long ncl = 0, nnt = 0, nnf = 0;
+  long long ncl = 0, nnt = 0, nnf = 0, nor = 0;
   const int sa = lane >> 2, cq = lane & 3;  // row inside a sub-tile, column group (cq, cq + 4)
   for (int w = 0; w < 2 * NSUB - 1; ++w) {
     const int p0 = w - (NSUB - 1) > 0 ? w - (NSUB - 1) : 0;
@@ -443,7 +443,12 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       const double tq = Tq[r * SLD + cc];
       const double qr = (tq + 6755399441055744.0) - 6755399441055744.0;
       const double qv = qr < lo ? lo : (qr > hi ? hi : qr);
-      code[k] = (int)(qv + zq + a.code_off);
+      // an unclamped integer beyond the int8 range is stored saturated and counted
+      // (only the symmetric byte output can be unclamped: zero points and packing
+      // require clamping, which keeps every code inside its byte)
+      const double qs = a.clamp ? qv : fmin(fmax(qv, -128.0), 127.0);
+      nor += (qs != qv) && isfinite(tq);
+      code[k] = (int)(qs + zq + a.code_off);
       const double res = Sdl[r] * Sdr[cc] * sr * (tq - qv);
       loss += res * res;
       ncl += (qv != qr);
@@ -465,27 +470,30 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
 
   // ---- tile statistics (fixed reduction order: deterministic)
   __shared__ double red_l[SWEEP_THREADS / 32];
-  __shared__ long long red_c[SWEEP_THREADS / 32][3];
+  __shared__ long long red_c[SWEEP_THREADS / 32][4];
   for (int o = 16; o > 0; o >>= 1) {
     loss += __shfl_down_sync(0xffffffffu, loss, o);
     ncl += __shfl_down_sync(0xffffffffu, ncl, o);
     nnt += __shfl_down_sync(0xffffffffu, nnt, o);
     nnf += __shfl_down_sync(0xffffffffu, nnf, o);
+    nor += __shfl_down_sync(0xffffffffu, nor, o);
   }
   if (lane == 0) {
     red_l[warp] = loss;
     red_c[warp][0] = ncl;
     red_c[warp][1] = nnt;
     red_c[warp][2] = nnf;
+    red_c[warp][3] = nor;
   }
   __syncthreads();
   if (tid == 0) {
-    TileStat st{0.0, 0, 0, 0};
+    TileStat st{0.0, 0, 0, 0, 0};
     for (int w2 = 0; w2 < SWEEP_THREADS / 32; ++w2) {
       st.loss += red_l[w2];
       st.clamped += red_c[w2][0];
       st.near_tie += red_c[w2][1];
       st.nonfinite += red_c[w2][2];
+      st.out_of_range += red_c[w2][3];
     }
     a.part[(int64_t)I * a.Tn + J] = st;
   }
@@ -794,20 +802,22 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
 __global__ void __launch_bounds__(256) finalize_kernel(const TileStat* part, int ntiles,
                                                        const int* err, gptq2d_stats* out) {
   __shared__ double sl[256];
-  __shared__ long long sc[256][3];
+  __shared__ long long sc[256][4];
   const int tid = threadIdx.x;
   double l = 0.0;
-  long long c0 = 0, c1 = 0, c2 = 0;
+  long long c0 = 0, c1 = 0, c2 = 0, c3 = 0;
   for (int i = tid; i < ntiles; i += 256) {
     l += part[i].loss;
     c0 += part[i].clamped;
     c1 += part[i].near_tie;
     c2 += part[i].nonfinite;
+    c3 += part[i].out_of_range;
   }
   sl[tid] = l;
   sc[tid][0] = c0;
   sc[tid][1] = c1;
   sc[tid][2] = c2;
+  sc[tid][3] = c3;
   __syncthreads();
   for (int o = 128; o > 0; o >>= 1) {
     if (tid < o) {
@@ -815,6 +825,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(const TileStat* part, int
       sc[tid][0] += sc[tid + o][0];
       sc[tid][1] += sc[tid + o][1];
       sc[tid][2] += sc[tid + o][2];
+      sc[tid][3] += sc[tid + o][3];
     }
     __syncthreads();
   }
@@ -824,14 +835,16 @@ __global__ void __launch_bounds__(256) finalize_kernel(const TileStat* part, int
     st.n_clamped = sc[0][0];
     st.n_near_tie = sc[0][1];
     st.n_nonfinite = sc[0][2];
+    st.n_out_of_range = sc[0][3];
     st.status = *err != 0 ? GPTQ2D_ERR_TIMEOUT
-                : sc[0][2] > 0 ? GPTQ2D_ERR_NONFINITE : GPTQ2D_OK;
+                : sc[0][2] > 0 ? GPTQ2D_ERR_NONFINITE
+                : sc[0][3] > 0 ? GPTQ2D_ERR_RANGE : GPTQ2D_OK;
     *out = st;
   }
 }
 
 __global__ void zero_stats_kernel(gptq2d_stats* out) {
-  gptq2d_stats st{0.0, 0, 0, 0, GPTQ2D_OK};
+  gptq2d_stats st{0.0, 0, 0, 0, GPTQ2D_OK, 0};
   *out = st;
 }
 

@@ -4,7 +4,6 @@
 namespace gptq2d {
 
 namespace {
-constexpr int kMaxDevices = 64;
 DevStreams g_dev[kMaxDevices];
 }  // namespace
 
