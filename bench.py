@@ -602,6 +602,140 @@ def run_block70b(args, rank: int = 0, world: int = 1):
             "block_workspace_gb": ws.numel() / 1e9, "layers": layers}
 
 
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count()
+
+
+def run_configs(args):
+    """Every workload of the rounding's configuration list, each timed on the GPU
+    (prepare_pair + quantize, CUDA events, best of 3 after a warm-up pass) beside the
+    fp64 oracle on this host's cores:
+      tiny   64 x 64 fp64, unit scales, no clamp: the naive mn x mn Kronecker sweep and
+             the anti-diagonal oracle, both in full;
+      small  512 x 512, INT4, seeds 0-3: the anti-diagonal oracle in full;
+      attn   4096 x 4096 INT4; mlp 4096 x 14336 INT4 and INT3: the oracle's factors in
+             full and its rounding on the leading 1024 x 1024 prefix (a problem of its
+             own), scaled to the layer by mn(m + n) (the rounding's work; the scaling
+             exponent is checked on prefixes from 512 to 4096, see DESIGN.md);
+    and the quantize call's fp64 rate against the cuBLAS DGEMM peak measured here."""
+    import torch
+    import oracle as O
+    import two_sided_adaptive_b200 as g
+    import workloads as WL
+    from two_sided_adaptive_b200 import build as gbuild
+    gbuild.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peak = measure_dgemm_tflops()
+    cores = cpu_cores()
+
+    def gpu_gram(X):
+        Xt = torch.from_numpy(X).cuda()
+        return (Xt.T @ Xt).cpu().numpy()
+
+    def gpu_time(pb, wdtype):
+        m, n = pb.shape
+        W = torch.from_numpy(np.ascontiguousarray(pb.W)).to(dev).to(wdtype)
+        HL = torch.from_numpy(np.ascontiguousarray(pb.H_L)).to(dev)
+        HR = torch.from_numpy(np.ascontiguousarray(pb.H_R)).to(dev)
+        sc = torch.from_numpy(pb.scales).to(dev)
+        ML = torch.empty((m, m), dtype=torch.float64, device=dev)
+        MR = torch.empty((n, n), dtype=torch.float64, device=dev)
+        wsP = torch.empty(512, dtype=torch.uint8, device=dev)
+        wsQ = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
+        Q = torch.empty((m, n), dtype=torch.int8, device=dev)
+        st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+        best = None
+        for rep in range(4):  # the first pass warms up
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            torch.cuda.synchronize()
+            e[0].record()
+            g.prepare_pair(HL, HR, out_l=ML, out_r=MR, workspace=wsP, check=False)
+            e[1].record()
+            g.quantize(W, ML, MR, sc, pb.bits, pb.clamp, out=Q, stats=st, workspace=wsQ)
+            e[2].record()
+            torch.cuda.synchronize()
+            t = (e[0].elapsed_time(e[1]) / 1e3, e[1].elapsed_time(e[2]) / 1e3)
+            if rep > 0 and (best is None or sum(t) < sum(best)):
+                best = t
+        sd = g.stats_dict(st)
+        Qh = Q.cpu().numpy()
+        del W, HL, HR, sc, ML, MR, wsP, wsQ, Q, st
+        torch.cuda.empty_cache()
+        return best, sd, Qh
+
+    rows = []
+
+    def record(name, pb, wdtype, cpu_s, cpu_how, agree=None):
+        m, n = pb.shape
+        (tp, tq), sd, _ = gpu_time(pb, wdtype)
+        tf = m * n * (m + n) / tq / 1e12
+        row = {"config": name, "m": m, "n": n, "bits": pb.bits if pb.clamp else None,
+               "w_dtype": str(wdtype).replace("torch.", ""),
+               "gpu_s_per_layer": tp + tq, "prepare_s": tp, "quantize_s": tq,
+               "entries_per_s": m * n / (tp + tq),
+               "quantize_fp64_tflops": tf, "quantize_frac_of_dgemm": tf / peak,
+               "status": sd["status"], "n_near_tie": sd["n_near_tie"],
+               "cpu_oracle_s_per_layer": cpu_s, "cpu_cores": cores, "cpu_how": cpu_how}
+        if agree is not None:
+            row["q_equals_oracle"] = agree
+        rows.append(row)
+        print(json.dumps(row), file=sys.stderr, flush=True)
+
+    # tiny: both CPU oracles in full
+    pb = WL.tiny(0)
+    t0 = time.perf_counter()
+    Q1, _ = O.babai_kron_sweep(pb.W, pb.H_L, pb.H_R, pb.scales.astype(np.float64), pb.bits,
+                               pb.clamp)
+    t_naive = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    r = O.gptq2d(pb.W, pb.H_L, pb.H_R, pb.scales.astype(np.float64), pb.bits, pb.clamp)
+    t_o2 = time.perf_counter() - t0
+    _, _, Qg = gpu_time(pb, torch.float64)
+    record("tiny 64x64 fp64 (s=1, no clamp)", pb, torch.float64, t_o2,
+           f"anti-diagonal oracle in full ({t_o2:.3f} s); naive mn x mn Kronecker sweep in full "
+           f"({t_naive:.2f} s)", bool(np.array_equal(Qg, r.Q) and np.array_equal(Q1, r.Q)))
+    # small, seeds 0-3: the anti-diagonal oracle in full
+    for seed in range(4):
+        pb = WL.small(seed)
+        t0 = time.perf_counter()
+        r = O.gptq2d(pb.W.astype(np.float64), pb.H_L, pb.H_R, pb.scales.astype(np.float64),
+                     pb.bits, pb.clamp)
+        t_o2 = time.perf_counter() - t0
+        _, _, Qg = gpu_time(pb, torch.float32)
+        record(f"small 512x512 INT4 seed {seed}", pb, torch.float32, t_o2,
+               "anti-diagonal oracle in full (LAPACK factors included)",
+               bool(np.array_equal(Qg, r.Q)))
+    # attn and mlp: factors in full, rounding on a 1024 x 1024 prefix, scaled by mn(m+n)
+    k = 1024
+    for name, pb in (("attn 4096x4096 INT4", WL.attn(0, matmul=gpu_gram)),
+                     ("mlp 4096x14336 INT4", WL.mlp(0, bits=4, matmul=gpu_gram)),
+                     ("mlp 4096x14336 INT3", WL.mlp(0, bits=3, matmul=gpu_gram))):
+        m, n = pb.shape
+        t0 = time.perf_counter()
+        ML = O.reverse_cholesky(pb.H_L)
+        MR = O.reverse_cholesky(pb.H_R)
+        t_f = time.perf_counter() - t0
+        W64 = torch.from_numpy(pb.W).to(torch.bfloat16).double().numpy()
+        t0 = time.perf_counter()
+        O.gptq2d_antidiagonal(W64[:k, :k], ML[:k, :k], MR[:k, :k],
+                              pb.scales[:k].astype(np.float64), pb.bits, pb.clamp)
+        t_r = time.perf_counter() - t0
+        scale = m * n * (m + n) / (k * k * 2 * k)
+        record(name, pb, torch.bfloat16, t_f + t_r * scale,
+               f"LAPACK factors in full ({t_f:.2f} s) + anti-diagonal rounding of the leading "
+               f"{k}x{k} prefix ({t_r:.2f} s) x {scale:.1f} (mn(m+n) ratio): extrapolated")
+        del ML, MR
+    return {"metric": "seconds per layer and entries/s for every configuration (1 B200), "
+                      "beside the fp64 CPU oracle",
+            "value": None, "unit": "s", "n_gpus": 1, "higher_is_better": False, "dtype": "f64",
+            "data": "synthetic", "dgemm_peak_tflops": peak, "cpu_cores": cores,
+            "config": {"workload": "configs"}, "configs": rows}
+
+
 def run_kron3(args):
     """A Hessian with three Kronecker factors: W is a 4096 x 64 x 64 tensor (a 4096 x 4096
     layer whose input dimension is split into 64 groups of 64, each mode with its own
@@ -816,16 +950,17 @@ def run_gram(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=80)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=("attn", "mlp", "small", "block70b", "kron3", "grid128",
-                                           "gram"),
+                                           "gram", "configs"),
                     default="attn",
                     help="block70b: seconds per layer for one 70B-class block; kron3: a "
                          "three-factor Kronecker Hessian; grid128: the attention layer on an "
                          "asymmetric 128-column-group packed INT4 grid; gram: the Kronecker "
-                         "factors from activations on the tensor cores (reports, not the "
+                         "factors from activations on the tensor cores; configs: every "
+                         "configuration with the CPU oracle beside it (reports, not the "
                          "headline metric)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -860,10 +995,10 @@ def main():
         if rank == 0:
             print(json.dumps(res), flush=True)
         return
-    if args.workload in ("block70b", "kron3", "grid128", "gram"):
+    if args.workload in ("block70b", "kron3", "grid128", "gram", "configs"):
         if rank == 0:
             run = {"block70b": run_block70b, "kron3": run_kron3, "grid128": run_grid128,
-                   "gram": run_gram}[args.workload]
+                   "gram": run_gram, "configs": run_configs}[args.workload]
             res = run(args)
             if res is not None:
                 print(json.dumps(res), flush=True)
