@@ -355,6 +355,18 @@ def run_ours(args, rank, world, local_rank):
                                              workspace=wsQ), reps),
     }
 
+    # the proxy loss of round-to-nearest on the same factors (the pages' baseline), and of
+    # the rounding's own Q as a full quadratic form, outside the timed region
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    rtn_loss = g.proxy_loss(W, M_L, M_R, s, None, pb.bits, pb.clamp)
+    f1.record()
+    own_loss = g.proxy_loss(W, M_L, M_R, s, Q, pb.bits, pb.clamp)
+    torch.cuda.synchronize()
+    stats["rtn_loss"] = float(rtn_loss.item())
+    stats["proxy_loss_quadratic_form"] = float(own_loss.item())
+    stats["proxy_loss_ms"] = f0.elapsed_time(f1)
+
     # end to end through the C ABI from pinned host memory
     e2e = None
     if not args.no_e2e:
@@ -662,6 +674,7 @@ def run_configs(args):
             if rep > 0 and (best is None or sum(t) < sum(best)):
                 best = t
         sd = g.stats_dict(st)
+        sd["rtn_loss"] = float(g.proxy_loss(W, ML, MR, sc, None, pb.bits, pb.clamp).item())
         Qh = Q.cpu().numpy()
         del W, HL, HR, sc, ML, MR, wsP, wsQ, Q, st
         torch.cuda.empty_cache()
@@ -679,6 +692,7 @@ def run_configs(args):
                "entries_per_s": m * n / (tp + tq),
                "quantize_fp64_tflops": tf, "quantize_frac_of_dgemm": tf / peak,
                "status": sd["status"], "n_near_tie": sd["n_near_tie"],
+               "proxy_loss": sd["proxy_loss"], "rtn_loss": sd["rtn_loss"],
                "cpu_oracle_s_per_layer": cpu_s, "cpu_cores": cores, "cpu_how": cpu_how}
         if agree is not None:
             row["q_equals_oracle"] = agree
@@ -964,7 +978,7 @@ def main():
                          "headline metric)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample", type=int, default=768)
+    ap.add_argument("--cpu-sample", type=int, default=1024)
     ap.add_argument("--ref-sample", type=int, default=384)
     ap.add_argument("--profile-step", action="store_true",
                     help="run one step of the path only (input for ncu captures); prints nothing")

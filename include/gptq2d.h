@@ -33,6 +33,14 @@
  *   - All floating-point arithmetic on the path is IEEE fp64.
  *   - Results are deterministic: identical inputs on the same device give a
  *     bitwise identical Q and statistics.
+ *   - Every pointer a device entry point dereferences on the GPU must belong to
+ *     the CURRENT device (cudaSetDevice) or be managed or page-locked host
+ *     memory; another device's memory or pageable host memory is refused with
+ *     GPTQ2D_ERR_INVALID_ARG before anything is enqueued.
+ *   - The library keeps per-device state, created on a device's first call:
+ *     internal streams and events, and the address of the no-allocation
+ *     scratch.  A cudaDeviceReset invalidates that state; do not call the
+ *     library on a device after resetting it in the same process.
  */
 #ifndef GPTQ2D_H_
 #define GPTQ2D_H_
@@ -282,6 +290,40 @@ int gptq2d_quantize(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ld
                     const float* scales, int bits, int clamp,
                     int8_t* Q, int64_t ldq, gptq2d_stats* stats,
                     void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* The proxy loss of a given rounding, and of round-to-nearest (the baseline   */
+/* the pages compare GPTQ-2D with: arxivlens, Abstract; mind-verse.de,         */
+/* "GPTQ-2D: Eine Weiterentwicklung der adaptiven Rundung")                    */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace gptq2d_proxy_loss needs for an m x n problem (two tile-padded
+ * fp64 m x n buffers and one double per 64 x 64 tile); 0 for sizes out of range. */
+size_t gptq2d_proxy_loss_workspace_size(int64_t m, int64_t n);
+
+/* L(Q) = tr(dW^T H_L dW H_R) = || M_L dW M_R^T ||_F^2 with dW = W - diag(s) Q, written
+ * to *loss (one DEVICE double) on `stream`.
+ *
+ *   W, w_dtype, ldw : device, m x n, GPTQ2D_F32, GPTQ2D_BF16 or GPTQ2D_F64.
+ *   Q, ldq          : device int8, m x n (row stride ldq >= n): the integers to score, e.g.
+ *                     gptq2d_quantize's output; NULL scores round-to-nearest,
+ *                     q = clamp(rint(W / s)) on the grid of bits / clamp (as in
+ *                     gptq2d_quantize).
+ *   scales          : device fp32 [m], the per-row grid steps.
+ *   M_L, M_R        : the lower factors (M^T M = H) as for gptq2d_quantize; only their
+ *                     lower triangles are read.
+ *   loss            : device pointer to one double.
+ *   ws, ws_bytes    : device workspace, >= gptq2d_proxy_loss_workspace_size(m, n),
+ *                     256-byte aligned.
+ *
+ * This is a full quadratic form (two triangular matrix products, about mn(m + n)
+ * flops on the FP64 tensor cores, as much work as the rounding), so the rounding does
+ * not compute it: its own loss comes from the nearest-plane residual identity in
+ * gptq2d_stats.  Deterministic (fixed reduction order).  m == 0 or n == 0 writes 0. */
+int gptq2d_proxy_loss(const void* W, int w_dtype, int64_t m, int64_t n, int64_t ldw,
+                      const int8_t* Q, int64_t ldq, const float* scales, int bits, int clamp,
+                      const double* M_L, int64_t ldl, const double* M_R, int64_t ldr,
+                      double* loss, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* Grid variants (the pages fix only a 4-bit integer grid: mind-verse.de       */

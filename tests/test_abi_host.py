@@ -221,3 +221,30 @@ def test_block_rejects_invalid_arguments(L):
     lay[0].grid.bits = 4
     assert L.gptq2d_quantize_block(lay, 1, 256, 10, None, None, None, None) == g.Status.WORKSPACE
     assert L.gptq2d_block_workspace_size(lay, 1) >= 2 * 2 * 64 * 64 * 8
+
+
+def test_proxy_loss_workspace_size(L):
+    assert L.gptq2d_proxy_loss_workspace_size(-1, 4) == 0
+    assert L.gptq2d_proxy_loss_workspace_size(0, 5) == 256
+    # two tile-padded fp64 buffers and one double per 64 x 64 tile
+    assert L.gptq2d_proxy_loss_workspace_size(100, 70) == 2 * 128 * 128 * 8 + 256
+
+
+@pytest.mark.parametrize("bad", [
+    dict(m=-1), dict(bits=1), dict(bits=9), dict(clamp=2), dict(W=None), dict(scales=None),
+    dict(ML=None), dict(ldw=5), dict(ldl=9), dict(ldr=5), dict(Q=16, ldq=3), dict(loss=None),
+    dict(w_dtype=7)])
+def test_proxy_loss_rejects_invalid_arguments(L, bad):
+    a = dict(W=16, w_dtype=0, m=10, n=6, ldw=6, Q=None, ldq=6, scales=16, bits=4, clamp=1,
+             ML=16, ldl=10, MR=16, ldr=6, loss=16, ws=256, ws_bytes=1 << 20)
+    a.update(bad)
+    assert L.gptq2d_proxy_loss(a["W"], a["w_dtype"], a["m"], a["n"], a["ldw"], a["Q"], a["ldq"],
+                               a["scales"], a["bits"], a["clamp"], a["ML"], a["ldl"], a["MR"],
+                               a["ldr"], a["loss"], a["ws"], a["ws_bytes"], None) == \
+        g.Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("ws, nbytes", [(None, 1 << 20), (256 + 8, 1 << 20), (256, 1000)])
+def test_proxy_loss_rejects_bad_workspace(L, ws, nbytes):
+    assert L.gptq2d_proxy_loss(16, 0, 10, 6, 6, None, 6, 16, 4, 1, 16, 10, 16, 6, 16, ws, nbytes,
+                               None) == g.Status.WORKSPACE

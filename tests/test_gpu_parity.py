@@ -336,6 +336,11 @@ def test_attention_layer_4096(g):
     assert st["proxy_loss"] == pytest.approx(direct, rel=LOSS_RTOL)
     rtn_loss = O.proxy_loss(W64, O.rtn(W64, s64, pb.bits, pb.clamp), s64, pb.H_L, pb.H_R)
     assert st["proxy_loss"] < rtn_loss
+    gpu_rtn = float(g.proxy_loss(dev(pb.W), ML, MR, dev(pb.scales), None, pb.bits,
+                                 pb.clamp).item())
+    assert gpu_rtn == pytest.approx(rtn_loss, rel=1e-9)
+    print(f"attn 4096^2: GPTQ-2D loss {st['proxy_loss']:.6g}, round-to-nearest {gpu_rtn:.6g} "
+          f"(ratio {st['proxy_loss'] / gpu_rtn:.4f})")
 
 
 @pytest.mark.slow
@@ -465,6 +470,36 @@ def test_unclamped_integers_beyond_int8_are_saturated_and_reported(g):
     assert big.sum() > 0 and st["n_out_of_range"] == int(big.sum())
     assert st["status"] == g.Status.RANGE
     np.testing.assert_array_equal(Qg, np.clip(r.Q, -128, 127))
+
+
+# --------------------------------------------------------------------------- #
+# the proxy loss of a given rounding and of round-to-nearest (gptq2d_proxy_loss)
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("shape, wdt, bits, clamp", [
+    ((1, 1), torch.float32, 4, True), ((70, 9), torch.float64, 3, True),
+    ((130, 449), torch.bfloat16, 4, True), ((257, 64), torch.float32, 4, False),
+    ((64, 200), torch.float32, 8, True)], ids=str)
+def test_proxy_loss_matches_the_direct_trace(g, shape, wdt, bits, clamp):
+    """gptq2d_proxy_loss of the rounding's own Q equals the loss the rounding reports
+    (the nearest-plane residual identity) and the oracle's direct trace; with Q = None
+    it scores round-to-nearest, against the oracle's trace of its RTN."""
+    m, n = shape
+    pb = WL.small(7, m, n, bits)
+    W = dev(pb.W).to(wdt)
+    W64 = W.double().cpu().numpy()
+    s = dev(pb.scales)
+    s64 = pb.scales.astype(np.float64)
+    ML, MR = g.prepare(dev(pb.H_L)), g.prepare(dev(pb.H_R))
+    Q, st = g.quantize(W, ML, MR, s, bits, clamp)
+    own = float(g.proxy_loss(W, ML, MR, s, Q, bits, clamp).item())
+    direct = O.proxy_loss(W64, Q.cpu().numpy(), s64, pb.H_L, pb.H_R)
+    assert own == pytest.approx(direct, rel=1e-9, abs=1e-300)
+    # the identity sums d^2 s^2 (t - q)^2 from t = y / s: relative rounding of order 1e-8
+    # where the loss is tiny (y close to the grid), so the rounding's own bound applies
+    assert own == pytest.approx(g.stats_dict(st)["proxy_loss"], rel=LOSS_RTOL, abs=1e-300)
+    rtn = float(g.proxy_loss(W, ML, MR, s, None, bits, clamp).item())
+    ref = O.proxy_loss(W64, O.rtn(W64, s64, bits, clamp), s64, pb.H_L, pb.H_R)
+    assert rtn == pytest.approx(ref, rel=1e-9, abs=1e-300)
 
 
 # --------------------------------------------------------------------------- #

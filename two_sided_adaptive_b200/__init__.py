@@ -22,7 +22,8 @@ __all__ = [
     "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS", "quantize_grid",
     "gram_accumulate", "gram_finalize", "gram", "quantize_block", "block_workspace_size",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
-    "round_host_workspace_size", "quantize_noalloc", "check_wait_timeout", "profile_enable",
+    "round_host_workspace_size", "quantize_noalloc", "proxy_loss", "check_wait_timeout",
+    "profile_enable",
     "profile_reset", "profile_read", "profile_timeline",
     "KERNEL_CLASSES", "STATS_WORDS", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F64",
 ]
@@ -134,6 +135,12 @@ def lib():
         L.gptq2d_quantize_noalloc.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p,
                                               _c_i64, _c_p, _c_i64, _c_p, ctypes.c_int,
                                               ctypes.c_int, _c_p, _c_i64, _c_p, _c_p]
+        L.gptq2d_proxy_loss_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_proxy_loss_workspace_size.argtypes = [_c_i64, _c_i64]
+        L.gptq2d_proxy_loss.restype = ctypes.c_int
+        L.gptq2d_proxy_loss.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
+                                        _c_p, ctypes.c_int, ctypes.c_int, _c_p, _c_i64, _c_p,
+                                        _c_i64, _c_p, _c_p, ctypes.c_size_t, _c_p]
         L.gptq2d_round_host_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_round_host_workspace_size.argtypes = [_c_i64, _c_i64, ctypes.c_int, ctypes.c_int]
         L.gptq2d_round_host.restype = ctypes.c_int
@@ -596,6 +603,33 @@ def quantize_noalloc(W, M_L, M_R, scales, bits: int = 4, clamp: bool = True, *, 
     if rc != Status.OK:
         raise GPTQ2DError(rc, "gptq2d_quantize_noalloc")
     return Q, st
+
+
+@_device_scoped
+def proxy_loss(W, M_L, M_R, scales, Q=None, bits: int = 4, clamp: bool = True, *, out=None,
+               workspace=None, stream=None):
+    """tr(dW^T H_L dW H_R) = ||M_L dW M_R^T||_F^2 of the integers Q (int8 m x n), or of
+    round-to-nearest on the bits / clamp grid when Q is None (gptq2d_proxy_loss).
+    Returns a one-element fp64 device tensor."""
+    torch = _torch()
+    _check_device(W, M_L, M_R, scales, Q, out, workspace)
+    m, n = W.shape
+    if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous fp32 vector of length m")
+    if M_L.dtype != torch.float64 or M_R.dtype != torch.float64:
+        raise ValueError("factors must be fp64")
+    if Q is not None and (Q.dtype != torch.int8 or tuple(Q.shape) != (m, n)):
+        raise ValueError("Q must be int8 m x n")
+    res = out if out is not None else torch.empty(1, dtype=torch.float64, device=W.device)
+    ws = _workspace(int(lib().gptq2d_proxy_loss_workspace_size(m, n)), W.device, workspace)
+    rc = lib().gptq2d_proxy_loss(W.data_ptr(), _dtype_code(W), m, n, _ld(W),
+                                 Q.data_ptr() if Q is not None else None,
+                                 _ld(Q) if Q is not None else n, scales.data_ptr(), int(bits),
+                                 int(clamp), M_L.data_ptr(), _ld(M_L), M_R.data_ptr(), _ld(M_R),
+                                 res.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_proxy_loss")
+    return res
 
 
 def stats_dict(st) -> dict:

@@ -22,7 +22,9 @@
 // address, so the first call on each device resolves the real address with
 // cudaGetSymbolAddress while that device is current, and caches it.  That
 // first call may load the library's device code and should therefore come
-// before any stream capture.  No call allocates: no cudaMalloc, cudaFree or
+// before any stream capture.  A cudaDeviceReset makes the cached address stale
+// (as it does the library's internal streams): the library must not be called
+// on a device after it was reset.  No call allocates: no cudaMalloc, cudaFree or
 // allocating library routine is used on this path.
 #include <mutex>
 
