@@ -938,6 +938,14 @@ def run_gram(args):
             e1.record()
             torch.cuda.synchronize()
             best = min(best, e0.elapsed_time(e1))
+        best_acc = 1e30  # gram_accumulate alone
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.gram_accumulate(Xb, H, accumulate=False, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            best_acc = min(best_acc, e0.elapsed_time(e1))
         fl = float(rows) * k * (k + 128)
         Xd = Xb.double()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -952,6 +960,8 @@ def run_gram(args):
         torch.cuda.empty_cache()
         out.append({"k": k, "rows": rows, "ms": best, "tflops": fl / (best * 1e-3) / 1e12,
                     "frac_of_bf16_peak": fl / (best * 1e-3) / 1e12 / peak,
+                    "accumulate_ms": best_acc,
+                    "accumulate_tflops": fl / (best_acc * 1e-3) / 1e12,
                     "fp64_matmul_ms": t64})
     return {"metric": "Gram X^T X / N + damping from bf16 activations (tensor cores), TFLOP/s",
             "value": out[-1]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,

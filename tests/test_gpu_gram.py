@@ -42,7 +42,8 @@ def _lower_block_mask(k, b=128):
 
 
 @pytest.mark.parametrize("rows,k", [(1, 8), (5, 8), (64, 128), (100, 136), (300, 256),
-                                    (4096, 384), (130, 520), (63, 64), (129, 1024)])
+                                    (4096, 384), (130, 520), (63, 64), (129, 1024),
+                                    (257, 1160)])
 def test_integer_activations_are_exact(g, rows, k):
     rng = np.random.default_rng(rows * 1000 + k)
     X = rng.integers(-4, 5, (rows, k)).astype(np.float32)

@@ -6,21 +6,23 @@
 // H = A^T A.  The damping (a fraction of the mean diagonal added to the diagonal)
 // is GPTQ's usual one; the pages give none.
 //
-// gram_kernel: one CTA per 128 x 128 block (bi, bj), bj <= bi, of the lower block
-// triangle of H.  The block is D = X[:, I]^T X[:, J] over all rows, accumulated in
-// fp32 in tensor memory by tcgen05.mma (kind::f16, bf16 operands, M = N = 128,
-// K = 16 per instruction).  Both operands are chunks of 64 rows of X, and X is
-// row-major (features contiguous), so A (128 features x 64 rows) and B are
-// "MN-major".  Each operand is two TMA boxes of 64 features x 64 rows
-// (cp.async.bulk.tensor, 128-byte swizzle; zero fill past the last row or
-// column): a box holds the rows as 128-byte lines, swizzled in groups of 8 lines,
-// which is the canonical 128B-swizzled MN-major layout of the operand descriptor
-// (stride byte offset 1024 between 8-row groups, leading byte offset 8192 between
-// the two 64-feature boxes).
+// gram_kernel: one CTA per pair of 128 x 128 blocks (bi, 2c), (bi, 2c + 1) of the
+// lower block triangle of H, or per diagonal block (bi, bi) of an even block row
+// (then 2c = bi).  The product is D = X[:, I]^T X[:, J] over all rows, 128 x 256 (or
+// 128 x 128), accumulated in fp32 in tensor memory by tcgen05.mma (kind::f16, bf16
+// operands, M = 128, N = 256 or 128, K = 16 per instruction): the wide tile reads
+// 12 KB of shared memory per 2^20 flops where two 128 x 128 tiles read 16 KB.  Both
+// operands are chunks of 64 rows of X, and X is row-major (features contiguous), so
+// A (128 features x 64 rows) and B (256 or 128 features) are "MN-major".  Each
+// operand is a run of TMA boxes of 64 features x 64 rows (cp.async.bulk.tensor,
+// 128-byte swizzle; zero fill past the last row or column): a box holds the rows
+// as 128-byte lines, swizzled in groups of 8 lines, which is the canonical
+// 128B-swizzled MN-major layout of the operand descriptor (stride byte offset 1024
+// between 8-row groups, leading byte offset 8192 between 64-feature boxes).
 //   warp 1, one thread  fills a 4-stage ring: it waits for the stage's empty
 //                       barrier, arms the full barrier with the stage's bytes and
-//                       issues the 2 (diagonal block) or 4 box loads;
-//   warp 0              allocates 128 columns of tensor memory; its elected thread
+//                       issues the 2 (diagonal block: B = A) or 6 box loads;
+//   warp 0              allocates 256 columns of tensor memory; its elected thread
 //                       waits for a full stage, issues the stage's four MMAs and
 //                       frees the stage with tcgen05.commit on its empty barrier.
 //                       A last commit signals the end.
@@ -42,17 +44,17 @@ namespace gptq2d {
 
 namespace {
 
-constexpr int GB = 128;                      // block edge (MMA M = N)
+constexpr int GB = 128;                      // block edge (MMA M; N is one or two blocks)
 constexpr int GK = 64;                       // rows of X per stage
 constexpr int GSTAGES = 4;
 constexpr int GTHREADS = 128;
 constexpr int G_BOX = 64 * GK * 2;           // one TMA box: 64 features x 64 rows, 8 KB
-constexpr int G_TILE = 2 * G_BOX;            // one bf16 operand tile: 16 KB
-constexpr int G_STAGE = 2 * G_TILE;          // A and B
+constexpr int G_TILE = 2 * G_BOX;            // one bf16 operand tile of 128 features: 16 KB
+constexpr int G_STAGE = 3 * G_TILE;          // A (128 features) and B (up to 256)
 constexpr int G_SMEM = GSTAGES * G_STAGE + 1024;  // + room to align the ring to 1024 bytes
 constexpr uint32_t G_SBO = 1024;             // between 8-row groups
 constexpr uint32_t G_LBO = G_BOX;            // between the two 64-feature boxes
-constexpr uint32_t G_TMEM_COLS = GB;         // fp32 accumulator: 128 lanes x 128 columns
+constexpr uint32_t G_TMEM_COLS = 2 * GB;     // fp32 accumulator: 128 lanes x up to 256 columns
 
 // Shared-memory operand descriptor: start address, leading and stride byte offsets
 // (all in 16-byte units), descriptor version 1, 128-byte swizzle (layout type 2).
@@ -78,8 +80,47 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x
 
 // Instruction descriptor (kind::f16): fp32 accumulator (bit 4), bf16 A (bit 7) and
 // B (bit 10), both MN-major (bits 15, 16), N / 8 at bit 17, M / 16 at bit 24.
-constexpr uint32_t G_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                             ((uint32_t)(GB >> 3) << 17) | ((uint32_t)(GB >> 4) << 24);
+__host__ __device__ constexpr uint32_t g_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(GB >> 4) << 24);
+}
+
+// CTAs of block rows 0 .. B - 1: row bi holds ceil((bi + 1) / 2) of them.
+__host__ __device__ inline int g_ctas_before(int B) { return (B + 1) * (B + 1) / 4; }
+
+// CTA order.  Block rows are taken in bands of GBAND; within a band the CTAs go
+// column pair by column pair (all the band's rows of pair c, then of c + 1), so the
+// CTAs resident at one time share a few row blocks and a few column blocks of X and
+// read them from L2, where a row-by-row order would stream a whole block row's
+// columns from HBM once per wave.
+constexpr int GBAND = 16;
+
+// CTA t -> (block row bi, column pair c) for nb block rows.
+__host__ __device__ inline void g_cta_block(int t, int nb, int& bi, int& c) {
+  // the band is the one holding t's block row in row-by-row order
+  int r = (int)(2.0f * sqrtf((float)t)) - 1;
+  if (r < 0) r = 0;
+  while (g_ctas_before(r + 1) <= t) ++r;
+  while (r > 0 && g_ctas_before(r) > t) --r;
+  const int b0 = r - r % GBAND;
+  const int gb = min(GBAND, nb - b0);  // rows in the band
+  int u = t - g_ctas_before(b0);
+  const int c_full = b0 / 2 + 1;       // pairs c with 2c <= b0: present in every row
+  if (u < c_full * gb) {
+    c = u / gb;
+    bi = b0 + u % gb;
+    return;
+  }
+  u -= c_full * gb;
+  for (c = c_full;; ++c) {             // pair c is in rows 2c .. b0 + gb - 1
+    const int nc = b0 + gb - 2 * c;
+    if (u < nc) {
+      bi = 2 * c + u;
+      return;
+    }
+    u -= nc;
+  }
+}
 
 __device__ __forceinline__ void tc_mma(uint32_t tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -123,14 +164,14 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a,
   __shared__ long long issued;  // chunks whose loads were issued
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // block (bi, bj), bj <= bi, of the lower block triangle
-  const int t = blockIdx.x;
-  int bi = (int)((sqrtf(8.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
-  while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
-  while (bi * (bi + 1) / 2 > t) --bi;
-  const int bj = t - bi * (bi + 1) / 2;
-  const int i0 = bi * GB, j0 = bj * GB;
-  const bool diag = bi == bj;
+  // blocks (bi, bj0) and (bi, bj0 + 1) of the lower block triangle, bj0 = 2c (one
+  // block when bj0 = bi): a 128 x 256 (or 128 x 128) product
+  int bi, cp;
+  g_cta_block(blockIdx.x, (a.k + GB - 1) / GB, bi, cp);
+  const int bj0 = 2 * cp;
+  const int nbj = bj0 + 1 <= bi ? 2 : 1;
+  const int nw = nbj * GB;  // output columns
+  const int i0 = bi * GB, j0 = bj0 * GB;
 
   if (tid == 0) {
     for (int s = 0; s < GSTAGES; ++s) {
@@ -157,7 +198,8 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a,
 
   if (warp == 1 && lane == 0) {
     // ---- producer: chunk c into stage c % GSTAGES, after the MMAs of chunk c - GSTAGES
-    const unsigned bytes = (diag ? 1 : 2) * G_TILE;
+    const bool diag = nbj == 1;  // the one-block tile is a diagonal block: B = A
+    const unsigned bytes = (diag ? 1 : 3) * G_TILE;
     long long c = 0;
     for (; c < nchunks; ++c) {
       const int st = (int)(c % GSTAGES);
@@ -172,10 +214,9 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a,
       mbar_arrive_expect_tx(&full_bar[st], bytes);
       tma_box(sA, &tmap, i0, y, &full_bar[st]);
       tma_box(sA + G_BOX, &tmap, i0 + 64, y, &full_bar[st]);
-      if (!diag) {
-        tma_box(sA + G_TILE, &tmap, j0, y, &full_bar[st]);
-        tma_box(sA + G_TILE + G_BOX, &tmap, j0 + 64, y, &full_bar[st]);
-      }
+      if (!diag)
+        for (int q = 0; q < 4; ++q)  // B: 64-feature boxes, LBO = G_BOX apart
+          tma_box(sA + G_TILE + q * G_BOX, &tmap, j0 + 64 * q, y, &full_bar[st]);
     }
     issued = c;
   } else if (warp == 0 && lane == 0) {
@@ -189,11 +230,12 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a,
       if (*(volatile int*)&abort_flag) break;
       tc_fence_after();
       const uint32_t aaddr = smem_u32(gsm + st * G_STAGE);
-      const uint32_t baddr = diag ? aaddr : aaddr + G_TILE;
+      const uint32_t baddr = nbj == 1 ? aaddr : aaddr + G_TILE;
+      const uint32_t idesc = g_idesc(nw);
       // K step s16 = rows 16 s16 .. 16 s16 + 15: two 8-row groups further (2 * SBO)
 #pragma unroll
       for (int s16 = 0; s16 < GK / 16; ++s16)
-        tc_mma(tmem, g_desc(aaddr + s16 * 2 * G_SBO), g_desc(baddr + s16 * 2 * G_SBO), G_IDESC,
+        tc_mma(tmem, g_desc(aaddr + s16 * 2 * G_SBO), g_desc(baddr + s16 * 2 * G_SBO), idesc,
                (c > 0 || s16 > 0) ? 1u : 0u);
       tc_commit(&empty_bar[st]);
     }
@@ -217,7 +259,7 @@ __global__ void __launch_bounds__(GTHREADS, 1) gram_kernel(GramArgs a,
   const int row = warp * 32 + lane;
   const int gi = i0 + row;
 #pragma unroll 1
-  for (int cb = 0; cb < GB / 32; ++cb) {
+  for (int cb = 0; cb < nw / 32; ++cb) {
     uint32_t v[32];
     const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cb * 32);
     asm volatile(
@@ -268,20 +310,20 @@ __global__ void __launch_bounds__(256) gram_diag_kernel(const float* H, int k, i
 }
 
 // H <- H / N on the lower block triangle (blocks of 128), H_ii += damp * mean(H_ii / N).
-// One CTA per 128-row stripe.
+// One CTA per row; row r covers columns 0 .. end of its diagonal block, read and
+// written once (coalesced, four independent loads in flight per thread).
 __global__ void __launch_bounds__(256) gram_finalize_kernel(float* H, int k, int64_t ldh,
                                                             double inv_n, double damp,
                                                             const double* diag_sum) {
   const double shift = damp * (*diag_sum) * inv_n / (double)k;
-  const int r0 = blockIdx.x * GB;
-  const int cend = min(k, r0 + GB);  // end of the stripe's diagonal block
-  for (int r = r0; r < min(k, r0 + GB); ++r) {
-    float* hr = H + (int64_t)r * ldh;
-    for (int c = threadIdx.x; c < cend; c += 256) {
-      double v = (double)hr[c] * inv_n;
-      if (c == r) v += shift;
-      hr[c] = (float)v;
-    }
+  const int r = blockIdx.x;
+  const int cend = min(k, (r / GB + 1) * GB);  // end of the row's diagonal block
+  float* hr = H + (int64_t)r * ldh;
+#pragma unroll 4
+  for (int c = threadIdx.x; c < cend; c += 256) {
+    double v = (double)hr[c] * inv_n;
+    if (c == r) v += shift;
+    hr[c] = (float)v;
   }
 }
 
@@ -325,18 +367,17 @@ int gram_accumulate_launch(const void* X, int64_t N, int k, int64_t ldx, float* 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return GPTQ2D_ERR_CUDA;
   }
-  const int blocks = nb * (nb + 1) / 2;
+  const int blocks = g_ctas_before(nb);
   GPTQ2D_LAUNCH(KC_OTHER, s, gram_kernel<<<blocks, GTHREADS, G_SMEM, s>>>(a, tmap));
   return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
 int gram_finalize_launch(float* H, int k, int64_t ldh, int64_t total_rows, double damp,
                          double* diag_sum, cudaStream_t s) {
-  const int nb = (k + GB - 1) / GB;
   GPTQ2D_LAUNCH(KC_OTHER, s, gram_diag_kernel<<<1, 256, 0, s>>>(H, k, ldh, diag_sum));
   GPTQ2D_LAUNCH(KC_OTHER, s,
-                gram_finalize_kernel<<<nb, 256, 0, s>>>(H, k, ldh, 1.0 / (double)total_rows, damp,
-                                                        diag_sum));
+                gram_finalize_kernel<<<k, 256, 0, s>>>(H, k, ldh, 1.0 / (double)total_rows, damp,
+                                                       diag_sum));
   return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
 }
 
