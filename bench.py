@@ -896,7 +896,8 @@ def run_gram(args):
     GPU.  Algorithmic work: the lower block triangle, rows * k * (k + 128) flops (the
     128-wide diagonal blocks are computed whole).  Timed with CUDA events, best of K steps
     after W warm-ups, against MEASURED_PEAKS.json's bf16 burst figure; the fp64 matmul that
-    forms the same Gram (torch, cuBLAS DGEMM) is timed beside it for context."""
+    forms the same Gram (torch, cuBLAS DGEMM) and cuBLAS's bf16 product X^T X (the whole
+    square, twice the triangle's work) are timed beside it for context."""
     import torch
     import two_sided_adaptive_b200 as g
     from two_sided_adaptive_b200 import build as gbuild
@@ -930,6 +931,9 @@ def run_gram(args):
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
+        sampler = ClockSampler(bus_id_of(dev))
+        sampler.start()
+        time.sleep(0.3)
         best = 1e30
         for _ in range(args.steps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -938,6 +942,7 @@ def run_gram(args):
             e1.record()
             torch.cuda.synchronize()
             best = min(best, e0.elapsed_time(e1))
+        clocks = sampler.stop()
         best_acc = 1e30  # gram_accumulate alone
         for _ in range(args.steps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -956,13 +961,28 @@ def run_gram(args):
         e1.record()
         torch.cuda.synchronize()
         t64 = e0.elapsed_time(e1)
-        del Xd, Xb, H
+        del Xd
+        # cuBLAS on the same bf16 operands (the whole square, fp32 accumulation), for
+        # context: best of 5
+        torch.matmul(Xb.T, Xb)
+        t16 = 1e30
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(Xb.T, Xb)
+            e1.record()
+            torch.cuda.synchronize()
+            t16 = min(t16, e0.elapsed_time(e1))
+        del Xb, H
         torch.cuda.empty_cache()
         out.append({"k": k, "rows": rows, "ms": best, "tflops": fl / (best * 1e-3) / 1e12,
                     "frac_of_bf16_peak": fl / (best * 1e-3) / 1e12 / peak,
+                    "clocks": clocks,
                     "accumulate_ms": best_acc,
                     "accumulate_tflops": fl / (best_acc * 1e-3) / 1e12,
-                    "fp64_matmul_ms": t64})
+                    "fp64_matmul_ms": t64,
+                    "cublas_bf16_square_ms": t16,
+                    "cublas_bf16_square_tflops": 2.0 * rows * k * k / (t16 * 1e-3) / 1e12})
     return {"metric": "Gram X^T X / N + damping from bf16 activations (tensor cores), TFLOP/s",
             "value": out[-1]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16 operands, f32 accumulation",
