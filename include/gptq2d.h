@@ -199,7 +199,8 @@ size_t gptq2d_gram_workspace_size(void);
 
 /* Accumulate the Gram of a batch of activation rows.
  *   X, x_dtype, rows, k, ldx : DEVICE, rows x k, GPTQ2D_BF16 only, row-major;
- *                              k and ldx multiples of 8, X 16-byte aligned.
+ *                              k and ldx multiples of 8, X 16-byte aligned;
+ *                              rows <= 2^31 - 1 (split larger batches into calls).
  *   H, ldh                   : DEVICE fp32 k x k.  The lower 128-block triangle
  *                              (every 128 x 128 block on or below the diagonal, so
  *                              every j <= i and a few j > i near the diagonal) is
@@ -211,7 +212,7 @@ size_t gptq2d_gram_workspace_size(void);
  * Products of bf16 values are exact in fp32; the sums are fp32 (tensor-core order).
  * rows == 0 with accumulate = 0 writes zeros.  k == 0 is a no-op.  A bounded
  * device-side wait that gives up sets the error word (read by gptq2d_gram_finalize
- * when it is given a HOST status pointer). */
+ * when it is given a HOST status pointer); H is then unspecified. */
 int gptq2d_gram_accumulate(const void* X, int x_dtype, int64_t rows, int64_t k, int64_t ldx,
                            float* H, int64_t ldh, int accumulate, void* ws, size_t ws_bytes,
                            void* stream);

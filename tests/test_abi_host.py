@@ -182,9 +182,10 @@ def _ga(L, **kw):
 
 @pytest.mark.parametrize("bad", [dict(dt=g.DTYPE_F32), dict(k=60, ldx=64, ldh=64), dict(ldx=68),
                                  dict(ldx=60), dict(X=4096 + 8), dict(H=None), dict(ldh=63),
-                                 dict(acc=2), dict(rows=-1), dict(X=None)])
+                                 dict(acc=2), dict(rows=-1), dict(X=None), dict(rows=2 ** 31)])
 def test_gram_accumulate_rejects_invalid_arguments(L, bad):
-    """Checked on the host: bf16 only, k and ldx multiples of 8, a 16-byte aligned X."""
+    """Checked on the host: bf16 only, k and ldx multiples of 8, a 16-byte aligned X,
+    rows that fit the 32-bit TMA row coordinate."""
     assert _ga(L, **bad) == g.Status.INVALID_ARG
 
 

@@ -58,6 +58,30 @@ def test_integer_activations_are_exact(g, rows, k):
     assert np.all(np.isnan(Hg[~m]))  # nothing outside the lower block triangle is written
 
 
+@pytest.mark.parametrize("rows,k", [(200, 5000), (65, 6664)])
+def test_many_tiles_per_cluster_pair_exact(g, rows, k):
+    """Widths with more 256 x 256 tiles than three per SM pair (210 and 351 tiles on
+    74 pairs): each pair reuses both tensor-memory accumulators, so the epilogue's
+    hand-back to the MMA thread is exercised.  Two batches (overwrite, then add)."""
+    rng = np.random.default_rng(rows + k)
+    X1 = rng.integers(-4, 5, (rows, k)).astype(np.float32)
+    X2 = rng.integers(-4, 5, (rows // 2 + 1, k)).astype(np.float32)
+    H = torch.full((k, k), float("nan"), dtype=torch.float32, device="cuda")
+    ws = _ws(g)
+    g.gram_accumulate(torch.from_numpy(X1).cuda().to(torch.bfloat16), H, accumulate=False,
+                      workspace=ws)
+    g.gram_accumulate(torch.from_numpy(X2).cuda().to(torch.bfloat16), H, accumulate=True,
+                      workspace=ws)
+    torch.cuda.synchronize()
+    Hg = H.cpu().numpy()
+    # small integers: every sum is exact in fp64 (and in fp32 on the GPU)
+    X1d, X2d = X1.astype(np.float64), X2.astype(np.float64)
+    ref = X1d.T @ X1d + X2d.T @ X2d
+    m = _lower_block_mask(k)
+    np.testing.assert_array_equal(Hg[m], ref[m].astype(np.float32))
+    assert np.all(np.isnan(Hg[~m]))
+
+
 def test_real_activations_within_fp32_bound(g):
     rng = np.random.default_rng(7)
     rows, k = 2048, 256

@@ -229,7 +229,9 @@ size_t gptq2d_gram_workspace_size(void) { return 256; }
 int gptq2d_gram_accumulate(const void* X, int x_dtype, int64_t rows, int64_t k, int64_t ldx,
                            float* H, int64_t ldh, int accumulate, void* ws, size_t ws_bytes,
                            void* stream) {
-  if (x_dtype != GPTQ2D_BF16 || rows < 0 || k < 0 || k > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  // rows: the TMA row coordinate is a 32-bit integer
+  if (x_dtype != GPTQ2D_BF16 || rows < 0 || rows > INT32_MAX || k < 0 || k > kMaxDim)
+    return GPTQ2D_ERR_INVALID_ARG;
   if (accumulate != 0 && accumulate != 1) return GPTQ2D_ERR_INVALID_ARG;
   if (k == 0) return GPTQ2D_OK;
   if (!H || ldh < k || k % 8 != 0) return GPTQ2D_ERR_INVALID_ARG;
