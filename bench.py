@@ -751,21 +751,24 @@ def run_configs(args):
 
 
 def run_kron3(args):
-    """A Hessian with three Kronecker factors: W is a 4096 x 64 x 64 tensor (a 4096 x 4096
-    layer whose input dimension is split into 64 groups of 64, each mode with its own
-    factor), H = H_1 kron H_2 kron H_3 with H_1 4096^2 and H_2, H_3 64^2, INT4 per-mode-1
-    absmax scales, W ~ N(0, 0.02^2) in bf16, Grams from Student-t(4) activations times
-    U(0.1, 10) column scales (4096 rows for H_1, 256 for H_2 and H_3) plus 1%
-    mean-diagonal damping, generated on the GPU.  One step = prepare(H_1), prepare(H_2),
-    prepare(H_3), kron_factor(M_2, M_3) and quantize of the 4096 x 4096 view, inputs
-    resident in HBM, timed with CUDA events over K steps after W warm-up steps."""
+    """Hessians with three Kronecker factors.  The line's workload: W is a 4096 x 64 x 64
+    tensor (a 4096 x 4096 layer whose input dimension is split into 64 groups of 64, each
+    mode with its own factor), H = H_1 kron H_2 kron H_3 with H_1 4096^2 and H_2, H_3
+    64^2; beside it a wide case, 1024 x 128 x 64 (n = 8192 columns: the right factor
+    dominates).  INT4 per-mode-1 absmax scales, W ~ N(0, 0.02^2) in bf16, Grams from
+    Student-t(4) activations times U(0.1, 10) column scales (4096 rows for a factor of
+    width >= 1024, else 4 x width) plus 1% mean-diagonal damping, generated on the GPU.
+    Two routes, each timed with CUDA events over K steps after W warm-up steps, inputs
+    resident in HBM:
+      per-mode: prepare(H_1), prepare(H_2), prepare(H_3), quantize_kron (the right
+                factor kept per mode; the line's value);
+      dense:    the same prepares, kron_factor(M_2, M_3) and quantize of the m x n view
+                with the n x n right factor."""
     import torch
     import two_sided_adaptive_b200 as g
     from two_sided_adaptive_b200 import build as gbuild
     gbuild.build()
     dev = torch.device("cuda", 0)
-    torch.manual_seed(77)
-    dims = (4096, 64, 64)
 
     def gram(width, rows):
         z = torch.randn(rows, width, device=dev, dtype=torch.float64)
@@ -777,54 +780,82 @@ def run_kron3(args):
         G.diagonal().add_(0.01 * G.diagonal().mean())
         return G.float()
 
-    Hs = [gram(d, 4096 if d == dims[0] else 4 * d) for d in dims]
-    m, n = dims[0], dims[1] * dims[2]
-    W = (torch.randn(dims, device=dev, dtype=torch.float32) * 0.02).to(torch.bfloat16)
-    W2 = W.reshape(m, n)
-    s = (W2.float().abs().amax(dim=1) / 7.0).clamp_min(1e-30).contiguous()
-    Ms = [torch.empty((d, d), dtype=torch.float64, device=dev) for d in dims]
-    wsP = [torch.empty(max(g.prepare_workspace_size(d), 256), dtype=torch.uint8, device=dev)
-           for d in dims]
-    MR = torch.empty((n, n), dtype=torch.float64, device=dev)
-    wsQ = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
-    Q = torch.empty((m, n), dtype=torch.int8, device=dev)
-    st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+    def case(dims, seed):
+        torch.manual_seed(seed)
+        Hs = [gram(d, 4096 if d >= 1024 else 4 * d) for d in dims]
+        m, n = dims[0], dims[1] * dims[2]
+        W = (torch.randn(dims, device=dev, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+        W2 = W.reshape(m, n)
+        s = (W2.float().abs().amax(dim=1) / 7.0).clamp_min(1e-30).contiguous()
+        Ms = [torch.empty((d, d), dtype=torch.float64, device=dev) for d in dims]
+        wsP = [torch.empty(max(g.prepare_workspace_size(d), 256), dtype=torch.uint8, device=dev)
+               for d in dims]
+        wsK = torch.empty(g.quantize_kron_workspace_size(m, dims[1:]), dtype=torch.uint8,
+                          device=dev)
+        Q = torch.empty((m, n), dtype=torch.int8, device=dev)
+        Qd = torch.empty((m, n), dtype=torch.int8, device=dev)
+        st = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+        std = torch.empty(g.STATS_WORDS, dtype=torch.int64, device=dev)
+        dense_ws = {}
 
-    def step(ev=None):
-        if ev:
-            ev[0].record()
-        for H, M, ws in zip(Hs, Ms, wsP):
-            g.prepare(H, out=M, workspace=ws, check=False)
-        g.kron_factor(Ms[1:], out=MR)
-        if ev:
-            ev[1].record()
-        g.quantize(W2, Ms[0], MR, s, 4, True, out=Q, stats=st, workspace=wsQ)
-        if ev:
-            ev[2].record()
+        def step(dense, ev=None):
+            if ev:
+                ev[0].record()
+            for H, M, ws in zip(Hs, Ms, wsP):
+                g.prepare(H, out=M, workspace=ws, check=False)
+            if dense:
+                g.kron_factor(Ms[1:], out=dense_ws["MR"])
+            if ev:
+                ev[1].record()
+            if dense:
+                g.quantize(W2, Ms[0], dense_ws["MR"], s, 4, True, out=Qd, stats=std,
+                           workspace=dense_ws["ws"])
+            else:
+                g.quantize_kron(W2, Ms[0], Ms[1:], s, 4, True, out=Q, stats=st, workspace=wsK)
+            if ev:
+                ev[2].record()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    tp = tq = 0.0
-    for _ in range(args.steps):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        step(ev)
-        torch.cuda.synchronize()
-        tp += ev[0].elapsed_time(ev[1])
-        tq += ev[1].elapsed_time(ev[2])
-    tp /= args.steps
-    tq /= args.steps
-    sd = g.stats_dict(st)
+        def timed(dense):
+            for _ in range(args.warmup):
+                step(dense)
+            torch.cuda.synchronize()
+            tp = tq = 0.0
+            for _ in range(args.steps):
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                step(dense, ev)
+                torch.cuda.synchronize()
+                tp += ev[0].elapsed_time(ev[1])
+                tq += ev[1].elapsed_time(ev[2])
+            return tp / args.steps, tq / args.steps
+
+        tp, tq = timed(False)
+        dense_ws["MR"] = torch.empty((n, n), dtype=torch.float64, device=dev)
+        dense_ws["ws"] = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
+        tpd, tqd = timed(True)
+        sd, sdd = g.stats_dict(st), g.stats_dict(std)
+        out = {"dims": list(dims), "ms_per_step": tp + tq, "entries_per_s": m * n / ((tp + tq) * 1e-3),
+               "prepare_ms": tp, "quantize_kron_ms": tq,
+               "per_mode_workspace_bytes": wsK.numel(),
+               "dense_route": {"ms_per_step": tpd + tqd, "prepare_and_kron_ms": tpd,
+                               "quantize_ms": tqd,
+                               "workspace_bytes": dense_ws["ws"].numel() + dense_ws["MR"].numel() * 8},
+               "routes_differ_at": int((Q != Qd).sum()), "status": sd["status"],
+               "dense_status": sdd["status"], "n_near_tie": sd["n_near_tie"],
+               "proxy_loss": sd["proxy_loss"], "dense_proxy_loss": sdd["proxy_loss"]}
+        del dense_ws["MR"], dense_ws["ws"], Hs, Ms, wsP, wsK
+        torch.cuda.empty_cache()
+        return out
+
+    main = case((4096, 64, 64), 77)
+    wide = case((1024, 128, 64), 78)
     return {"metric": "weight entries rounded per second, 3-factor Kronecker Hessian (INT4, 1 B200)",
-            "value": m * n / ((tp + tq) * 1e-3), "unit": "entries/s", "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tp + tq,
+            "value": main["entries_per_s"], "unit": "entries/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
             "higher_is_better": True, "dtype": "f64",
             "data": "synthetic (generated on the GPU, see run_kron3)",
-            "config": {"workload": "kron3", "dims": list(dims), "bits": 4,
-                       "step": "prepare x3 + kron_factor + quantize (4096 x 4096 view)"},
-            "phases": {"prepare_and_kron_ms": tp, "quantize_ms": tq,
-                       "quantize_fp64_tflops": m * n * (m + n) / (tq * 1e-3) / 1e12},
-            "status": sd["status"], "n_near_tie": sd["n_near_tie"]}
+            "config": {"workload": "kron3", "dims": main["dims"], "bits": 4,
+                       "step": "prepare x3 + quantize_kron (per-mode right factor)"},
+            "cases": [main, wide]}
 
 
 def run_grid128(args):

@@ -258,6 +258,46 @@ int gptq2d_gram_finalize(float* H, int64_t k, int64_t ldh, int64_t total_rows, d
 int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
                        double* out, int64_t ldo, void* stream);
 
+/* Bytes of device workspace gptq2d_quantize_kron needs for an m x prod(dims)
+ * rounding with these trailing modes; 0 when the per-mode path does not apply
+ * (see gptq2d_quantize_kron) or the arguments are out of range. */
+size_t gptq2d_quantize_kron_workspace_size(int64_t m, int nf, const int64_t* dims);
+
+/* The k-way rounding of gptq2d_kron_factor + gptq2d_quantize with the right factor
+ * kept per mode: M_R = M[0] (x) ... (x) M[nf-1] is never formed, and the right-hand
+ * error feedback is applied mode by mode (the separable feedback of the abstract's
+ * extension to several Kronecker factors).  With the normalised factors
+ * Lh_f = diag(M_f)^-1 M_f, the last factors whose sizes multiply to m_in form the
+ * inner group, where m_in is the largest product of a suffix of dims that divides 64
+ * (the tile width); the path applies when m_in >= 8.  Then a 64-column tile holds
+ * a = 64 / m_in consecutive indices of the outer modes, every block of the
+ * normalised right factor between two tiles is (an a x a block of the outer
+ * factors' product) (x) (the inner factor), and a tile's right feedback from
+ * tiles two or more to its left costs a multiply-adds per entry per source tile
+ * instead of a 64 x 64 x 64 product; the inner factor is applied once per tile.
+ * Memory: the factors as given plus O(m n); no n x n matrix.
+ *   W, w_dtype, m, ldw     : as gptq2d_quantize, W is m x n with n = prod dims
+ *                            (the tensor of shape (m, dims...) in C order).
+ *   M_L, ldl               : the mode-1 factor, as gptq2d_quantize's M_L.
+ *   nf, M, dims, ldm       : HOST arrays of nf <= GPTQ2D_MAX_KRON_FACTORS entries;
+ *                            M[f] a DEVICE fp64 lower factor of dims[f] x dims[f]
+ *                            (gptq2d_prepare of H_{f+2}), leading dimension
+ *                            ldm[f] >= dims[f]; strict upper triangles not read.
+ *                            prod dims <= 2^20.
+ *   scales, bits, clamp, Q, ldq, stats : as gptq2d_quantize.
+ *   ws, ws_bytes           : DEVICE workspace >= gptq2d_quantize_kron_workspace_size,
+ *                            256-byte aligned.
+ * The result is gptq2d_quantize's with M_R = gptq2d_kron_factor(M) up to the
+ * rounding order (the factor entries are formed as products of normalised entries):
+ * Q may differ only at near-ties.  Returns GPTQ2D_ERR_INVALID_ARG when the path does
+ * not apply (m_in < 8, e.g. a last mode of 3 or 100); the dense
+ * gptq2d_kron_factor + gptq2d_quantize route handles every shape. */
+int gptq2d_quantize_kron(const void* W, int w_dtype, int64_t m, int64_t ldw, const double* M_L,
+                         int64_t ldl, int nf, const double* const* M, const int64_t* dims,
+                         const int64_t* ldm, const float* scales, int bits, int clamp, int8_t* Q,
+                         int64_t ldq, gptq2d_stats* stats, void* ws, size_t ws_bytes,
+                         void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* Rounding                                                                    */
 /* ------------------------------------------------------------------------- */

@@ -249,3 +249,56 @@ def test_proxy_loss_rejects_invalid_arguments(L, bad):
 def test_proxy_loss_rejects_bad_workspace(L, ws, nbytes):
     assert L.gptq2d_proxy_loss(16, 0, 10, 6, 6, None, 6, 16, 4, 1, 16, 10, 16, 6, 16, ws, nbytes,
                                None) == g.Status.WORKSPACE
+
+
+def _qk(L, dims=(16, 16), nf=None, ws_bytes=None, **kw):
+    """gptq2d_quantize_kron with fake (never dereferenced) pointers: host checks only."""
+    nf = len(dims) if nf is None else nf
+    n = 1
+    for d in dims:
+        n *= d
+    a = dict(W=4096, dt=g.DTYPE_F32, m=32, ldw=n, ML=8192, ldl=32, S=12288,
+             bits=4, clamp=1, Q=16384, ldq=n, st=20480, ws=256)
+    a.update(kw)
+    k = max(len(dims), 1)
+    ptrs = (ctypes.c_void_p * k)(*([24576] * k))
+    da = (ctypes.c_int64 * k)(*dims)
+    lds = (ctypes.c_int64 * k)(*dims)
+    wsb = L.gptq2d_quantize_kron_workspace_size(a["m"], len(dims), da) if ws_bytes is None else ws_bytes
+    return L.gptq2d_quantize_kron(a["W"], a["dt"], a["m"], a["ldw"], a["ML"], a["ldl"], nf, ptrs,
+                                  da, lds, a["S"], a["bits"], a["clamp"], a["Q"], a["ldq"], a["st"],
+                                  a["ws"], wsb, None)
+
+
+def test_quantize_kron_workspace_size(L):
+    """Zero when the per-mode path does not apply or the sizes are out of range; else it
+    omits the n x n normalised right factor of the dense route."""
+    ws = lambda m, dims: L.gptq2d_quantize_kron_workspace_size(
+        m, len(dims), (ctypes.c_int64 * len(dims))(*dims))
+    assert ws(64, [5, 3]) == 0        # suffix products 3, 15: none divides 64 and is >= 8
+    assert ws(64, [128]) == 0         # 128 does not divide 64
+    assert ws(64, [4]) == 0           # 4 < 8
+    assert ws(64, [0]) == 0
+    assert ws(64, [2 ** 11, 2 ** 10]) == 0  # more than 2^20 columns
+    assert ws(64, [3, 8]) > 0 and ws(64, [64, 64]) > 0
+    n = 64 * 64
+    # the dense route's n x n right factor against the inner factor's 64 x 64
+    assert L.gptq2d_quantize_workspace_size(64, n) - ws(64, [64, 64]) >= 8 * (n * n - 64 * 64)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(nf=0), "INVALID_ARG"), (dict(nf=9), "INVALID_ARG"),
+    (dict(dims=(5, 3)), "INVALID_ARG"),             # the per-mode path does not apply
+    (dict(bits=9), "INVALID_ARG"), (dict(clamp=2), "INVALID_ARG"),
+    (dict(ldw=255), "INVALID_ARG"), (dict(ldl=31), "INVALID_ARG"), (dict(ldq=10), "INVALID_ARG"),
+    (dict(W=None), "INVALID_ARG"), (dict(st=None), "INVALID_ARG"), (dict(dt=7), "INVALID_ARG"),
+    (dict(ws_bytes=1024), "WORKSPACE"), (dict(ws=None), "WORKSPACE"), (dict(ws=272), "WORKSPACE"),
+])
+def test_quantize_kron_rejects_invalid_arguments(L, kw, code):
+    assert _qk(L, **kw) == getattr(g.Status, code)
+
+
+def test_quantize_kron_checks_pointers_before_any_launch(L):
+    """Valid sizes but host addresses: rejected as INVALID_ARG by the device-pointer
+    check (nothing is launched)."""
+    assert _qk(L) == g.Status.INVALID_ARG

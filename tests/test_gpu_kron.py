@@ -136,3 +136,93 @@ def test_quantize_tensor_end_to_end(g):
     assert g.stats_dict(st)["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
     assert O.proxy_loss_tensor(W.astype(np.float64), Q.cpu().numpy(), s.astype(np.float64), Hs) == \
         pytest.approx(rep.result.loss_identity, rel=1e-6)
+
+
+# The per-mode right factor (gptq2d_quantize_kron): trailing modes whose last sizes
+# multiply to m_in in {8, 16, 32, 64}.  Shapes with one to four outer modes, a tile
+# holding 1, 2, 4 or 8 outer indices, ragged last column and row tiles, and right
+# feedback two or more tiles away (n >= 192).
+PER_MODE = [(97, 16, 16), (70, 24, 32), (65, 3, 4, 16), (300, 6, 8, 8), (100, 12, 64),
+            (48, 2, 3, 2, 8), (200, 5, 16), (33, 3, 8), (130, 8, 8, 2),
+            (40, 2, 2, 2, 2, 2, 2, 2), (64, 4, 2), (130, 64)]
+
+
+@pytest.mark.parametrize("shape", PER_MODE, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("bits,clamp", [(4, True), (3, True), (4, False)])
+def test_per_mode_rounding_matches_oracle(g, shape, bits, clamp):
+    assert g.kron_inner_size(shape[1:]) > 0
+    W, Hs, s = _case(7 * bits + clamp, shape)
+    s = s if clamp else (s * 4).astype(np.float32)
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    W2 = torch.from_numpy(W.reshape(shape[0], -1)).cuda()
+    Q, st = g.quantize_kron(W2, torch.from_numpy(Ms[0]).cuda(),
+                            [torch.from_numpy(M).cuda() for M in Ms[1:]],
+                            torch.from_numpy(s).cuda(), bits, clamp)
+    torch.cuda.synchronize()
+    Qg = Q.cpu().numpy()
+    st = g.stats_dict(st)
+    s64 = s.astype(np.float64)
+    rep = check_against_oracle(W.reshape(shape[0], -1).astype(np.float64), Ms[0],
+                               O.kron_factor(Ms[1:]), s64, bits, clamp, Qg)
+    assert st["status"] == 0
+    assert st["n_clamped"] == rep.result.n_clamped
+    assert st["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+    if not rep.flips and len(shape) <= 4:
+        rk = O.gptq_kron_hyperplane(W.astype(np.float64), Ms, s64, bits, clamp)
+        np.testing.assert_array_equal(rk.Q.reshape(shape[0], -1), Qg)
+
+
+def test_per_mode_equals_the_dense_kronecker_factor(g):
+    """The two routes of the library agree entry for entry away from near-ties, and the
+    per-mode one needs no n x n matrix: its workspace is smaller by n^2 doubles, less
+    the inner factor's 64 x 64, at n = 768."""
+    shape = (128, 12, 64)
+    W, Hs, s = _case(3, shape)
+    Ms = [torch.from_numpy(O.reverse_cholesky(H)).cuda() for H in Hs]
+    W2 = torch.from_numpy(W.reshape(shape[0], -1)).cuda()
+    sc = torch.from_numpy(s).cuda()
+    Qk, stk = g.quantize_kron(W2, Ms[0], Ms[1:], sc, 4, True)
+    Qd, std = g.quantize(W2, Ms[0], g.kron_factor(Ms[1:]), sc, 4, True)
+    torch.cuda.synchronize()
+    a, b = g.stats_dict(stk), g.stats_dict(std)
+    diff = int((Qk != Qd).sum())
+    assert diff <= a["n_near_tie"] + b["n_near_tie"]
+    if diff == 0:
+        assert a["proxy_loss"] == pytest.approx(b["proxy_loss"], rel=1e-12)
+    n = 12 * 64
+    assert g.quantize_workspace_size(128, n) - g.quantize_kron_workspace_size(128, [12, 64]) >= \
+        8 * (n * n - 64 * 64)
+
+
+def test_per_mode_rejects_shapes_it_does_not_cover(g):
+    """A last mode of 3 (no suffix product of 8..64 dividing 64): INVALID_ARG, and the
+    workspace query says 0; quantize_tensor then takes the dense route."""
+    assert g.quantize_kron_workspace_size(16, [5, 3]) == 0
+    shape = (16, 5, 3)
+    W, Hs, s = _case(1, shape)
+    Ms = [torch.from_numpy(O.reverse_cholesky(H)).cuda() for H in Hs]
+    with pytest.raises(g.GPTQ2DError):
+        g.quantize_kron(torch.from_numpy(W.reshape(16, -1)).cuda(), Ms[0], Ms[1:],
+                        torch.from_numpy(s).cuda(), 4, True)
+    Q, st = g.quantize_tensor(torch.from_numpy(W).cuda(), [torch.from_numpy(H).cuda() for H in Hs],
+                              torch.from_numpy(s).cuda(), 4, True)
+    torch.cuda.synchronize()
+    assert g.stats_dict(st)["status"] == 0
+
+
+def test_quantize_tensor_per_mode_end_to_end(g):
+    """prepare each mode's factor on the GPU and round with the per-mode right factor
+    (the default route for these modes): the k-way tensor result and its loss."""
+    shape = (96, 6, 4, 16)
+    assert g.kron_inner_size(shape[1:]) == 64
+    W, Hs, s = _case(12, shape)
+    Q, st = g.quantize_tensor(torch.from_numpy(W).cuda(), [torch.from_numpy(H).cuda() for H in Hs],
+                              torch.from_numpy(s).cuda(), 4, True)
+    torch.cuda.synchronize()
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    rep = check_against_oracle(W.reshape(shape[0], -1).astype(np.float64), Ms[0],
+                               O.kron_factor(Ms[1:]), s.astype(np.float64), 4, True,
+                               Q.cpu().numpy().reshape(shape[0], -1))
+    assert g.stats_dict(st)["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+    assert O.proxy_loss_tensor(W.astype(np.float64), Q.cpu().numpy(), s.astype(np.float64), Hs) == \
+        pytest.approx(rep.result.loss_identity, rel=1e-6)

@@ -20,6 +20,7 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS", "quantize_grid",
+    "quantize_kron", "quantize_kron_workspace_size", "kron_inner_size",
     "gram_accumulate", "gram_finalize", "gram", "quantize_block", "block_workspace_size",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
     "round_host_workspace_size", "quantize_noalloc", "proxy_loss", "check_wait_timeout",
@@ -121,6 +122,13 @@ def lib():
                                            ctypes.c_size_t, _c_p, ctypes.POINTER(ctypes.c_int)]
         L.gptq2d_kron_factor.restype = ctypes.c_int
         L.gptq2d_kron_factor.argtypes = [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p]
+        L.gptq2d_quantize_kron_workspace_size.restype = ctypes.c_size_t
+        L.gptq2d_quantize_kron_workspace_size.argtypes = [_c_i64, ctypes.c_int, _c_p]
+        L.gptq2d_quantize_kron.restype = ctypes.c_int
+        L.gptq2d_quantize_kron.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_i64,
+                                           ctypes.c_int, _c_p, _c_p, _c_p, _c_p, ctypes.c_int,
+                                           ctypes.c_int, _c_p, _c_i64, _c_p, _c_p, ctypes.c_size_t,
+                                           _c_p]
         L.gptq2d_quantize_grid.restype = ctypes.c_int
         L.gptq2d_quantize_grid.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_i64,
                                            _c_p, _c_i64, ctypes.POINTER(_Grid), _c_p, _c_i64, _c_p,
@@ -438,16 +446,83 @@ def prepare_kron(Hs, *, stream=None, check: bool = True):
     return Ms[0], (Ms[1] if len(Ms) == 2 else kron_factor(Ms[1:], stream=stream))
 
 
+def kron_inner_size(dims) -> int:
+    """m_in of gptq2d_quantize_kron for these trailing modes: the largest product of a
+    suffix of ``dims`` dividing 64 when it is at least 8, else 0 (the per-mode path
+    does not apply)."""
+    p, best = 1, 0
+    for d in reversed([int(x) for x in dims]):
+        if d < 1 or p * d > 64 or 64 % (p * d) != 0:
+            break
+        p *= d
+        if p >= 8:
+            best = p
+    return best
+
+
+def quantize_kron_workspace_size(m: int, dims) -> int:
+    nf = len(dims)
+    arr = (_c_i64 * nf)(*[int(d) for d in dims])
+    return int(lib().gptq2d_quantize_kron_workspace_size(int(m), nf, arr))
+
+
 @_device_scoped
-def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, stream=None):
+def quantize_kron(W, M_L, Ms, scales, bits: int = 4, clamp: bool = True, *, out=None, stats=None,
+                  workspace=None, stream=None):
+    """The k-way rounding with the right factor kept per mode (gptq2d_quantize_kron): W is
+    the m x (m_2 ... m_k) matrix of the tensor, M_L = prepare(H_1), Ms = [prepare(H_2), ...,
+    prepare(H_k)].  Returns (Q int8 m x n, stats on the device)."""
+    torch = _torch()
+    _check_device(W, M_L, scales, out, stats, workspace, *Ms)
+    m, n = W.shape
+    if not 1 <= len(Ms) <= MAX_KRON_FACTORS:
+        raise ValueError(f"1 to {MAX_KRON_FACTORS} trailing factors")
+    for M in Ms:
+        if M.dtype != torch.float64 or M.dim() != 2 or M.shape[0] != M.shape[1]:
+            raise ValueError("factors must be square fp64 matrices")
+    dims = [int(M.shape[0]) for M in Ms]
+    if int(np.prod(dims)) != n:
+        raise ValueError("the factors' sizes must multiply to W's column count")
+    if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous fp32 vector of length m")
+    if M_L.dtype != torch.float64:
+        raise ValueError("factors must be fp64")
+    Q = out if out is not None else torch.empty((m, n), dtype=torch.int8, device=W.device)
+    st = stats if stats is not None else torch.empty(STATS_WORDS, dtype=torch.int64, device=W.device)
+    ws = _workspace(max(quantize_kron_workspace_size(m, dims), 256), W.device, workspace)
+    nf = len(Ms)
+    ptrs = (ctypes.c_void_p * nf)(*[M.data_ptr() for M in Ms])
+    dimsa = (_c_i64 * nf)(*dims)
+    lds = (_c_i64 * nf)(*[_ld(M) for M in Ms])
+    rc = lib().gptq2d_quantize_kron(W.data_ptr(), _dtype_code(W), m, _ld(W), M_L.data_ptr(),
+                                    _ld(M_L), nf, ptrs, dimsa, lds, scales.data_ptr(), int(bits),
+                                    int(clamp), Q.data_ptr(), _ld(Q), st.data_ptr(), ws.data_ptr(),
+                                    ws.numel(), _stream(stream))
+    if rc != Status.OK:
+        raise GPTQ2DError(rc, "gptq2d_quantize_kron")
+    return Q, st
+
+
+@_device_scoped
+def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, per_mode=None,
+                    stream=None):
     """GPTQ-2D rounding of a k-way tensor W (m_1 x ... x m_k, C order) under
     H_1 kron ... kron H_k with per-mode-1 scales: the m_1 x (m_2 ... m_k) problem with
-    M_L = prepare(H_1), M_R = M_2 kron ... kron M_k.  Returns (Q shaped like W, stats)."""
+    M_L = prepare(H_1) and the right factor M_2 kron ... kron M_k.  per_mode=None picks
+    the per-mode right factor (quantize_kron) when it applies to the trailing modes
+    (kron_inner_size > 0) and the dense Kronecker factor (kron_factor + quantize)
+    otherwise; True or False forces one.  Returns (Q shaped like W, stats)."""
     if W.dim() != len(Hs) or W.dim() < 2:
         raise ValueError("one Hessian factor per mode, at least two modes")
-    M_L, M_R = prepare_kron(Hs, stream=stream)
     W2 = W.reshape(W.shape[0], -1)
-    Q, st = quantize(W2, M_L, M_R, scales, bits, clamp, stream=stream)
+    dims = list(W.shape[1:])
+    use = kron_inner_size(dims) > 0 if per_mode is None else bool(per_mode)
+    if use:
+        Ms = [prepare(H, stream=stream) for H in Hs]
+        Q, st = quantize_kron(W2, Ms[0], Ms[1:], scales, bits, clamp, stream=stream)
+    else:
+        M_L, M_R = prepare_kron(Hs, stream=stream)
+        Q, st = quantize(W2, M_L, M_R, scales, bits, clamp, stream=stream)
     return Q.reshape(W.shape), st
 
 

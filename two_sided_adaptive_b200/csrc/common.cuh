@@ -213,12 +213,29 @@ struct GridSpec {
   int packed = 0;                 // two 4-bit codes per byte
 };
 
+// The right factor of a k-way rounding given per mode (gptq2d_quantize_kron):
+// M_R = M[0] (x) ... (x) M[nf-1], never formed.  The last factors whose sizes
+// multiply to m_in (8, 16, 32 or 64, a divisor of the 64-column tile) form the
+// inner group; kron_inner finds it.
+struct KronSpec {
+  int nf = 0;
+  const double* const* M = nullptr;  // HOST array of DEVICE pointers
+  const int64_t* dims = nullptr;
+  const int64_t* ldm = nullptr;
+};
+// m_in of these modes (the product of the longest suffix of dims dividing 64, when
+// it is at least 8), or 0 when the per-mode path does not apply; *nin = its factors.
+int kron_inner(int nf, const int64_t* dims, int* nin);
+size_t quantize_kron_ws_bytes(int64_t m, int nf, const int64_t* dims);
+
 // Optional row events: row_ev[k] is recorded once the tile rows 0..row_tile[k] of
-// Q are final (row_tile ascending), so a caller can copy them out early.
+// Q are final (row_tile ascending), so a caller can copy them out early.  With
+// `kron`, MR and ldr are unused and the workspace is quantize_kron_ws_bytes.
 int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const double* ML,
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
                     int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
                     cudaStream_t s, int n_row_ev = 0, const int* row_tile = nullptr,
-                    cudaEvent_t* row_ev = nullptr, const GridSpec* grid = nullptr);
+                    cudaEvent_t* row_ev = nullptr, const GridSpec* grid = nullptr,
+                    const KronSpec* kron = nullptr);
 
 }  // namespace gptq2d

@@ -56,6 +56,27 @@ namespace {
 constexpr int SLD = TB + 4;  // 68 doubles: [row][k] tiles (conflict-free DMMA fragments)
 constexpr int SWEEP_THREADS = 512;
 
+// The right factor given per mode (k-way rounding): R^ = Lh_0 (x) ... (x) Lh_{nf-1},
+// Lh_f = diag(M_f)^-1 M_f, generated where it is used.  A column j has the mixed-
+// radix digits d_f(j) = (j / stride_f) % dim_f (last factor fastest).  The last
+// nf - nout factors form the inner group of size m_in (dividing the tile width), so
+// a tile holds a = TB / m_in consecutive outer indices u = j / m_in, and a block of
+// R^ between tiles is (a x a outer block of Ah) (x) Lin, with Ah the outer factors'
+// product and Lin the inner one's.
+constexpr int KMAXF = 8;
+constexpr int KMAXA = 8;  // a = TB / m_in with m_in >= 8
+struct KronDesc {
+  int nf, nout;
+  int m_in, a;
+  int U;                    // outer extent n / m_in
+  int dim[KMAXF];
+  int ustride[KMAXF];       // stride_f / m_in for the outer factors
+  int vstride[KMAXF];       // stride_f for the inner factors
+  const double* M[KMAXF];   // the factors as given (lower, fp64)
+  int64_t ld[KMAXF];
+  const double* lin;        // Lin, m_in x m_in, unit diagonal, zero above (workspace)
+};
+
 struct QArgs {
   const void* W;
   int64_t ldw;
@@ -86,7 +107,27 @@ struct QArgs {
   double* dR;     // M_R[j,j] (np)
   TileStat* part; // Tm x Tn
   int Tm, Tn;
+  int kron;       // 1: the right factor is kd (Rh is not formed)
+  KronDesc kd;
 };
+
+// One normalised factor entry Lh_f[r][c]: 1 on the diagonal, M_f[r][c] / M_f[r][r]
+// below it, 0 above.
+__device__ __forceinline__ double kron_factor_entry(const KronDesc& k, int f, int r, int c) {
+  if (r == c) return 1.0;
+  if (c > r) return 0.0;
+  const double* Mf = k.M[f] + (int64_t)r * k.ld[f];
+  return Mf[c] / Mf[r];
+}
+// Ah[u][u'] (outer indices u, u' < U).
+__device__ __forceinline__ double kron_outer(const KronDesc& k, int u, int up) {
+  double v = 1.0;
+  for (int f = 0; f < k.nout && v != 0.0; ++f) {
+    const int r = (u / k.ustride[f]) % k.dim[f], c = (up / k.ustride[f]) % k.dim[f];
+    v *= kron_factor_entry(k, f, r, c);
+  }
+  return v;
+}
 
 // ---------------------------------------------------------------------------
 // small PTX helpers
@@ -130,6 +171,36 @@ __global__ void __launch_bounds__(256) normalize_kernel(QArgs a) {
   }
 }
 
+// The per-mode right factor's set-up: Lin (the inner group's normalised factor,
+// m_in x m_in, into the workspace) and dR[j] = M_R[j][j] = prod_f M_f[d_f(j)][d_f(j)]
+// (zero on the padding columns).  Grid-stride over m_in^2 + np entries.
+__global__ void __launch_bounds__(256) kron_setup_kernel(QArgs a) {
+  const KronDesc& k = a.kd;
+  const int64_t nlin = (int64_t)k.m_in * k.m_in, total = nlin + a.np;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    if (e < nlin) {
+      const int v = (int)(e / k.m_in), vp = (int)(e % k.m_in);
+      double x = 1.0;
+      for (int f = k.nout; f < k.nf && x != 0.0; ++f)
+        x *= kron_factor_entry(k, f, (v / k.vstride[f]) % k.dim[f], (vp / k.vstride[f]) % k.dim[f]);
+      const_cast<double*>(k.lin)[e] = x;
+    } else {
+      const int64_t j = e - nlin;
+      double d = 0.0;
+      if (j < a.n) {
+        d = 1.0;
+        const int u = (int)(j / k.m_in), v = (int)(j % k.m_in);
+        for (int f = 0; f < k.nf; ++f) {
+          const int r = f < k.nout ? (u / k.ustride[f]) % k.dim[f] : (v / k.vstride[f]) % k.dim[f];
+          d *= k.M[f][(int64_t)r * k.ld[f] + r];
+        }
+      }
+      a.dR[j] = d;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // the tile sweep
 // ---------------------------------------------------------------------------
@@ -162,7 +233,9 @@ constexpr int NSUB = TB / SUB;     // sub-tiles per tile edge
 // right of it (P[p][q'] += dW[p][q] Rh[q'][q]^T) and its final P below it
 // (V[p'][q] += Lh[p'][p] P[p][q]) as 8x8x8 FP64 tensor-core products, one warp
 // per target sub-tile.
-template <typename TW>
+// KRON: the right factor is given per mode (a.kron); a separate instantiation, so
+// that the dense route's code is not touched by it.
+template <typename TW, bool KRON>
 __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D, int I0) {
   extern __shared__ __align__(128) double sm[];
   double* Pt = sm;                 // P of the tile
@@ -185,12 +258,39 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   //   down:  V += Lh[I,I-1] P_final[I-1,J]   (warps 8..15)
   // All operand tiles and the tile's own P and E arrive in two async batches; the
   // two products run side by side on the DMMA units.
+  //   With the right factor given per mode, P holds the far-field sum before the
+  //   inner factor (see kron_push_kernel) and the right product is
+  //   P = (P + dW[I,J-1] mixed by the outer block Ah[J,J-1]) (I_a (x) Lin)^T.
   const bool has_r = J > 0, has_d = I > 0;
+  constexpr bool kron = KRON;
+  __shared__ double KN[KRON ? KMAXA : 1][KMAXA], KA[KRON ? KMAXA : 1][KMAXA];  // Ah[J,J-1], Ah[J,J]
+  if constexpr (KRON) {
+    if (tid < 2 * KMAXA * KMAXA) {
+      const KronDesc& k = a.kd;
+      const bool diag = tid >= KMAXA * KMAXA;
+      const int x = (tid % (KMAXA * KMAXA)) / KMAXA, y = tid % KMAXA;
+      const int u = J * k.a + x, up = (J - (diag ? 0 : 1)) * k.a + y;
+      const double v =
+          (x < k.a && y < k.a && u < k.U && up >= 0 && up < k.U) ? kron_outer(k, u, up) : 0.0;
+      (diag ? KA : KN)[x][y] = v;
+    }
+  }
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
     const int r = x >> 5, c2 = (x & 31) * 2;
     if (has_r) {
       cp_async16_zfill(Dt + r * SLD + c2, a.Dl + ts - TB + (int64_t)r * np + c2, true);
-      cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 - TB + c2, true);
+      if (kron && a.kd.a == 1) {  // I_a (x) Lin = Lin, [target column][source column]
+        cp_async16_zfill(Rt + r * SLD + c2, a.kd.lin + r * TB + c2, c0 + r < a.n);
+      } else if (kron) {
+        const int mi = a.kd.m_in;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = c2 + e;
+          Rt[r * SLD + c] = (r / mi == c / mi && c0 + r < a.n) ? a.kd.lin[(r % mi) * mi + c % mi] : 0.0;
+        }
+      } else {
+        cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 - TB + c2, true);
+      }
     }
     if (has_d) {
       cp_async16_zfill(Lt + r * SLD + c2, a.Lh + (int64_t)(r0 + r) * a.mp + r0 - TB + c2, true);
@@ -200,9 +300,19 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
   cp_async_commit_group();
   // far-field feedback reaches a tile only from two or more tiles away: P needs
   // J >= 2 and E needs I >= 2 (else zero; those buffers may not be zeroed yet)
+  // (with the right factor per mode, P is an operand of the right product: it goes
+  // with the first batch)
+  if constexpr (KRON) {
+    for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
+      const int r = x >> 5, c2 = (x & 31) * 2;
+      cp_async16_zfill(Pt + r * SLD + c2, J >= 2 ? a.P + ts + (int64_t)r * np + c2 : a.P, J >= 2);
+    }
+    cp_async_commit_group();
+  }
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
     const int r = x >> 5, c2 = (x & 31) * 2;
-    cp_async16_zfill(Pt + r * SLD + c2, J >= 2 ? a.P + ts + (int64_t)r * np + c2 : a.P, J >= 2);
+    if (!kron)
+      cp_async16_zfill(Pt + r * SLD + c2, J >= 2 ? a.P + ts + (int64_t)r * np + c2 : a.P, J >= 2);
     cp_async16_zfill(Vt + r * SLD + c2, I >= 2 ? a.E + ts + (int64_t)r * np + c2 : a.E, I >= 2);
   }
   cp_async_commit_group();
@@ -241,12 +351,29 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
                 ? to_f64(static_cast<const TW*>(a.W)[(int64_t)(r0 + r) * a.ldw + c0 + c])
                 : 0.0;
   }
-  cp_async_wait_group<1>();
+  if (kron) {
+    // P += dW[I,J-1] mixed by Ah[J,J-1]: column (x, v) of the tile takes
+    // sum_y Ah[Ja+x][(J-1)a+y] dW[I,J-1][., (y, v)]
+    cp_async_wait_group<1>();
+    __syncthreads();
+    if (has_r) {
+      const int mi = a.kd.m_in, na = a.kd.a;
+      for (int e = tid; e < TB * TB; e += SWEEP_THREADS) {
+        const int r = e >> 6, c = e & 63, xq = c / mi, v = c % mi;
+        double sacc = Pt[r * SLD + c];
+        for (int y = 0; y < na; ++y) sacc = fma(KN[xq][y], Dt[r * SLD + y * mi + v], sacc);
+        Pt[r * SLD + c] = sacc;
+      }
+    }
+  } else {
+    cp_async_wait_group<1>();
+  }
   __syncthreads();
   {
     // warp w8 = warp % 8 owns rows (w8>>1)*16..+16, columns (w8&1)*32..+32
     const int w8 = warp & 7, nr = (w8 >> 1) * 16, nc = (w8 & 1) * 32;
     const bool right = warp < 8;
+    const double* Ar = kron ? Pt : Dt;  // the right product's A operand
     double acc[2][4][2] = {};
     if (right ? has_r : has_d) {
 #pragma unroll 4
@@ -255,7 +382,7 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int r = nr + i * 8 + g;
-          av[i] = right ? Dt[r * SLD + kk + t4] : Lt[r * SLD + kk + t4];
+          av[i] = right ? Ar[r * SLD + kk + t4] : Lt[r * SLD + kk + t4];
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -271,20 +398,35 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
     cp_async_wait_group<0>();
     __syncthreads();
     double* C = right ? Pt : Vt;
+    const bool overwrite = right && kron;  // the mixed sum was the product's operand
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         double* c = C + (nr + i * 8 + g) * SLD + nc + j * 8 + 2 * t4;
-        c[0] += acc[i][j][0];
-        c[1] += acc[i][j][1];
+        c[0] = overwrite ? acc[i][j][0] : c[0] + acc[i][j][0];
+        c[1] = overwrite ? acc[i][j][1] : c[1] + acc[i][j][1];
       }
   }
   __syncthreads();
   // ---- W -> Dt, V += W; diagonal blocks of the normalised factors -> Rt, Lt
   for (int x = tid; x < TB * TB / 2; x += SWEEP_THREADS) {
     const int r = x >> 5, c2 = (x & 31) * 2;
-    cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 + c2, true);
+    if (kron && a.kd.a == 1) {
+      // Rh[J,J] = Lin; the sweep reads only its strictly lower part
+      cp_async16_zfill(Rt + r * SLD + c2, a.kd.lin + r * TB + c2, c0 + r < a.n);
+    } else if (kron) {  // Rh[J,J] = Ah[J,J] (x) Lin, strictly lower
+      const int mi = a.kd.m_in;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = c2 + e;
+        Rt[r * SLD + c] = (c < r && c0 + r < a.n)
+                              ? KA[r / mi][c / mi] * a.kd.lin[(r % mi) * mi + c % mi]
+                              : 0.0;
+      }
+    } else {
+      cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 + c2, true);
+    }
     cp_async16_zfill(Lt + r * SLD + c2, a.Lh + (int64_t)(r0 + r) * a.mp + r0 + c2, true);
   }
   cp_async_commit_group();
@@ -661,7 +803,8 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
     auto group_count = [&](int g) -> int {
       const bool dn = g >= pl.nt;
       const int I = pl.I0 + (dn ? g - pl.nt : g), J = pl.D - I;
-      return min(pl.cap, dn ? a.Tm - I - pl.dist0 : a.Tn - J - pl.dist0);
+      // (with the right factor given per mode, kron_push_kernel does the right tasks)
+      return min(pl.cap, dn ? a.Tm - I - pl.dist0 : (a.kron ? 0 : a.Tn - J - pl.dist0));
     };
     unsigned help_done = 0;  // help groups found empty
     for (int g = next_group(); ok; g = next_group()) {
@@ -798,6 +941,68 @@ __global__ void __launch_bounds__(FAR_THREADS, 1) far_kernel(QArgs a, FarPlan pl
   if (lane == 0) atomicExch(a.err, 1);  // a wait gave up
 }
 
+// Far-field right feedback with the right factor given per mode.  The product
+// dW[I,J] Rh[J',J]^T (J' >= J + 2) factors as (dW[I,J] mixed by the outer block
+// Ah[J',J]) (I_a (x) Lin)^T, and the inner factor is common to every source of a
+// target, so the sources add only their mixed dW into P[I,J'] (column (x, v) takes
+// sum_y Ah[J'a+x][Ja+y] dW[I,J][., (y, v)]: a multiply-adds per entry, no product);
+// the target's sweep applies Lin once, with its near neighbour (sweep_kernel).  One
+// CTA per source tile of wavefront D and run of KP_RUN targets (one: a late
+// wavefront has few sources, and a CTA's targets run one after another), with
+// dW[I,J] read into shared memory from L2.  Each entry of P gets one addition per
+// launch (one source per tile row on a wavefront), so the sums do not depend on the
+// order of the CTAs.
+constexpr int KP_RUN = 1;
+constexpr int KP_THREADS = 256;
+constexpr int KP_SMEM = TB * SLD * (int)sizeof(double);
+
+inline __host__ __device__ int kp_targets(int J, int Tn) { return Tn - J - 2 > 0 ? Tn - J - 2 : 0; }
+
+__global__ void __launch_bounds__(KP_THREADS) kron_push_kernel(QArgs a, int D, int I0, int nt) {
+  extern __shared__ __align__(16) double dws[];  // dW[I,J], row stride SLD
+  __shared__ double cc[KMAXA][KMAXA];
+  const KronDesc& k = a.kd;
+  // this CTA's source tile and run of targets
+  int b = blockIdx.x, i = 0;
+  for (; i < nt; ++i) {
+    const int runs = (kp_targets(D - (I0 + i), a.Tn) + KP_RUN - 1) / KP_RUN;
+    if (b < runs) break;
+    b -= runs;
+  }
+  if (i >= nt) return;
+  const int I = I0 + i, J = D - I;
+  const int rows = min(TB, a.m - I * TB);
+  const int t0 = J + 2 + b * KP_RUN, t1 = min(a.Tn, t0 + KP_RUN);
+  const int64_t np = a.np;
+  const double* src = a.Dl + (int64_t)I * TB * np + (int64_t)J * TB;
+  for (int x = threadIdx.x; x < TB * TB / 2; x += KP_THREADS) {
+    const int r = x >> 5, c2 = (x & 31) * 2;
+    cp_async16_zfill(dws + r * SLD + c2, src + (int64_t)r * np + c2, true);
+  }
+  cp_async_commit_group();
+  const int mi = k.m_in, na = k.a;
+  for (int Jt = t0; Jt < t1; ++Jt) {
+    if (threadIdx.x < KMAXA * KMAXA) {
+      const int x = threadIdx.x / KMAXA, y = threadIdx.x % KMAXA;
+      const int u = Jt * na + x, up = J * na + y;
+      cc[x][y] = (x < na && y < na && u < k.U && up < k.U) ? kron_outer(k, u, up) : 0.0;
+    }
+    cp_async_wait_group<0>();
+    __syncthreads();
+    const int cols = min(TB, a.n - Jt * TB);
+    double* dst = a.P + (int64_t)I * TB * np + (int64_t)Jt * TB;
+    for (int e = threadIdx.x; e < TB * TB; e += KP_THREADS) {
+      const int r = e >> 6, c = e & 63;
+      if (r >= rows || c >= cols) continue;
+      const int xq = c / mi, v = c % mi;
+      double acc = 0.0;
+      for (int y = 0; y < na; ++y) acc = fma(cc[xq][y], dws[r * SLD + y * mi + v], acc);
+      red_add(dst + (int64_t)r * np + c, acc);
+    }
+    __syncthreads();  // cc is rewritten for the next target
+  }
+}
+
 // Sums the per-tile statistics in a fixed order into the caller's gptq2d_stats.
 __global__ void __launch_bounds__(256) finalize_kernel(const TileStat* part, int ntiles,
                                                        const int* err, gptq2d_stats* out) {
@@ -854,7 +1059,7 @@ __global__ void zero_stats_kernel(gptq2d_stats* out) {
 struct WsLayout {
   int64_t mp, np;
   int Tm, Tn;
-  size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_part, off_cnt, total;
+  size_t off_Lh, off_Rh, off_P, off_E, off_D, off_dL, off_dR, off_lin, off_part, off_cnt, total;
   int n_cnt;  // far-field plans (MAX_GROUPS group counters each)
 };
 
@@ -865,7 +1070,8 @@ inline int wave_tiles(int D, int Tm, int Tn) {
   return std::min(D, Tm - 1) - wave_i0(D, Tn) + 1;
 }
 
-WsLayout layout(int64_t m, int64_t n) {
+// m_in > 0: the right factor is given per mode (no Rh; Lin of m_in x m_in instead).
+WsLayout layout(int64_t m, int64_t n, int m_in = 0) {
   WsLayout L;
   L.mp = round_up(m, TB);
   L.np = round_up(n, TB);
@@ -874,12 +1080,13 @@ WsLayout layout(int64_t m, int64_t n) {
   const size_t mat = align256((size_t)L.mp * L.np * sizeof(double));
   size_t o = 0;
   L.off_Lh = o; o += align256((size_t)L.mp * L.mp * sizeof(double));
-  L.off_Rh = o; o += align256((size_t)L.np * L.np * sizeof(double));
+  L.off_Rh = o; o += m_in > 0 ? 0 : align256((size_t)L.np * L.np * sizeof(double));
   L.off_P = o; o += mat;
   L.off_E = o; o += mat;
   L.off_D = o; o += mat;
   L.off_dL = o; o += align256(L.mp * sizeof(double));
   L.off_dR = o; o += align256(L.np * sizeof(double));
+  L.off_lin = o; o += align256((size_t)m_in * m_in * sizeof(double));
   L.off_part = o; o += align256((size_t)L.Tm * L.Tn * sizeof(TileStat));
   L.n_cnt = 0;
   for (int D = 0; D < L.Tm + L.Tn - 1; ++D)  // one far-field plan per MAX_GROUPS/2 tiles
@@ -889,14 +1096,16 @@ WsLayout layout(int64_t m, int64_t n) {
   return L;
 }
 
-std::atomic<uint64_t> g_sweep_smem_set[3];
+std::atomic<uint64_t> g_sweep_smem_set[6];  // per weight type, dense and per mode
 std::atomic<uint64_t> g_far_smem_set{0};
 
 template <typename TW>
 int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s, int wslot,
                int n_row_ev, const int* row_tile, cudaEvent_t* row_ev) {
   constexpr int SW_SMEM = sweep_smem_bytes<TW>();
-  if (ensure_smem(sweep_kernel<TW>, SW_SMEM, g_sweep_smem_set[wslot]) != cudaSuccess ||
+  if (ensure_smem(sweep_kernel<TW, false>, SW_SMEM, g_sweep_smem_set[wslot]) != cudaSuccess ||
+      (a.kron &&
+       ensure_smem(sweep_kernel<TW, true>, SW_SMEM, g_sweep_smem_set[3 + wslot]) != cudaSuccess) ||
       ensure_smem(far_kernel, FAR_SMEM, g_far_smem_set) != cudaSuccess)
     return GPTQ2D_ERR_CUDA;
   DevStreams* ds = nullptr;
@@ -913,7 +1122,13 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
   // them); zero P and E and the counters on the low-priority one, where only the
   // far-field launches, which run after it, write them (the sweeps of tiles with
   // I < 2 or J < 2, which get no far-field feedback, do not read them)
-  GPTQ2D_LAUNCH(KC_OTHER, hi, normalize_kernel<<<(int)(L.mp + L.np), 256, 0, hi>>>(a));
+  GPTQ2D_LAUNCH(KC_OTHER, hi,
+                normalize_kernel<<<(int)(a.kron ? L.mp : L.mp + L.np), 256, 0, hi>>>(a));
+  if (a.kron) {
+    const int64_t work = (int64_t)a.kd.m_in * a.kd.m_in + L.np;
+    const int blocks = (int)std::min<int64_t>((work + 255) / 256, 4 * (int64_t)ds->sms);
+    GPTQ2D_LAUNCH(KC_OTHER, hi, kron_setup_kernel<<<blocks, 256, 0, hi>>>(a));
+  }
   ok = ok && cudaMemsetAsync(a.P, 0, (size_t)(L.off_D - L.off_P), lo) == cudaSuccess;
   int* counters = a.err + 1;
   ok = ok && cudaMemsetAsync(a.err, 0, (1 + (size_t)L.n_cnt * MAX_GROUPS) * sizeof(int), lo) ==
@@ -937,7 +1152,8 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
       ok = cudaStreamWaitEvent(hi, ds->far[(D - 2) % RING], 0) == cudaSuccess;
     far_recorded[D % RING] = false;
     GPTQ2D_LAUNCH(KC_SWEEP, hi,
-                  sweep_kernel<TW><<<nt, SWEEP_THREADS, SW_SMEM, hi>>>(a, D, I0));
+                  (a.kron ? sweep_kernel<TW, true> : sweep_kernel<TW, false>)<<<nt, SWEEP_THREADS,
+                                                                               SW_SMEM, hi>>>(a, D, I0));
     // tile row I is final after the sweep of its last tile, on wavefront I + Tn - 1
     for (int k = 0; k < n_row_ev && ok; ++k)
       if (D == row_tile[k] + a.Tn - 1) ok = cudaEventRecord(row_ev[k], hi) == cudaSuccess;
@@ -948,13 +1164,18 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
     prev_plans.clear();
     prev_b.clear();
 
-    // band products of wavefront D to tiles two or more tiles away
-    long long total = 0;
+    // band products of wavefront D to tiles two or more tiles away (with the right
+    // factor given per mode, the right ones are kron_push_kernel's mixed adds)
+    long long total = 0, kp_runs = 0;
     for (int i = 0; i < nt; ++i) {
       const int I = I0 + i, J = D - I;
-      total += std::max(0, a.Tn - J - 2) + std::max(0, a.Tm - I - 2);
+      if (a.kron)
+        kp_runs += (kp_targets(J, a.Tn) + KP_RUN - 1) / KP_RUN;
+      else
+        total += std::max(0, a.Tn - J - 2);
+      total += std::max(0, a.Tm - I - 2);
     }
-    if (total == 0) continue;
+    if (total == 0 && kp_runs == 0) continue;
     const int nt_next = wave_tiles(D + 1, a.Tm, a.Tn);
     const int a_ctas = std::max(sms / 4, sms - nt_next);
     // a second launch pays when the work outlasts the next sweep on a_ctas SMs
@@ -978,7 +1199,8 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
       int nonempty = 0;
       for (int gidx = 0; gidx < G; ++gidx) {
         const int I = pl.I0 + (gidx < pl.nt ? gidx : gidx - pl.nt), J = D - I;
-        cnt[gidx] = gidx < pl.nt ? std::max(0, a.Tn - J - 2) : std::max(0, a.Tm - I - 2);
+        cnt[gidx] = gidx < pl.nt ? (a.kron ? 0 : std::max(0, a.Tn - J - 2))
+                                 : std::max(0, a.Tm - I - 2);
         tasks += cnt[gidx];
         nonempty += cnt[gidx] > 0;
       }
@@ -1028,6 +1250,9 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
         prev_b.push_back(b_ctas);
       }
     }
+    if (kp_runs > 0)
+      GPTQ2D_LAUNCH(KC_PROPAGATE, lo,
+                    kron_push_kernel<<<(int)kp_runs, KP_THREADS, KP_SMEM, lo>>>(a, D, I0, nt));
     ok = ok && cudaEventRecord(ds->far[D % RING], lo) == cudaSuccess;
     far_recorded[D % RING] = true;
   }
@@ -1042,6 +1267,30 @@ int launch_all(QArgs& a, const WsLayout& L, gptq2d_stats* stats, cudaStream_t s,
 }  // namespace
 
 size_t quantize_ws_bytes(int64_t m, int64_t n) { return layout(m, n).total; }
+
+int kron_inner(int nf, const int64_t* dims, int* nin) {
+  int64_t p = 1;
+  int best = 0, cnt = 0;
+  for (int f = nf - 1; f >= 0; --f) {
+    if (dims[f] < 1 || p * dims[f] > TB || TB % (p * dims[f]) != 0) break;
+    p *= dims[f];
+    ++cnt;
+    if (p >= 8) {
+      best = (int)p;
+      *nin = cnt;
+    }
+  }
+  return best;
+}
+
+size_t quantize_kron_ws_bytes(int64_t m, int nf, const int64_t* dims) {
+  int nin = 0;
+  const int m_in = kron_inner(nf, dims, &nin);
+  if (m_in == 0) return 0;
+  int64_t n = 1;
+  for (int f = 0; f < nf; ++f) n *= dims[f];
+  return layout(m, n, m_in).total;
+}
 
 namespace {
 __device__ int g_wait_status;
@@ -1065,12 +1314,15 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
                     int64_t ldl, const double* MR, int64_t ldr, const float* scales, int bits,
                     int clamp, int8_t* Q, int64_t ldq, gptq2d_stats* stats, void* ws,
                     cudaStream_t s, int n_row_ev, const int* row_tile, cudaEvent_t* row_ev,
-                    const GridSpec* grid) {
+                    const GridSpec* grid, const KronSpec* kron) {
   if (m == 0 || n == 0) {
     GPTQ2D_LAUNCH(KC_OTHER, s, zero_stats_kernel<<<1, 1, 0, s>>>(stats));
     return cudaGetLastError() == cudaSuccess ? GPTQ2D_OK : GPTQ2D_ERR_CUDA;
   }
-  const WsLayout L = layout(m, n);
+  int nin = 0;
+  const int m_in = kron ? kron_inner(kron->nf, kron->dims, &nin) : 0;
+  if (kron && (m_in == 0 || kron->nf > KMAXF)) return GPTQ2D_ERR_INVALID_ARG;
+  const WsLayout L = layout(m, n, m_in);
   char* base = static_cast<char*>(ws);
   QArgs a;
   a.W = W;
@@ -1107,6 +1359,26 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
   a.err = reinterpret_cast<int*>(base + L.off_cnt);
   a.Tm = L.Tm;
   a.Tn = L.Tn;
+  a.kron = kron ? 1 : 0;
+  a.kd = KronDesc{};
+  if (kron) {
+    KronDesc& k = a.kd;
+    k.nf = kron->nf;
+    k.nout = kron->nf - nin;
+    k.m_in = m_in;
+    k.a = TB / m_in;
+    k.U = n / m_in;
+    int64_t stride = 1;
+    for (int f = k.nf - 1; f >= 0; --f) {
+      k.dim[f] = (int)kron->dims[f];
+      k.M[f] = kron->M[f];
+      k.ld[f] = kron->ldm[f];
+      k.vstride[f] = f >= k.nout ? (int)stride : 1;
+      k.ustride[f] = f < k.nout ? (int)(stride / m_in) : 1;
+      stride *= kron->dims[f];
+    }
+    k.lin = reinterpret_cast<const double*>(base + L.off_lin);
+  }
   int rc;
   switch (w_dtype) {
     case GPTQ2D_F32: rc = launch_all<float>(a, L, stats, s, 0, n_row_ev, row_tile, row_ev); break;
