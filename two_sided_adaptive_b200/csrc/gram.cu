@@ -7,43 +7,45 @@
 // is GPTQ's usual one; the pages give none.
 //
 // gram_kernel: persistent CTA pairs (clusters of two CTAs on neighbouring SMs, one
-// pair per two SMs) over the 256 x 256 tiles (BI, BJ), BJ <= BI, of the lower
-// triangle of 256-blocks of H; pair p takes tiles p, p + pairs, ... of the order
-// below.  A tile is D = X[:, I]^T X[:, J] over all rows, accumulated in fp32 in
-// tensor memory by tcgen05.mma.cta_group::2 (kind::f16, bf16 operands, M = N = 256,
-// K = 16 per instruction): CTA r of the pair holds rows 128 r .. 128 r + 127 of A
-// (features 256 BI + 128 r ..) and columns 128 r .. of B (features 256 BJ + 128 r ..)
-// in its own shared memory, and receives rows 128 r .. of D (all 256 columns) in its
-// own tensor memory.  Per 2^20 flops each SM moves 8 KB of operands from shared
-// memory into the MMA, where a one-SM 128 x 256 tile moves 12 KB.  Both operands are
-// chunks of 64 rows of X, and X is row-major (features contiguous), so A and B are
-// "MN-major".  Each operand half is two TMA boxes of 64 features x 64 rows
-// (cp.async.bulk.tensor, 128-byte swizzle; zero fill past the last row or
-// column): a box holds the rows as 128-byte lines, swizzled in groups of 8 lines,
-// which is the canonical 128B-swizzled MN-major layout of the operand descriptor
-// (stride byte offset 1024 between 8-row groups, leading byte offset 8192 between
-// the two 64-feature boxes).  On a diagonal tile B = A in each CTA.
-//   warp 1, one thread  (both CTAs) fills a 6-stage ring, chunk after chunk, tile
+// pair per two SMs) over the 256 x 512 tiles (BI, C) of the lower triangle of H:
+// rows 256 BI .. 256 BI + 255 and columns 512 C .. 512 C + 511, 2C <= BI; pair p
+// takes tiles p, p + pairs, ... of the order below.  A tile is D = X[:, I]^T X[:, J]
+// over all rows, accumulated in fp32 in tensor memory by two
+// tcgen05.mma.cta_group::2 products per 16 rows (kind::f16, bf16 operands, M = N =
+// 256, K = 16 per instruction), one per 256-column half, sharing A: CTA r of the
+// pair holds rows 128 r .. 128 r + 127 of A (features 256 BI + 128 r ..) and
+// columns 128 r .. of each half of B in its own shared memory, and receives rows
+// 128 r .. of D (all 512 columns, the whole tensor memory) in its own tensor memory.
+// Per 2^20 flops each SM loads 6 KB of operands from L2 (8 KB for a 256 x 256 tile,
+// 12 KB for a one-SM 128 x 256 one).  Both operands are chunks of 64 rows of X, and
+// X is row-major (features contiguous), so A and B are "MN-major".  Each operand
+// half is two TMA boxes of 64 features x 64 rows (cp.async.bulk.tensor, 128-byte
+// swizzle; zero fill past the last row or column): a box holds the rows as 128-byte
+// lines, swizzled in groups of 8 lines, which is the canonical 128B-swizzled
+// MN-major layout of the operand descriptor (stride byte offset 1024 between 8-row
+// groups, leading byte offset 8192 between the two 64-feature boxes).  When the
+// first half of B is A's own block (2C = BI) it is not loaded again; when the
+// second half lies above the diagonal (2C + 1 > BI) it is neither loaded nor
+// multiplied.
+//   warp 1, one thread  (both CTAs) fills a 4-stage ring, chunk after chunk, tile
 //                       after tile: it waits for the stage's empty barrier and
 //                       issues its CTA's box loads, which complete on the
 //                       LEADER's full barrier (.cta_group::2); the leader's thread
 //                       first arms that barrier with both CTAs' bytes;
 //   warp 0              (both CTAs) allocates all 512 columns of tensor memory for
-//                       the pair: two 256-column accumulators, tile t in
-//                       accumulator t % 2.  In the leader (rank 0) one thread waits
-//                       until both CTAs' epilogues have emptied the accumulator,
-//                       then, per full stage, issues the stage's four MMAs and
-//                       frees the stage in both CTAs with a multicast
-//                       tcgen05.commit; after a tile's last chunk a multicast
-//                       commit marks the accumulator full in both CTAs;
-//   warps 2..5          (both CTAs, the epilogue) wait for a full accumulator, read
-//                       their 32 lanes (rows) of it with tcgen05.ld, 32 columns at
-//                       a time, tell the leader it is empty, and write (or add) the
-//                       rows into H, each 32 x 32 chunk turned around in shared
+//                       the pair.  In the leader (rank 0) one thread waits until
+//                       both CTAs' epilogues have read the previous tile, then, per
+//                       full stage, issues the stage's MMAs and frees the stage in
+//                       both CTAs with a multicast tcgen05.commit; after a tile's
+//                       last chunk a multicast commit marks the accumulator full in
+//                       both CTAs;
+//   warps 2..5          (both CTAs, the epilogue) wait for the full accumulator,
+//                       read their 32 lanes (rows) of it with tcgen05.ld, 32 columns
+//                       at a time, tell the leader it is read, and write (or add)
+//                       the rows into H, each 32 x 32 chunk turned around in shared
 //                       memory so that a store writes 32 consecutive floats of one
-//                       row; the 128 x 128 block above the diagonal of a diagonal
-//                       tile is skipped.  This runs beside the next tile's loads
-//                       and MMAs.
+//                       row; 128 x 128 blocks above the diagonal are skipped.  The
+//                       next tile's loads run meanwhile; its MMAs wait for the read.
 // Every wait is bounded (%globaltimer); a wait that gives up sets the error word and
 // stops the pair (H is then unspecified); the pair lets copies in flight land (a
 // fixed 200 us) and exchanges the outcome across the cluster before either frees
@@ -65,16 +67,16 @@ namespace {
 constexpr int GB = 128;                      // block edge of H's lower block triangle
 constexpr int GT = 2 * GB;                   // tile edge of a CTA pair (MMA M = N)
 constexpr int GK = 64;                       // rows of X per stage
-constexpr int GSTAGES = 6;
+constexpr int GSTAGES = 4;
 constexpr int GTHREADS = 192;                // warp 0 MMA, warp 1 loads, warps 2..5 epilogue
 constexpr int G_BOX = 64 * GK * 2;           // one TMA box: 64 features x 64 rows, 8 KB
 constexpr int G_TILE = 2 * G_BOX;            // one CTA's operand half, 128 features: 16 KB
-constexpr int G_STAGE = 2 * G_TILE;          // A half and B half
+constexpr int G_STAGE = 3 * G_TILE;          // A half and two B halves
 constexpr int G_TR = 4 * 32 * 33 * 4;       // the epilogue warps' 32 x 32 transposes
 constexpr int G_SMEM = GSTAGES * G_STAGE + G_TR + 1024;  // + room to align the ring to 1024 bytes
 constexpr uint32_t G_SBO = 1024;             // between 8-row groups
 constexpr uint32_t G_LBO = G_BOX;            // between the two 64-feature boxes
-constexpr uint32_t G_TMEM_COLS = 2 * GT;     // two fp32 accumulators of 128 lanes x 256 columns
+constexpr uint32_t G_TMEM_COLS = 2 * GT;     // fp32 accumulator: 128 lanes x 512 columns
 constexpr unsigned long long G_DRAIN_NS = 200000;  // copies in flight after a timeout
 
 // Shared-memory operand descriptor: start address, leading and stride byte offsets
@@ -122,39 +124,40 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x
 constexpr uint32_t G_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                              ((uint32_t)(GT >> 3) << 17) | ((uint32_t)(GT >> 4) << 24);
 
-// Tiles of tile rows 0 .. B - 1 (row BI holds BI + 1 of them).
-__host__ __device__ inline int g_tiles_before(int B) { return B * (B + 1) / 2; }
+// Tiles of tile rows 0 .. B - 1: row BI holds the column pairs C with 2C <= BI.
+__host__ __device__ inline int g_tiles_before(int B) { return (B + 1) * (B + 1) / 4; }
 
 // Tile order.  Tile rows are taken in bands of GBAND; within a band the pairs go
-// column by column (all the band's rows of column BJ, then of BJ + 1), so the pairs
-// resident at one time share a few row blocks and a few column blocks of X and read
-// them from L2, where a row-by-row order would stream a whole tile row's columns
-// from HBM once per wave.
+// column pair by column pair (all the band's rows of pair C, then of C + 1), so the
+// CTA pairs resident at one time share a few row blocks and a few column blocks of
+// X and read them from L2, where a row-by-row order would stream a whole tile row's
+// columns from HBM once per wave.
 constexpr int GBAND = 8;
 
-// Pair t -> tile (BI, BJ) for NB tile rows.
-__host__ __device__ inline void g_pair_tile(int t, int NB, int& BI, int& BJ) {
+// Pair t -> tile (BI, C) for NB tile rows: rows 256 BI .., columns 512 C ...
+__host__ __device__ inline void g_pair_tile(int t, int NB, int& BI, int& C) {
   // the band is the one holding t's tile row in row-by-row order
-  int r = (int)((sqrtf(8.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
+  int r = (int)(2.0f * sqrtf((float)t)) - 1;
   if (r < 0) r = 0;
   while (g_tiles_before(r + 1) <= t) ++r;
   while (r > 0 && g_tiles_before(r) > t) --r;
   const int b0 = r - r % GBAND;
   const int gb = min(GBAND, NB - b0);  // rows in the band
   int u = t - g_tiles_before(b0);
-  if (u < (b0 + 1) * gb) {             // columns BJ <= b0: present in every row
-    BJ = u / gb;
+  const int c_full = b0 / 2 + 1;       // pairs C with 2C <= b0: present in every row
+  if (u < c_full * gb) {
+    C = u / gb;
     BI = b0 + u % gb;
     return;
   }
-  u -= (b0 + 1) * gb;
-  for (BJ = b0 + 1;; ++BJ) {           // column BJ is in rows BJ .. b0 + gb - 1
-    const int n = b0 + gb - BJ;
-    if (u < n) {
-      BI = BJ + u;
+  u -= c_full * gb;
+  for (C = c_full;; ++C) {             // pair C is in rows 2C .. b0 + gb - 1
+    const int nc = b0 + gb - 2 * C;
+    if (u < nc) {
+      BI = 2 * C + u;
       return;
     }
-    u -= n;
+    u -= nc;
   }
 }
 
@@ -206,7 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
   uint8_t* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
   float* trs = reinterpret_cast<float*>(gsm + GSTAGES * G_STAGE);
   __shared__ __align__(8) uint64_t full_bar[GSTAGES], empty_bar[GSTAGES];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+  __shared__ __align__(8) uint64_t acc_full, acc_empty;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -222,10 +225,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
       mbar_init(&full_bar[s], 1);   // the leader's arm; both CTAs' bytes
       mbar_init(&empty_bar[s], 1);  // the leader's commit
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);   // the leader's commit
-      mbar_init(&acc_empty[b], 8);  // one lane of each epilogue warp of both CTAs
-    }
+    mbar_init(&acc_full, 1);   // the leader's commit
+    mbar_init(&acc_empty, 8);  // one lane of each epilogue warp of both CTAs
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -250,11 +251,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
       const uint32_t full0 = cluster_addr(&full_bar[0], 0);
       long long g = 0;
       for (int t = pair; t < ntiles && !*(volatile int*)&abort_flag; t += npairs) {
-        int BI, BJ;
-        g_pair_tile(t, NB, BI, BJ);
-        const bool diag = BI == BJ;
-        const int ia = BI * GT + (int)rank * GB, jb = BJ * GT + (int)rank * GB;
-        const unsigned bytes = (diag ? 1 : 2) * G_TILE;  // per CTA
+        int BI, C;
+        g_pair_tile(t, NB, BI, C);
+        const bool diag = 2 * C == BI;      // B0 = A
+        const bool wide = 2 * C + 1 <= BI;  // B1 (the second 256 columns) below the diagonal
+        const int ia = BI * GT + (int)rank * GB;
+        const int jb0 = 2 * C * GT + (int)rank * GB, jb1 = jb0 + GT;
+        const unsigned bytes = (1 + (diag ? 0 : 1) + (wide ? 1 : 0)) * G_TILE;  // per CTA
         for (long long c = 0; c < nchunks; ++c, ++g) {
           const int st = (int)(g % GSTAGES);
           if (g >= GSTAGES &&
@@ -270,8 +273,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
           tma_box(sA, &tmap, ia, y, fb);
           tma_box(sA + G_BOX, &tmap, ia + 64, y, fb);
           if (!diag) {
-            tma_box(sA + G_TILE, &tmap, jb, y, fb);
-            tma_box(sA + G_TILE + G_BOX, &tmap, jb + 64, y, fb);
+            tma_box(sA + G_TILE, &tmap, jb0, y, fb);
+            tma_box(sA + G_TILE + G_BOX, &tmap, jb0 + 64, y, fb);
+          }
+          if (wide) {
+            tma_box(sA + 2 * G_TILE, &tmap, jb1, y, fb);
+            tma_box(sA + 2 * G_TILE + G_BOX, &tmap, jb1 + 64, y, fb);
           }
         }
       }
@@ -282,17 +289,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
       long long g = 0;
       int it = 0;  // this pair's tile count
       for (int t = pair; t < ntiles && !*(volatile int*)&abort_flag; t += npairs, ++it) {
-        int BI, BJ;
-        g_pair_tile(t, NB, BI, BJ);
-        const bool diag = BI == BJ;
-        const int b = it & 1;
-        // accumulator b was last used by tile it - 2: both epilogues must have read it
-        if (it >= 2 && !mbar_wait(&acc_empty[b], (uint32_t)(((it >> 1) - 1) & 1))) {
+        int BI, C;
+        g_pair_tile(t, NB, BI, C);
+        const bool diag = 2 * C == BI, wide = 2 * C + 1 <= BI;
+        // the accumulator was last used by tile it - 1: both epilogues must have read it
+        if (it >= 1 && !mbar_wait(&acc_empty, (uint32_t)((it - 1) & 1))) {
           atomicExch(&abort_flag, 1);
           break;
         }
         tc_fence_after();
-        const uint32_t dt = tmem + (uint32_t)(b * GT);
         bool ok = true;
         for (int64_t c = 0; c < nchunks; ++c, ++g) {
           const int st = (int)(g % GSTAGES);
@@ -302,19 +307,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
           }
           tc_fence_after();
           const uint32_t aaddr = smem_u32(gsm + st * G_STAGE);
-          const uint32_t baddr = diag ? aaddr : aaddr + G_TILE;
-          // K step s16 = rows 16 s16 .. 16 s16 + 15: two 8-row groups further (2 * SBO)
+          const uint32_t b0addr = diag ? aaddr : aaddr + G_TILE, b1addr = aaddr + 2 * G_TILE;
+          // K step s16 = rows 16 s16 .. 16 s16 + 15: two 8-row groups further (2 * SBO);
+          // columns 0..255 of the tile into accumulator columns 0..255, 256..511 into
+          // 256..511
 #pragma unroll
-          for (int s16 = 0; s16 < GK / 16; ++s16)
-            tc_mma(dt, g_desc(aaddr + s16 * 2 * G_SBO), g_desc(baddr + s16 * 2 * G_SBO),
-                   G_IDESC, (c > 0 || s16 > 0) ? 1u : 0u);
+          for (int s16 = 0; s16 < GK / 16; ++s16) {
+            const uint64_t ad = g_desc(aaddr + s16 * 2 * G_SBO);
+            const uint32_t acc = (c > 0 || s16 > 0) ? 1u : 0u;
+            tc_mma(tmem, ad, g_desc(b0addr + s16 * 2 * G_SBO), G_IDESC, acc);
+            if (wide) tc_mma(tmem + (uint32_t)GT, ad, g_desc(b1addr + s16 * 2 * G_SBO), G_IDESC, acc);
+          }
           tc_commit_pair(&empty_bar[st]);
         }
         if (!ok) {
           atomicExch(&abort_flag, 1);
           break;
         }
-        tc_commit_pair(&acc_full[b]);  // the tile's MMAs are complete in both CTAs
+        tc_commit_pair(&acc_full);  // the tile's MMAs are complete in both CTAs
       }
     }
   } else {
@@ -322,23 +332,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
     // 32 (w % 4) .. + 31, i.e. rows 32 (w % 4) .. of this CTA's half of the tile
     const int q = warp & 3;
     float* tr = trs + (warp - 2) * 32 * 33;
-    const uint32_t empty0 = cluster_addr(&acc_empty[0], 0);
+    const uint32_t empty0 = cluster_addr(&acc_empty, 0);
     // (every decision below is taken by the whole warp: tcgen05.ld is warp-wide)
     int it = 0;
     for (int t = pair; t < ntiles && !__any_sync(0xffffffffu, *(volatile int*)&abort_flag);
          t += npairs, ++it) {
-      int BI, BJ;
-      g_pair_tile(t, NB, BI, BJ);
-      const int b = it & 1;
-      const int ia = BI * GT + (int)rank * GB, j0 = BJ * GT;
-      // 32-column chunks in 128-blocks at or left of this CTA's diagonal block
-      const int ncb = (2 * BJ + 2 <= 2 * BI + (int)rank + 1 ? 2 : 1) * (GB / 32);
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[b], (uint32_t)((it >> 1) & 1)))) {
+      int BI, C;
+      g_pair_tile(t, NB, BI, C);
+      const int ia = BI * GT + (int)rank * GB, j0 = 2 * C * GT;
+      // 32-column chunks in the tile's 128-blocks 4C .. 4C + 3 at or left of this
+      // CTA's diagonal block 2 BI + rank (a prefix of them)
+      const int ncb = min(4, 2 * BI + (int)rank - 4 * C + 1) * (GB / 32);
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full, (uint32_t)(it & 1)))) {
         if (lane == 0) atomicExch(&abort_flag, 1);
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * GT);
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
       for (int cb = 0; cb < ncb; ++cb) {
         uint32_t v[32];
@@ -357,7 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GTHREADS, 1)
           // the accumulator is read: hand it back to the leader's MMA thread
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_remote(empty0 + (uint32_t)(b * sizeof(uint64_t)));
+          if (lane == 0) mbar_arrive_remote(empty0);
         }
         // turn the 32 x 32 chunk around so that each store writes 32 consecutive
         // floats of one row
