@@ -866,6 +866,16 @@ def run_kron3(args):
         torch.cuda.empty_cache()
         return out
 
+    if args.profile_step:  # one per-mode rounding of the 4096 x 64 x 64 case (ncu input)
+        torch.manual_seed(77)
+        dims = (4096, 64, 64)
+        Hs = [gram(d, 4096 if d >= 1024 else 4 * d) for d in dims]
+        W2 = (torch.randn((dims[0], dims[1] * dims[2]), device=dev) * 0.02).to(torch.bfloat16)
+        s = (W2.float().abs().amax(dim=1) / 7.0).clamp_min(1e-30).contiguous()
+        Ms = [g.prepare(H, check=False) for H in Hs]
+        g.quantize_kron(W2, Ms[0], Ms[1:], s, 4, True)
+        torch.cuda.synchronize()
+        return None
     main = case((4096, 64, 64), 77)
     wide = case((1024, 128, 64), 78)
     return {"metric": "weight entries rounded per second, 3-factor Kronecker Hessian (INT4, 1 B200)",

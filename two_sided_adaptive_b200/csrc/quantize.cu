@@ -68,6 +68,7 @@ constexpr int KMAXA = 8;  // a = TB / m_in with m_in >= 8
 struct KronDesc {
   int nf, nout;
   int m_in, a;
+  int lg;                   // log2 m_in (m_in is a power of two: it divides 64)
   int U;                    // outer extent n / m_in
   int dim[KMAXF];
   int ustride[KMAXF];       // stride_f / m_in for the outer factors
@@ -282,11 +283,13 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       if (kron && a.kd.a == 1) {  // I_a (x) Lin = Lin, [target column][source column]
         cp_async16_zfill(Rt + r * SLD + c2, a.kd.lin + r * TB + c2, c0 + r < a.n);
       } else if (kron) {
-        const int mi = a.kd.m_in;
+        const int lg = a.kd.lg, mk = a.kd.m_in - 1;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int c = c2 + e;
-          Rt[r * SLD + c] = (r / mi == c / mi && c0 + r < a.n) ? a.kd.lin[(r % mi) * mi + c % mi] : 0.0;
+          Rt[r * SLD + c] = ((r >> lg) == (c >> lg) && c0 + r < a.n)
+                                ? a.kd.lin[((r & mk) << lg) + (c & mk)]
+                                : 0.0;
         }
       } else {
         cp_async16_zfill(Rt + r * SLD + c2, a.Rh + (int64_t)(c0 + r) * np + c0 - TB + c2, true);
@@ -357,11 +360,11 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
     cp_async_wait_group<1>();
     __syncthreads();
     if (has_r) {
-      const int mi = a.kd.m_in, na = a.kd.a;
+      const int lg = a.kd.lg, v_mask = a.kd.m_in - 1, na = a.kd.a;
       for (int e = tid; e < TB * TB; e += SWEEP_THREADS) {
-        const int r = e >> 6, c = e & 63, xq = c / mi, v = c % mi;
+        const int r = e >> 6, c = e & 63, xq = c >> lg, v = c & v_mask;
         double sacc = Pt[r * SLD + c];
-        for (int y = 0; y < na; ++y) sacc = fma(KN[xq][y], Dt[r * SLD + y * mi + v], sacc);
+        for (int y = 0; y < na; ++y) sacc = fma(KN[xq][y], Dt[r * SLD + (y << lg) + v], sacc);
         Pt[r * SLD + c] = sacc;
       }
     }
@@ -416,12 +419,12 @@ __global__ void __launch_bounds__(SWEEP_THREADS, 1) sweep_kernel(QArgs a, int D,
       // Rh[J,J] = Lin; the sweep reads only its strictly lower part
       cp_async16_zfill(Rt + r * SLD + c2, a.kd.lin + r * TB + c2, c0 + r < a.n);
     } else if (kron) {  // Rh[J,J] = Ah[J,J] (x) Lin, strictly lower
-      const int mi = a.kd.m_in;
+      const int lg = a.kd.lg, mk = a.kd.m_in - 1;
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int c = c2 + e;
         Rt[r * SLD + c] = (c < r && c0 + r < a.n)
-                              ? KA[r / mi][c / mi] * a.kd.lin[(r % mi) * mi + c % mi]
+                              ? KA[r >> lg][c >> lg] * a.kd.lin[((r & mk) << lg) + (c & mk)]
                               : 0.0;
       }
     } else {
@@ -980,7 +983,7 @@ __global__ void __launch_bounds__(KP_THREADS) kron_push_kernel(QArgs a, int D, i
     cp_async16_zfill(dws + r * SLD + c2, src + (int64_t)r * np + c2, true);
   }
   cp_async_commit_group();
-  const int mi = k.m_in, na = k.a;
+  const int lg = k.lg, v_mask = k.m_in - 1, na = k.a;
   for (int Jt = t0; Jt < t1; ++Jt) {
     if (threadIdx.x < KMAXA * KMAXA) {
       const int x = threadIdx.x / KMAXA, y = threadIdx.x % KMAXA;
@@ -994,9 +997,9 @@ __global__ void __launch_bounds__(KP_THREADS) kron_push_kernel(QArgs a, int D, i
     for (int e = threadIdx.x; e < TB * TB; e += KP_THREADS) {
       const int r = e >> 6, c = e & 63;
       if (r >= rows || c >= cols) continue;
-      const int xq = c / mi, v = c % mi;
+      const int xq = c >> lg, v = c & v_mask;
       double acc = 0.0;
-      for (int y = 0; y < na; ++y) acc = fma(cc[xq][y], dws[r * SLD + y * mi + v], acc);
+      for (int y = 0; y < na; ++y) acc = fma(cc[xq][y], dws[r * SLD + (y << lg) + v], acc);
       red_add(dst + (int64_t)r * np + c, acc);
     }
     __syncthreads();  // cc is rewritten for the next target
@@ -1367,6 +1370,8 @@ int quantize_launch(const void* W, int w_dtype, int m, int n, int64_t ldw, const
     k.nout = kron->nf - nin;
     k.m_in = m_in;
     k.a = TB / m_in;
+    k.lg = 0;
+    while ((1 << k.lg) < m_in) ++k.lg;
     k.U = n / m_in;
     int64_t stride = 1;
     for (int f = k.nf - 1; f >= 0; --f) {
