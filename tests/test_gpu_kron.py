@@ -226,3 +226,34 @@ def test_quantize_tensor_per_mode_end_to_end(g):
     assert g.stats_dict(st)["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
     assert O.proxy_loss_tensor(W.astype(np.float64), Q.cpu().numpy(), s.astype(np.float64), Hs) == \
         pytest.approx(rep.result.loss_identity, rel=1e-6)
+
+
+@pytest.mark.parametrize("wdt", ["bfloat16", "float64"])
+def test_per_mode_weight_dtypes(g, wdt):
+    """The per-mode sweep is instantiated per weight type: bf16 and fp64 W against the
+    oracle on the same (upcast) weights."""
+    shape = (97, 16, 16)
+    W, Hs, s = _case(21, shape)
+    Wt = torch.from_numpy(W.reshape(shape[0], -1)).to(getattr(torch, wdt)).cuda()
+    W64 = Wt.double().cpu().numpy()
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    Q, st = g.quantize_kron(Wt, torch.from_numpy(Ms[0]).cuda(),
+                            [torch.from_numpy(M).cuda() for M in Ms[1:]],
+                            torch.from_numpy(s).cuda(), 4, True)
+    torch.cuda.synchronize()
+    rep = check_against_oracle(W64, Ms[0], O.kron_factor(Ms[1:]), s.astype(np.float64), 4, True,
+                               Q.cpu().numpy())
+    assert g.stats_dict(st)["status"] == 0
+    assert g.stats_dict(st)["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+
+
+def test_per_mode_zero_rows(g):
+    """m = 0: nothing to round; the statistics are zero and the status OK."""
+    Ms = [torch.eye(d, dtype=torch.float64, device="cuda") for d in (8, 8, 8)]
+    W = torch.empty((0, 64), dtype=torch.float32, device="cuda")
+    s = torch.empty(0, dtype=torch.float32, device="cuda")
+    Q, st = g.quantize_kron(W, torch.empty((0, 0), dtype=torch.float64, device="cuda"), Ms[1:],
+                            s, 4, True)
+    torch.cuda.synchronize()
+    d = g.stats_dict(st)
+    assert d["status"] == 0 and d["n_clamped"] == 0 and d["proxy_loss"] == 0.0
