@@ -651,8 +651,9 @@ def run_configs(args):
       small  512 x 512, INT4, seeds 0-3: the anti-diagonal oracle in full;
       attn   4096 x 4096 INT4; mlp 4096 x 14336 INT4 and INT3: the oracle's factors in
              full and its rounding on the leading 1024 x 1024 prefix (a problem of its
-             own), scaled to the layer by mn(m + n) (the rounding's work; the scaling
-             exponent is checked on prefixes from 512 to 4096, see DESIGN.md);
+             own), scaled to the layer by mn(m + n) (the rounding's work; the oracle's
+             time grows as about k^3.07 over full k x k runs from 512 to 4096 on 16
+             host cores, so the scaled figure is a lower bound);
     and the quantize call's fp64 rate against the cuBLAS DGEMM peak measured here."""
     import torch
     import oracle as O
