@@ -302,3 +302,29 @@ def test_quantize_kron_checks_pointers_before_any_launch(L):
     """Valid sizes but host addresses: rejected as INVALID_ARG by the device-pointer
     check (nothing is launched)."""
     assert _qk(L) == g.Status.INVALID_ARG
+
+
+def test_per_mode_order_moves_an_inner_group_last():
+    """The chosen order of the trailing modes ends in modes whose sizes multiply to the
+    largest of 64, 32, 16, 8 any subset reaches (checked by brute force), keeps the
+    other modes' order, and keeps the given order when it already reaches it."""
+    import itertools
+    cases = [[64, 64], [32, 128], [3, 3, 64], [3, 3, 256], [24, 5], [16, 128], [2, 128],
+             [5, 3], [8, 8, 2], [6, 4, 16], [12, 64], [64, 12], [3, 41], [2] * 7, [1, 7, 4, 2]]
+    for dims in cases:
+        best = 0
+        for r in range(1, len(dims) + 1):
+            for sel in itertools.combinations(range(len(dims)), r):
+                p = 1
+                for i in sel:
+                    p *= dims[i]
+                if p in (8, 16, 32, 64):
+                    best = max(best, p)
+        order = g.per_mode_order(dims)
+        if best == 0:
+            assert order is None, dims
+            continue
+        assert sorted(order) == list(range(len(dims)))
+        assert g.kron_inner_size([dims[i] for i in order]) == best, (dims, order)
+        if g.kron_inner_size(dims) == best:
+            assert order == list(range(len(dims)))

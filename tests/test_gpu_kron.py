@@ -257,3 +257,26 @@ def test_per_mode_zero_rows(g):
     torch.cuda.synchronize()
     d = g.stats_dict(st)
     assert d["status"] == 0 and d["n_clamped"] == 0 and d["proxy_loss"] == 0.0
+
+
+@pytest.mark.parametrize("shape", [(40, 32, 3), (24, 16, 128), (30, 64, 3, 3), (36, 5, 8, 8, 2)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_quantize_tensor_reorders_trailing_modes(g, shape):
+    """Trailing modes whose given order has no inner group of 8..64 (a last mode of 3
+    or 128) are rounded with the eligible modes moved last; the result, put back in
+    W's order, is the oracle's rounding of the original order (the rounding depends
+    only on each entry's dominated orthant)."""
+    order = g.per_mode_order(shape[1:])
+    assert order is not None and order != list(range(len(shape) - 1))
+    W, Hs, s = _case(31, shape)
+    Q, st = g.quantize_tensor(torch.from_numpy(W).cuda(), [torch.from_numpy(H).cuda() for H in Hs],
+                              torch.from_numpy(s).cuda(), 4, True)
+    torch.cuda.synchronize()
+    assert tuple(Q.shape) == shape
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    rep = check_against_oracle(W.reshape(shape[0], -1).astype(np.float64), Ms[0],
+                               O.kron_factor(Ms[1:]), s.astype(np.float64), 4, True,
+                               Q.cpu().numpy().reshape(shape[0], -1))
+    d = g.stats_dict(st)
+    assert d["status"] == 0
+    assert d["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)

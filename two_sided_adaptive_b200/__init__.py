@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "Status", "GPTQ2DError", "lib", "library_path", "prepare", "quantize", "round_host",
     "kron_factor", "prepare_kron", "quantize_tensor", "MAX_KRON_FACTORS", "quantize_grid",
-    "quantize_kron", "quantize_kron_workspace_size", "kron_inner_size",
+    "quantize_kron", "quantize_kron_workspace_size", "kron_inner_size", "per_mode_order",
     "gram_accumulate", "gram_finalize", "gram", "quantize_block", "block_workspace_size",
     "stats_dict", "launch_count", "prepare_workspace_size", "quantize_workspace_size",
     "round_host_workspace_size", "quantize_noalloc", "proxy_loss", "check_wait_timeout",
@@ -503,26 +503,58 @@ def quantize_kron(W, M_L, Ms, scales, bits: int = 4, clamp: bool = True, *, out=
     return Q, st
 
 
+def per_mode_order(dims):
+    """An order of the trailing modes for quantize_kron, or None: the subset of modes
+    whose sizes multiply to the largest of 64, 32, 16, 8 goes last (the inner group),
+    the rest keep their order in front.  The k-way rounding depends only on each
+    entry's dominated orthant, so reordering the trailing modes permutes the result
+    and nothing else.  The given order is kept when it already reaches that size."""
+    dims = [int(d) for d in dims]
+    k = len(dims)
+    best, best_p = None, 0
+    for mask in range(1, 1 << k):
+        sel = [i for i in range(k) if (mask >> i) & 1]
+        p = int(np.prod([dims[i] for i in sel]))
+        if p in (8, 16, 32, 64) and p > best_p:
+            best, best_p = sel, p
+    if best is None:
+        return None
+    if kron_inner_size(dims) == best_p:
+        return list(range(k))
+    return [i for i in range(k) if i not in best] + best
+
+
 @_device_scoped
 def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, per_mode=None,
                     stream=None):
     """GPTQ-2D rounding of a k-way tensor W (m_1 x ... x m_k, C order) under
     H_1 kron ... kron H_k with per-mode-1 scales: the m_1 x (m_2 ... m_k) problem with
     M_L = prepare(H_1) and the right factor M_2 kron ... kron M_k.  per_mode=None picks
-    the per-mode right factor (quantize_kron) when it applies to the trailing modes
-    (kron_inner_size > 0) and the dense Kronecker factor (kron_factor + quantize)
+    the per-mode right factor (quantize_kron) when some order of the trailing modes
+    allows it (per_mode_order: the tensor is rounded with those modes reordered and Q
+    is put back in W's order), and the dense Kronecker factor (kron_factor + quantize)
     otherwise; True or False forces one.  Returns (Q shaped like W, stats)."""
     if W.dim() != len(Hs) or W.dim() < 2:
         raise ValueError("one Hessian factor per mode, at least two modes")
-    W2 = W.reshape(W.shape[0], -1)
     dims = list(W.shape[1:])
-    use = kron_inner_size(dims) > 0 if per_mode is None else bool(per_mode)
-    if use:
+    order = per_mode_order(dims) if per_mode is None or per_mode else None
+    if per_mode and order is None:
+        raise ValueError("no order of the trailing modes has an inner group of 8 to 64")
+    if order is not None:
         Ms = [prepare(H, stream=stream) for H in Hs]
-        Q, st = quantize_kron(W2, Ms[0], Ms[1:], scales, bits, clamp, stream=stream)
-    else:
-        M_L, M_R = prepare_kron(Hs, stream=stream)
-        Q, st = quantize(W2, M_L, M_R, scales, bits, clamp, stream=stream)
+        perm = [0] + [1 + i for i in order]
+        Wp = W.permute(*perm).contiguous() if order != list(range(len(dims))) else W
+        Q, st = quantize_kron(Wp.reshape(W.shape[0], -1), Ms[0], [Ms[1 + i] for i in order],
+                              scales, bits, clamp, stream=stream)
+        Q = Q.reshape(Wp.shape)
+        if order != list(range(len(dims))):
+            inv = [0] * len(perm)
+            for a_, b_ in enumerate(perm):
+                inv[b_] = a_
+            Q = Q.permute(*inv).contiguous()
+        return Q, st
+    M_L, M_R = prepare_kron(Hs, stream=stream)
+    Q, st = quantize(W.reshape(W.shape[0], -1), M_L, M_R, scales, bits, clamp, stream=stream)
     return Q.reshape(W.shape), st
 
 
