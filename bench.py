@@ -779,6 +779,8 @@ def run_kron3(args):
     dominates).  INT4 per-mode-1 absmax scales, W ~ N(0, 0.02^2) in bf16, Grams from
     Student-t(4) activations times U(0.1, 10) column scales (4096 rows for a factor of
     width >= 1024, else 4 x width) plus 1% mean-diagonal damping, generated on the GPU.
+    A third case, 256 x 4096 x 64 (n = 262,144 columns), runs the per-mode route only:
+    the dense route's n x n factor would take 550 GB.
     Two routes, each timed with CUDA events over K steps after W warm-up steps, inputs
     resident in HBM:
       per-mode: prepare(H_1), prepare(H_2), prepare(H_3), quantize_kron (the right
@@ -801,7 +803,7 @@ def run_kron3(args):
         G.diagonal().add_(0.01 * G.diagonal().mean())
         return G.float()
 
-    def case(dims, seed):
+    def case(dims, seed, dense=True):
         torch.manual_seed(seed)
         Hs = [gram(d, 4096 if d >= 1024 else 4 * d) for d in dims]
         m, n = dims[0], dims[1] * dims[2]
@@ -850,10 +852,21 @@ def run_kron3(args):
             return tp / args.steps, tq / args.steps
 
         tp, tq = timed(False)
+        sd = g.stats_dict(st)
+        if not dense:  # the dense route's n x n factor would not fit
+            out = {"dims": list(dims), "ms_per_step": tp + tq,
+                   "entries_per_s": m * n / ((tp + tq) * 1e-3), "prepare_ms": tp,
+                   "quantize_kron_ms": tq, "per_mode_workspace_bytes": wsK.numel(),
+                   "dense_route": {"n_by_n_factor_bytes": 8 * n * n, "run": False},
+                   "status": sd["status"], "n_near_tie": sd["n_near_tie"],
+                   "proxy_loss": sd["proxy_loss"]}
+            del Hs, Ms, wsP, wsK
+            torch.cuda.empty_cache()
+            return out
         dense_ws["MR"] = torch.empty((n, n), dtype=torch.float64, device=dev)
         dense_ws["ws"] = torch.empty(g.quantize_workspace_size(m, n), dtype=torch.uint8, device=dev)
         tpd, tqd = timed(True)
-        sd, sdd = g.stats_dict(st), g.stats_dict(std)
+        sdd = g.stats_dict(std)
         out = {"dims": list(dims), "ms_per_step": tp + tq, "entries_per_s": m * n / ((tp + tq) * 1e-3),
                "prepare_ms": tp, "quantize_kron_ms": tq,
                "per_mode_workspace_bytes": wsK.numel(),
@@ -879,6 +892,7 @@ def run_kron3(args):
         return None
     main = case((4096, 64, 64), 77)
     wide = case((1024, 128, 64), 78)
+    huge = case((256, 4096, 64), 79, dense=False)
     return {"metric": "weight entries rounded per second, 3-factor Kronecker Hessian (INT4, 1 B200)",
             "value": main["entries_per_s"], "unit": "entries/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
@@ -886,7 +900,7 @@ def run_kron3(args):
             "data": "synthetic (generated on the GPU, see run_kron3)",
             "config": {"workload": "kron3", "dims": main["dims"], "bits": 4,
                        "step": "prepare x3 + quantize_kron (per-mode right factor)"},
-            "cases": [main, wide]}
+            "cases": [main, wide, huge]}
 
 
 def run_grid128(args):
