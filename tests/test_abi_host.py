@@ -328,3 +328,22 @@ def test_per_mode_order_moves_an_inner_group_last():
         assert g.kron_inner_size([dims[i] for i in order]) == best, (dims, order)
         if g.kron_inner_size(dims) == best:
             assert order == list(range(len(dims)))
+
+
+def test_per_mode_eligibility_agrees_between_library_and_binding():
+    """The library's workspace query (0 when the per-mode path does not apply) and the
+    binding's kron_inner_size agree on every trailing-mode list up to three modes of
+    sizes 1..12, 16, 32, 64, 100, 128."""
+    import itertools
+    sizes = list(range(1, 13)) + [16, 32, 64, 100, 128]
+    for k in (1, 2, 3):
+        for dims in itertools.product(sizes, repeat=k):
+            if k == 3 and (dims[0] > 4 or dims[1] > 8):
+                continue  # keep the sweep small
+            arr = (ctypes.c_int64 * k)(*dims)
+            lib_ok = L_global().gptq2d_quantize_kron_workspace_size(16, k, arr) > 0
+            assert lib_ok == (g.kron_inner_size(dims) > 0), dims
+
+
+def L_global():
+    return g.lib()
