@@ -414,6 +414,16 @@ int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64
                          const gptq2d_grid* grid, void* Q, int64_t ldq, gptq2d_stats* stats,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* gptq2d_quantize_kron on a grid variant: the k-way rounding with the right factor
+ * kept per mode (arguments, applicability and workspace as gptq2d_quantize_kron)
+ * on group-wise scales, integer zero points or packed 4-bit output (grid, Q and ldq
+ * as gptq2d_quantize_grid; scale groups run along the flattened trailing modes). */
+int gptq2d_quantize_kron_grid(const void* W, int w_dtype, int64_t m, int64_t ldw,
+                              const double* M_L, int64_t ldl, int nf, const double* const* M,
+                              const int64_t* dims, const int64_t* ldm, const gptq2d_grid* grid,
+                              void* Q, int64_t ldq, gptq2d_stats* stats, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* A block of layers (the pages quantize whole models, block by block:         */
 /* arxivlens, Abstract, Llama-3.1-70B-Instruct on one GPU)                     */

@@ -280,3 +280,55 @@ def test_quantize_tensor_reorders_trailing_modes(g, shape):
     d = g.stats_dict(st)
     assert d["status"] == 0
     assert d["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+
+
+KRON_GRID = [  # tensor shape, group size, asymmetric, bits, packed
+    ((70, 24, 32), 32, True, 4, True),
+    ((65, 3, 4, 16), 64, False, 4, False),
+    ((97, 16, 16), 16, True, 3, False),
+    ((48, 2, 3, 2, 8), 8, True, 4, True),
+]
+
+
+@pytest.mark.parametrize("case", KRON_GRID, ids=lambda c: "x".join(map(str, c[0])) + "_G%d_%s_b%d_%s" % (
+    c[1], "asym" if c[2] else "sym", c[3], "packed" if c[4] else "bytes"))
+def test_per_mode_grid_variant_matches_oracle(g, case):
+    """gptq2d_quantize_kron_grid: group-wise scales along the flattened trailing modes,
+    integer zero points and packed 4-bit codes on the per-mode route, against the
+    oracle's rounding with the same per-entry grid; the stored bytes are the oracle's
+    codes."""
+    shape, G, asym, bits, packed = case
+    W, Hs, _ = _case(41, shape)
+    m, n = shape[0], int(np.prod(shape[1:]))
+    W2 = W.reshape(m, n).astype(np.float64)
+    if asym:
+        S, Z = WL.group_minmax_grid(W2, bits, G)
+    else:
+        S, Z = WL.group_absmax_scales(W2, bits, G), None
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    Qb, st = g.quantize_kron(torch.from_numpy(W.reshape(m, n)).cuda(), torch.from_numpy(Ms[0]).cuda(),
+                             [torch.from_numpy(M).cuda() for M in Ms[1:]],
+                             torch.from_numpy(np.ascontiguousarray(S, np.float32)).cuda(), bits, True,
+                             group_size=G, zeros=torch.from_numpy(Z).cuda() if Z is not None else None,
+                             packed=packed)
+    torch.cuda.synchronize()
+    B = Qb.cpu().numpy().astype(np.int64)
+    if packed:
+        codes = np.zeros((m, n), np.int64)
+        codes[:, 0::2] = B[:, : (n + 1) // 2] & 15
+        codes[:, 1::2] = (B[:, : n // 2] >> 4) & 15
+        q = codes - (1 << (bits - 1)) if Z is None else codes - np.asarray(Z, np.int64)[:, np.arange(n) // G]
+    else:
+        codes = B if Z is not None else Qb.cpu().numpy().astype(np.int8).astype(np.int64)
+        q = codes if Z is None else codes - np.asarray(Z, np.int64)[:, np.arange(n) // G]
+    grid = O.expand_grid(m, n, S.astype(np.float64), bits, True, G, Z)
+    rep = check_against_oracle(W2, Ms[0], O.kron_factor(Ms[1:]), None, bits, True, q, grid=grid)
+    d = g.stats_dict(st)
+    assert d["status"] == 0 and d["n_nonfinite"] == 0
+    assert d["n_clamped"] == rep.result.n_clamped
+    assert d["proxy_loss"] == pytest.approx(rep.result.loss_identity, rel=1e-5)
+    if packed:
+        np.testing.assert_array_equal(Qb.cpu().numpy(),
+                                      O.pack_nibbles(O.packed_codes(rep.result.Q, m, n, bits, G, Z)))
+    else:
+        np.testing.assert_array_equal(codes, O.stored_codes(rep.result.Q, m, n, bits, G, Z))

@@ -124,6 +124,11 @@ def lib():
         L.gptq2d_kron_factor.argtypes = [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p]
         L.gptq2d_quantize_kron_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_quantize_kron_workspace_size.argtypes = [_c_i64, ctypes.c_int, _c_p]
+        L.gptq2d_quantize_kron_grid.restype = ctypes.c_int
+        L.gptq2d_quantize_kron_grid.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_i64,
+                                                ctypes.c_int, _c_p, _c_p, _c_p,
+                                                ctypes.POINTER(_Grid), _c_p, _c_i64, _c_p, _c_p,
+                                                ctypes.c_size_t, _c_p]
         L.gptq2d_quantize_kron.restype = ctypes.c_int
         L.gptq2d_quantize_kron.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_i64,
                                            ctypes.c_int, _c_p, _c_p, _c_p, _c_p, ctypes.c_int,
@@ -467,13 +472,16 @@ def quantize_kron_workspace_size(m: int, dims) -> int:
 
 
 @_device_scoped
-def quantize_kron(W, M_L, Ms, scales, bits: int = 4, clamp: bool = True, *, out=None, stats=None,
-                  workspace=None, stream=None):
+def quantize_kron(W, M_L, Ms, scales, bits: int = 4, clamp: bool = True, *, group_size: int = 0,
+                  zeros=None, packed: bool = False, out=None, stats=None, workspace=None,
+                  stream=None):
     """The k-way rounding with the right factor kept per mode (gptq2d_quantize_kron): W is
     the m x (m_2 ... m_k) matrix of the tensor, M_L = prepare(H_1), Ms = [prepare(H_2), ...,
-    prepare(H_k)].  Returns (Q int8 m x n, stats on the device)."""
+    prepare(H_k)].  group_size / zeros / packed select a grid variant as in quantize_grid
+    (gptq2d_quantize_kron_grid).  Returns (Q bytes m x n, or m x ceil(n/2) packed; stats
+    on the device)."""
     torch = _torch()
-    _check_device(W, M_L, scales, out, stats, workspace, *Ms)
+    _check_device(W, M_L, scales, zeros, out, stats, workspace, *Ms)
     m, n = W.shape
     if not 1 <= len(Ms) <= MAX_KRON_FACTORS:
         raise ValueError(f"1 to {MAX_KRON_FACTORS} trailing factors")
@@ -483,23 +491,49 @@ def quantize_kron(W, M_L, Ms, scales, bits: int = 4, clamp: bool = True, *, out=
     dims = [int(M.shape[0]) for M in Ms]
     if int(np.prod(dims)) != n:
         raise ValueError("the factors' sizes must multiply to W's column count")
-    if scales.dtype != torch.float32 or scales.numel() != m or not scales.is_contiguous():
-        raise ValueError("scales must be a contiguous fp32 vector of length m")
     if M_L.dtype != torch.float64:
         raise ValueError("factors must be fp64")
-    Q = out if out is not None else torch.empty((m, n), dtype=torch.int8, device=W.device)
+    if scales.dtype != torch.float32:
+        raise ValueError("scales must be fp32")
+    grid = group_size != 0 or zeros is not None or packed
+    if grid:
+        S = scales.reshape(m, -1) if scales.dim() == 1 else scales
+        if S.shape[0] != m or S.stride(1) != 1:
+            raise ValueError("scales must have m rows with unit column stride")
+        if zeros is not None:
+            if zeros.dtype != torch.uint8 or tuple(zeros.reshape(m, -1).shape) != tuple(S.shape):
+                raise ValueError("zeros must be uint8, shaped like the scales")
+            Z = zeros.reshape(m, -1)
+            if Z.stride(0) != S.stride(0) or Z.stride(1) != 1:
+                raise ValueError("zeros must share the scales' layout")
+    elif scales.numel() != m or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous fp32 vector of length m")
+    qdt = torch.uint8 if (zeros is not None or packed) else torch.int8
+    ncol = (n + 1) // 2 if packed else n
+    Q = out if out is not None else torch.empty((m, ncol), dtype=qdt, device=W.device)
     st = stats if stats is not None else torch.empty(STATS_WORDS, dtype=torch.int64, device=W.device)
     ws = _workspace(max(quantize_kron_workspace_size(m, dims), 256), W.device, workspace)
     nf = len(Ms)
     ptrs = (ctypes.c_void_p * nf)(*[M.data_ptr() for M in Ms])
     dimsa = (_c_i64 * nf)(*dims)
     lds = (_c_i64 * nf)(*[_ld(M) for M in Ms])
-    rc = lib().gptq2d_quantize_kron(W.data_ptr(), _dtype_code(W), m, _ld(W), M_L.data_ptr(),
-                                    _ld(M_L), nf, ptrs, dimsa, lds, scales.data_ptr(), int(bits),
-                                    int(clamp), Q.data_ptr(), _ld(Q), st.data_ptr(), ws.data_ptr(),
-                                    ws.numel(), _stream(stream))
+    if grid:
+        gr = _Grid(int(bits), int(clamp), int(group_size), S.data_ptr(), S.stride(0) if m else 1,
+                   zeros.data_ptr() if zeros is not None else None, int(bool(packed)))
+        rc = lib().gptq2d_quantize_kron_grid(W.data_ptr(), _dtype_code(W), m, _ld(W), M_L.data_ptr(),
+                                             _ld(M_L), nf, ptrs, dimsa, lds, ctypes.byref(gr),
+                                             Q.data_ptr(), _ld(Q) if Q.numel() else ncol,
+                                             st.data_ptr(), ws.data_ptr(), ws.numel(),
+                                             _stream(stream))
+        name = "gptq2d_quantize_kron_grid"
+    else:
+        rc = lib().gptq2d_quantize_kron(W.data_ptr(), _dtype_code(W), m, _ld(W), M_L.data_ptr(),
+                                        _ld(M_L), nf, ptrs, dimsa, lds, scales.data_ptr(),
+                                        int(bits), int(clamp), Q.data_ptr(), _ld(Q),
+                                        st.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+        name = "gptq2d_quantize_kron"
     if rc != Status.OK:
-        raise GPTQ2DError(rc, "gptq2d_quantize_kron")
+        raise GPTQ2DError(rc, name)
     return Q, st
 
 

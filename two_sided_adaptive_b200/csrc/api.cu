@@ -293,58 +293,6 @@ int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, cons
   return kron_factor_launch(nf, M, dims, ldm, out, ldo, static_cast<cudaStream_t>(stream));
 }
 
-size_t gptq2d_quantize_kron_workspace_size(int64_t m, int nf, const int64_t* dims) {
-  if (m < 0 || m > kMaxDim || nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !dims) return 0;
-  int64_t n = 1;
-  for (int f = 0; f < nf; ++f) {
-    if (dims[f] < 1 || dims[f] > kMaxDim) return 0;
-    n *= dims[f];
-    if (n > kMaxDim) return 0;
-  }
-  return quantize_kron_ws_bytes(m, nf, dims);
-}
-
-int gptq2d_quantize_kron(const void* W, int w_dtype, int64_t m, int64_t ldw, const double* M_L,
-                         int64_t ldl, int nf, const double* const* M, const int64_t* dims,
-                         const int64_t* ldm, const float* scales, int bits, int clamp, int8_t* Q,
-                         int64_t ldq, gptq2d_stats* stats, void* ws, size_t ws_bytes,
-                         void* stream) {
-  if (m < 0 || m > kMaxDim || nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !M || !dims || !ldm)
-    return GPTQ2D_ERR_INVALID_ARG;
-  if (elem_size(w_dtype) == 0) return GPTQ2D_ERR_INVALID_ARG;
-  if (bits < 2 || bits > 8 || (clamp != 0 && clamp != 1)) return GPTQ2D_ERR_INVALID_ARG;
-  if (!stats) return GPTQ2D_ERR_INVALID_ARG;
-  int64_t n = 1;
-  for (int f = 0; f < nf; ++f) {
-    if (dims[f] < 0 || dims[f] > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
-    n *= dims[f];
-    if (n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
-  }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (m == 0 || n == 0)
-    return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, nullptr, 0, scales, bits,
-                           clamp, Q, ldq, stats, ws, s);
-  int nin = 0;
-  if (kron_inner(nf, dims, &nin) == 0) return GPTQ2D_ERR_INVALID_ARG;
-  if (!W || !M_L || !scales || !Q) return GPTQ2D_ERR_INVALID_ARG;
-  if (ldw < n || ldl < m || ldq < n) return GPTQ2D_ERR_INVALID_ARG;
-  for (int f = 0; f < nf; ++f)
-    if (!M[f] || ldm[f] < dims[f]) return GPTQ2D_ERR_INVALID_ARG;
-  if (!ws || !aligned256(ws) || ws_bytes < quantize_kron_ws_bytes(m, nf, dims))
-    return GPTQ2D_ERR_WORKSPACE;
-  if (check_device_pointers({W, M_L, scales, Q, stats, ws}) != GPTQ2D_OK)
-    return GPTQ2D_ERR_INVALID_ARG;
-  for (int f = 0; f < nf; ++f)
-    if (check_device_pointers({M[f]}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
-  KronSpec ks;
-  ks.nf = nf;
-  ks.M = M;
-  ks.dims = dims;
-  ks.ldm = ldm;
-  return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, nullptr, 0, scales, bits,
-                         clamp, Q, ldq, stats, ws, s, 0, nullptr, nullptr, nullptr, &ks);
-}
-
 int gptq2d_prepare_pair(const void* H_L, int64_t m, int64_t ldhl, const void* H_R, int64_t n,
                         int64_t ldhr, int h_dtype, double* M_L, int64_t ldml, double* M_R,
                         int64_t ldmr, void* ws, size_t ws_bytes, void* stream,
@@ -461,6 +409,77 @@ int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64
   return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, M_R, ldr, grid->scales,
                          grid->bits, grid->clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0,
                          nullptr, nullptr, &gs);
+}
+
+size_t gptq2d_quantize_kron_workspace_size(int64_t m, int nf, const int64_t* dims) {
+  if (m < 0 || m > kMaxDim || nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !dims) return 0;
+  int64_t n = 1;
+  for (int f = 0; f < nf; ++f) {
+    if (dims[f] < 1 || dims[f] > kMaxDim) return 0;
+    n *= dims[f];
+    if (n > kMaxDim) return 0;
+  }
+  return quantize_kron_ws_bytes(m, nf, dims);
+}
+
+int gptq2d_quantize_kron_grid(const void* W, int w_dtype, int64_t m, int64_t ldw,
+                              const double* M_L, int64_t ldl, int nf, const double* const* M,
+                              const int64_t* dims, const int64_t* ldm, const gptq2d_grid* grid,
+                              void* Q, int64_t ldq, gptq2d_stats* stats, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (m < 0 || m > kMaxDim || nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !M || !dims || !ldm)
+    return GPTQ2D_ERR_INVALID_ARG;
+  int64_t n = 1;
+  for (int f = 0; f < nf; ++f) {
+    if (dims[f] < 0 || dims[f] > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+    n *= dims[f];
+    if (n > kMaxDim) return GPTQ2D_ERR_INVALID_ARG;
+  }
+  GridSpec gs;
+  const int rc = check_grid_call(W, w_dtype, m, n, ldw, grid, Q, ldq, stats, &gs);
+  if (rc != GPTQ2D_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (m == 0 || n == 0)
+    return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, nullptr, 0, grid->scales,
+                           grid->bits, grid->clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0,
+                           nullptr, nullptr, &gs);
+  int nin = 0;
+  if (kron_inner(nf, dims, &nin) == 0) return GPTQ2D_ERR_INVALID_ARG;
+  if (!M_L || ldl < m) return GPTQ2D_ERR_INVALID_ARG;
+  for (int f = 0; f < nf; ++f)
+    if (!M[f] || ldm[f] < dims[f]) return GPTQ2D_ERR_INVALID_ARG;
+  if (!ws || !aligned256(ws) || ws_bytes < quantize_kron_ws_bytes(m, nf, dims))
+    return GPTQ2D_ERR_WORKSPACE;
+  if (check_device_pointers({W, M_L, grid->scales, grid->zeros, Q, stats, ws}) != GPTQ2D_OK)
+    return GPTQ2D_ERR_INVALID_ARG;
+  for (int f = 0; f < nf; ++f)
+    if (check_device_pointers({M[f]}) != GPTQ2D_OK) return GPTQ2D_ERR_INVALID_ARG;
+  KronSpec ks;
+  ks.nf = nf;
+  ks.M = M;
+  ks.dims = dims;
+  ks.ldm = ldm;
+  return quantize_launch(W, w_dtype, (int)m, (int)n, ldw, M_L, ldl, nullptr, 0, grid->scales,
+                         grid->bits, grid->clamp, static_cast<int8_t*>(Q), ldq, stats, ws, s, 0,
+                         nullptr, nullptr, &gs, &ks);
+}
+
+int gptq2d_quantize_kron(const void* W, int w_dtype, int64_t m, int64_t ldw, const double* M_L,
+                         int64_t ldl, int nf, const double* const* M, const int64_t* dims,
+                         const int64_t* ldm, const float* scales, int bits, int clamp, int8_t* Q,
+                         int64_t ldq, gptq2d_stats* stats, void* ws, size_t ws_bytes,
+                         void* stream) {
+  // the symmetric grid with one scale per row
+  gptq2d_grid g{};
+  g.bits = bits;
+  g.clamp = clamp;
+  g.group_size = 0;
+  g.scales = scales;
+  g.ld_scales = 1;
+  g.zeros = nullptr;
+  g.packed = 0;
+  return gptq2d_quantize_kron_grid(W, w_dtype, m, ldw, M_L, ldl, nf, M, dims, ldm, &g, Q, ldq,
+                                   stats, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
