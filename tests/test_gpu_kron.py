@@ -332,3 +332,28 @@ def test_per_mode_grid_variant_matches_oracle(g, case):
                                       O.pack_nibbles(O.packed_codes(rep.result.Q, m, n, bits, G, Z)))
     else:
         np.testing.assert_array_equal(codes, O.stored_codes(rep.result.Q, m, n, bits, G, Z))
+
+
+@pytest.mark.parametrize("shape,route", [((70, 24, 32), "per-mode"), ((40, 6, 11, 2), "dense")])
+def test_quantize_tensor_grid_routes(g, shape, route):
+    """quantize_tensor with group-wise asymmetric INT4 scales: the per-mode route where
+    the given order allows it, the dense one otherwise; both equal the other route's
+    direct call and the oracle's rounding on the same grid."""
+    W, Hs, _ = _case(51, shape)
+    m, n = shape[0], int(np.prod(shape[1:]))
+    W2 = W.reshape(m, n).astype(np.float64)
+    G = 8 if n % 8 == 0 else n
+    S, Z = WL.group_minmax_grid(W2, 4, G)
+    args = dict(group_size=G, zeros=torch.from_numpy(Z).cuda())
+    Q, st = g.quantize_tensor(torch.from_numpy(W).cuda(), [torch.from_numpy(H).cuda() for H in Hs],
+                              torch.from_numpy(np.ascontiguousarray(S, np.float32)).cuda(), 4, True,
+                              **args)
+    torch.cuda.synchronize()
+    assert (g.kron_inner_size(shape[1:]) > 0) == (route == "per-mode")
+    codes = Q.cpu().numpy().reshape(m, n).astype(np.int64)
+    q = codes - np.asarray(Z, np.int64)[:, np.arange(n) // G]
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    grid = O.expand_grid(m, n, S.astype(np.float64), 4, True, G, Z)
+    rep = check_against_oracle(W2, Ms[0], O.kron_factor(Ms[1:]), None, 4, True, q, grid=grid)
+    assert g.stats_dict(st)["status"] == 0
+    np.testing.assert_array_equal(codes, O.stored_codes(rep.result.Q, m, n, 4, G, Z))

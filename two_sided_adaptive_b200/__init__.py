@@ -559,36 +559,54 @@ def per_mode_order(dims):
 
 
 @_device_scoped
-def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, per_mode=None,
-                    stream=None):
+def quantize_tensor(W, Hs, scales, bits: int = 4, clamp: bool = True, *, group_size: int = 0,
+                    zeros=None, packed: bool = False, per_mode=None, stream=None):
     """GPTQ-2D rounding of a k-way tensor W (m_1 x ... x m_k, C order) under
-    H_1 kron ... kron H_k with per-mode-1 scales: the m_1 x (m_2 ... m_k) problem with
-    M_L = prepare(H_1) and the right factor M_2 kron ... kron M_k.  per_mode=None picks
-    the per-mode right factor (quantize_kron) when some order of the trailing modes
-    allows it (per_mode_order: the tensor is rounded with those modes reordered and Q
-    is put back in W's order), and the dense Kronecker factor (kron_factor + quantize)
-    otherwise; True or False forces one.  Returns (Q shaped like W, stats)."""
+    H_1 kron ... kron H_k with scales per index of mode 1: the m_1 x (m_2 ... m_k) problem
+    with M_L = prepare(H_1) and the right factor M_2 kron ... kron M_k.  per_mode=None picks
+    the per-mode right factor (quantize_kron) when some order of the trailing modes allows
+    it (per_mode_order: the tensor is rounded with those modes reordered and Q is put back
+    in W's order), and the dense Kronecker factor (kron_factor + quantize) otherwise; True
+    or False forces one.  group_size / zeros / packed select a grid variant as in
+    quantize_grid, with the scale groups along the flattened trailing modes; a grid keeps
+    the given mode order (a reorder would break the groups), so the per-mode route then
+    needs that order to allow it.  Returns (Q shaped like W, or m_1 x ceil(n/2) bytes
+    when packed; stats)."""
     if W.dim() != len(Hs) or W.dim() < 2:
         raise ValueError("one Hessian factor per mode, at least two modes")
     dims = list(W.shape[1:])
-    order = per_mode_order(dims) if per_mode is None or per_mode else None
+    grid = dict(group_size=group_size, zeros=zeros, packed=packed) \
+        if (group_size or zeros is not None or packed) else None
+    ident = list(range(len(dims)))
+    if grid is not None:
+        order = ident if kron_inner_size(dims) > 0 else None
+    else:
+        order = per_mode_order(dims)
+    if per_mode is False:
+        order = None
     if per_mode and order is None:
-        raise ValueError("no order of the trailing modes has an inner group of 8 to 64")
+        raise ValueError("no usable order of the trailing modes has an inner group of 8 to 64")
+    m = W.shape[0]
     if order is not None:
         Ms = [prepare(H, stream=stream) for H in Hs]
         perm = [0] + [1 + i for i in order]
-        Wp = W.permute(*perm).contiguous() if order != list(range(len(dims))) else W
-        Q, st = quantize_kron(Wp.reshape(W.shape[0], -1), Ms[0], [Ms[1 + i] for i in order],
-                              scales, bits, clamp, stream=stream)
+        Wp = W.permute(*perm).contiguous() if order != ident else W
+        Q, st = quantize_kron(Wp.reshape(m, -1), Ms[0], [Ms[1 + i] for i in order], scales, bits,
+                              clamp, stream=stream, **(grid or {}))
+        if grid is not None and packed:
+            return Q, st
         Q = Q.reshape(Wp.shape)
-        if order != list(range(len(dims))):
+        if order != ident:
             inv = [0] * len(perm)
             for a_, b_ in enumerate(perm):
                 inv[b_] = a_
             Q = Q.permute(*inv).contiguous()
         return Q, st
     M_L, M_R = prepare_kron(Hs, stream=stream)
-    Q, st = quantize(W.reshape(W.shape[0], -1), M_L, M_R, scales, bits, clamp, stream=stream)
+    if grid is not None:
+        Q, st = quantize_grid(W.reshape(m, -1), M_L, M_R, scales, bits, clamp, stream=stream, **grid)
+        return (Q, st) if packed else (Q.reshape(W.shape), st)
+    Q, st = quantize(W.reshape(m, -1), M_L, M_R, scales, bits, clamp, stream=stream)
     return Q.reshape(W.shape), st
 
 
