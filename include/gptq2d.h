@@ -258,6 +258,19 @@ int gptq2d_gram_finalize(float* H, int64_t k, int64_t ldh, int64_t total_rows, d
 int gptq2d_kron_factor(int nf, const double* const* M, const int64_t* dims, const int64_t* ldm,
                        double* out, int64_t ldo, void* stream);
 
+/* An order of trailing modes for gptq2d_quantize_kron (host only, no GPU work).  The
+ * k-way rounding depends only on each entry's dominated orthant, so reordering modes
+ * 2..k permutes the result and nothing else: a caller may permute W's trailing modes
+ * (and the factors) by `order`, round, and permute Q back.  The subset of modes whose
+ * sizes multiply to the largest of 64, 32, 16, 8 goes last (the inner group), the
+ * others keep their order in front; the given order is kept when it already reaches
+ * that size.
+ *   nf, dims : HOST, the trailing modes' sizes (1 <= nf <= GPTQ2D_MAX_KRON_FACTORS).
+ *   order    : HOST, nf entries: order[p] = the given index of the mode placed p-th.
+ * Returns the inner size m_in the reordered modes give (8, 16, 32 or 64), or 0 when
+ * no subset reaches 8 (order is then the identity); -1 for invalid arguments. */
+int gptq2d_per_mode_order(int nf, const int64_t* dims, int* order);
+
 /* Bytes of device workspace gptq2d_quantize_kron needs for an m x prod(dims)
  * rounding with these trailing modes; 0 when the per-mode path does not apply
  * (see gptq2d_quantize_kron) or the arguments are out of range. */

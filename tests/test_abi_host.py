@@ -347,3 +347,29 @@ def test_per_mode_eligibility_agrees_between_library_and_binding():
 
 def L_global():
     return g.lib()
+
+
+def test_library_per_mode_order_equals_the_binding():
+    """gptq2d_per_mode_order (C, host only) returns the binding's order and the inner
+    size that order gives, on every list up to three modes of sizes 1..12, 16, 32, 64,
+    100, 128; invalid arguments give -1."""
+    import itertools
+    L = g.lib()
+    sizes = list(range(1, 13)) + [16, 32, 64, 100, 128]
+    for k in (1, 2, 3):
+        for dims in itertools.product(sizes, repeat=k):
+            if k == 3 and (dims[0] > 4 or dims[1] > 8):
+                continue
+            da = (ctypes.c_int64 * k)(*dims)
+            oa = (ctypes.c_int * k)()
+            r = L.gptq2d_per_mode_order(k, da, oa)
+            want = g.per_mode_order(list(dims))
+            if want is None:
+                assert r == 0 and list(oa) == list(range(k)), dims
+            else:
+                assert list(oa) == want, (dims, list(oa), want)
+                assert r == g.kron_inner_size([dims[i] for i in want]), dims
+    oa = (ctypes.c_int * 2)()
+    assert L.gptq2d_per_mode_order(0, (ctypes.c_int64 * 1)(8), oa) == -1
+    assert L.gptq2d_per_mode_order(2, (ctypes.c_int64 * 2)(8, 0), oa) == -1
+    assert L.gptq2d_per_mode_order(2, None, oa) == -1

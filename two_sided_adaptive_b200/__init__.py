@@ -124,6 +124,8 @@ def lib():
         L.gptq2d_kron_factor.argtypes = [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p]
         L.gptq2d_quantize_kron_workspace_size.restype = ctypes.c_size_t
         L.gptq2d_quantize_kron_workspace_size.argtypes = [_c_i64, ctypes.c_int, _c_p]
+        L.gptq2d_per_mode_order.restype = ctypes.c_int
+        L.gptq2d_per_mode_order.argtypes = [ctypes.c_int, _c_p, _c_p]
         L.gptq2d_quantize_kron_grid.restype = ctypes.c_int
         L.gptq2d_quantize_kron_grid.argtypes = [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_i64,
                                                 ctypes.c_int, _c_p, _c_p, _c_p,

@@ -411,6 +411,33 @@ int gptq2d_quantize_grid(const void* W, int w_dtype, int64_t m, int64_t n, int64
                          nullptr, nullptr, &gs);
 }
 
+int gptq2d_per_mode_order(int nf, const int64_t* dims, int* order) {
+  if (nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !dims || !order) return -1;
+  for (int f = 0; f < nf; ++f)
+    if (dims[f] < 1) return -1;
+  for (int f = 0; f < nf; ++f) order[f] = f;
+  int best_mask = 0;
+  int64_t best_p = 0;
+  for (int mask = 1; mask < (1 << nf); ++mask) {
+    int64_t p = 1;
+    for (int f = 0; f < nf && p <= 64; ++f)
+      if ((mask >> f) & 1) p *= dims[f];
+    if ((p == 8 || p == 16 || p == 32 || p == 64) && p > best_p) {
+      best_p = p;
+      best_mask = mask;
+    }
+  }
+  if (best_p == 0) return 0;
+  int nin = 0;
+  if (kron_inner(nf, dims, &nin) == best_p) return (int)best_p;  // the given order reaches it
+  int k = 0;
+  for (int f = 0; f < nf; ++f)
+    if (!((best_mask >> f) & 1)) order[k++] = f;
+  for (int f = 0; f < nf; ++f)
+    if ((best_mask >> f) & 1) order[k++] = f;
+  return (int)best_p;
+}
+
 size_t gptq2d_quantize_kron_workspace_size(int64_t m, int nf, const int64_t* dims) {
   if (m < 0 || m > kMaxDim || nf < 1 || nf > GPTQ2D_MAX_KRON_FACTORS || !dims) return 0;
   int64_t n = 1;
