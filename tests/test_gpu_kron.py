@@ -357,3 +357,32 @@ def test_quantize_tensor_grid_routes(g, shape, route):
     rep = check_against_oracle(W2, Ms[0], O.kron_factor(Ms[1:]), None, 4, True, q, grid=grid)
     assert g.stats_dict(st)["status"] == 0
     np.testing.assert_array_equal(codes, O.stored_codes(rep.result.Q, m, n, 4, G, Z))
+
+
+@pytest.mark.slow
+def test_per_mode_4096x64x64_every_entry(g):
+    """The per-mode route at full size (the kron3 bench's 4096 x 64 x 64 tensor, INT4,
+    bf16 weights): every one of the 16.8 M entries is the rounding of its own y computed
+    from the GPU's integers with the dense Kronecker factor (tests/parity.py fixed
+    point), and the in-kernel loss equals the oracle's identity from the same check."""
+    from tests.parity import check_fixed_point
+    rng = np.random.default_rng(4096)
+    dims = (4096, 64, 64)
+    Hs = [_spd(rng, d) for d in dims]
+    W = rng.normal(0, 0.02, dims).astype(np.float32)
+    m, n = 4096, 4096
+    Wb = torch.from_numpy(W.reshape(m, n)).to(torch.bfloat16)
+    W64 = Wb.double().numpy()
+    s = WL.absmax_scales(W64, 4).astype(np.float32)
+    Ms = [O.reverse_cholesky(H) for H in Hs]
+    Q, st = g.quantize_kron(Wb.cuda(), torch.from_numpy(Ms[0]).cuda(),
+                            [torch.from_numpy(M).cuda() for M in Ms[1:]],
+                            torch.from_numpy(s).cuda(), 4, True)
+    torch.cuda.synchronize()
+    d = g.stats_dict(st)
+    assert d["status"] == 0
+    rep = check_fixed_point(W64, Ms[0], O.kron_factor(Ms[1:]), s.astype(np.float64), 4, True,
+                            Q.cpu().numpy())
+    assert rep.n_entries == m * n
+    print(f"per-mode 4096x64x64: {rep.n_entries} entries checked, near-ties {rep.n_near_tie} "
+          f"(GPU counted {d['n_near_tie']}), other neighbour taken at {rep.n_other_neighbour}")
